@@ -1,0 +1,167 @@
+"""fp64 NumPy oracle: the plain definition of softmax attention and its gradient.
+
+TEST INFRASTRUCTURE ONLY (see the package docstring): the product path never
+imports this module.
+
+Arrays are [B, H, N, d] (queries, keys, values, output, output gradient) and
+[B, H, N] (log-sum-exp).  Inputs may be any real dtype; they are upcast exactly
+to float64 before any arithmetic, so the oracle sees precisely the 16-bit values
+the GPU sees.  Per (batch, head) slice the full score rows are materialised for a
+chunk of query rows (memory is chunk x N, never N x N for large N), the softmax
+of each row is taken exactly (subtract the row maximum, exponentiate, divide by
+the sum) and the rest are ordinary matrix products.  Nothing here is tiled over
+keys or computed incrementally: that is the GPU path's business, and the point
+of this module is to be the reference it is checked against.
+
+Sources (page title, section):
+  * "Flash Attention spiegata: una guida completa" (datacamp), "Attention
+    standard vs Flash attention": the fast method computes exactly standard
+    attention.
+  * "FlashAttention-2" (systems-analysis.info wiki), "Предпосылки": standard
+    attention materialises the full score matrix -- which is what this oracle
+    does, a chunk of rows at a time.
+  * "Flash Attention spiegata", "Ricomputazione": the backward pass recomputes
+    the probabilities from the scores; here they are recomputed from scratch
+    per chunk as well.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+_ROW_CHUNK = 1024
+
+
+def _f64(x) -> np.ndarray:
+    """Exact upcast to float64 (torch tensors are converted through numpy)."""
+    if hasattr(x, "detach"):  # torch.Tensor without importing torch here
+        x = x.detach().cpu().double().numpy()
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+
+
+def _check_shapes(q, k, v):
+    if q.ndim != 4 or k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k, v must all be [B, H, N, d] with equal shapes")
+
+
+def _scores(q_rows: np.ndarray, k: np.ndarray, row0: int, scale: float,
+            causal: bool) -> tuple[np.ndarray, int]:
+    """Scaled scores S = scale * q_rows k^T for query rows row0..row0+len-1.
+
+    With ``causal`` the keys after each row's own position are set to -inf and
+    only keys 0..row_last are formed at all.  Returns (S, number of keys used).
+    """
+    n_rows = q_rows.shape[0]
+    n_keys = min(k.shape[0], row0 + n_rows) if causal else k.shape[0]
+    s = scale * (q_rows @ k[:n_keys].T)
+    if causal:
+        rows = row0 + np.arange(n_rows)[:, None]
+        cols = np.arange(n_keys)[None, :]
+        s = np.where(cols > rows, -np.inf, s)
+    return s, n_keys
+
+
+def _softmax_rows(s: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
+    """Exact row softmax and row log-sum-exp of a score block (fp64)."""
+    m = s.max(axis=1, keepdims=True)
+    e = np.exp(s - m)
+    z = e.sum(axis=1, keepdims=True)
+    return e / z, (m + np.log(z))[:, 0]
+
+
+def attn_fwd_rows_ref(q, k, v, scale: float, causal: bool, bh: int,
+                      rows) -> tuple[np.ndarray, np.ndarray]:
+    """O and LSE of selected query rows of one flattened (batch*head) slice.
+
+    ``q, k, v`` are [B, H, N, d]; ``bh`` indexes the flattened B*H axis; ``rows``
+    is a sequence of query row indices.  Returns (O [len(rows), d],
+    LSE [len(rows)]), fp64.  Used to check full-size GPU runs on a sample of
+    rows without forming every row.
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    _check_shapes(q, k, v)
+    B, H, N, d = q.shape
+    b, h = divmod(int(bh), H)
+    rows = np.asarray(rows, dtype=np.int64)
+    out = np.empty((rows.size, d))
+    lse = np.empty(rows.size)
+    for t, r in enumerate(rows):
+        s, nk = _scores(q[b, h, r:r + 1], k[b, h], int(r), scale, causal)
+        p, l = _softmax_rows(s)
+        out[t] = (p @ v[b, h, :nk])[0]
+        lse[t] = l[0]
+    return out, lse
+
+
+def attn_fwd_ref(q, k, v, scale: float, causal: bool,
+                 row_chunk: int = _ROW_CHUNK) -> tuple[np.ndarray, np.ndarray]:
+    """Forward attention: O = softmax(scale * Q K^T [causal mask]) V, and LSE.
+
+    Returns (O [B,H,N,d], LSE [B,H,N]) in fp64.
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    _check_shapes(q, k, v)
+    B, H, N, d = q.shape
+    out = np.empty((B, H, N, d))
+    lse = np.empty((B, H, N))
+    for b in range(B):
+        for h in range(H):
+            for r0 in range(0, N, row_chunk):
+                r1 = min(N, r0 + row_chunk)
+                s, nk = _scores(q[b, h, r0:r1], k[b, h], r0, scale, causal)
+                p, l = _softmax_rows(s)
+                out[b, h, r0:r1] = p @ v[b, h, :nk]
+                lse[b, h, r0:r1] = l
+    return out, lse
+
+
+def attn_probs_ref(q, k, scale: float, causal: bool) -> np.ndarray:
+    """The full probability matrix P [B,H,N,N] (tiny shapes only; for pins)."""
+    q, k = _f64(q), _f64(k)
+    B, H, N, d = q.shape
+    p_all = np.zeros((B, H, N, N))
+    for b in range(B):
+        for h in range(H):
+            s, nk = _scores(q[b, h], k[b, h], 0, scale, causal)
+            p, _ = _softmax_rows(s)
+            p_all[b, h, :, :nk] = p
+    return p_all
+
+
+def attn_bwd_ref(q, k, v, do, scale: float, causal: bool,
+                 row_chunk: int = _ROW_CHUNK, heads=None):
+    """Gradients of L = sum(O * dO) with respect to Q, K and V (fp64).
+
+    The probabilities are recomputed from the scores of each chunk of query
+    rows; D_i = sum_j P_ij dP_ij is taken from P and dP directly (not from the
+    forward output).  ``heads`` optionally restricts the work to a list of
+    flattened (batch*head) indices; other slices of the results are left as
+    NaN.  Returns (dQ, dK, dV), each [B,H,N,d].
+    """
+    q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
+    _check_shapes(q, k, v)
+    if do.shape != q.shape:
+        raise ValueError("do must have the shape of q")
+    B, H, N, d = q.shape
+    dq = np.full((B, H, N, d), np.nan)
+    dk = np.full((B, H, N, d), np.nan)
+    dv = np.full((B, H, N, d), np.nan)
+    todo = range(B * H) if heads is None else [int(x) for x in heads]
+    for bh in todo:
+        b, h = divmod(bh, H)
+        dk_bh = np.zeros((N, d))
+        dv_bh = np.zeros((N, d))
+        for r0 in range(0, N, row_chunk):
+            r1 = min(N, r0 + row_chunk)
+            s, nk = _scores(q[b, h, r0:r1], k[b, h], r0, scale, causal)
+            p, _ = _softmax_rows(s)
+            do_c = do[b, h, r0:r1]
+            dv_bh[:nk] += p.T @ do_c
+            dp = do_c @ v[b, h, :nk].T
+            dd = (p * dp).sum(axis=1, keepdims=True)
+            ds = p * (dp - dd)
+            dq[b, h, r0:r1] = scale * (ds @ k[b, h, :nk])
+            dk_bh[:nk] += scale * (ds.T @ q[b, h, r0:r1])
+        dk[b, h] = dk_bh
+        dv[b, h] = dv_bh
+    return dq, dk, dv

@@ -1,0 +1,357 @@
+"""Pins of the fp64 CPU oracle against things other than itself.
+
+Each pin is a function of the oracle's two entry points (forward, backward), so
+the same pins can be run against deliberately broken copies of the oracle
+(``test_pins_catch_planted_mistakes``): every planted mistake -- a wrong causal
+diagonal, a dropped scale, a dropped term of the softmax gradient, a transposed
+probability matrix, a log in the wrong base -- must fail at least one pin.
+
+What the pins rest on:
+  * the scalar C brute force (independent code);
+  * PyTorch's fp64 CPU attention and autograd (library routines);
+  * closed forms (Q = 0, N = 1, constant V, causal row 0);
+  * invariances (a common shift of all keys, a permutation of the keys);
+  * central finite differences of L = sum(O * dO).
+The pages say the method is exact up to rounding ("Flash Attention spiegata",
+"Attention standard vs Flash attention"; "Flash Attention 2: attivarla",
+"Perché Flash Attention 2"), so all of these must hold to fp64 rounding.
+"""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle import attention as oatt
+from oracle.brute import brute_bwd, brute_fwd
+from exact_io_aware_74_b200.workloads import WORKLOADS, make_inputs, workload_inputs
+
+RTOL = 1e-12
+
+
+def _rand(shape, seed, scale=1.0):
+    rng = np.random.default_rng(seed)
+    return scale * rng.standard_normal(shape)
+
+
+def _close(a, b, tol=RTOL):
+    a, b = np.asarray(a), np.asarray(b)
+    denom = max(1.0, float(np.max(np.abs(b))) if b.size else 1.0)
+    err = float(np.max(np.abs(a - b))) if a.size else 0.0
+    assert err <= tol * denom, f"max abs err {err:.3e} > {tol:.1e} * {denom:.3e}"
+
+
+def _torch_sdpa(q, k, v, scale, causal):
+    tq, tk, tv = (torch.from_numpy(np.asarray(x, dtype=np.float64)) for x in (q, k, v))
+    return torch.nn.functional.scaled_dot_product_attention(
+        tq, tk, tv, is_causal=causal, scale=scale).numpy()
+
+
+# ----------------------------------------------------------------------------------
+# pins, each a function of (fwd, bwd)
+# ----------------------------------------------------------------------------------
+
+SMALL_SHAPES = [(1, 2, 1, 4), (1, 2, 5, 4), (1, 2, 33, 4), (1, 2, 33, 64), (2, 1, 17, 8)]
+
+
+def pin_brute_force(fwd, bwd):
+    for i, shape in enumerate(SMALL_SHAPES):
+        for causal in (False, True):
+            q, k, v, do = (_rand(shape, 10 * i + j) for j in range(4))
+            s = 1.0 / math.sqrt(shape[-1])
+            o, lse = fwd(q, k, v, s, causal)
+            bo, blse = brute_fwd(q, k, v, s, causal)
+            _close(o, bo)
+            _close(lse, blse)
+            dq, dk, dv = bwd(q, k, v, do, s, causal)
+            bq, bk, bv = brute_bwd(q, k, v, do, s, causal)
+            _close(dq, bq)
+            _close(dk, bk)
+            _close(dv, bv)
+
+
+def pin_torch_library(fwd, bwd):
+    for i, (B, H, N, d) in enumerate([(2, 3, 37, 16), (1, 2, 64, 32)]):
+        for causal in (False, True):
+            q, k, v, do = (_rand((B, H, N, d), 100 + 4 * i + j) for j in range(4))
+            s = 0.3 + 0.1 * i
+            o, lse = fwd(q, k, v, s, causal)
+            _close(o, _torch_sdpa(q, k, v, s, causal))
+            tq, tk, tv = (torch.tensor(x, requires_grad=True) for x in (q, k, v))
+            sc = s * tq @ tk.transpose(-1, -2)
+            if causal:
+                sc = sc.masked_fill(torch.ones(N, N, dtype=torch.bool).triu(1), float("-inf"))
+            _close(lse, torch.logsumexp(sc, dim=-1).detach().numpy())
+            to = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, is_causal=causal,
+                                                                  scale=s)
+            (to * torch.from_numpy(do)).sum().backward()
+            dq, dk, dv = bwd(q, k, v, do, s, causal)
+            _close(dq, tq.grad.numpy(), 1e-10)
+            _close(dk, tk.grad.numpy(), 1e-10)
+            _close(dv, tv.grad.numpy(), 1e-10)
+
+
+def pin_rows_sum_to_one(fwd, bwd):
+    q, k = _rand((1, 2, 29, 8), 1), _rand((1, 2, 29, 8), 2)
+    for causal in (False, True):
+        p = oracle.attn_probs_ref(q, k, 0.5, causal)
+        _close(p.sum(-1), np.ones((1, 2, 29)))
+        if causal:
+            assert np.all(np.triu(p[0, 0], 1) == 0)
+
+
+def pin_constant_v(fwd, bwd):
+    B, H, N, d = 1, 2, 40, 8
+    q, k = _rand((B, H, N, d), 3, 3.0), _rand((B, H, N, d), 4, 3.0)
+    row = _rand((d,), 5)
+    v = np.broadcast_to(row, (B, H, N, d)).copy()
+    for causal in (False, True):
+        o, _ = fwd(q, k, v, 0.7, causal)
+        _close(o, v)
+
+
+def pin_causal_row0_and_n1(fwd, bwd):
+    B, H, N, d = 2, 2, 9, 8
+    q, k, v = (_rand((B, H, N, d), 6 + j) for j in range(3))
+    s = 0.4
+    o, lse = fwd(q, k, v, s, True)
+    _close(o[:, :, 0], v[:, :, 0])
+    _close(lse[:, :, 0], s * np.einsum("bhc,bhc->bh", q[:, :, 0], k[:, :, 0]))
+    for causal in (False, True):
+        o1, l1 = fwd(q[:, :, :1], k[:, :, :1], v[:, :, :1], s, causal)
+        _close(o1, v[:, :, :1])
+        _close(l1[:, :, 0], s * np.einsum("bhc,bhc->bh", q[:, :, 0], k[:, :, 0]))
+
+
+def pin_zero_queries(fwd, bwd):
+    B, H, N, d = 1, 3, 21, 8
+    q = np.zeros((B, H, N, d))
+    k, v = _rand((B, H, N, d), 9), _rand((B, H, N, d), 10)
+    o, lse = fwd(q, k, v, 1.3, False)
+    _close(o, np.broadcast_to(v.mean(axis=2, keepdims=True), o.shape))
+    _close(lse, np.full((B, H, N), math.log(N)))
+    o, lse = fwd(q, k, v, 1.3, True)
+    counts = np.arange(1, N + 1)
+    _close(o, np.cumsum(v, axis=2) / counts[None, None, :, None])
+    _close(lse, np.broadcast_to(np.log(counts), (B, H, N)))
+
+
+def pin_key_shift(fwd, bwd):
+    """K' = K + 1 u^T adds s q_i.u to every visible score of row i."""
+    B, H, N, d = 1, 2, 33, 16
+    q, k, v, do = (_rand((B, H, N, d), 20 + j) for j in range(4))
+    u = _rand((d,), 30, 4.0)
+    s = 0.25
+    for causal in (False, True):
+        o, lse = fwd(q, k, v, s, causal)
+        o2, lse2 = fwd(q, k + u, v, s, causal)
+        _close(o2, o, 1e-11)
+        _close(lse2, lse + s * np.einsum("bhnc,c->bhn", q, u), 1e-11)
+        # the loss does not depend on a common shift of the keys: sum_j dK_j = 0
+        dq, dk, dv = bwd(q, k, v, do, s, causal)
+        _close(dk.sum(axis=2), np.zeros((B, H, d)), 1e-11)
+        # rows of P sum to one: sum_j dV_j = sum_i dO_i
+        _close(dv.sum(axis=2), do.sum(axis=2), 1e-11)
+
+
+def pin_key_permutation(fwd, bwd):
+    B, H, N, d = 2, 2, 31, 8
+    q, k, v, do = (_rand((B, H, N, d), 40 + j) for j in range(4))
+    perm = np.random.default_rng(7).permutation(N)
+    o, lse = fwd(q, k, v, 0.6, False)
+    o2, lse2 = fwd(q, k[:, :, perm], v[:, :, perm], 0.6, False)
+    _close(o2, o)
+    _close(lse2, lse)
+    _, dk, dv = bwd(q, k, v, do, 0.6, False)
+    _, dk2, dv2 = bwd(q, k[:, :, perm], v[:, :, perm], do, 0.6, False)
+    _close(dk2, dk[:, :, perm])
+    _close(dv2, dv[:, :, perm])
+
+
+def pin_finite_differences(fwd, bwd):
+    eps = 1e-6
+    for N, causal in ((3, False), (5, True), (5, False)):
+        B, H, d = 1, 1, 4
+        q, k, v, do = (_rand((B, H, N, d), 50 + N + j) for j in range(4))
+        s = 0.8
+
+        def loss(qq, kk, vv):
+            o, _ = fwd(qq, kk, vv, s, causal)
+            return float((o * do).sum())
+
+        grads = bwd(q, k, v, do, s, causal)
+        for which, g in enumerate(grads):
+            num = np.zeros_like(g)
+            args = [q, k, v]
+            for idx in np.ndindex(*g.shape):
+                plus = [a.copy() for a in args]
+                minus = [a.copy() for a in args]
+                plus[which][idx] += eps
+                minus[which][idx] -= eps
+                num[idx] = (loss(*plus) - loss(*minus)) / (2 * eps)
+            _close(g, num, 1e-6)
+
+
+PINS = [pin_brute_force, pin_torch_library, pin_rows_sum_to_one, pin_constant_v,
+        pin_causal_row0_and_n1, pin_zero_queries, pin_key_shift, pin_key_permutation,
+        pin_finite_differences]
+
+
+@pytest.mark.parametrize("pin", PINS, ids=[p.__name__ for p in PINS])
+def test_oracle_pin(pin):
+    pin(oracle.attn_fwd_ref, oracle.attn_bwd_ref)
+
+
+# ----------------------------------------------------------------------------------
+# planted mistakes (in copies of the oracle, on the CPU) must fail some pin
+# ----------------------------------------------------------------------------------
+
+def _mut_scores_diag(q_rows, k, row0, scale, causal):
+    """Causal mask that also hides the diagonal (j >= i instead of j > i)."""
+    n_rows = q_rows.shape[0]
+    n_keys = min(k.shape[0], row0 + n_rows) if causal else k.shape[0]
+    s = scale * (q_rows @ k[:n_keys].T)
+    if causal:
+        rows = row0 + np.arange(n_rows)[:, None]
+        cols = np.arange(n_keys)[None, :]
+        s = np.where(cols >= rows, -np.inf, s)
+        s[:, 0] = np.where(np.isinf(s[:, 0]), 0.0, s[:, 0])  # keep row 0 finite
+    return s, n_keys
+
+
+def _mut_softmax_log2(s):
+    m = s.max(axis=1, keepdims=True)
+    e = np.exp(s - m)
+    z = e.sum(axis=1, keepdims=True)
+    return e / z, (m + np.log2(z))[:, 0]
+
+
+def _bwd_variant(kind):
+    def bwd(q, k, v, do, scale, causal):
+        q, k, v, do = (np.asarray(x, dtype=np.float64) for x in (q, k, v, do))
+        B, H, N, d = q.shape
+        dq, dk, dv = (np.zeros((B, H, N, d)) for _ in range(3))
+        for b in range(B):
+            for h in range(H):
+                s, nk = oatt._scores(q[b, h], k[b, h], 0, scale, causal)
+                p, _ = oatt._softmax_rows(s)
+                dp = do[b, h] @ v[b, h, :nk].T
+                dd = 0.0 if kind == "drop_D" else (p * dp).sum(1, keepdims=True)
+                ds = p * (dp - dd)
+                ks = 1.0 if kind == "drop_dk_scale" else scale
+                pv = p if kind == "transpose_dv" else p.T
+                dv[b, h, :nk] = pv @ do[b, h] if kind != "transpose_dv" else (pv @ do[b, h])[:nk]
+                dq[b, h] = scale * ds @ k[b, h, :nk]
+                dk[b, h, :nk] = ks * ds.T @ q[b, h]
+        return dq, dk, dv
+    return bwd
+
+
+MUTANTS = ["causal_diag", "lse_log2", "drop_D", "drop_dk_scale", "transpose_dv"]
+
+
+@pytest.mark.parametrize("mutant", MUTANTS)
+def test_pins_catch_planted_mistakes(mutant, monkeypatch):
+    fwd, bwd = oracle.attn_fwd_ref, oracle.attn_bwd_ref
+    if mutant == "causal_diag":
+        monkeypatch.setattr(oatt, "_scores", _mut_scores_diag)
+    elif mutant == "lse_log2":
+        monkeypatch.setattr(oatt, "_softmax_rows", _mut_softmax_log2)
+    else:
+        bwd = _bwd_variant(mutant)
+    failed = []
+    for pin in PINS:
+        if pin is pin_finite_differences and mutant in ("causal_diag", "lse_log2"):
+            continue  # forward mutants are caught faster elsewhere
+        try:
+            pin(fwd, bwd)
+        except AssertionError:
+            failed.append(pin.__name__)
+    assert failed, f"planted mistake {mutant!r} passed every pin"
+
+
+def test_bwd_variant_is_exact_when_unmutated():
+    """The mutant scaffold itself reproduces the oracle when nothing is planted."""
+    q, k, v, do = (_rand((1, 2, 13, 8), 70 + j) for j in range(4))
+    for causal in (False, True):
+        a = _bwd_variant("none")(q, k, v, do, 0.5, causal)
+        b = oracle.attn_bwd_ref(q, k, v, do, 0.5, causal)
+        for x, y in zip(a, b):
+            _close(x, y)
+
+
+# ----------------------------------------------------------------------------------
+# internal consistency of the oracle's own entry points
+# ----------------------------------------------------------------------------------
+
+def test_row_chunking_and_row_sampler_agree():
+    q, k, v, do = (_rand((2, 2, 70, 16), 80 + j) for j in range(4))
+    for causal in (False, True):
+        o, lse = oracle.attn_fwd_ref(q, k, v, 0.3, causal)
+        o7, lse7 = oracle.attn_fwd_ref(q, k, v, 0.3, causal, row_chunk=7)
+        _close(o7, o)
+        _close(lse7, lse)
+        rows = [0, 1, 33, 69]
+        bo, blse = brute_fwd(q, k, v, 0.3, causal)
+        ro, rl = oracle.attn_fwd_rows_ref(q, k, v, 0.3, causal, bh=3, rows=rows)
+        _close(ro, bo[1, 1, rows])
+        _close(rl, blse[1, 1, rows])
+        g = oracle.attn_bwd_ref(q, k, v, do, 0.3, causal)
+        g9 = oracle.attn_bwd_ref(q, k, v, do, 0.3, causal, row_chunk=9, heads=[2])
+        for x, y in zip(g9, g):
+            _close(x[1, 0], y[1, 0])
+            assert np.isnan(x[0, 0]).all()
+
+
+def test_D_equals_rowdot_of_output():
+    """D_i = sum_j P_ij dP_ij equals sum_c dO_ic O_ic (used by the GPU backward)."""
+    q, k, v, do = (_rand((1, 1, 24, 8), 90 + j) for j in range(4))
+    for causal in (False, True):
+        o, _ = oracle.attn_fwd_ref(q, k, v, 0.5, causal)
+        p = oracle.attn_probs_ref(q, k, 0.5, causal)[0, 0]
+        dp = do[0, 0] @ v[0, 0].T
+        _close((p * dp).sum(1), (do[0, 0] * o[0, 0]).sum(1))
+
+
+# ----------------------------------------------------------------------------------
+# the seeded input recipe
+# ----------------------------------------------------------------------------------
+
+def test_inputs_are_seeded_and_exact_in_fp64():
+    a = make_inputs(1, 2, 64, 16, "bf16", 5, with_do=True)
+    b = make_inputs(1, 2, 64, 16, "bf16", 5, with_do=True)
+    for key in ("q", "k", "v", "do"):
+        assert a[key].dtype == torch.bfloat16
+        assert torch.equal(a[key], b[key])
+        # upcast to fp64 and back is lossless
+        assert torch.equal(a[key].double().to(torch.bfloat16), a[key])
+    c = make_inputs(1, 2, 64, 16, "bf16", 6)
+    assert not torch.equal(a["q"], c["q"])
+
+
+def test_outlier_rows_recipe():
+    w = WORKLOADS["fwd_bf16_b1h32_n32768_d128_causal_outliers"]
+    x = make_inputs(1, 2, 1000, 8, "bf16", w.seed, outlier_frac=0.01, outlier_mult=8.0)
+    plain = make_inputs(1, 2, 1000, 8, "bf16", w.seed)
+    rows = x["outlier_rows"]
+    assert rows.shape == (1, 2, 10)
+    for h in range(2):
+        idx = rows[0, h]
+        assert len(set(idx.tolist())) == 10
+        mask = torch.zeros(1000, dtype=torch.bool)
+        mask[idx] = True
+        # non-outlier rows unchanged, outlier rows exactly x8 (power of two)
+        assert torch.equal(x["k"][0, h, ~mask], plain["k"][0, h, ~mask])
+        assert torch.equal(x["k"][0, h, mask].float(), 8 * plain["k"][0, h, mask].float())
+
+
+def test_workload_table():
+    flops = {n: w.fwd_flops for n, w in WORKLOADS.items()}
+    assert flops["fwd_fp16_b1h2_n128_d64"] == 4 * 2 * 128 * 128 * 64
+    assert flops["fwd_bf16_b2h32_n8192_d128"] == pytest.approx(2.199e12, rel=1e-3)
+    w4 = WORKLOADS["fwdbwd_bf16_b8h16_n4096_d128_causal"]
+    assert w4.bwd_flops == pytest.approx(1.374e12, rel=1e-3)
+    small = workload_inputs(WORKLOADS["fwd_fp16_b1h2_n128_d64"])
+    assert small["q"].dtype == torch.float16 and small["q"].shape == (1, 2, 128, 64)
