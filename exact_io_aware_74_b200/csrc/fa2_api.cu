@@ -1,0 +1,257 @@
+// Host side of libfa2.so: argument validation, TMA descriptor encoding, kernel
+// launch and the device status word.  Declarations and the contract of every
+// entry point are in include/fa2.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstdlib>
+#include <mutex>
+
+#include "../../include/fa2.h"
+#include "fa2_bwd.cuh"
+#include "fa2_fwd.cuh"
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr unsigned int kDefaultWaitMs = 2000;
+
+std::mutex g_mu;
+unsigned int* g_status[kMaxDevices] = {};  // one device word per device, lazily allocated
+std::atomic<int> g_fault{0};
+std::atomic<unsigned int> g_wait_ms{kDefaultWaitMs};
+std::atomic<unsigned long long> g_launches{0};
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return static_cast<EncodeTiledFn>(nullptr);
+    return reinterpret_cast<EncodeTiledFn>(p);
+  }();
+  return fn;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool overlaps(const void* a, const void* b, size_t bytes) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + bytes && y < x + bytes;
+}
+
+// Common checks of fa2_fwd / fa2_bwd that need no CUDA call.
+int check_sizes(int B, int H, int N, int d, float scale, int causal, int dtype) {
+  if (B < 1 || H < 1 || N < 1) return FA2_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return FA2_ERR_INVALID_ARG;
+  if (dtype != FA2_FP16 && dtype != FA2_BF16) return FA2_ERR_INVALID_ARG;
+  if (!std::isfinite(scale) || !(scale > 0.f)) return FA2_ERR_INVALID_ARG;
+  if (static_cast<long long>(B) * H > (1ll << 30) || N > (1 << 30)) return FA2_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA2_ERR_UNSUPPORTED;
+  return FA2_OK;
+}
+
+// Current device must be compute capability 10.0; returns its ordinal in *dev.
+int check_device(int* dev) {
+  if (cudaGetDevice(dev) != cudaSuccess) {
+    cudaGetLastError();
+    return FA2_ERR_CUDA;
+  }
+  int major = 0, minor = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, *dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, *dev) != cudaSuccess) {
+    cudaGetLastError();
+    return FA2_ERR_CUDA;
+  }
+  if (major != 10 || minor != 0) return FA2_ERR_ARCH;
+  if (*dev < 0 || *dev >= kMaxDevices) return FA2_ERR_CUDA;
+  return FA2_OK;
+}
+
+unsigned int* status_word(int dev) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (!g_status[dev]) {
+    void* p = nullptr;
+    if (cudaMalloc(&p, 256) != cudaSuccess) return nullptr;
+    if (cudaMemset(p, 0, 256) != cudaSuccess) return nullptr;
+    g_status[dev] = static_cast<unsigned int*>(p);
+  }
+  return g_status[dev];
+}
+
+// [BH][N][d] 16-bit tensor viewed as a 3-D TMA map with 128-row x 64-column
+// boxes and 128-byte swizzle; rows past N read as zeros.
+bool make_map(CUtensorMap* map, const void* base, int BH, int N, int d, int dtype) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
+                              static_cast<cuuint64_t>(BH)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
+                                 static_cast<cuuint64_t>(N) * d * 2};
+  const cuuint32_t box[3] = {64, 128, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUtensorMapDataType ty =
+      dtype == FA2_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  return enc(map, ty, 3, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+unsigned long long wait_ns() { return static_cast<unsigned long long>(g_wait_ms.load()) * 1000000ull; }
+
+template <int D, bool BF16, bool CAUSAL>
+int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+               const fa2::FwdParams& p, cudaStream_t stream) {
+  using Cfg = fa2::FwdCfg<D>;
+  auto kern = fa2::fa2_fwd_kernel<D, BF16, CAUSAL>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM) !=
+      cudaSuccess) {
+    cudaGetLastError();
+    return FA2_ERR_CUDA;
+  }
+  const unsigned int grid = static_cast<unsigned int>(p.n_qblk) * static_cast<unsigned int>(p.BH);
+  kern<<<grid, Cfg::THREADS, Cfg::SMEM, stream>>>(mq, mk, mv, p);
+  if (cudaGetLastError() != cudaSuccess) return FA2_ERR_CUDA;
+  g_launches.fetch_add(1);
+  return FA2_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int fa2_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, int B, int H,
+            int N, int d, float scale, int causal, int dtype, fa2_stream_t stream) {
+  if (!Q || !K || !V || !O || !LSE) return FA2_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(LSE))
+    return FA2_ERR_INVALID_ARG;
+  int rc = check_sizes(B, H, N, d, scale, causal, dtype);
+  if (rc != FA2_OK) return rc;
+  const int BH = B * H;
+  const size_t bytes = static_cast<size_t>(BH) * N * d * 2;
+  if (overlaps(O, Q, bytes) || overlaps(O, K, bytes) || overlaps(O, V, bytes) ||
+      overlaps(LSE, O, bytes))
+    return FA2_ERR_INVALID_ARG;
+  int dev = 0;
+  rc = check_device(&dev);
+  if (rc != FA2_OK) return rc;
+  unsigned int* st = status_word(dev);
+  if (!st) return FA2_ERR_CUDA;
+
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, Q, BH, N, d, dtype) || !make_map(&mk, K, BH, N, d, dtype) ||
+      !make_map(&mv, V, BH, N, d, dtype))
+    return FA2_ERR_CUDA;
+
+  fa2::FwdParams p{};
+  p.O = O;
+  p.LSE = LSE;
+  p.N = N;
+  p.BH = BH;
+  p.n_qblk = (N + 255) / 256;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.status = st;
+  p.wait_ns = wait_ns();
+  p.fault = g_fault.load();
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const bool bf = dtype == FA2_BF16;
+  if (d == 64) {
+    if (bf) return causal ? launch_fwd<64, true, true>(mq, mk, mv, p, s) : launch_fwd<64, true, false>(mq, mk, mv, p, s);
+    return causal ? launch_fwd<64, false, true>(mq, mk, mv, p, s) : launch_fwd<64, false, false>(mq, mk, mv, p, s);
+  }
+  if (bf) return causal ? launch_fwd<128, true, true>(mq, mk, mv, p, s) : launch_fwd<128, true, false>(mq, mk, mv, p, s);
+  return causal ? launch_fwd<128, false, true>(mq, mk, mv, p, s) : launch_fwd<128, false, false>(mq, mk, mv, p, s);
+}
+
+size_t fa2_bwd_workspace_size(int B, int H, int N, int d) {
+  if (check_sizes(B, H, N, d, 1.0f, 0, FA2_BF16) != FA2_OK) return 0;
+  return fa2::bwd_workspace_bytes(static_cast<size_t>(B) * H, N, d);
+}
+
+int fa2_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO,
+            const float* LSE, void* dQ, void* dK, void* dV, void* workspace,
+            size_t workspace_bytes, int B, int H, int N, int d, float scale, int causal,
+            int dtype, fa2_stream_t stream) {
+  if (!Q || !K || !V || !O || !dO || !LSE || !dQ || !dK || !dV) return FA2_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(dO) ||
+      !aligned16(LSE) || !aligned16(dQ) || !aligned16(dK) || !aligned16(dV))
+    return FA2_ERR_INVALID_ARG;
+  int rc = check_sizes(B, H, N, d, scale, causal, dtype);
+  if (rc != FA2_OK) return rc;
+  const int BH = B * H;
+  const size_t bytes = static_cast<size_t>(BH) * N * d * 2;
+  const void* ins[6] = {Q, K, V, O, dO, LSE};
+  void* outs[3] = {dQ, dK, dV};
+  for (void* o : outs) {
+    for (const void* in : ins)
+      if (overlaps(o, in, bytes)) return FA2_ERR_INVALID_ARG;
+  }
+  if (overlaps(dQ, dK, bytes) || overlaps(dQ, dV, bytes) || overlaps(dK, dV, bytes))
+    return FA2_ERR_INVALID_ARG;
+  const size_t need = fa2::bwd_workspace_bytes(static_cast<size_t>(BH), N, d);
+  if (!workspace || workspace_bytes < need ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return FA2_ERR_WORKSPACE;
+  int dev = 0;
+  rc = check_device(&dev);
+  if (rc != FA2_OK) return rc;
+  unsigned int* st = status_word(dev);
+  if (!st) return FA2_ERR_CUDA;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  rc = fa2::launch_bwd(Q, K, V, O, dO, LSE, dQ, dK, dV, workspace, BH, N, d, scale, causal != 0,
+                       dtype == FA2_BF16, st, wait_ns(), s);
+  if (rc == FA2_OK) g_launches.fetch_add(fa2::kBwdKernelsPerCall);
+  return rc;
+}
+
+int fa2_get_device_status(fa2_stream_t stream, int* site) {
+  if (site) *site = 0;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return FA2_ERR_CUDA;
+  }
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return FA2_ERR_CUDA;
+  unsigned int* st = status_word(dev);
+  if (!st) return FA2_ERR_CUDA;
+  unsigned int w = 0;
+  if (cudaMemcpy(&w, st, sizeof(w), cudaMemcpyDeviceToHost) != cudaSuccess) return FA2_ERR_CUDA;
+  if (w != 0 && cudaMemset(st, 0, sizeof(w)) != cudaSuccess) return FA2_ERR_CUDA;
+  if (site) *site = static_cast<int>((w >> 8) & 0xFFu);
+  const unsigned int code = w & 0xFFu;
+  return code == 0 ? FA2_OK : static_cast<int>(code);
+}
+
+const char* fa2_status_string(int status) {
+  switch (status) {
+    case FA2_OK: return "FA2_OK";
+    case FA2_ERR_INVALID_ARG: return "FA2_ERR_INVALID_ARG";
+    case FA2_ERR_UNSUPPORTED: return "FA2_ERR_UNSUPPORTED";
+    case FA2_ERR_ARCH: return "FA2_ERR_ARCH";
+    case FA2_ERR_CUDA: return "FA2_ERR_CUDA";
+    case FA2_ERR_TIMEOUT: return "FA2_ERR_TIMEOUT";
+    case FA2_ERR_WORKSPACE: return "FA2_ERR_WORKSPACE";
+    default: return "FA2_ERR_UNKNOWN";
+  }
+}
+
+void fa2_debug_set(int fault, unsigned int wait_limit_ms) {
+  g_fault.store(fault == 1 ? 1 : 0);
+  g_wait_ms.store(wait_limit_ms == 0 ? kDefaultWaitMs : wait_limit_ms);
+}
+
+unsigned long long fa2_launch_count(void) { return g_launches.load(); }
+
+}  // extern "C"

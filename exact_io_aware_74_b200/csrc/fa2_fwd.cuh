@@ -1,0 +1,383 @@
+// Forward pass of exact attention on sm_100a: O = softmax(scale Q K^T [causal]) V
+// and the row log-sum-exp, tile by tile, with no N x N matrix in HBM.
+//
+// Sources (page title, section):
+//   "Flash Attention spiegata: una guida completa" (datacamp), "Tiling": Q, K
+//   and V are split into tiles that sit in fast on-chip memory and each tile is
+//   processed end to end with the softmax applied incrementally.
+//   "FlashAttention-2" (systems-analysis.info wiki), "Техническая архитектура и
+//   принципы работы": (1) fewer non-matmul operations -- here the running
+//   maximum is only applied to the output when it grows by more than 2^8, and
+//   the 1/l normalisation happens once at the end; (2) parallelism over the
+//   sequence -- every CTA owns 256 query rows of one (batch, head); (3) work
+//   split across warps so that softmax statistics never go through shared
+//   memory -- here one thread owns one query row, read straight from TMEM.
+//   "Flash Attention spiegata", "Specializzazione dei warp" and "TMA":
+//   producer and consumer warps and asynchronous tile copies (Hopper-era prior
+//   art, restated for tcgen05).
+//
+// CTA layout (320 threads):
+//   warps 0-3  softmax warpgroup for query tile 0 (rows r0 .. r0+127)
+//   warps 4-7  softmax warpgroup for query tile 1 (rows r0+128 .. r0+255)
+//   warp  8    TMA producer (Q once, then a ring of K and V tiles)
+//   warp  9    MMA issuer (tcgen05, one thread)
+// TMEM (512 columns x 128 lanes, fp32): S_t at column 128 t, O_t at 256 + D t.
+// P_t (16-bit) overwrites the first 64 columns of S_t and feeds the P V MMA
+// straight from TMEM.  The MMA warp alternates between the two query tiles so
+// that one warpgroup's softmax overlaps the other tile's matrix products.
+#pragma once
+
+#include "ptx.cuh"
+
+namespace fa2 {
+
+struct FwdParams {
+  void* O;                     // [BH][N][D] 16-bit
+  float* LSE;                  // [BH][N]
+  int N;                       // sequence length
+  int BH;                      // batch * heads
+  int n_qblk;                  // ceil(N / 256)
+  float scale_log2;            // scale * log2(e)
+  unsigned int* status;        // device status word
+  unsigned long long wait_ns;  // budget of one bounded wait
+  int fault;                   // test hook: 1 = skip the first K load
+};
+
+template <int D>
+struct FwdCfg {
+  static constexpr int BM = 128;                  // query rows per tile
+  static constexpr int BN = 128;                  // keys per tile
+  static constexpr int QT = 2;                    // query tiles per CTA
+  static constexpr int KCH = D / 64;              // 128-byte swizzle chunks along d
+  static constexpr int CHUNK = 128 * 128;         // bytes of one 128-row x 64-col chunk
+  static constexpr int TILE = 128 * D * 2;        // bytes of one 128-row tile
+  static constexpr int KS = (D == 64) ? 4 : 2;    // K ring stages
+  static constexpr int VS = (D == 64) ? 4 : 2;    // V ring stages
+  static constexpr int SMEM = (QT + KS + VS) * TILE + 1024;
+  static constexpr int THREADS = 320;
+  static constexpr uint32_t S_COL0 = 0, S_COL1 = 128;
+  static constexpr uint32_t O_COL0 = 256, O_COL1 = 256 + D;
+};
+
+// Wait-site ids reported through the status word.
+enum FwdSite : uint32_t {
+  kSiteProdKEmpty = 1, kSiteProdVEmpty, kSiteMmaQ, kSiteMmaK, kSiteMmaV, kSiteMmaP,
+  kSiteMmaDrain, kSiteSoftS, kSiteSoftO, kSiteSoftOEnd, kSiteProdDrain
+};
+
+template <int D, bool BF16, bool CAUSAL>
+__global__ void __launch_bounds__(320, 1)
+fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+               const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
+  using C = FwdCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* sQ = smem;
+  uint8_t* sK = sQ + C::QT * C::TILE;
+  uint8_t* sV = sK + C::KS * C::TILE;
+
+  __shared__ uint64_t bar_q, k_full[C::KS], k_empty[C::KS], v_full[C::VS], v_empty[C::VS];
+  __shared__ uint64_t s_full[2], p_ready[2], o_done[2], drain;
+  __shared__ uint32_t tmem_slot;
+  __shared__ int abort_flag;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int N = p.N;
+
+  // Heaviest query blocks first (they see the most keys when causal).
+  const int qb = p.n_qblk - 1 - static_cast<int>(blockIdx.x) / p.BH;
+  const int bh = static_cast<int>(blockIdx.x) % p.BH;
+  const int n_kv_all = (N + C::BN - 1) / C::BN;
+  int row0[2], n_kv[2];
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    row0[t] = qb * 256 + t * 128;
+    if (row0[t] >= N) {
+      n_kv[t] = 0;
+    } else if (CAUSAL) {
+      n_kv[t] = min(n_kv_all, row0[t] / C::BN + 1);
+    } else {
+      n_kv[t] = n_kv_all;
+    }
+  }
+  const int n_kv_max = max(n_kv[0], n_kv[1]);
+
+  WaitCtl wc{p.status, &abort_flag, p.wait_ns};
+
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    mbar_init(&bar_q, 1);
+    for (int s = 0; s < C::KS; ++s) { mbar_init(&k_full[s], 1); mbar_init(&k_empty[s], 1); }
+    for (int s = 0; s < C::VS; ++s) { mbar_init(&v_full[s], 1); mbar_init(&v_empty[s], 1); }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&s_full[t], 1);
+      mbar_init(&p_ready[t], 4);
+      mbar_init(&o_done[t], 1);
+    }
+    mbar_init(&drain, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(&tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = tmem_slot;
+
+  if (warp == 8) {
+    // ------------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      const uint64_t keep = policy_evict_last();
+      uint32_t q_bytes = 0;
+      for (int t = 0; t < 2; ++t) q_bytes += (n_kv[t] > 0) ? C::TILE : 0;
+      mbar_arrive_expect_tx(&bar_q, q_bytes);
+      for (int t = 0; t < 2; ++t) {
+        if (n_kv[t] == 0) continue;
+        for (int c = 0; c < C::KCH; ++c)
+          tma_load_3d(sQ + t * C::TILE + c * C::CHUNK, &tmQ, &bar_q, c * 64, row0[t], bh);
+      }
+      int k_issued = 0, v_issued = 0;  // loads issued so far
+      bool ok = true;
+      for (int j = 0; j < n_kv_max && ok; ++j) {
+        const int ks = j % C::KS, vs = j % C::VS;
+        if (j >= C::KS && !mbar_wait(&k_empty[ks], ((j / C::KS) - 1) & 1, wc, kSiteProdKEmpty)) {
+          ok = false;
+          break;
+        }
+        if (!(p.fault == 1 && j == 0)) {
+          mbar_arrive_expect_tx(&k_full[ks], C::TILE);
+          for (int c = 0; c < C::KCH; ++c)
+            tma_load_3d_hint(sK + ks * C::TILE + c * C::CHUNK, &tmK, &k_full[ks], c * 64,
+                             j * C::BN, bh, keep);
+          k_issued = j + 1;
+        }
+        if (j >= C::VS && !mbar_wait(&v_empty[vs], ((j / C::VS) - 1) & 1, wc, kSiteProdVEmpty)) {
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(&v_full[vs], C::TILE);
+        for (int c = 0; c < C::KCH; ++c)
+          tma_load_3d_hint(sV + vs * C::TILE + c * C::CHUNK, &tmV, &v_full[vs], c * 64,
+                           j * C::BN, bh, keep);
+        v_issued = j + 1;
+      }
+      if (!ok) {
+        // Let every copy already issued land before the CTA exits.
+        volatile int no_abort = 0;
+        WaitCtl dw{p.status, &no_abort, 100000000ull};
+        // The last load put into each ring slot is load jj; its phase is jj / stages.
+        for (int jj = max(0, k_issued - C::KS); jj < k_issued; ++jj)
+          if (!(p.fault == 1 && jj == 0))
+            mbar_wait(&k_full[jj % C::KS], (jj / C::KS) & 1, dw, kSiteProdDrain);
+        for (int jj = max(0, v_issued - C::VS); jj < v_issued; ++jj)
+          mbar_wait(&v_full[jj % C::VS], (jj / C::VS) & 1, dw, kSiteProdDrain);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 9) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t id_qk = idesc_f16(128, 128, BF16, false, false);
+      constexpr uint32_t id_pv = idesc_f16(128, D, BF16, false, true);
+      const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV);
+
+      auto issue_qk = [&](int t, int ks) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * C::CHUNK + (kk & 3) * 32;
+          umma_ss(tbase + (t ? C::S_COL1 : C::S_COL0), sdesc_sw128(sQa + t * C::TILE + off, 16, 1024),
+                  sdesc_sw128(sKa + ks * C::TILE + off, 16, 1024), id_qk, kk > 0);
+        }
+      };
+      auto issue_pv = [&](int t, int vs, bool acc) {
+#pragma unroll
+        for (int kk = 0; kk < C::BN / 16; ++kk) {
+          umma_ts(tbase + (t ? C::O_COL1 : C::O_COL0), tbase + (t ? C::S_COL1 : C::S_COL0) + kk * 8,
+                  sdesc_sw128(sVa + vs * C::TILE + kk * 2048, C::CHUNK, 1024), id_pv,
+                  (acc || kk > 0) ? 1u : 0u);
+        }
+      };
+
+      bool ok = mbar_wait(&bar_q, 0, wc, kSiteMmaQ) && mbar_wait(&k_full[0], 0, wc, kSiteMmaK);
+      if (ok) {
+        tc_fence_after();
+        issue_qk(0, 0);
+        umma_commit(&s_full[0]);
+        if (n_kv[1] > 0) {
+          issue_qk(1, 0);
+          umma_commit(&s_full[1]);
+        }
+        umma_commit(&k_empty[0]);
+      }
+      for (int j = 0; j < n_kv_max && ok; ++j) {
+        const int vs = j % C::VS;
+        const int ks1 = (j + 1) % C::KS;
+        const bool has_next = j + 1 < n_kv_max;
+        bool k_next_ready = false;
+        if (!mbar_wait(&v_full[vs], (j / C::VS) & 1, wc, kSiteMmaV)) { ok = false; break; }
+        auto tile_step = [&](int t, int nkv_t) -> bool {
+          if (j >= nkv_t) return true;
+          if (!mbar_wait(&p_ready[t], j & 1, wc, kSiteMmaP)) return false;
+          tc_fence_after();
+          issue_pv(t, vs, j > 0);
+          umma_commit(&o_done[t]);
+          if (j + 1 < nkv_t) {
+            if (!k_next_ready) {
+              if (!mbar_wait(&k_full[ks1], ((j + 1) / C::KS) & 1, wc, kSiteMmaK)) return false;
+              tc_fence_after();
+              k_next_ready = true;
+            }
+            issue_qk(t, ks1);
+            umma_commit(&s_full[t]);
+          }
+          return true;
+        };
+        ok = tile_step(0, n_kv[0]) && tile_step(1, n_kv[1]);
+        if (!ok) break;
+        umma_commit(&v_empty[vs]);
+        if (has_next) umma_commit(&k_empty[ks1]);
+      }
+      // Every MMA issued above completes before TMEM is released.
+      umma_commit(&drain);
+      volatile int no_abort = 0;
+      WaitCtl dw{p.status, &no_abort, p.wait_ns};
+      mbar_wait(&drain, 0, dw, kSiteMmaDrain);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------------ softmax
+    const int t = warp >> 2;      // query tile of this warpgroup
+    const int wq = warp & 3;      // TMEM lane quadrant
+    const int r_loc = wq * 32 + lane;
+    const int my_row0 = t ? row0[1] : row0[0];
+    const int my_nkv = t ? n_kv[1] : n_kv[0];
+    const int row = my_row0 + r_loc;
+    const uint32_t s_col = t ? C::S_COL1 : C::S_COL0;
+    const uint32_t o_col = t ? C::O_COL1 : C::O_COL0;
+    const uint32_t lane_base = static_cast<uint32_t>(wq * 32);
+    const float sl2 = p.scale_log2;  // > 0 (checked on the host)
+    float m = -INFINITY;  // running max, log2 units of scaled scores
+    float l = 0.f;        // running sum of exp2(s * sl2 - m)
+    bool ok = my_nkv > 0;
+    for (int j = 0; j < my_nkv && ok; ++j) {
+      // Warp-uniform wait: the TMEM loads and stores below are warp-collective.
+      ok = __all_sync(0xffffffffu, mbar_wait(&s_full[t], j & 1, wc, kSiteSoftS));
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t sr[128];
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+        tmem_ld32(tmem_addr(tbase, lane_base, s_col + 32 * c),
+                  *reinterpret_cast<uint32_t(*)[32]>(&sr[32 * c]));
+      tmem_wait_ld();
+      reg_fence(sr);
+      const int key0 = j * C::BN;
+      const bool need_mask = (CAUSAL && key0 + C::BN - 1 > my_row0) || (key0 + C::BN > N);
+      if (need_mask) {
+        const int lim = CAUSAL ? min(row - key0 + 1, N - key0) : (N - key0);
+#pragma unroll
+        for (int i = 0; i < 128; ++i)
+          if (i >= lim) sr[i] = __float_as_uint(-INFINITY);
+      }
+      float mx[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) mx[k] = __uint_as_float(sr[k]);
+#pragma unroll
+      for (int i = 8; i < 128; ++i) mx[i & 7] = fmaxf(mx[i & 7], __uint_as_float(sr[i]));
+#pragma unroll
+      for (int k = 4; k >= 1; k >>= 1)
+#pragma unroll
+        for (int q = 0; q < k; ++q) mx[q] = fmaxf(mx[q], mx[q + k]);
+      const float m_new = fmaxf(m, mx[0] * sl2);
+      if (j == 0) {
+        m = m_new;
+      } else {
+        // Lazy rescale: the stale maximum is kept unless it fell behind by more
+        // than 8 (a factor 256 in the exponentials); the output accumulator is
+        // only touched in that case, after the previous P V product landed.
+        const bool need = m_new - m > 8.0f;
+        if (__any_sync(0xffffffffu, need)) {
+          const float f = need ? ex2_approx(m - m_new) : 1.0f;
+          if (need) m = m_new;
+          l *= f;
+          ok = __all_sync(0xffffffffu, mbar_wait(&o_done[t], (j - 1) & 1, wc, kSiteSoftO));
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t r[32];
+            tmem_ld32(tmem_addr(tbase, lane_base, o_col + 32 * c), r);
+            tmem_wait_ld();
+            reg_fence(r);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * f);
+            tmem_st32(tmem_addr(tbase, lane_base, o_col + 32 * c), r);
+          }
+        }
+      }
+      const float neg_m = -m;
+      float sum[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float a = ex2_approx(fmaf(__uint_as_float(sr[64 * h + 2 * i]), sl2, neg_m));
+          const float b = ex2_approx(fmaf(__uint_as_float(sr[64 * h + 2 * i + 1]), sl2, neg_m));
+          sum[(2 * i) & 3] += a;
+          sum[(2 * i + 1) & 3] += b;
+          pk[i] = pack2<BF16>(a, b);
+        }
+        tmem_st32(tmem_addr(tbase, lane_base, s_col + 32 * h), pk);
+      }
+      l += (sum[0] + sum[1]) + (sum[2] + sum[3]);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_ready[t]);
+    }
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&o_done[t], (my_nkv - 1) & 1, wc, kSiteSoftOEnd));
+    if (ok) {
+      tc_fence_after();
+      const float inv_l = 1.0f / l;
+      uint8_t* orow = reinterpret_cast<uint8_t*>(p.O) +
+                      (static_cast<size_t>(bh) * N + row) * (D * 2);
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld32(tmem_addr(tbase, lane_base, o_col + 32 * c), r);
+        tmem_wait_ld();
+        reg_fence(r);
+        uint4 v[4];
+        uint32_t* pv = reinterpret_cast<uint32_t*>(v);
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          pv[i] = pack2<BF16>(__uint_as_float(r[2 * i]) * inv_l,
+                              __uint_as_float(r[2 * i + 1]) * inv_l);
+        if (row < N) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + c * 64);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) dst[i] = v[i];
+        }
+      }
+      if (row < N)
+        p.LSE[static_cast<size_t>(bh) * N + row] = (m + __log2f(l)) * 0.69314718055994531f;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tbase, 512);
+  }
+}
+
+}  // namespace fa2

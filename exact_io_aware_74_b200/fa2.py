@@ -1,0 +1,162 @@
+"""ctypes binding of libfa2.so (declared in include/fa2.h).
+
+Argument marshalling only: every step of the attention computation runs in the
+library's CUDA kernels.  Tensors are torch CUDA tensors (PyTorch provides device
+memory and streams); they are passed to the C ABI as raw device pointers.  A
+missing or unloadable library raises ``RuntimeError`` -- there is no fallback.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libfa2.so")
+
+FA2_OK = 0
+FA2_ERR_INVALID_ARG = 1
+FA2_ERR_UNSUPPORTED = 2
+FA2_ERR_ARCH = 3
+FA2_ERR_CUDA = 4
+FA2_ERR_TIMEOUT = 5
+FA2_ERR_WORKSPACE = 6
+FA2_FP16 = 0
+FA2_BF16 = 1
+
+# Every symbol include/fa2.h declares.
+EXPORTS = ("fa2_fwd", "fa2_bwd_workspace_size", "fa2_bwd", "fa2_get_device_status",
+           "fa2_status_string", "fa2_debug_set", "fa2_launch_count")
+
+_lib = None
+
+
+class FA2Error(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} ({status})")
+
+
+def load() -> ctypes.CDLL:
+    """Open libfa2.so (once) and declare the C signatures."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                           "`python -m exact_io_aware_74_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    lib.fa2_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, i, vp]
+    lib.fa2_fwd.restype = i
+    lib.fa2_bwd_workspace_size.argtypes = [i, i, i, i]
+    lib.fa2_bwd_workspace_size.restype = sz
+    lib.fa2_bwd.argtypes = [vp] * 10 + [sz, i, i, i, i, f, i, i, vp]
+    lib.fa2_bwd.restype = i
+    lib.fa2_get_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_int)]
+    lib.fa2_get_device_status.restype = i
+    lib.fa2_status_string.argtypes = [i]
+    lib.fa2_status_string.restype = ctypes.c_char_p
+    lib.fa2_debug_set.argtypes = [i, ctypes.c_uint]
+    lib.fa2_debug_set.restype = None
+    lib.fa2_launch_count.argtypes = []
+    lib.fa2_launch_count.restype = ctypes.c_ulonglong
+    _lib = lib
+    return lib
+
+
+def status_string(status: int) -> str:
+    return load().fa2_status_string(int(status)).decode()
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return FA2_BF16
+    if t.dtype == torch.float16:
+        return FA2_FP16
+    raise TypeError(f"unsupported dtype {t.dtype}; use float16 or bfloat16")
+
+
+def _ptr(t) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _check_layout(*ts):
+    for t in ts:
+        if not (t.is_cuda and t.is_contiguous()):
+            raise ValueError("tensors must be contiguous CUDA tensors")
+
+
+def fa2_fwd(q, k, v, o, lse, scale: float, causal: bool, stream=None) -> int:
+    """Raw call: q, k, v, o [B,H,N,d] 16-bit; lse [B,H,N] float32.  Returns the status."""
+    _check_layout(q, k, v, o, lse)
+    B, H, N, d = q.shape
+    return load().fa2_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d,
+                          float(scale), int(bool(causal)), _dtype_code(q), _stream(stream))
+
+
+def fa2_bwd_workspace_size(B: int, H: int, N: int, d: int) -> int:
+    return int(load().fa2_bwd_workspace_size(B, H, N, d))
+
+
+def fa2_bwd(q, k, v, o, do, lse, dq, dk, dv, workspace, scale: float, causal: bool,
+            stream=None) -> int:
+    """Raw call; ``workspace`` is a uint8 CUDA tensor.  Returns the status."""
+    _check_layout(q, k, v, o, do, lse, dq, dk, dv)
+    B, H, N, d = q.shape
+    ws_ptr = _ptr(workspace)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    return load().fa2_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse), _ptr(dq),
+                          _ptr(dk), _ptr(dv), ws_ptr, ws_bytes, B, H, N, d, float(scale),
+                          int(bool(causal)), _dtype_code(q), _stream(stream))
+
+
+def fa2_get_device_status(stream=None) -> tuple[int, int]:
+    """(status, wait site) of the current device; synchronises ``stream``."""
+    site = ctypes.c_int(0)
+    rc = load().fa2_get_device_status(_stream(stream), ctypes.byref(site))
+    return rc, site.value
+
+
+def fa2_debug_set(fault: int, wait_limit_ms: int = 0) -> None:
+    load().fa2_debug_set(int(fault), int(wait_limit_ms))
+
+
+def fa2_launch_count() -> int:
+    return int(load().fa2_launch_count())
+
+
+# ------------------------------------------------------------------------------------
+# allocating conveniences (PyTorch owns the memory)
+# ------------------------------------------------------------------------------------
+
+def forward(q, k, v, scale: float, causal: bool, stream=None):
+    """Allocates O and LSE, calls fa2_fwd, raises FA2Error on a bad status."""
+    B, H, N, d = q.shape
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    rc = fa2_fwd(q, k, v, o, lse, scale, causal, stream)
+    if rc != FA2_OK:
+        raise FA2Error(rc, "fa2_fwd")
+    return o, lse
+
+
+def backward(q, k, v, o, do, lse, scale: float, causal: bool, workspace=None, stream=None):
+    """Allocates dQ, dK, dV (and the workspace if not given), calls fa2_bwd."""
+    B, H, N, d = q.shape
+    if workspace is None:
+        workspace = torch.empty(fa2_bwd_workspace_size(B, H, N, d), dtype=torch.uint8,
+                                device=q.device)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    rc = fa2_bwd(q, k, v, o, do, lse, dq, dk, dv, workspace, scale, causal, stream)
+    if rc != FA2_OK:
+        raise FA2Error(rc, "fa2_bwd")
+    return dq, dk, dv

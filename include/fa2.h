@@ -1,0 +1,135 @@
+/*
+ * fa2.h -- C ABI of the B200 (sm_100a) exact-attention library libfa2.so.
+ *
+ * The library computes exact scaled-dot-product attention
+ *
+ *     O = softmax(Q K^T * scale [+ causal mask]) V
+ *
+ * tile by tile in on-chip memory, never writing an N x N matrix to HBM, and its
+ * gradient by recomputing the probabilities from the saved log-sum-exp.
+ *
+ * Sources (page title, section):
+ *   [DC]  "Flash Attention spiegata: una guida completa" (datacamp):
+ *         "Attention standard vs Flash attention" (exact, not an approximation;
+ *         tiles in fast on-chip memory, softmax applied incrementally);
+ *         "Tiling"; "Ricomputazione" (the backward pass recomputes scores).
+ *   [RU]  "FlashAttention-2" (systems-analysis.info wiki):
+ *         "Предпосылки" (IO-aware tiling, memory linear in N);
+ *         "Техническая архитектура и принципы работы" (fewer non-matmul
+ *         operations, parallelism over the sequence, work split across warps).
+ *   [QL]  "Flash Attention 2: attivarla (llama.cpp, Ollama, vLLM)" (qualellm.it):
+ *         "Perché Flash Attention 2" (same mathematical result);
+ *         troubleshooting "Errore unsupported head dimension" (unsupported head
+ *         sizes are reported as an error).
+ *
+ * Conventions shared by every call
+ *   - Tensors are dense, contiguous, row-major [B][H][N][d] in the 16-bit
+ *     dtype given by ``dtype``; LSE and the backward's D are [B][H][N] float.
+ *   - All pointers are DEVICE pointers on the current CUDA device, owned by the
+ *     caller, 16-byte aligned.  The library keeps no reference after a call
+ *     returns (work is enqueued on ``stream``).
+ *   - ``causal`` = 1 lets query row i see keys 0..i; 0 lets it see all keys.
+ *   - LSE_i = ln sum_j exp(S_ij) over the keys row i sees, S = scale * Q K^T.
+ *   - The return value reports argument validation and launch only; the kernels
+ *     run asynchronously.  Failures inside a kernel (a bounded wait that ran out)
+ *     are reported by fa2_get_device_status().
+ *   - Head dims 64 and 128 are supported; any other d returns
+ *     FA2_ERR_UNSUPPORTED and launches nothing (no silent fallback).
+ *   - Only compute capability 10.0 devices (B200, sm_100a) are supported;
+ *     others return FA2_ERR_ARCH.
+ *   - The library allocates one small device status word per device on first
+ *     use and nothing per call.
+ */
+#ifndef FA2_H_
+#define FA2_H_
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Opaque CUDA stream (cudaStream_t); NULL is the legacy default stream. */
+typedef struct CUstream_st* fa2_stream_t;
+
+typedef enum {
+  FA2_OK = 0,
+  FA2_ERR_INVALID_ARG = 1, /* null / misaligned pointer, bad size, flag or scale */
+  FA2_ERR_UNSUPPORTED = 2, /* head dim other than 64 or 128 */
+  FA2_ERR_ARCH = 3,        /* current device is not compute capability 10.0 */
+  FA2_ERR_CUDA = 4,        /* a CUDA runtime / driver call failed */
+  FA2_ERR_TIMEOUT = 5,     /* a bounded in-kernel wait ran out (device status) */
+  FA2_ERR_WORKSPACE = 6    /* backward workspace null or too small */
+} fa2_status;
+
+typedef enum { FA2_FP16 = 0, FA2_BF16 = 1 } fa2_dtype;
+
+/*
+ * Forward pass.  [DC] "Tiling", "Attention standard vs Flash attention";
+ * [RU] "Техническая архитектура и принципы работы".
+ *
+ *   Q, K, V : in,  [B][H][N][d] dtype
+ *   O       : out, [B][H][N][d] dtype, O_i = sum_j softmax_j(S_i) V_j
+ *   LSE     : out, [B][H][N] float (natural log, scaled-score units)
+ *   B, H, N : >= 1; d in {64, 128}; scale finite; causal in {0, 1};
+ *   dtype   : FA2_FP16 or FA2_BF16
+ * O must not overlap Q, K or V.  Results are bitwise repeatable run to run.
+ */
+int fa2_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, int B, int H,
+            int N, int d, float scale, int causal, int dtype, fa2_stream_t stream);
+
+/*
+ * Bytes of device workspace fa2_bwd needs for these sizes (the per-row
+ * D = rowsum(dO * O) and a float32 dQ accumulator), a multiple of 256.
+ * Returns 0 for sizes fa2_bwd would reject.
+ */
+size_t fa2_bwd_workspace_size(int B, int H, int N, int d);
+
+/*
+ * Backward pass.  [DC] "Ricomputazione": the probabilities are recomputed from
+ * Q, K and the saved LSE, then dV = P^T dO, dP = dO V^T, D = rowsum(dO * O),
+ * dS = P * (dP - D), dQ = scale dS K, dK = scale dS^T Q.
+ *
+ *   Q, K, V, O, dO : in,  [B][H][N][d] dtype (O and LSE as fa2_fwd wrote them)
+ *   LSE            : in,  [B][H][N] float
+ *   dQ, dK, dV     : out, [B][H][N][d] dtype
+ *   workspace      : scratch of at least fa2_bwd_workspace_size() bytes,
+ *                    256-byte aligned, owned by the caller; its contents on
+ *                    entry do not matter and on return are unspecified
+ * Other arguments as for fa2_fwd.  dQ is accumulated with float atomics, so it
+ * may differ in the last bits from run to run; dK and dV are repeatable.
+ */
+int fa2_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO,
+            const float* LSE, void* dQ, void* dK, void* dV, void* workspace,
+            size_t workspace_bytes, int B, int H, int N, int d, float scale, int causal,
+            int dtype, fa2_stream_t stream);
+
+/*
+ * Synchronises ``stream``, then returns and clears the current device's status
+ * word: FA2_OK, or FA2_ERR_TIMEOUT if a kernel gave up a bounded wait since the
+ * last call (the kernel then skipped its output and exited cleanly; the CUDA
+ * context stays usable).  FA2_ERR_CUDA if the synchronisation itself failed.
+ * If ``site`` is not NULL it receives the id of the wait that ran out (0 if none).
+ */
+int fa2_get_device_status(fa2_stream_t stream, int* site);
+
+/* Human-readable name of a status code (static storage). */
+const char* fa2_status_string(int status);
+
+/*
+ * Test hook.  ``wait_limit_ms`` sets the wall-clock budget of every bounded
+ * in-kernel wait (0 restores the default of 2000 ms).  ``fault`` = 1 makes the
+ * next forward launches skip their first K-tile load, so a consumer's wait
+ * runs out and the timeout path is exercised without any GPU fault; 0 turns it
+ * off.  Not for production use.
+ */
+void fa2_debug_set(int fault, unsigned int wait_limit_ms);
+
+/* Number of kernels this library has launched in this process (all devices). */
+unsigned long long fa2_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA2_H_ */

@@ -1,0 +1,101 @@
+"""Host-side checks of the C ABI that need no GPU.
+
+The library must load and export every symbol include/fa2.h declares, and argument
+validation must reject bad calls before any CUDA call is made (so these run on a
+machine without a GPU).
+"""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from exact_io_aware_74_b200 import fa2
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _header_functions():
+    src = open(os.path.join(ROOT, "include", "fa2.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(fa2_[a-z_]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from exact_io_aware_74_b200 import build
+    build.build()
+    return fa2.load()
+
+
+def test_header_declarations_match_binding():
+    assert _header_functions() == sorted(fa2.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in _header_functions():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings(lib):
+    assert fa2.status_string(fa2.FA2_OK) == "FA2_OK"
+    assert fa2.status_string(fa2.FA2_ERR_TIMEOUT) == "FA2_ERR_TIMEOUT"
+    assert fa2.status_string(99) == "FA2_ERR_UNKNOWN"
+
+
+P = 1 << 20  # a fake, 16-byte aligned "device pointer": never dereferenced on these paths
+
+
+@pytest.mark.parametrize("args,expect", [
+    ((0, P, P, P, P, 1, 1, 64, 64, 0.1, 0, 1), fa2.FA2_ERR_INVALID_ARG),        # null Q
+    ((P + 2, P, P, 2 * P, 3 * P, 1, 1, 64, 64, 0.1, 0, 1), fa2.FA2_ERR_INVALID_ARG),  # misaligned
+    ((P, P, P, 2 * P, 3 * P, 0, 1, 64, 64, 0.1, 0, 1), fa2.FA2_ERR_INVALID_ARG),  # B = 0
+    ((P, P, P, 2 * P, 3 * P, 1, 1, 0, 64, 0.1, 0, 1), fa2.FA2_ERR_INVALID_ARG),   # N = 0
+    ((P, P, P, 2 * P, 3 * P, 1, 1, 64, 64, 0.1, 2, 1), fa2.FA2_ERR_INVALID_ARG),  # causal = 2
+    ((P, P, P, 2 * P, 3 * P, 1, 1, 64, 64, 0.1, 0, 5), fa2.FA2_ERR_INVALID_ARG),  # dtype
+    ((P, P, P, 2 * P, 3 * P, 1, 1, 64, 64, float("nan"), 0, 1), fa2.FA2_ERR_INVALID_ARG),
+    ((P, P, P, 2 * P, 3 * P, 1, 1, 64, 64, -0.5, 0, 1), fa2.FA2_ERR_INVALID_ARG),  # scale <= 0
+    ((P, P, P, P, 3 * P, 1, 1, 64, 64, 0.1, 0, 1), fa2.FA2_ERR_INVALID_ARG),     # O aliases Q
+    ((P, P, P, 2 * P, 3 * P, 1, 1, 64, 96, 0.1, 0, 1), fa2.FA2_ERR_UNSUPPORTED),  # d = 96
+    ((P, P, P, 2 * P, 3 * P, 1, 1, 64, 256, 0.1, 0, 1), fa2.FA2_ERR_UNSUPPORTED),
+])
+def test_fwd_validation_without_device(lib, args, expect):
+    assert lib.fa2_fwd(*args, None) == expect
+
+
+def test_bwd_validation_without_device(lib):
+    ws = fa2.fa2_bwd_workspace_size(2, 3, 1000, 128)
+    assert ws > 0 and ws % 256 == 0
+    # D and LSE*log2(e) padded to 128 rows per head, then the fp32 dQ accumulator
+    assert ws >= 2 * 3 * 1000 * 128 * 4
+    assert fa2.fa2_bwd_workspace_size(2, 3, 1000, 96) == 0
+    ptrs = [P * (i + 1) for i in range(9)]
+    # workspace too small
+    rc = lib.fa2_bwd(*ptrs, 16 * P, 256, 1, 1, 64, 64, 0.1, 0, 1, None)
+    assert rc == fa2.FA2_ERR_WORKSPACE
+    # null dK
+    bad = list(ptrs)
+    bad[7] = 0
+    assert lib.fa2_bwd(*bad, 16 * P, ws, 1, 1, 64, 64, 0.1, 0, 1, None) == fa2.FA2_ERR_INVALID_ARG
+    # dQ aliasing Q
+    bad = list(ptrs)
+    bad[6] = bad[0]
+    assert lib.fa2_bwd(*bad, 16 * P, ws, 1, 1, 64, 64, 0.1, 0, 1, None) == fa2.FA2_ERR_INVALID_ARG
+
+
+def test_device_calls_fail_cleanly_without_gpu(lib):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    rc = lib.fa2_fwd(P, 2 * P, 3 * P, 4 * P, 5 * P, 1, 1, 64, 64, 0.1, 0, 1, None)
+    assert rc in (fa2.FA2_ERR_CUDA, fa2.FA2_ERR_ARCH)
+    site = ctypes.c_int(7)
+    assert lib.fa2_get_device_status(None, ctypes.byref(site)) == fa2.FA2_ERR_CUDA
+
+
+def test_binding_fails_loudly_when_library_missing(monkeypatch, tmp_path):
+    monkeypatch.setattr(fa2, "_lib", None)
+    monkeypatch.setattr(fa2, "LIB_PATH", str(tmp_path / "libfa2.so"))
+    with pytest.raises(RuntimeError, match="missing"):
+        fa2.load()
