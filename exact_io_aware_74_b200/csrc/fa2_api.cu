@@ -45,9 +45,10 @@ EncodeTiledFn encode_fn() {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-bool overlaps(const void* a, const void* b, size_t bytes) {
+// True when [a, a + a_bytes) and [b, b + b_bytes) share a byte.
+bool overlaps(const void* a, size_t a_bytes, const void* b, size_t b_bytes) {
   const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
-  return x < y + bytes && y < x + bytes;
+  return x < y + b_bytes && y < x + a_bytes;
 }
 
 // Common checks of fa2_fwd / fa2_bwd that need no CUDA call.
@@ -140,8 +141,11 @@ int fa2_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, in
   if (rc != FA2_OK) return rc;
   const int BH = B * H;
   const size_t bytes = static_cast<size_t>(BH) * N * d * 2;
-  if (overlaps(O, Q, bytes) || overlaps(O, K, bytes) || overlaps(O, V, bytes) ||
-      overlaps(LSE, O, bytes))
+  const size_t lse_bytes = static_cast<size_t>(BH) * N * sizeof(float);
+  if (overlaps(O, bytes, Q, bytes) || overlaps(O, bytes, K, bytes) ||
+      overlaps(O, bytes, V, bytes) || overlaps(LSE, lse_bytes, O, bytes) ||
+      overlaps(LSE, lse_bytes, Q, bytes) || overlaps(LSE, lse_bytes, K, bytes) ||
+      overlaps(LSE, lse_bytes, V, bytes))
     return FA2_ERR_INVALID_ARG;
   int dev = 0;
   rc = check_device(&dev);
@@ -191,13 +195,16 @@ int fa2_bwd(const void* Q, const void* K, const void* V, const void* O, const vo
   if (rc != FA2_OK) return rc;
   const int BH = B * H;
   const size_t bytes = static_cast<size_t>(BH) * N * d * 2;
+  const size_t lse_bytes = static_cast<size_t>(BH) * N * sizeof(float);
   const void* ins[6] = {Q, K, V, O, dO, LSE};
+  const size_t in_bytes[6] = {bytes, bytes, bytes, bytes, bytes, lse_bytes};
   void* outs[3] = {dQ, dK, dV};
   for (void* o : outs) {
-    for (const void* in : ins)
-      if (overlaps(o, in, bytes)) return FA2_ERR_INVALID_ARG;
+    for (int i = 0; i < 6; ++i)
+      if (overlaps(o, bytes, ins[i], in_bytes[i])) return FA2_ERR_INVALID_ARG;
   }
-  if (overlaps(dQ, dK, bytes) || overlaps(dQ, dV, bytes) || overlaps(dK, dV, bytes))
+  if (overlaps(dQ, bytes, dK, bytes) || overlaps(dQ, bytes, dV, bytes) ||
+      overlaps(dK, bytes, dV, bytes))
     return FA2_ERR_INVALID_ARG;
   const size_t need = fa2::bwd_workspace_bytes(static_cast<size_t>(BH), N, d);
   if (!workspace || workspace_bytes < need ||

@@ -64,6 +64,21 @@ def test_fwd_validation_without_device(lib, args, expect):
     assert lib.fa2_fwd(*args, None) == expect
 
 
+def test_fwd_overlap_checks_use_each_buffer_size(lib):
+    """An LSE buffer placed right below O (or right after it) is not an alias."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("these fake pointers are only safe without a device")
+    B, H, N, d = 1, 2, 64, 64
+    o_bytes, lse_bytes = B * H * N * d * 2, B * H * N * 4
+    O = 64 * P
+    for lse in (O - lse_bytes, O + o_bytes):
+        rc = lib.fa2_fwd(P, 2 * P, 3 * P, O, lse, B, H, N, d, 0.1, 0, 1, None)
+        assert rc in (fa2.FA2_ERR_CUDA, fa2.FA2_ERR_ARCH)  # validation passed
+    rc = lib.fa2_fwd(P, 2 * P, 3 * P, O, O + 16, B, H, N, d, 0.1, 0, 1, None)
+    assert rc == fa2.FA2_ERR_INVALID_ARG
+
+
 def test_bwd_validation_without_device(lib):
     ws = fa2.fa2_bwd_workspace_size(2, 3, 1000, 128)
     assert ws > 0 and ws % 256 == 0
