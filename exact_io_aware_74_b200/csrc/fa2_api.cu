@@ -43,6 +43,14 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
+}  // namespace
+
+namespace fa2 {
+bool make_tile_map(CUtensorMap* map, const void* base, int BH, int N, int d, bool bf16);
+}  // namespace fa2
+
+namespace {
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // True when [a, a + a_bytes) and [b, b + b_bytes) share a byte.
@@ -90,9 +98,13 @@ unsigned int* status_word(int dev) {
   return g_status[dev];
 }
 
+}  // namespace
+
+namespace fa2 {
+
 // [BH][N][d] 16-bit tensor viewed as a 3-D TMA map with 128-row x 64-column
 // boxes and 128-byte swizzle; rows past N read as zeros.
-bool make_map(CUtensorMap* map, const void* base, int BH, int N, int d, int dtype) {
+bool make_tile_map(CUtensorMap* map, const void* base, int BH, int N, int d, bool bf16) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
   const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
@@ -102,11 +114,19 @@ bool make_map(CUtensorMap* map, const void* base, int BH, int N, int d, int dtyp
   const cuuint32_t box[3] = {64, 128, 1};
   const cuuint32_t estr[3] = {1, 1, 1};
   const CUtensorMapDataType ty =
-      dtype == FA2_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+      bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
   return enc(map, ty, 3, const_cast<void*>(base), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace fa2
+
+namespace {
+
+bool make_map(CUtensorMap* map, const void* base, int BH, int N, int d, int dtype) {
+  return fa2::make_tile_map(map, base, BH, N, d, dtype == FA2_BF16);
 }
 
 unsigned long long wait_ns() { return static_cast<unsigned long long>(g_wait_ms.load()) * 1000000ull; }

@@ -1,18 +1,569 @@
-// Backward pass (placeholder launcher while the kernels are written).
+// Backward pass of exact attention on sm_100a.
+//
+// Source: "Flash Attention spiegata: una guida completa" (datacamp), section
+// "Ricomputazione": instead of keeping the probabilities for the backward pass,
+// the scores are recomputed from Q and K (cheap next to the memory traffic they
+// would cost).  Here P is rebuilt from the saved log-sum-exp, so no N x N matrix
+// is ever stored.  With dO = dL/dO:
+//   dV = P^T dO,  dP = dO V^T,  D_i = sum_c dO_ic O_ic,
+//   dS = P * (dP - D),  dQ = scale dS K,  dK = scale dS^T Q.
+//
+// Three kernels per call, all on the caller's stream:
+//   1. fa2_bwd_pre_kernel  : D and LSE * log2(e) per query row (padded to a
+//                            multiple of 128 rows), and a zeroed fp32 dQ
+//                            accumulator;
+//   2. fa2_bwd_kernel      : one CTA per (128-key tile, batch*head); loops over
+//                            the query tiles that see those keys;
+//   3. fa2_bwd_dq_kernel   : dQ = scale * accumulator, rounded to 16 bits.
+//
+// Main kernel, CTA layout (192 threads):
+//   warps 0-3 compute warpgroup: thread r owns key row r of the tile for P^T and
+//             dS^T, and query row r of the current query tile when it moves the
+//             dQ partial from TMEM to the fp32 accumulator (vector atomics);
+//   warp  4   TMA producer: K_j and V_j once, then a 2-stage ring of (Q_i, dO_i);
+//   warp  5   tcgen05 MMA issuer (one thread).
+// TMEM (fp32 columns): S^T [0,128) -- P^T (16-bit, packed) overwrites [0,64) and
+// dS^T [64,128); dP^T [128,256); dV [256,256+D); dK [256+D,256+2D); the dQ
+// partial reuses [128,256) when D = 128 and has [384,448) when D = 64.
+// Products (M = 128 rows of the first operand, K = 16 per instruction):
+//   S^T  = K_j  Q_i^T   (A = K smem K-major, B = Q smem K-major)
+//   dP^T = V_j  dO_i^T  (A = V smem K-major, B = dO smem K-major)
+//   dV  += P^T  dO_i    (A = P^T TMEM, B = dO smem MN-major)
+//   dK  += dS^T Q_i     (A = dS^T TMEM, B = Q smem MN-major)
+//   dQ_i = dS   K_j     (A = dS^T smem MN-major, B = K smem MN-major)
 #pragma once
+
+#include <cuda_fp16.h>
+
 #include "ptx.cuh"
+
 namespace fa2 {
+
 constexpr int kBwdKernelsPerCall = 3;
+
+// Workspace: D [BH][Npad] f32 | L2 = LSE*log2(e) [BH][Npad] f32 | dQacc [BH][N][d] f32.
+inline size_t bwd_npad(int N) { return (static_cast<size_t>(N) + 127) / 128 * 128; }
+inline size_t bwd_rowstat_bytes(size_t BH, int N) {
+  return (2 * BH * bwd_npad(N) * 4 + 255) / 256 * 256;
+}
 inline size_t bwd_workspace_bytes(size_t BH, int N, int d) {
-  const size_t npad = (static_cast<size_t>(N) + 127) / 128 * 128;
-  size_t b = 2 * BH * npad * 4;
-  b = (b + 255) / 256 * 256;
-  b += BH * static_cast<size_t>(N) * d * 4;
-  return (b + 255) / 256 * 256;
+  return bwd_rowstat_bytes(BH, N) + (BH * static_cast<size_t>(N) * d * 4 + 255) / 256 * 256;
 }
-inline int launch_bwd(const void*, const void*, const void*, const void*, const void*, const float*,
-                      void*, void*, void*, void*, int, int, int, float, bool, bool, unsigned int*,
-                      unsigned long long, cudaStream_t) {
-  return 2;
+
+// ------------------------------------------------------------------------------------
+// 1. preprocess
+// ------------------------------------------------------------------------------------
+
+template <int D, bool BF16>
+__global__ void __launch_bounds__(256)
+fa2_bwd_pre_kernel(const uint16_t* __restrict__ O, const uint16_t* __restrict__ dO,
+                   const float* __restrict__ LSE, float* __restrict__ Dg,
+                   float* __restrict__ Lg, float* __restrict__ dQacc, int N, int Npad,
+                   long long total_rows) {
+  constexpr int TPR = D / 8;  // threads per row, 8 elements (16 bytes) each
+  constexpr int RPB = 256 / TPR;
+  const int sub = threadIdx.x % TPR;
+  const long long r = static_cast<long long>(blockIdx.x) * RPB + threadIdx.x / TPR;
+  const bool in_range = r < total_rows;  // no early exit: the shuffle below is warp-wide
+  const long long bh = in_range ? r / Npad : 0;
+  const int q = in_range ? static_cast<int>(r % Npad) : N;
+  float acc = 0.f;
+  if (q < N) {
+    const size_t off = (static_cast<size_t>(bh) * N + q) * D + sub * 8;
+    const uint4 a = *reinterpret_cast<const uint4*>(O + off);
+    const uint4 b = *reinterpret_cast<const uint4*>(dO + off);
+    const uint32_t* pa = reinterpret_cast<const uint32_t*>(&a);
+    const uint32_t* pb = reinterpret_cast<const uint32_t*>(&b);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float a0, a1, b0, b1;
+      if constexpr (BF16) {
+        a0 = __uint_as_float(pa[i] << 16); a1 = __uint_as_float(pa[i] & 0xFFFF0000u);
+        b0 = __uint_as_float(pb[i] << 16); b1 = __uint_as_float(pb[i] & 0xFFFF0000u);
+      } else {
+        const __half2 ha = *reinterpret_cast<const __half2*>(&pa[i]);
+        const __half2 hb = *reinterpret_cast<const __half2*>(&pb[i]);
+        a0 = __low2float(ha); a1 = __high2float(ha);
+        b0 = __low2float(hb); b1 = __high2float(hb);
+      }
+      acc = fmaf(a0, b0, acc);
+      acc = fmaf(a1, b1, acc);
+    }
+    float4* z = reinterpret_cast<float4*>(dQacc + off);
+    z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+    z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+#pragma unroll
+  for (int o = TPR / 2; o >= 1; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o, TPR);
+  if (in_range && sub == 0) {
+    Dg[r] = q < N ? acc : 0.f;
+    Lg[r] = q < N ? LSE[static_cast<size_t>(bh) * N + q] * 1.4426950408889634f : INFINITY;
+  }
 }
+
+// ------------------------------------------------------------------------------------
+// 3. dQ finalise
+// ------------------------------------------------------------------------------------
+
+template <bool BF16>
+__global__ void __launch_bounds__(256)
+fa2_bwd_dq_kernel(const float* __restrict__ dQacc, uint16_t* __restrict__ dQ, float scale,
+                  long long n8) {
+  const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= n8) return;
+  const float4 a = reinterpret_cast<const float4*>(dQacc)[2 * i];
+  const float4 b = reinterpret_cast<const float4*>(dQacc)[2 * i + 1];
+  uint4 out;
+  out.x = pack2<BF16>(a.x * scale, a.y * scale);
+  out.y = pack2<BF16>(a.z * scale, a.w * scale);
+  out.z = pack2<BF16>(b.x * scale, b.y * scale);
+  out.w = pack2<BF16>(b.z * scale, b.w * scale);
+  reinterpret_cast<uint4*>(dQ)[i] = out;
+}
+
+// ------------------------------------------------------------------------------------
+// 2. main kernel
+// ------------------------------------------------------------------------------------
+
+struct BwdParams {
+  const float* Dg;    // [BH][Npad]
+  const float* Lg;    // [BH][Npad]
+  float* dQacc;       // [BH][N][D]
+  void* dK;           // [BH][N][D] 16-bit
+  void* dV;           // [BH][N][D] 16-bit
+  int N, Npad, BH, n_kv;
+  float scale, scale_log2;
+  unsigned int* status;
+  unsigned long long wait_ns;
+};
+
+template <int D>
+struct BwdCfg {
+  static constexpr int KCH = D / 64;
+  static constexpr int CHUNK = 128 * 128;
+  static constexpr int TILE = 128 * D * 2;
+  static constexpr int ST = 2;                 // (Q, dO) ring stages
+  static constexpr int DS_BYTES = 128 * 128 * 2;
+  static constexpr int SMEM = (2 + 2 * ST) * TILE + DS_BYTES + 1024;
+  static constexpr int THREADS = 192;
+  static constexpr uint32_t C_S = 0, C_P = 0, C_DS = 64, C_DP = 128;
+  static constexpr uint32_t C_DV = 256, C_DK = 256 + D;
+  static constexpr uint32_t C_DQ = (D == 128) ? 128 : 384;
+};
+
+enum BwdSite : uint32_t {
+  kBSiteProdEmpty = 32, kBSiteMmaKV, kBSiteMmaQ, kBSiteMmaDrained, kBSiteMmaP, kBSiteMmaDS,
+  kBSiteMmaDrain, kBSiteCmpQ, kBSiteCmpS, kBSiteCmpDP, kBSiteCmpDQ, kBSiteProdDrain
+};
+
+__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
+  asm volatile("red.relaxed.gpu.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a),
+               "f"(b), "f"(c), "f"(d)
+               : "memory");
+}
+
+template <int D, bool BF16, bool CAUSAL>
+__global__ void __launch_bounds__(192, 1)
+fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+               const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
+               const BwdParams p) {
+  using C = BwdCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* sK = smem;
+  uint8_t* sV = sK + C::TILE;
+  uint8_t* sQ = sV + C::TILE;                // ST tiles
+  uint8_t* sdO = sQ + C::ST * C::TILE;       // ST tiles
+  uint8_t* sDS = sdO + C::ST * C::TILE;      // dS^T, MN-major for the dQ product
+
+  __shared__ uint64_t bar_kv, qdo_full[C::ST], qdo_empty[C::ST];
+  __shared__ uint64_t s_full, dp_full, p_ready, ds_ready, dq_full, dq_drained, drain;
+  __shared__ uint32_t tmem_slot;
+  __shared__ int abort_flag;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int N = p.N;
+  const int j = static_cast<int>(blockIdx.x) / p.BH;   // key tile (heaviest first when causal)
+  const int bh = static_cast<int>(blockIdx.x) % p.BH;
+  const int n_q = p.n_kv;
+  const int i_begin = CAUSAL ? j : 0;
+  const int n_it = n_q - i_begin;
+
+  WaitCtl wc{p.status, &abort_flag, p.wait_ns};
+
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    mbar_init(&bar_kv, 1);
+    for (int s = 0; s < C::ST; ++s) { mbar_init(&qdo_full[s], 1); mbar_init(&qdo_empty[s], 1); }
+    mbar_init(&s_full, 1);
+    mbar_init(&dp_full, 1);
+    mbar_init(&p_ready, 4);
+    mbar_init(&ds_ready, 4);
+    mbar_init(&dq_full, 1);
+    mbar_init(&dq_drained, 4);
+    mbar_init(&drain, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(&tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = tmem_slot;
+
+  if (warp == 4) {
+    // ------------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      tma_prefetch_desc(&tmdO);
+      mbar_arrive_expect_tx(&bar_kv, 2 * C::TILE);
+      for (int c = 0; c < C::KCH; ++c) {
+        tma_load_3d(sK + c * C::CHUNK, &tmK, &bar_kv, c * 64, j * 128, bh);
+        tma_load_3d(sV + c * C::CHUNK, &tmV, &bar_kv, c * 64, j * 128, bh);
+      }
+      const uint64_t keep = policy_evict_last();
+      int issued = 0;
+      bool ok = true;
+      for (int it = 0; it < n_it; ++it) {
+        const int st = it % C::ST;
+        if (it >= C::ST &&
+            !mbar_wait(&qdo_empty[st], ((it / C::ST) - 1) & 1, wc, kBSiteProdEmpty)) {
+          ok = false;
+          break;
+        }
+        const int row = (i_begin + it) * 128;
+        mbar_arrive_expect_tx(&qdo_full[st], 2 * C::TILE);
+        for (int c = 0; c < C::KCH; ++c) {
+          tma_load_3d_hint(sQ + st * C::TILE + c * C::CHUNK, &tmQ, &qdo_full[st], c * 64, row,
+                           bh, keep);
+          tma_load_3d_hint(sdO + st * C::TILE + c * C::CHUNK, &tmdO, &qdo_full[st], c * 64,
+                           row, bh, keep);
+        }
+        issued = it + 1;
+      }
+      volatile int no_abort = 0;
+      WaitCtl dw{p.status, &no_abort, 100000000ull};
+      if (!ok) {
+        for (int it = max(0, issued - C::ST); it < issued; ++it)
+          mbar_wait(&qdo_full[it % C::ST], (it / C::ST) & 1, dw, kBSiteProdDrain);
+      }
+      // K and V always land before exit, even on an aborted run.
+      mbar_wait(&bar_kv, 0, dw, kBSiteProdDrain);
+    }
+    __syncwarp();
+  } else if (warp == 5) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t id_kk = idesc_f16(128, 128, BF16, false, false);  // S^T, dP^T
+      constexpr uint32_t id_tb = idesc_f16(128, D, BF16, false, true);     // dV, dK (B MN-major)
+      constexpr uint32_t id_dq = idesc_f16(128, D, BF16, true, true);      // dQ (A, B MN-major)
+      const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aQ = smem_u32(sQ),
+                     adO = smem_u32(sdO), aDS = smem_u32(sDS);
+      bool ok = mbar_wait(&bar_kv, 0, wc, kBSiteMmaKV);
+      for (int it = 0; it < n_it && ok; ++it) {
+        const int st = it % C::ST;
+        if (!mbar_wait(&qdo_full[st], (it / C::ST) & 1, wc, kBSiteMmaQ)) { ok = false; break; }
+        tc_fence_after();
+        // S^T = K Q^T
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * C::CHUNK + (kk & 3) * 32;
+          umma_ss(tbase + C::C_S, sdesc_sw128(aK + off, 16, 1024),
+                  sdesc_sw128(aQ + st * C::TILE + off, 16, 1024), id_kk, kk > 0);
+        }
+        umma_commit(&s_full);
+        // dP^T = V dO^T (its columns hold the previous dQ partial when D = 128)
+        if (D == 128 && it > 0) {
+          if (!mbar_wait(&dq_drained, (it - 1) & 1, wc, kBSiteMmaDrained)) { ok = false; break; }
+          tc_fence_after();
+        }
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * C::CHUNK + (kk & 3) * 32;
+          umma_ss(tbase + C::C_DP, sdesc_sw128(aV + off, 16, 1024),
+                  sdesc_sw128(adO + st * C::TILE + off, 16, 1024), id_kk, kk > 0);
+        }
+        umma_commit(&dp_full);
+        // dV += P^T dO
+        if (!mbar_wait(&p_ready, it & 1, wc, kBSiteMmaP)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          umma_ts(tbase + C::C_DV, tbase + C::C_P + kk * 8,
+                  sdesc_sw128(adO + st * C::TILE + kk * 2048, C::CHUNK, 1024), id_tb,
+                  (it > 0 || kk > 0) ? 1u : 0u);
+        // dK += dS^T Q
+        if (!mbar_wait(&ds_ready, it & 1, wc, kBSiteMmaDS)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          umma_ts(tbase + C::C_DK, tbase + C::C_DS + kk * 8,
+                  sdesc_sw128(aQ + st * C::TILE + kk * 2048, C::CHUNK, 1024), id_tb,
+                  (it > 0 || kk > 0) ? 1u : 0u);
+        // dQ_i = dS K (its own columns when D = 64: wait for the previous drain)
+        if (D == 64 && it > 0) {
+          if (!mbar_wait(&dq_drained, (it - 1) & 1, wc, kBSiteMmaDrained)) { ok = false; break; }
+          tc_fence_after();
+        }
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          umma_ss(tbase + C::C_DQ, sdesc_sw128(aDS + kk * 2048, C::CHUNK, 1024),
+                  sdesc_sw128(aK + kk * 2048, C::CHUNK, 1024), id_dq, kk > 0);
+        umma_commit(&dq_full);
+        umma_commit(&qdo_empty[st]);
+      }
+      umma_commit(&drain);
+      volatile int no_abort = 0;
+      WaitCtl dw{p.status, &no_abort, p.wait_ns};
+      mbar_wait(&drain, 0, dw, kBSiteMmaDrain);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------------ compute
+    const int r = warp * 32 + lane;            // key row (P^T, dS^T) / query row (dQ)
+    const int key = j * 128 + r;
+    const uint32_t lb = static_cast<uint32_t>(warp * 32);
+    const float sl2 = p.scale_log2;
+    const size_t stat_base = static_cast<size_t>(bh) * p.Npad;
+    bool ok = true;
+    for (int it = 0; it < n_it && ok; ++it) {
+      const int i = i_begin + it;
+      const float4* L4 = reinterpret_cast<const float4*>(p.Lg + stat_base + i * 128);
+      const float4* D4 = reinterpret_cast<const float4*>(p.Dg + stat_base + i * 128);
+      ok = __all_sync(0xffffffffu, mbar_wait(&s_full, it & 1, wc, kBSiteCmpS));
+      if (!ok) break;
+      tc_fence_after();
+      // P^T row: exp2(S^T * scale * log2e - LSE * log2e), zero where masked.
+      float pr[128];
+      const bool diag = CAUSAL && i == j;
+      const bool key_oob = key >= N;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t sr[32];
+        tmem_ld32(tmem_addr(tbase, lb, C::C_S + 32 * c), sr);
+        tmem_wait_ld();
+        reg_fence(sr);
+#pragma unroll
+        for (int v = 0; v < 8; ++v) {
+          const float4 l4 = __ldg(L4 + c * 8 + v);
+          const float ls[4] = {l4.x, l4.y, l4.z, l4.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int qc = c * 32 + v * 4 + e;
+            float x = ex2_approx(fmaf(__uint_as_float(sr[v * 4 + e]), sl2, -ls[e]));
+            if ((diag && qc < r) || key_oob) x = 0.f;
+            pr[qc] = x;
+          }
+        }
+      }
+      {
+        uint32_t pk[32];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) pk[e] = pack2<BF16>(pr[64 * h + 2 * e], pr[64 * h + 2 * e + 1]);
+          tmem_st32(tmem_addr(tbase, lb, C::C_P + 32 * h), pk);
+        }
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_ready);
+      // dS^T = P^T * (dP^T - D)
+      ok = __all_sync(0xffffffffu, mbar_wait(&dp_full, it & 1, wc, kBSiteCmpDP));
+      if (!ok) break;
+      tc_fence_after();
+      // 32 queries at a time: TMEM dP^T chunk -> dS^T -> 16-bit pairs, written to
+      // TMEM (A operand of dK) and to shared memory (A operand of dQ).  The shared
+      // copy is MN-major with 128-byte swizzle: chunk qc holds queries
+      // 64 qc .. 64 qc + 63 of every key row; 16-byte unit u of row r sits at
+      // unit u ^ (r % 8).
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t dr[32];
+        tmem_ld32(tmem_addr(tbase, lb, C::C_DP + 32 * c), dr);
+        tmem_wait_ld();
+        reg_fence(dr);
+        uint32_t dsk[16];
+#pragma unroll
+        for (int v = 0; v < 8; ++v) {
+          const float4 d4 = __ldg(D4 + c * 8 + v);
+          const int q0 = c * 32 + v * 4;
+          const float a0 = pr[q0 + 0] * (__uint_as_float(dr[v * 4 + 0]) - d4.x);
+          const float a1 = pr[q0 + 1] * (__uint_as_float(dr[v * 4 + 1]) - d4.y);
+          const float a2 = pr[q0 + 2] * (__uint_as_float(dr[v * 4 + 2]) - d4.z);
+          const float a3 = pr[q0 + 3] * (__uint_as_float(dr[v * 4 + 3]) - d4.w);
+          dsk[2 * v] = pack2<BF16>(a0, a1);
+          dsk[2 * v + 1] = pack2<BF16>(a2, a3);
+        }
+        tmem_st16(tmem_addr(tbase, lb, C::C_DS + 16 * c), dsk);
+        const int qc = c >> 1;
+#pragma unroll
+        for (int uu = 0; uu < 4; ++uu) {
+          const int u = (c & 1) * 4 + uu;
+          const uint4 val = make_uint4(dsk[4 * uu], dsk[4 * uu + 1], dsk[4 * uu + 2], dsk[4 * uu + 3]);
+          *reinterpret_cast<uint4*>(sDS + qc * C::CHUNK + r * 128 + ((u ^ (r & 7)) << 4)) = val;
+        }
+      }
+      fence_proxy_async_smem();
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ds_ready);
+      // dQ partial (row r = query i*128 + r) -> fp32 accumulator
+      ok = __all_sync(0xffffffffu, mbar_wait(&dq_full, it & 1, wc, kBSiteCmpDQ));
+      if (!ok) break;
+      tc_fence_after();
+      const int q = i * 128 + r;
+      float* dst = p.dQacc + (static_cast<size_t>(bh) * N + q) * D;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t qr[32];
+        tmem_ld32(tmem_addr(tbase, lb, C::C_DQ + 32 * c), qr);
+        tmem_wait_ld();
+        reg_fence(qr);
+        if (c == D / 32 - 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&dq_drained);
+        }
+        if (q < N) {
+#pragma unroll
+          for (int v = 0; v < 8; ++v)
+            red_add_v4(dst + c * 32 + v * 4, __uint_as_float(qr[4 * v]),
+                       __uint_as_float(qr[4 * v + 1]), __uint_as_float(qr[4 * v + 2]),
+                       __uint_as_float(qr[4 * v + 3]));
+        }
+      }
+    }
+    if (ok) {
+      // dV and dK are final once the last dQ product (issued after them) landed.
+      uint8_t* dv_row = reinterpret_cast<uint8_t*>(p.dV) + (static_cast<size_t>(bh) * N + key) * (D * 2);
+      uint8_t* dk_row = reinterpret_cast<uint8_t*>(p.dK) + (static_cast<size_t>(bh) * N + key) * (D * 2);
+#pragma unroll
+      for (int which = 0; which < 2; ++which) {
+        const uint32_t col = which ? C::C_DK : C::C_DV;
+        const float mul = which ? p.scale : 1.0f;
+        uint8_t* row = which ? dk_row : dv_row;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t rr[32];
+          tmem_ld32(tmem_addr(tbase, lb, col + 32 * c), rr);
+          tmem_wait_ld();
+          reg_fence(rr);
+          uint4 v[4];
+          uint32_t* pv = reinterpret_cast<uint32_t*>(v);
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            pv[e] = pack2<BF16>(__uint_as_float(rr[2 * e]) * mul, __uint_as_float(rr[2 * e + 1]) * mul);
+          if (key < N) {
+            uint4* dst4 = reinterpret_cast<uint4*>(row + c * 64);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) dst4[e] = v[e];
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tbase, 512);
+  }
+}
+
+// ------------------------------------------------------------------------------------
+// host launcher
+// ------------------------------------------------------------------------------------
+
+bool make_tile_map(CUtensorMap* map, const void* base, int BH, int N, int d, bool bf16);
+
+template <int D, bool BF16, bool CAUSAL>
+int launch_bwd_t(const void* Q, const void* K, const void* V, const void* O, const void* dO,
+                 const float* LSE, void* dQ, void* dK, void* dV, void* workspace, int BH, int N,
+                 float scale, unsigned int* status, unsigned long long wait_ns,
+                 cudaStream_t stream) {
+  using Cfg = BwdCfg<D>;
+  const int Npad = static_cast<int>(bwd_npad(N));
+  float* Dg = static_cast<float*>(workspace);
+  float* Lg = Dg + static_cast<size_t>(BH) * Npad;
+  float* dQacc = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
+                                          bwd_rowstat_bytes(static_cast<size_t>(BH), N));
+  CUtensorMap mq, mk, mv, mdo;
+  if (!make_tile_map(&mq, Q, BH, N, D, BF16) || !make_tile_map(&mk, K, BH, N, D, BF16) ||
+      !make_tile_map(&mv, V, BH, N, D, BF16) || !make_tile_map(&mdo, dO, BH, N, D, BF16))
+    return 4;  // FA2_ERR_CUDA
+  // 1. preprocess
+  {
+    const long long rows = static_cast<long long>(BH) * Npad;
+    constexpr int RPB = 256 / (D / 8);
+    const unsigned int grid = static_cast<unsigned int>((rows + RPB - 1) / RPB);
+    fa2_bwd_pre_kernel<D, BF16><<<grid, 256, 0, stream>>>(
+        static_cast<const uint16_t*>(O), static_cast<const uint16_t*>(dO), LSE, Dg, Lg, dQacc, N,
+        Npad, rows);
+    if (cudaGetLastError() != cudaSuccess) return 4;
+  }
+  // 2. main
+  {
+    auto kern = fa2_bwd_kernel<D, BF16, CAUSAL>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM) !=
+        cudaSuccess) {
+      cudaGetLastError();
+      return 4;
+    }
+    BwdParams bp{};
+    bp.Dg = Dg;
+    bp.Lg = Lg;
+    bp.dQacc = dQacc;
+    bp.dK = dK;
+    bp.dV = dV;
+    bp.N = N;
+    bp.Npad = Npad;
+    bp.BH = BH;
+    bp.n_kv = Npad / 128;
+    bp.scale = scale;
+    bp.scale_log2 = scale * 1.4426950408889634f;
+    bp.status = status;
+    bp.wait_ns = wait_ns;
+    const unsigned int grid = static_cast<unsigned int>(bp.n_kv) * static_cast<unsigned int>(BH);
+    kern<<<grid, Cfg::THREADS, Cfg::SMEM, stream>>>(mq, mk, mv, mdo, bp);
+    if (cudaGetLastError() != cudaSuccess) return 4;
+  }
+  // 3. dQ finalise
+  {
+    const long long n8 = static_cast<long long>(BH) * N * D / 8;
+    const unsigned int grid = static_cast<unsigned int>((n8 + 255) / 256);
+    fa2_bwd_dq_kernel<BF16><<<grid, 256, 0, stream>>>(dQacc, static_cast<uint16_t*>(dQ), scale,
+                                                      n8);
+    if (cudaGetLastError() != cudaSuccess) return 4;
+  }
+  return 0;
+}
+
+inline int launch_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO,
+                      const float* LSE, void* dQ, void* dK, void* dV, void* workspace, int BH,
+                      int N, int d, float scale, bool causal, bool bf16, unsigned int* status,
+                      unsigned long long wait_ns, cudaStream_t s) {
+#define FA2_BWD_CALL(D_, BF_, CA_)                                                          \
+  return launch_bwd_t<D_, BF_, CA_>(Q, K, V, O, dO, LSE, dQ, dK, dV, workspace, BH, N, scale, \
+                                    status, wait_ns, s)
+  if (d == 64) {
+    if (bf16) { if (causal) FA2_BWD_CALL(64, true, true); FA2_BWD_CALL(64, true, false); }
+    if (causal) FA2_BWD_CALL(64, false, true);
+    FA2_BWD_CALL(64, false, false);
+  }
+  if (bf16) { if (causal) FA2_BWD_CALL(128, true, true); FA2_BWD_CALL(128, true, false); }
+  if (causal) FA2_BWD_CALL(128, false, true);
+  FA2_BWD_CALL(128, false, false);
+#undef FA2_BWD_CALL
+}
+
 }  // namespace fa2
