@@ -66,27 +66,32 @@ def input_bytes(w) -> int:
     return n * (4 if w.backward else 3)
 
 
-def csrc_hash() -> str:
+# Device sources of each C-ABI call's kernels.
+KERNEL_SOURCES = {"fa2_fwd": ("ptx.cuh", "fa2_fwd.cuh"), "fa2_bwd": ("ptx.cuh", "fa2_bwd.cuh")}
+
+
+def csrc_hash(call: str) -> str:
+    """Hash of the device source files of one call's kernels."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "exact_io_aware_74_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in KERNEL_SOURCES[call]:
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
 
 
 def traffic_from_profiles(kernel_key: str) -> int | None:
-    """DRAM bytes per launch recorded by an ncu capture of the current kernel source.
+    """DRAM bytes per call recorded by an ncu capture of the current kernel source.
 
-    ``profiles/dram_traffic.txt`` holds lines ``<key> <csrc hash> <bytes>``; a
-    record taken from another version of the kernels does not count.
+    ``profiles/dram_traffic.txt`` holds lines ``<call>:<workload> <source hash>
+    <bytes>``; a record taken from another version of the kernels does not count.
     """
     path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
     try:
         lines = open(path).read().splitlines()
     except OSError:
         return None
-    cur = csrc_hash()
+    cur = csrc_hash(kernel_key.split(":")[0])
     for ln in lines:
         parts = ln.split()
         if len(parts) == 3 and parts[0] == kernel_key and parts[1] == cur:

@@ -65,13 +65,16 @@ def test_traffic_record_requires_current_kernel_source(tmp_path, monkeypatch):
     (tmp_path / "exact_io_aware_74_b200").mkdir()
     csrc = tmp_path / "exact_io_aware_74_b200" / "csrc"
     csrc.mkdir()
-    (csrc / "k.cu").write_text("kernel v1")
+    for name in ("ptx.cuh", "fa2_fwd.cuh", "fa2_bwd.cuh"):
+        (csrc / name).write_text(name + " v1")
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
-    h = bench.csrc_hash()
+    h = bench.csrc_hash("fa2_bwd")
     (prof / "dram_traffic.txt").write_text(f"fa2_bwd:w {h} 12345\nfa2_fwd:w deadbeef 99\n")
     assert bench.traffic_from_profiles("fa2_bwd:w") == 12345
     assert bench.traffic_from_profiles("fa2_fwd:w") is None
-    (csrc / "k.cu").write_text("kernel v2")
+    (csrc / "fa2_fwd.cuh").write_text("fa2_fwd.cuh v2")   # another kernel: record stands
+    assert bench.traffic_from_profiles("fa2_bwd:w") == 12345
+    (csrc / "fa2_bwd.cuh").write_text("fa2_bwd.cuh v2")   # this kernel changed: void
     assert bench.traffic_from_profiles("fa2_bwd:w") is None
 
 
