@@ -1,0 +1,39 @@
+"""Runs fa2_fwd (and fa2_bwd) a few times on one shape, for profilers.
+
+    python -m exact_io_aware_74_b200.profile_case B H N d causal [reps] [--fwd-only]
+
+Seeded N(0, 1) bf16 inputs; exits non-zero if a call or the device status fails.
+Used to capture Nsight Compute profiles of one kernel on a small case.
+"""
+
+from __future__ import annotations
+
+import math
+import sys
+
+import torch
+
+from exact_io_aware_74_b200 import fa2
+from exact_io_aware_74_b200.workloads import make_inputs
+
+
+def main(argv: list[str]) -> int:
+    fwd_only = "--fwd-only" in argv
+    args = [a for a in argv if not a.startswith("--")]
+    B, H, N, d, causal = (int(a) for a in args[:5])
+    reps = int(args[5]) if len(args) > 5 else 2
+    x = make_inputs(B, H, N, d, "bf16", seed=5, with_do=not fwd_only)
+    q, k, v = (x[n].cuda() for n in ("q", "k", "v"))
+    do = None if fwd_only else x["do"].cuda()
+    scale = 1.0 / math.sqrt(d)
+    for _ in range(reps):
+        o, lse = fa2.forward(q, k, v, scale, bool(causal))
+        if not fwd_only:
+            fa2.backward(q, k, v, o, do, lse, scale, bool(causal))
+    rc, site = fa2.fa2_get_device_status()
+    print(f"status {fa2.status_string(rc)} site {site}")
+    return 0 if rc == fa2.FA2_OK else 1
+
+
+if __name__ == "__main__":
+    sys.exit(main(sys.argv[1:]))
