@@ -242,6 +242,92 @@ int fa2_bwd(const void* Q, const void* K, const void* V, const void* O, const vo
   return rc;
 }
 
+}  // extern "C"
+
+// ------------------------------------------------------------------------------------
+// Allocation-free backward.
+//
+// Some callers cannot call cudaMalloc: runtimes that hand out device memory only
+// from their own fixed pool, and latency-critical code that must not take the
+// device-wide synchronisation an allocation can cause.  They cannot provide the
+// workspace fa2_bwd asks for, so fa2_bwd_noalloc uses this file-scope buffer
+// instead.  Every GPU that loads the library holds it until the process exits.
+// ------------------------------------------------------------------------------------
+
+namespace {
+
+constexpr size_t kNoAllocBytes = static_cast<size_t>(32) << 20;  // 32 MiB
+constexpr size_t kNoAllocStatusBytes = 256;  // status word used when none exists yet
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocBytes];
+
+// Device address of g_noalloc_scratch, per device.  In host code the symbol's
+// name is only a host-side stand-in; the device address comes from
+// cudaGetSymbolAddress, called with that device current.
+void* g_noalloc_base[kMaxDevices] = {};
+
+void* noalloc_base(int dev) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (!g_noalloc_base[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) {
+      cudaGetLastError();
+      return nullptr;
+    }
+    g_noalloc_base[dev] = p;
+  }
+  return g_noalloc_base[dev];
+}
+
+unsigned int* existing_status_word(int dev) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  return g_status[dev];
+}
+
+}  // namespace
+
+extern "C" {
+
+int fa2_bwd_noalloc(const void* Q, const void* K, const void* V, const void* O, const void* dO,
+                    const float* LSE, void* dQ, void* dK, void* dV, int B, int H, int N, int d,
+                    float scale, int causal, int dtype, fa2_stream_t stream) {
+  if (!Q || !K || !V || !O || !dO || !LSE || !dQ || !dK || !dV) return FA2_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(dO) ||
+      !aligned16(LSE) || !aligned16(dQ) || !aligned16(dK) || !aligned16(dV))
+    return FA2_ERR_INVALID_ARG;
+  int rc = check_sizes(B, H, N, d, scale, causal, dtype);
+  if (rc != FA2_OK) return rc;
+  const int BH = B * H;
+  const size_t bytes = static_cast<size_t>(BH) * N * d * 2;
+  const size_t lse_bytes = static_cast<size_t>(BH) * N * sizeof(float);
+  const void* ins[6] = {Q, K, V, O, dO, LSE};
+  const size_t in_bytes[6] = {bytes, bytes, bytes, bytes, bytes, lse_bytes};
+  void* outs[3] = {dQ, dK, dV};
+  for (void* o : outs) {
+    for (int i = 0; i < 6; ++i)
+      if (overlaps(o, bytes, ins[i], in_bytes[i])) return FA2_ERR_INVALID_ARG;
+  }
+  if (overlaps(dQ, bytes, dK, bytes) || overlaps(dQ, bytes, dV, bytes) ||
+      overlaps(dK, bytes, dV, bytes))
+    return FA2_ERR_INVALID_ARG;
+  const size_t need = fa2::bwd_workspace_bytes(static_cast<size_t>(BH), N, d);
+  if (need > kNoAllocBytes - kNoAllocStatusBytes) return FA2_ERR_WORKSPACE;
+  int dev = 0;
+  rc = check_device(&dev);
+  if (rc != FA2_OK) return rc;
+  uint8_t* base = static_cast<uint8_t*>(noalloc_base(dev));  // first call on a device: set-up
+  if (!base) return FA2_ERR_CUDA;
+  // Timeouts go to the library's status word when it exists (so that
+  // fa2_get_device_status reports them); otherwise to a word in the buffer.
+  unsigned int* st = existing_status_word(dev);
+  if (!st) st = reinterpret_cast<unsigned int*>(base);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  rc = fa2::launch_bwd(Q, K, V, O, dO, LSE, dQ, dK, dV, base + kNoAllocStatusBytes, BH, N, d,
+                       scale, causal != 0, dtype == FA2_BF16, st, wait_ns(), s);
+  if (rc == FA2_OK) g_launches.fetch_add(fa2::kBwdKernelsPerCall);
+  return rc;
+}
+
 int fa2_get_device_status(fa2_stream_t stream, int* site) {
   if (site) *site = 0;
   int dev = 0;

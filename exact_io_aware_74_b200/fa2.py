@@ -27,8 +27,8 @@ FA2_FP16 = 0
 FA2_BF16 = 1
 
 # Every symbol include/fa2.h declares.
-EXPORTS = ("fa2_fwd", "fa2_bwd_workspace_size", "fa2_bwd", "fa2_get_device_status",
-           "fa2_status_string", "fa2_debug_set", "fa2_launch_count")
+EXPORTS = ("fa2_fwd", "fa2_bwd_workspace_size", "fa2_bwd", "fa2_bwd_noalloc",
+           "fa2_get_device_status", "fa2_status_string", "fa2_debug_set", "fa2_launch_count")
 
 _lib = None
 
@@ -55,6 +55,8 @@ def load() -> ctypes.CDLL:
     lib.fa2_bwd_workspace_size.restype = sz
     lib.fa2_bwd.argtypes = [vp] * 10 + [sz, i, i, i, i, f, i, i, vp]
     lib.fa2_bwd.restype = i
+    lib.fa2_bwd_noalloc.argtypes = [vp] * 9 + [i, i, i, i, f, i, i, vp]
+    lib.fa2_bwd_noalloc.restype = i
     lib.fa2_get_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_int)]
     lib.fa2_get_device_status.restype = i
     lib.fa2_status_string.argtypes = [i]
@@ -117,6 +119,16 @@ def fa2_bwd(q, k, v, o, do, lse, dq, dk, dv, workspace, scale: float, causal: bo
     return load().fa2_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse), _ptr(dq),
                           _ptr(dk), _ptr(dv), ws_ptr, ws_bytes, B, H, N, d, float(scale),
                           int(bool(causal)), _dtype_code(q), _stream(stream))
+
+
+def fa2_bwd_noalloc(q, k, v, o, do, lse, dq, dk, dv, scale: float, causal: bool,
+                    stream=None) -> int:
+    """Raw call of the allocation-free backward (library-owned scratch).  Returns the status."""
+    _check_layout(q, k, v, o, do, lse, dq, dk, dv)
+    B, H, N, d = q.shape
+    return load().fa2_bwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse),
+                                  _ptr(dq), _ptr(dk), _ptr(dv), B, H, N, d, float(scale),
+                                  int(bool(causal)), _dtype_code(q), _stream(stream))
 
 
 def fa2_get_device_status(stream=None) -> tuple[int, int]:

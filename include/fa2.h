@@ -105,6 +105,34 @@ int fa2_bwd(const void* Q, const void* K, const void* V, const void* O, const vo
             int dtype, fa2_stream_t stream);
 
 /*
+ * Allocation-free backward.  The paper has no counterpart: this entry point
+ * exists for callers that cannot call cudaMalloc -- runtimes that hand out device
+ * memory only from their own fixed pool, and latency-critical code that must not
+ * take the device-wide synchronisation an allocation can cause -- and so cannot
+ * provide the workspace fa2_bwd asks for.
+ *
+ * Same arguments, results and errors as fa2_bwd, minus the workspace: the
+ * scratch lives in a 32 MiB buffer that the library holds in device memory on
+ * every GPU that loads it, until the process exits.  Nothing is allocated.
+ *   - Sizes whose workspace (fa2_bwd_workspace_size) exceeds 32 MiB - 256 bytes
+ *     return FA2_ERR_WORKSPACE and launch nothing (e.g. B*H = 64, N = 1024,
+ *     d = 64 fits; B*H = 128, N = 4096, d = 128 does not).
+ *   - The first call on a device looks up the buffer's device address (set-up);
+ *     make that first call before any stream capture.
+ *   - Every call shares the one buffer and it keeps the last call's contents;
+ *     each call rewrites all of it that it reads (the dQ accumulator is zeroed
+ *     by the call itself).  Calls that overlap on the GPU -- on different
+ *     streams, or from several host threads -- race on the buffer and give
+ *     wrong results: serialise them.
+ *   - In-kernel wait timeouts are reported by fa2_get_device_status() once any
+ *     fa2_fwd / fa2_bwd call has run on the device; before that they are not
+ *     observable.
+ */
+int fa2_bwd_noalloc(const void* Q, const void* K, const void* V, const void* O, const void* dO,
+                    const float* LSE, void* dQ, void* dK, void* dV, int B, int H, int N, int d,
+                    float scale, int causal, int dtype, fa2_stream_t stream);
+
+/*
  * Synchronises ``stream``, then returns and clears the current device's status
  * word: FA2_OK, or FA2_ERR_TIMEOUT if a kernel gave up a bounded wait since the
  * last call (the kernel then skipped its output and exited cleanly; the CUDA
