@@ -136,6 +136,16 @@ int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& 
                const fa2::FwdParams& p, cudaStream_t stream) {
   using Cfg = fa2::FwdCfg<D>;
   auto kern = fa2::fa2_fwd_kernel<D, BF16, CAUSAL>;
+  // The kernel re-splits its registers between warpgroups; that is only sound
+  // when every thread was launched with exactly Cfg::LAUNCH_REGS registers.
+  static const bool regs_ok = [&] {
+    cudaFuncAttributes fa{};
+    return cudaFuncGetAttributes(&fa, kern) == cudaSuccess && fa.numRegs == Cfg::LAUNCH_REGS;
+  }();
+  if (!regs_ok) {
+    cudaGetLastError();
+    return FA2_ERR_CUDA;
+  }
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM) !=
       cudaSuccess) {
     cudaGetLastError();

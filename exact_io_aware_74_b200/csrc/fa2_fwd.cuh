@@ -16,11 +16,17 @@
 //   producer and consumer warps and asynchronous tile copies (Hopper-era prior
 //   art, restated for tcgen05).
 //
-// CTA layout (320 threads):
+// CTA layout (384 threads, three warpgroups):
 //   warps 0-3  softmax warpgroup for query tile 0 (rows r0 .. r0+127)
 //   warps 4-7  softmax warpgroup for query tile 1 (rows r0+128 .. r0+255)
 //   warp  8    TMA producer (Q once, then a ring of K and V tiles)
 //   warp  9    MMA issuer (tcgen05, one thread)
+//   warps 10-11 idle (they complete the third warpgroup)
+// The kernel is compiled for 168 registers per thread (384 x 168 = 64512); the
+// third warpgroup gives registers back (down to 40) and the two softmax
+// warpgroups take them (up to 232): 2 x 128 x 232 + 128 x 40 = 64512, so the
+// re-split never asks for more than the launch holds.  The host refuses to
+// launch a build whose register count is not 168.
 // TMEM (512 columns x 128 lanes, fp32): S_t at column 128 t, O_t at 256 + D t.
 // P_t (16-bit) overwrites the first 64 columns of S_t and feeds the P V MMA
 // straight from TMEM.  The MMA warp alternates between the two query tiles so
@@ -54,7 +60,12 @@ struct FwdCfg {
   static constexpr int KS = (D == 64) ? 4 : 2;    // K ring stages
   static constexpr int VS = (D == 64) ? 4 : 2;    // V ring stages
   static constexpr int SMEM = (QT + KS + VS) * TILE + 1024;
-  static constexpr int THREADS = 320;
+  static constexpr int THREADS = 384;
+  static constexpr int LAUNCH_REGS = 168;  // per thread, as compiled (checked on the host)
+  static constexpr int SOFT_REGS = 232;
+  static constexpr int OTHER_REGS = 40;
+  static_assert(2 * 128 * SOFT_REGS + 128 * OTHER_REGS <= THREADS * LAUNCH_REGS,
+                "register re-split exceeds the launch allocation");
   static constexpr uint32_t S_COL0 = 0, S_COL1 = 128;
   static constexpr uint32_t O_COL0 = 256, O_COL1 = 256 + D;
 };
@@ -66,7 +77,7 @@ enum FwdSite : uint32_t {
 };
 
 template <int D, bool BF16, bool CAUSAL>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(384, 1)
 fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
   using C = FwdCfg<D>;
@@ -128,7 +139,12 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   tc_fence_after();
   const uint32_t tbase = tmem_slot;
 
-  if (warp == 8) {
+  if (warp >= 8) {
+  // Third warpgroup: every warp executes the same register release first.
+  regs_dec<C::OTHER_REGS>();
+  if (warp >= 10) {
+    // idle warps of the third warpgroup
+  } else if (warp == 8) {
     // ------------------------------------------------------------------ producer
     if (lane == 0) {
       tma_prefetch_desc(&tmQ);
@@ -251,8 +267,10 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       mbar_wait(&drain, 0, dw, kSiteMmaDrain);
     }
     __syncwarp();
+  }
   } else {
     // ------------------------------------------------------------------ softmax
+    regs_inc<C::SOFT_REGS>();
     const int t = warp >> 2;      // query tile of this warpgroup
     const int wq = warp & 3;      // TMEM lane quadrant
     const int r_loc = wq * 32 + lane;

@@ -39,6 +39,16 @@ __device__ __forceinline__ bool elect_one() {
   return pred != 0;
 }
 
+// Warpgroup-wide register re-split (all 4 warps of the warpgroup execute it).
+template <uint32_t N>
+__device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // ------------------------------------------------------------------------------------
 // mbarriers
 // ------------------------------------------------------------------------------------
