@@ -70,6 +70,15 @@ struct FwdCfg {
   static constexpr uint32_t O_COL0 = 256, O_COL1 = 256 + D;
 };
 
+// Pairs i of a score row with (i & 3) >= kPolyFrom take the polynomial exp2
+// (4: none, 3: one pair in four, 2: half).  Measured on B200 (d = 128): the FMA
+// and ALU pipes, not the MUFU unit, bound the softmax, and moving exponentials
+// onto them slows the kernel (one in four: -13 %, half: -20 %), so none do.
+#ifndef FA2_POLY_FROM
+#define FA2_POLY_FROM 4
+#endif
+constexpr int kPolyFrom = FA2_POLY_FROM;
+
 // Wait-site ids reported through the status word.
 enum FwdSite : uint32_t {
   kSiteProdKEmpty = 1, kSiteProdVEmpty, kSiteMmaQ, kSiteMmaK, kSiteMmaV, kSiteMmaP,
@@ -306,13 +315,19 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       }
       float mx[8];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) mx[k] = __uint_as_float(sr[k]);
+      for (int k = 0; k < 8; ++k)
+        mx[k] = fmax3(__uint_as_float(sr[k]), __uint_as_float(sr[k + 8]), __uint_as_float(sr[k + 16]));
 #pragma unroll
-      for (int i = 8; i < 128; ++i) mx[i & 7] = fmaxf(mx[i & 7], __uint_as_float(sr[i]));
+      for (int i = 24; i < 120; i += 16)  // elements 24 .. 119
 #pragma unroll
-      for (int k = 4; k >= 1; k >>= 1)
+        for (int k = 0; k < 8; ++k)
+          mx[k] = fmax3(mx[k], __uint_as_float(sr[i + k]), __uint_as_float(sr[i + k + 8]));
 #pragma unroll
-        for (int q = 0; q < k; ++q) mx[q] = fmaxf(mx[q], mx[q + k]);
+      for (int k = 0; k < 8; ++k) mx[k] = fmaxf(mx[k], __uint_as_float(sr[120 + k]));
+      mx[0] = fmax3(mx[0], mx[1], mx[2]);
+      mx[3] = fmax3(mx[3], mx[4], mx[5]);
+      mx[6] = fmaxf(mx[6], mx[7]);
+      mx[0] = fmax3(mx[0], mx[3], mx[6]);
       const float m_new = fmaxf(m, mx[0] * sl2);
       if (j == 0) {
         m = m_new;
@@ -340,22 +355,39 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           }
         }
       }
-      const float neg_m = -m;
-      float sum[4] = {0.f, 0.f, 0.f, 0.f};
+      // P = 2^(s * scale * log2 e - m): arguments two at a time (f32x2),
+      // exponentials on the MUFU unit (or the polynomial, see kPolyFrom).
+      const uint64_t sl2x2 = f2_pack(sl2, sl2);
+      const uint64_t negm2 = f2_pack(-m, -m);
+      uint64_t sum2[4] = {0, 0, 0, 0};
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         uint32_t pk[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-          const float a = ex2_approx(fmaf(__uint_as_float(sr[64 * h + 2 * i]), sl2, neg_m));
-          const float b = ex2_approx(fmaf(__uint_as_float(sr[64 * h + 2 * i + 1]), sl2, neg_m));
-          sum[(2 * i) & 3] += a;
-          sum[(2 * i + 1) & 3] += b;
+          const uint64_t arg = f2_fma(f2_pack(__uint_as_float(sr[64 * h + 2 * i]),
+                                              __uint_as_float(sr[64 * h + 2 * i + 1])),
+                                      sl2x2, negm2);
+          float a, b;
+          f2_unpack(arg, a, b);
+          if ((i & 3) >= kPolyFrom) {
+            a = exp2_poly3(a);
+            b = exp2_poly3(b);
+          } else {
+            a = ex2_approx(a);
+            b = ex2_approx(b);
+          }
+          sum2[i & 3] = f2_add(sum2[i & 3], f2_pack(a, b));
           pk[i] = pack2<BF16>(a, b);
         }
         tmem_st32(tmem_addr(tbase, lane_base, s_col + 32 * h), pk);
       }
-      l += (sum[0] + sum[1]) + (sum[2] + sum[3]);
+      {
+        const uint64_t s01 = f2_add(f2_add(sum2[0], sum2[1]), f2_add(sum2[2], sum2[3]));
+        float lo, hi;
+        f2_unpack(s01, lo, hi);
+        l += lo + hi;
+      }
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();

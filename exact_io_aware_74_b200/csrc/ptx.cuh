@@ -369,6 +369,52 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+// max(a, b, c) in one instruction.
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// Two fp32 values in one 64-bit register pair, for the packed f32x2 operations.
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// 2^x on the FMA pipe, for x <= 127 (used for part of the softmax exponentials
+// so that they do not all queue on the MUFU unit).  Range reduction after Cody
+// and Waite: x = j + f with j = rint(x) (adding 1.5 * 2^23 rounds to an integer)
+// and f in [-1/2, 1/2]; 2^f is a degree-3 polynomial fitted for this library
+// (minimax in relative error on [-1/2, 1/2], max relative error 7.5e-5 in fp32
+// Horner evaluation); 2^j enters through the exponent bits.  x is clamped at
+// -125, so inputs below that (including -inf) give about 2^-125 instead of 0.
+__device__ __forceinline__ float exp2_poly3(float x) {
+  x = fmaxf(x, -125.0f);
+  const float kRound = 12582912.0f;  // 1.5 * 2^23
+  const float t = __fadd_rn(x, kRound);
+  const float j = __fsub_rn(t, kRound);
+  const float f = __fsub_rn(x, j);
+  float p = fmaf(f, 0.055171661f, 0.24261114f);
+  p = fmaf(f, p, 0.69326099f);
+  p = fmaf(f, p, 0.99992807f);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
 // Packs two fp32 values into a 32-bit pair of 16-bit values (round to nearest
 // even); ``lo`` goes to the low half.
 template <bool BF16>

@@ -355,3 +355,29 @@ def test_workload_table():
     assert w4.bwd_flops == pytest.approx(1.374e12, rel=1e-3)
     small = workload_inputs(WORKLOADS["fwd_fp16_b1h2_n128_d64"])
     assert small["q"].dtype == torch.float16 and small["q"].shape == (1, 2, 128, 64)
+
+
+# ----------------------------------------------------------------------------------
+# the FMA-pipe exp2 of the CUDA library (csrc/ptx.cuh, exp2_poly3), emulated in fp32
+# ----------------------------------------------------------------------------------
+
+def _exp2_poly3_f32(x):
+    """Step-by-step fp32 emulation of exp2_poly3: rint range reduction + cubic."""
+    f32 = np.float32
+    x = np.maximum(x.astype(f32), f32(-125.0))
+    t = (x + f32(12582912.0)).astype(f32)
+    j = (t - f32(12582912.0)).astype(f32)
+    f = (x - j).astype(f32)
+    p = (f.astype(np.float64) * f32(0.055171661) + f32(0.24261114)).astype(f32)
+    p = (f.astype(np.float64) * p + f32(0.69326099)).astype(f32)
+    p = (f.astype(np.float64) * p + f32(0.99992807)).astype(f32)
+    bits = (p.view(np.int32).astype(np.int64) + (t.view(np.int32).astype(np.int64) << 23))
+    return (bits & 0xFFFFFFFF).astype(np.uint32).view(np.float32)
+
+
+def test_exp2_poly3_relative_error_bound():
+    x = np.concatenate([np.linspace(-124.0, 8.0, 400001), np.linspace(-1.0, 1.0, 100001)])
+    got = _exp2_poly3_f32(x).astype(np.float64)
+    rel = np.abs(got / np.exp2(x.astype(np.float32).astype(np.float64)) - 1.0)
+    assert rel.max() < 1e-4  # fitted bound 7.5e-5, below the fp16 half-ulp 2.4e-4
+    assert 0 < _exp2_poly3_f32(np.array([-np.inf]))[0] < 1e-37  # clamped, not NaN
