@@ -16,12 +16,16 @@
 //                            the query tiles that see those keys;
 //   3. fa2_bwd_dq_kernel   : dQ = scale * accumulator, rounded to 16 bits.
 //
-// Main kernel, CTA layout (192 threads):
-//   warps 0-3 compute warpgroup: thread r owns key row r of the tile for P^T and
-//             dS^T, and query row r of the current query tile when it moves the
-//             dQ partial from TMEM to the fp32 accumulator (vector atomics);
-//   warp  4   TMA producer: K_j and V_j once, then a 2-stage ring of (Q_i, dO_i);
-//   warp  5   tcgen05 MMA issuer (one thread).
+// Main kernel, CTA layout (320 threads):
+//   warps 0-7 two compute warpgroups g = 0, 1.  Thread r of warpgroup g owns key
+//             row r of the tile for the query columns 64 g .. 64 g + 63 of P^T
+//             and dS^T, and query row r of the current query tile for the head
+//             columns g D/2 .. (g+1) D/2 - 1 when it moves the dQ partial from
+//             TMEM to the fp32 accumulator (vector atomics).  Splitting every
+//             row between the two warpgroups halves the per-tile chain
+//             P^T -> dS^T -> dQ drain that the products wait on;
+//   warp  8   TMA producer: K_j and V_j once, then a 2-stage ring of (Q_i, dO_i);
+//   warp  9   tcgen05 MMA issuer (one thread).
 // TMEM (fp32 columns): S^T [0,128) -- P^T (16-bit, packed) overwrites [0,64) and
 // dS^T [64,128); dP^T [128,256); dV [256,256+D); dK [256+D,256+2D); the dQ
 // partial reuses [128,256) when D = 128 and has [384,448) when D = 64.
@@ -144,15 +148,37 @@ struct BwdCfg {
   static constexpr int TILE = 128 * D * 2;
   static constexpr int ST = 2;                 // (Q, dO) ring stages
   static constexpr int DS_BYTES = 128 * 128 * 2;
-  static constexpr int SMEM = (2 + 2 * ST) * TILE + DS_BYTES + 1024;
-  static constexpr int THREADS = 192;
+  static constexpr int LD_BYTES = ST * 2 * 128 * 4;  // LSE*log2e and D rows of each stage
+  static constexpr int CTRL_BYTES = 256;              // barriers, TMEM address, abort flag
+  // No alignment slack: the dynamic region must start 1024-byte aligned (checked).
+  static constexpr int SMEM = (2 + 2 * ST) * TILE + DS_BYTES + LD_BYTES + CTRL_BYTES;
+  static constexpr int THREADS = 320;
   static constexpr uint32_t C_S = 0, C_P = 0, C_DS = 64, C_DP = 128;
   static constexpr uint32_t C_DV = 256, C_DK = 256 + D;
   static constexpr uint32_t C_DQ = (D == 128) ? 128 : 384;
 };
 
+// Control block at the end of the dynamic shared memory (no static shared memory,
+// so that the 1024-byte aligned tiles start at the base of the window).
+template <int ST>
+struct BwdCtrl {
+  uint64_t bar_kv, qdo_full[ST], qdo_empty[ST];
+  uint64_t s_full, dp_full, p_ready, ds_ready, dq_full, dq_drained, drain;
+  uint32_t tmem_slot;
+  int abort_flag;
+};
+
+__device__ __forceinline__ void bulk_load_1d(void* smem_dst, const void* gmem_src, uint32_t bytes,
+                                             uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(gmem_src)), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
 enum BwdSite : uint32_t {
-  kBSiteProdEmpty = 32, kBSiteMmaKV, kBSiteMmaQ, kBSiteMmaDrained, kBSiteMmaP, kBSiteMmaDS,
+  kBSiteAlign = 31, kBSiteProdEmpty = 32, kBSiteMmaKV, kBSiteMmaQ, kBSiteMmaDrained, kBSiteMmaP, kBSiteMmaDS,
   kBSiteMmaDrain, kBSiteCmpQ, kBSiteCmpS, kBSiteCmpDP, kBSiteCmpDQ, kBSiteProdDrain
 };
 
@@ -163,24 +189,38 @@ __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float 
 }
 
 template <int D, bool BF16, bool CAUSAL>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
 fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
                const BwdParams p) {
   using C = BwdCfg<D>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  if ((smem_u32(smem_raw) & 1023u) != 0) {
+    // The swizzled tiles need a 1024-byte aligned base; report and do nothing.
+    if (threadIdx.x == 0) atomicCAS(p.status, 0u, 4u | (kBSiteAlign << 8));
+    return;
+  }
+  uint8_t* smem = smem_raw;
   uint8_t* sK = smem;
   uint8_t* sV = sK + C::TILE;
   uint8_t* sQ = sV + C::TILE;                // ST tiles
   uint8_t* sdO = sQ + C::ST * C::TILE;       // ST tiles
   uint8_t* sDS = sdO + C::ST * C::TILE;      // dS^T, MN-major for the dQ product
-
-  __shared__ uint64_t bar_kv, qdo_full[C::ST], qdo_empty[C::ST];
-  __shared__ uint64_t s_full, dp_full, p_ready, ds_ready, dq_full, dq_drained, drain;
-  __shared__ uint32_t tmem_slot;
-  __shared__ int abort_flag;
+  float* sLD = reinterpret_cast<float*>(sDS + C::DS_BYTES);  // [ST][2][128]: L, D
+  BwdCtrl<C::ST>& ctl = *reinterpret_cast<BwdCtrl<C::ST>*>(sDS + C::DS_BYTES + C::LD_BYTES);
+  static_assert(sizeof(BwdCtrl<C::ST>) <= C::CTRL_BYTES, "control block too large");
+  uint64_t& bar_kv = ctl.bar_kv;
+  uint64_t* qdo_full = ctl.qdo_full;
+  uint64_t* qdo_empty = ctl.qdo_empty;
+  uint64_t& s_full = ctl.s_full;
+  uint64_t& dp_full = ctl.dp_full;
+  uint64_t& p_ready = ctl.p_ready;
+  uint64_t& ds_ready = ctl.ds_ready;
+  uint64_t& dq_full = ctl.dq_full;
+  uint64_t& dq_drained = ctl.dq_drained;
+  uint64_t& drain = ctl.drain;
+  uint32_t& tmem_slot = ctl.tmem_slot;
+  int& abort_flag = ctl.abort_flag;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -199,10 +239,10 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     for (int s = 0; s < C::ST; ++s) { mbar_init(&qdo_full[s], 1); mbar_init(&qdo_empty[s], 1); }
     mbar_init(&s_full, 1);
     mbar_init(&dp_full, 1);
-    mbar_init(&p_ready, 4);
-    mbar_init(&ds_ready, 4);
+    mbar_init(&p_ready, 8);
+    mbar_init(&ds_ready, 8);
     mbar_init(&dq_full, 1);
-    mbar_init(&dq_drained, 4);
+    mbar_init(&dq_drained, 8);
     mbar_init(&drain, 1);
     fence_mbar_init();
   }
@@ -215,7 +255,7 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   tc_fence_after();
   const uint32_t tbase = tmem_slot;
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ------------------------------------------------------------------ producer
     if (lane == 0) {
       tma_prefetch_desc(&tmQ);
@@ -238,7 +278,10 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           break;
         }
         const int row = (i_begin + it) * 128;
-        mbar_arrive_expect_tx(&qdo_full[st], 2 * C::TILE);
+        mbar_arrive_expect_tx(&qdo_full[st], 2 * C::TILE + 2 * 512);
+        const size_t stat = static_cast<size_t>(bh) * p.Npad + row;
+        bulk_load_1d(sLD + st * 256, p.Lg + stat, 512, &qdo_full[st]);
+        bulk_load_1d(sLD + st * 256 + 128, p.Dg + stat, 512, &qdo_full[st]);
         for (int c = 0; c < C::KCH; ++c) {
           tma_load_3d_hint(sQ + st * C::TILE + c * C::CHUNK, &tmQ, &qdo_full[st], c * 64, row,
                            bh, keep);
@@ -257,7 +300,7 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       mbar_wait(&bar_kv, 0, dw, kBSiteProdDrain);
     }
     __syncwarp();
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t id_kk = idesc_f16(128, 128, BF16, false, false);  // S^T, dP^T
@@ -326,38 +369,45 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     __syncwarp();
   } else {
     // ------------------------------------------------------------------ compute
-    const int r = warp * 32 + lane;            // key row (P^T, dS^T) / query row (dQ)
+    const int g = warp >> 2;                   // warpgroup: query columns 64 g .. 64 g + 63
+    const int wq = warp & 3;                   // TMEM lane quadrant
+    const int r = wq * 32 + lane;              // key row (P^T, dS^T) / query row (dQ)
     const int key = j * 128 + r;
-    const uint32_t lb = static_cast<uint32_t>(warp * 32);
+    const uint32_t lb = static_cast<uint32_t>(wq * 32);
     const float sl2 = p.scale_log2;
-    const size_t stat_base = static_cast<size_t>(bh) * p.Npad;
+    const int qoff = 64 * g;
     bool ok = true;
     for (int it = 0; it < n_it && ok; ++it) {
       const int i = i_begin + it;
-      const float4* L4 = reinterpret_cast<const float4*>(p.Lg + stat_base + i * 128);
-      const float4* D4 = reinterpret_cast<const float4*>(p.Dg + stat_base + i * 128);
+      const int st = it % C::ST;
+      // This tile's LSE*log2e and D rows arrive in shared memory with Q_i and dO_i.
+      const float4* L4 = reinterpret_cast<const float4*>(sLD + st * 256 + qoff);
+      const float4* D4 = reinterpret_cast<const float4*>(sLD + st * 256 + 128 + qoff);
+      ok = __all_sync(0xffffffffu, mbar_wait(&qdo_full[st], (it / C::ST) & 1, wc, kBSiteCmpQ));
+      if (!ok) break;
       ok = __all_sync(0xffffffffu, mbar_wait(&s_full, it & 1, wc, kBSiteCmpS));
       if (!ok) break;
       tc_fence_after();
-      // P^T row: exp2(S^T * scale * log2e - LSE * log2e), zero where masked.
-      float pr[128];
+      // P^T (this warpgroup's 64 query columns): exp2(S^T * scale * log2e - LSE * log2e),
+      // zero where the key comes after the query or lies past N.
+      float pr[64];
       const bool diag = CAUSAL && i == j;
       const bool key_oob = key >= N;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < 2; ++c) {
         uint32_t sr[32];
-        tmem_ld32(tmem_addr(tbase, lb, C::C_S + 32 * c), sr);
+        tmem_ld32(tmem_addr(tbase, lb, C::C_S + qoff + 32 * c), sr);
         tmem_wait_ld();
         reg_fence(sr);
 #pragma unroll
         for (int v = 0; v < 8; ++v) {
-          const float4 l4 = __ldg(L4 + c * 8 + v);
+          const float4 l4 = L4[c * 8 + v];
           const float ls[4] = {l4.x, l4.y, l4.z, l4.w};
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int qc = c * 32 + v * 4 + e;
             float x = ex2_approx(fmaf(__uint_as_float(sr[v * 4 + e]), sl2, -ls[e]));
-            if ((diag && qc < r) || key_oob) x = 0.f;
+            if ((diag && qoff + qc < r) || key_oob) x = 0.f;
             pr[qc] = x;
           }
         }
@@ -365,35 +415,30 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       {
         uint32_t pk[32];
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-#pragma unroll
-          for (int e = 0; e < 32; ++e) pk[e] = pack2<BF16>(pr[64 * h + 2 * e], pr[64 * h + 2 * e + 1]);
-          tmem_st32(tmem_addr(tbase, lb, C::C_P + 32 * h), pk);
-        }
+        for (int e = 0; e < 32; ++e) pk[e] = pack2<BF16>(pr[2 * e], pr[2 * e + 1]);
+        tmem_st32(tmem_addr(tbase, lb, C::C_P + 32 * g), pk);
       }
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_ready);
-      // dS^T = P^T * (dP^T - D)
+      // dS^T = P^T * (dP^T - D), 32 queries at a time, written to TMEM (A operand
+      // of dK) and to shared memory (A operand of dQ).  The shared copy is
+      // MN-major with 128-byte swizzle: chunk g holds queries 64 g .. 64 g + 63 of
+      // every key row; 16-byte unit u of row r sits at unit u ^ (r % 8).
       ok = __all_sync(0xffffffffu, mbar_wait(&dp_full, it & 1, wc, kBSiteCmpDP));
       if (!ok) break;
       tc_fence_after();
-      // 32 queries at a time: TMEM dP^T chunk -> dS^T -> 16-bit pairs, written to
-      // TMEM (A operand of dK) and to shared memory (A operand of dQ).  The shared
-      // copy is MN-major with 128-byte swizzle: chunk qc holds queries
-      // 64 qc .. 64 qc + 63 of every key row; 16-byte unit u of row r sits at
-      // unit u ^ (r % 8).
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < 2; ++c) {
         uint32_t dr[32];
-        tmem_ld32(tmem_addr(tbase, lb, C::C_DP + 32 * c), dr);
+        tmem_ld32(tmem_addr(tbase, lb, C::C_DP + qoff + 32 * c), dr);
         tmem_wait_ld();
         reg_fence(dr);
         uint32_t dsk[16];
 #pragma unroll
         for (int v = 0; v < 8; ++v) {
-          const float4 d4 = __ldg(D4 + c * 8 + v);
+          const float4 d4 = D4[c * 8 + v];
           const int q0 = c * 32 + v * 4;
           const float a0 = pr[q0 + 0] * (__uint_as_float(dr[v * 4 + 0]) - d4.x);
           const float a1 = pr[q0 + 1] * (__uint_as_float(dr[v * 4 + 1]) - d4.y);
@@ -402,13 +447,12 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           dsk[2 * v] = pack2<BF16>(a0, a1);
           dsk[2 * v + 1] = pack2<BF16>(a2, a3);
         }
-        tmem_st16(tmem_addr(tbase, lb, C::C_DS + 16 * c), dsk);
-        const int qc = c >> 1;
+        tmem_st16(tmem_addr(tbase, lb, C::C_DS + 32 * g + 16 * c), dsk);
 #pragma unroll
         for (int uu = 0; uu < 4; ++uu) {
-          const int u = (c & 1) * 4 + uu;
+          const int u = c * 4 + uu;
           const uint4 val = make_uint4(dsk[4 * uu], dsk[4 * uu + 1], dsk[4 * uu + 2], dsk[4 * uu + 3]);
-          *reinterpret_cast<uint4*>(sDS + qc * C::CHUNK + r * 128 + ((u ^ (r & 7)) << 4)) = val;
+          *reinterpret_cast<uint4*>(sDS + g * C::CHUNK + r * 128 + ((u ^ (r & 7)) << 4)) = val;
         }
       }
       fence_proxy_async_smem();
@@ -416,19 +460,20 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&ds_ready);
-      // dQ partial (row r = query i*128 + r) -> fp32 accumulator
+      // dQ partial: query row r, head columns g D/2 .. (g+1) D/2 - 1 -> fp32 accumulator
       ok = __all_sync(0xffffffffu, mbar_wait(&dq_full, it & 1, wc, kBSiteCmpDQ));
       if (!ok) break;
       tc_fence_after();
       const int q = i * 128 + r;
-      float* dst = p.dQacc + (static_cast<size_t>(bh) * N + q) * D;
+      constexpr int HALF = D / 2;
+      float* dst = p.dQacc + (static_cast<size_t>(bh) * N + q) * D + g * HALF;
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
+      for (int c = 0; c < HALF / 32; ++c) {
         uint32_t qr[32];
-        tmem_ld32(tmem_addr(tbase, lb, C::C_DQ + 32 * c), qr);
+        tmem_ld32(tmem_addr(tbase, lb, C::C_DQ + g * HALF + 32 * c), qr);
         tmem_wait_ld();
         reg_fence(qr);
-        if (c == D / 32 - 1) {
+        if (c == HALF / 32 - 1) {
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&dq_drained);
@@ -443,30 +488,27 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       }
     }
     if (ok) {
-      // dV and dK are final once the last dQ product (issued after them) landed.
-      uint8_t* dv_row = reinterpret_cast<uint8_t*>(p.dV) + (static_cast<size_t>(bh) * N + key) * (D * 2);
-      uint8_t* dk_row = reinterpret_cast<uint8_t*>(p.dK) + (static_cast<size_t>(bh) * N + key) * (D * 2);
+      // dV (warpgroup 0) and dK (warpgroup 1) are final once the last dQ product,
+      // issued after them, has landed.
+      const uint32_t col = g ? C::C_DK : C::C_DV;
+      const float mul = g ? p.scale : 1.0f;
+      uint8_t* row = reinterpret_cast<uint8_t*>(g ? p.dK : p.dV) +
+                     (static_cast<size_t>(bh) * N + key) * (D * 2);
 #pragma unroll
-      for (int which = 0; which < 2; ++which) {
-        const uint32_t col = which ? C::C_DK : C::C_DV;
-        const float mul = which ? p.scale : 1.0f;
-        uint8_t* row = which ? dk_row : dv_row;
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t rr[32];
+        tmem_ld32(tmem_addr(tbase, lb, col + 32 * c), rr);
+        tmem_wait_ld();
+        reg_fence(rr);
+        uint4 v[4];
+        uint32_t* pv = reinterpret_cast<uint32_t*>(v);
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t rr[32];
-          tmem_ld32(tmem_addr(tbase, lb, col + 32 * c), rr);
-          tmem_wait_ld();
-          reg_fence(rr);
-          uint4 v[4];
-          uint32_t* pv = reinterpret_cast<uint32_t*>(v);
+        for (int e = 0; e < 16; ++e)
+          pv[e] = pack2<BF16>(__uint_as_float(rr[2 * e]) * mul, __uint_as_float(rr[2 * e + 1]) * mul);
+        if (key < N) {
+          uint4* dst4 = reinterpret_cast<uint4*>(row + c * 64);
 #pragma unroll
-          for (int e = 0; e < 16; ++e)
-            pv[e] = pack2<BF16>(__uint_as_float(rr[2 * e]) * mul, __uint_as_float(rr[2 * e + 1]) * mul);
-          if (key < N) {
-            uint4* dst4 = reinterpret_cast<uint4*>(row + c * 64);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) dst4[e] = v[e];
-          }
+          for (int e = 0; e < 4; ++e) dst4[e] = v[e];
         }
       }
     }
