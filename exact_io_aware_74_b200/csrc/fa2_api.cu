@@ -47,6 +47,7 @@ EncodeTiledFn encode_fn() {
 
 namespace fa2 {
 bool make_tile_map(CUtensorMap* map, const void* base, int BH, int N, int d, bool bf16);
+bool make_acc_map(CUtensorMap* map, float* base, int BH, int N, int d);
 }  // namespace fa2
 
 namespace {
@@ -116,6 +117,23 @@ bool make_tile_map(CUtensorMap* map, const void* base, int BH, int N, int d, boo
   const CUtensorMapDataType ty =
       bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
   return enc(map, ty, 3, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// fp32 [BH][N][d] accumulator as a 3-D TMA map with 128-row x 32-column boxes
+// and 128-byte swizzle, for tiled reduce-adds; rows past N are clipped.
+bool make_acc_map(CUtensorMap* map, float* base, int BH, int N, int d) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
+                              static_cast<cuuint64_t>(BH)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 4,
+                                 static_cast<cuuint64_t>(N) * d * 4};
+  const cuuint32_t box[3] = {32, 128, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;

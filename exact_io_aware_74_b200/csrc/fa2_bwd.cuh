@@ -26,9 +26,12 @@
 //             P^T -> dS^T -> dQ drain that the products wait on;
 //   warp  8   TMA producer: K_j and V_j once, then a 2-stage ring of (Q_i, dO_i);
 //   warp  9   tcgen05 MMA issuer (one thread).
-// TMEM (fp32 columns): S^T [0,128) -- P^T (16-bit, packed) overwrites [0,64) and
-// dS^T [64,128); dP^T [128,256); dV [256,256+D); dK [256+D,256+2D); the dQ
-// partial reuses [128,256) when D = 128 and has [384,448) when D = 64.
+// TMEM (fp32 columns): S^T [0,128), warpgroup g's query columns at [64 g, 64 g + 64);
+// each warpgroup packs its P^T (16-bit pairs) into [64 g, 64 g + 32) and its dS^T
+// into [64 g + 32, 64 g + 64) -- inside its own score columns, which it has fully
+// read by then, never the other warpgroup's; dP^T [128,256); dV [256,256+D);
+// dK [256+D,256+2D); the dQ partial reuses [128,256) when D = 128 and has
+// [384,448) when D = 64.
 // Products (M = 128 rows of the first operand, K = 16 per instruction):
 //   S^T  = K_j  Q_i^T   (A = K smem K-major, B = Q smem K-major)
 //   dP^T = V_j  dO_i^T  (A = V smem K-major, B = dO smem K-major)
@@ -153,7 +156,10 @@ struct BwdCfg {
   // No alignment slack: the dynamic region must start 1024-byte aligned (checked).
   static constexpr int SMEM = (2 + 2 * ST) * TILE + DS_BYTES + LD_BYTES + CTRL_BYTES;
   static constexpr int THREADS = 320;
-  static constexpr uint32_t C_S = 0, C_P = 0, C_DS = 64, C_DP = 128;
+  static constexpr uint32_t C_S = 0, C_DP = 128;
+  // packed P^T / dS^T of warpgroup g: columns 64 g + (0 | 32) .. + 31
+  __host__ __device__ static constexpr uint32_t C_P(int g) { return 64u * g; }
+  __host__ __device__ static constexpr uint32_t C_DS(int g) { return 64u * g + 32u; }
   static constexpr uint32_t C_DV = 256, C_DK = 256 + D;
   static constexpr uint32_t C_DQ = (D == 128) ? 128 : 384;
 };
@@ -182,17 +188,11 @@ enum BwdSite : uint32_t {
   kBSiteMmaDrain, kBSiteCmpQ, kBSiteCmpS, kBSiteCmpDP, kBSiteCmpDQ, kBSiteProdDrain
 };
 
-__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
-  asm volatile("red.relaxed.gpu.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a),
-               "f"(b), "f"(c), "f"(d)
-               : "memory");
-}
-
 template <int D, bool BF16, bool CAUSAL>
 __global__ void __launch_bounds__(320, 1)
 fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
-               const BwdParams p) {
+               const __grid_constant__ CUtensorMap tmdQ, const BwdParams p) {
   using C = BwdCfg<D>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   if ((smem_u32(smem_raw) & 1023u) != 0) {
@@ -337,8 +337,8 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         if (!mbar_wait(&p_ready, it & 1, wc, kBSiteMmaP)) { ok = false; break; }
         tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          umma_ts(tbase + C::C_DV, tbase + C::C_P + kk * 8,
+        for (int kk = 0; kk < 8; ++kk)  // queries 16 kk .. 16 kk + 15: warpgroup kk / 4
+          umma_ts(tbase + C::C_DV, tbase + C::C_P(kk >> 2) + (kk & 3) * 8,
                   sdesc_sw128(adO + st * C::TILE + kk * 2048, C::CHUNK, 1024), id_tb,
                   (it > 0 || kk > 0) ? 1u : 0u);
         // dK += dS^T Q
@@ -346,7 +346,7 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          umma_ts(tbase + C::C_DK, tbase + C::C_DS + kk * 8,
+          umma_ts(tbase + C::C_DK, tbase + C::C_DS(kk >> 2) + (kk & 3) * 8,
                   sdesc_sw128(aQ + st * C::TILE + kk * 2048, C::CHUNK, 1024), id_tb,
                   (it > 0 || kk > 0) ? 1u : 0u);
         // dQ_i = dS K (its own columns when D = 64: wait for the previous drain)
@@ -376,6 +376,7 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     const uint32_t lb = static_cast<uint32_t>(wq * 32);
     const float sl2 = p.scale_log2;
     const int qoff = 64 * g;
+    const uint32_t wg_bar = 1 + g;             // named barrier of this warpgroup
     bool ok = true;
     for (int it = 0; it < n_it && ok; ++it) {
       const int i = i_begin + it;
@@ -383,9 +384,12 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       // This tile's LSE*log2e and D rows arrive in shared memory with Q_i and dO_i.
       const float4* L4 = reinterpret_cast<const float4*>(sLD + st * 256 + qoff);
       const float4* D4 = reinterpret_cast<const float4*>(sLD + st * 256 + 128 + qoff);
-      ok = __all_sync(0xffffffffu, mbar_wait(&qdo_full[st], (it / C::ST) & 1, wc, kBSiteCmpQ));
+      // Every wait of a compute warpgroup ends in a warpgroup-wide vote, so that all
+      // of its 128 threads leave together on a timeout (the named barriers below
+      // have no time limit and must never be left waiting).
+      ok = named_bar_and(wg_bar, 128, mbar_wait(&qdo_full[st], (it / C::ST) & 1, wc, kBSiteCmpQ));
       if (!ok) break;
-      ok = __all_sync(0xffffffffu, mbar_wait(&s_full, it & 1, wc, kBSiteCmpS));
+      ok = named_bar_and(wg_bar, 128, mbar_wait(&s_full, it & 1, wc, kBSiteCmpS));
       if (!ok) break;
       tc_fence_after();
       // P^T (this warpgroup's 64 query columns): exp2(S^T * scale * log2e - LSE * log2e),
@@ -416,7 +420,7 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         uint32_t pk[32];
 #pragma unroll
         for (int e = 0; e < 32; ++e) pk[e] = pack2<BF16>(pr[2 * e], pr[2 * e + 1]);
-        tmem_st32(tmem_addr(tbase, lb, C::C_P + 32 * g), pk);
+        tmem_st32(tmem_addr(tbase, lb, C::C_P(g)), pk);
       }
       tmem_wait_st();
       tc_fence_before();
@@ -426,9 +430,15 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       // of dK) and to shared memory (A operand of dQ).  The shared copy is
       // MN-major with 128-byte swizzle: chunk g holds queries 64 g .. 64 g + 63 of
       // every key row; 16-byte unit u of row r sits at unit u ^ (r % 8).
-      ok = __all_sync(0xffffffffu, mbar_wait(&dp_full, it & 1, wc, kBSiteCmpDP));
+      ok = named_bar_and(wg_bar, 128, mbar_wait(&dp_full, it & 1, wc, kBSiteCmpDP));
       if (!ok) break;
       tc_fence_after();
+      if (it > 0) {
+        // This warpgroup's dS^T chunk doubled as the staging tile of the previous
+        // dQ reduce: that bulk copy must have finished reading it.
+        if (r == 0) tma_store_wait_read();
+        named_bar_sync(wg_bar, 128);
+      }
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         uint32_t dr[32];
@@ -447,7 +457,7 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           dsk[2 * v] = pack2<BF16>(a0, a1);
           dsk[2 * v + 1] = pack2<BF16>(a2, a3);
         }
-        tmem_st16(tmem_addr(tbase, lb, C::C_DS + 32 * g + 16 * c), dsk);
+        tmem_st16(tmem_addr(tbase, lb, C::C_DS(g) + 16 * c), dsk);
 #pragma unroll
         for (int uu = 0; uu < 4; ++uu) {
           const int u = c * 4 + uu;
@@ -461,12 +471,16 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       __syncwarp();
       if (lane == 0) mbar_arrive(&ds_ready);
       // dQ partial: query row r, head columns g D/2 .. (g+1) D/2 - 1 -> fp32 accumulator
-      ok = __all_sync(0xffffffffu, mbar_wait(&dq_full, it & 1, wc, kBSiteCmpDQ));
+      ok = named_bar_and(wg_bar, 128, mbar_wait(&dq_full, it & 1, wc, kBSiteCmpDQ));
       if (!ok) break;
       tc_fence_after();
-      const int q = i * 128 + r;
+      // dQ partial, head columns g D/2 .. (g+1) D/2 - 1, 32 at a time: TMEM ->
+      // this warpgroup's dS^T chunk of shared memory (free: the dQ product that
+      // read it has completed), laid out as a 128-row x 32-float tile with
+      // 128-byte swizzle -> one TMA reduce-add into the fp32 accumulator (rows
+      // past N are clipped by the tensor map).
       constexpr int HALF = D / 2;
-      float* dst = p.dQacc + (static_cast<size_t>(bh) * N + q) * D + g * HALF;
+      uint8_t* stage = sDS + g * C::CHUNK;
 #pragma unroll
       for (int c = 0; c < HALF / 32; ++c) {
         uint32_t qr[32];
@@ -478,15 +492,26 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           __syncwarp();
           if (lane == 0) mbar_arrive(&dq_drained);
         }
-        if (q < N) {
-#pragma unroll
-          for (int v = 0; v < 8; ++v)
-            red_add_v4(dst + c * 32 + v * 4, __uint_as_float(qr[4 * v]),
-                       __uint_as_float(qr[4 * v + 1]), __uint_as_float(qr[4 * v + 2]),
-                       __uint_as_float(qr[4 * v + 3]));
+        if (c > 0) {
+          if (r == 0) tma_store_wait_read();
+          named_bar_sync(wg_bar, 128);
         }
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          *reinterpret_cast<uint4*>(stage + r * 128 + ((u ^ (r & 7)) << 4)) =
+              make_uint4(qr[4 * u], qr[4 * u + 1], qr[4 * u + 2], qr[4 * u + 3]);
+        fence_proxy_async_smem();
+        named_bar_sync(wg_bar, 128);
+        if (r == 0) {
+          tma_reduce_add_3d(&tmdQ, stage, g * HALF + 32 * c, i * 128, bh);
+          tma_store_commit();
+        }
+        __syncwarp();  // the TMEM loads that follow are warp-collective
       }
     }
+    // All reductions complete before the CTA (and its shared memory) goes away.
+    if (r == 0) tma_store_wait_all();
+    __syncwarp();
     if (ok) {
       // dV (warpgroup 0) and dK (warpgroup 1) are final once the last dQ product,
       // issued after them, has landed.
@@ -527,6 +552,7 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 // ------------------------------------------------------------------------------------
 
 bool make_tile_map(CUtensorMap* map, const void* base, int BH, int N, int d, bool bf16);
+bool make_acc_map(CUtensorMap* map, float* base, int BH, int N, int d);
 
 template <int D, bool BF16, bool CAUSAL>
 int launch_bwd_t(const void* Q, const void* K, const void* V, const void* O, const void* dO,
@@ -539,9 +565,10 @@ int launch_bwd_t(const void* Q, const void* K, const void* V, const void* O, con
   float* Lg = Dg + static_cast<size_t>(BH) * Npad;
   float* dQacc = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
                                           bwd_rowstat_bytes(static_cast<size_t>(BH), N));
-  CUtensorMap mq, mk, mv, mdo;
+  CUtensorMap mq, mk, mv, mdo, mdq;
   if (!make_tile_map(&mq, Q, BH, N, D, BF16) || !make_tile_map(&mk, K, BH, N, D, BF16) ||
-      !make_tile_map(&mv, V, BH, N, D, BF16) || !make_tile_map(&mdo, dO, BH, N, D, BF16))
+      !make_tile_map(&mv, V, BH, N, D, BF16) || !make_tile_map(&mdo, dO, BH, N, D, BF16) ||
+      !make_acc_map(&mdq, dQacc, BH, N, D))
     return 4;  // FA2_ERR_CUDA
   // 1. preprocess
   {
@@ -576,7 +603,7 @@ int launch_bwd_t(const void* Q, const void* K, const void* V, const void* O, con
     bp.status = status;
     bp.wait_ns = wait_ns;
     const unsigned int grid = static_cast<unsigned int>(bp.n_kv) * static_cast<unsigned int>(BH);
-    kern<<<grid, Cfg::THREADS, Cfg::SMEM, stream>>>(mq, mk, mv, mdo, bp);
+    kern<<<grid, Cfg::THREADS, Cfg::SMEM, stream>>>(mq, mk, mv, mdo, mdq, bp);
     if (cudaGetLastError() != cudaSuccess) return 4;
   }
   // 3. dQ finalise

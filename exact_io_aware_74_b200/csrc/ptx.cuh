@@ -186,6 +186,42 @@ __device__ __forceinline__ void tma_store_wait_read() {
   asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
 }
 
+// 3-D tiled reduce-add (fp32) from shared memory into global memory, bulk group
+// completion.  Rows outside the tensor are clipped.
+__device__ __forceinline__ void tma_reduce_add_3d(const CUtensorMap* map, const void* smem_src,
+                                                  int c0, int c1, int c2) {
+  asm volatile(
+      "cp.reduce.async.bulk.tensor.3d.global.shared::cta.add.tile.bulk_group"
+      " [%0, {%2, %3, %4}], [%1];" ::"l"(reinterpret_cast<uint64_t>(map)),
+      "r"(smem_u32(smem_src)), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+
+// Named barrier over ``n`` threads (a multiple of 32); id 0 is __syncthreads.
+// bar.sync is warp-aligned: the warp is reconverged first, otherwise a warp whose
+// lanes are still apart (one of them waiting on a bulk copy, say) could be
+// counted as arrived before that lane is done.
+__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t n) {
+  __syncwarp();
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
+// Named barrier that also returns the AND of ``pred`` over its ``n`` threads, so
+// that all of them take the same branch afterwards.
+__device__ __forceinline__ bool named_bar_and(uint32_t id, uint32_t n, bool pred) {
+  uint32_t r;
+  __syncwarp();  // warp-aligned barrier: reconverge first (see named_bar_sync)
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(pred)), "r"(id), "r"(n)
+      : "memory");
+  return r != 0;
+}
+
 // Makes generic-proxy writes to shared memory visible to the async proxy
 // (TMA stores, tcgen05 MMAs reading shared memory).
 __device__ __forceinline__ void fence_proxy_async_smem() {
