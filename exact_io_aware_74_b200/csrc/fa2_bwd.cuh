@@ -395,8 +395,10 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       // P^T (this warpgroup's 64 query columns): exp2(S^T * scale * log2e - LSE * log2e),
       // zero where the key comes after the query or lies past N.
       float pr[64];
-      const bool diag = CAUSAL && i == j;
-      const bool key_oob = key >= N;
+      // Masking (key after query on the diagonal tile, or key past N) is rare: one
+      // branch per tile, not a compare per element.
+      const bool masked = (CAUSAL && i == j) || key >= N;
+      const uint64_t sl2x2 = f2_pack(sl2, sl2);
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         uint32_t sr[32];
@@ -406,15 +408,24 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 #pragma unroll
         for (int v = 0; v < 8; ++v) {
           const float4 l4 = L4[c * 8 + v];
-          const float ls[4] = {l4.x, l4.y, l4.z, l4.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int qc = c * 32 + v * 4 + e;
-            float x = ex2_approx(fmaf(__uint_as_float(sr[v * 4 + e]), sl2, -ls[e]));
-            if ((diag && qoff + qc < r) || key_oob) x = 0.f;
-            pr[qc] = x;
-          }
+          const uint64_t a01 = f2_fma(f2_pack(__uint_as_float(sr[v * 4]), __uint_as_float(sr[v * 4 + 1])),
+                                      sl2x2, f2_pack(-l4.x, -l4.y));
+          const uint64_t a23 = f2_fma(f2_pack(__uint_as_float(sr[v * 4 + 2]), __uint_as_float(sr[v * 4 + 3])),
+                                      sl2x2, f2_pack(-l4.z, -l4.w));
+          float x0, x1, x2, x3;
+          f2_unpack(a01, x0, x1);
+          f2_unpack(a23, x2, x3);
+          const int q0 = c * 32 + v * 4;
+          pr[q0 + 0] = ex2_approx(x0);
+          pr[q0 + 1] = ex2_approx(x1);
+          pr[q0 + 2] = ex2_approx(x2);
+          pr[q0 + 3] = ex2_approx(x3);
         }
+      }
+      if (masked) {
+#pragma unroll
+        for (int qc = 0; qc < 64; ++qc)
+          if ((CAUSAL && i == j && qoff + qc < r) || key >= N) pr[qc] = 0.f;
       }
       {
         uint32_t pk[32];
@@ -450,10 +461,13 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         for (int v = 0; v < 8; ++v) {
           const float4 d4 = D4[c * 8 + v];
           const int q0 = c * 32 + v * 4;
-          const float a0 = pr[q0 + 0] * (__uint_as_float(dr[v * 4 + 0]) - d4.x);
-          const float a1 = pr[q0 + 1] * (__uint_as_float(dr[v * 4 + 1]) - d4.y);
-          const float a2 = pr[q0 + 2] * (__uint_as_float(dr[v * 4 + 2]) - d4.z);
-          const float a3 = pr[q0 + 3] * (__uint_as_float(dr[v * 4 + 3]) - d4.w);
+          const uint64_t t01 = f2_sub(f2_pack(__uint_as_float(dr[v * 4]), __uint_as_float(dr[v * 4 + 1])),
+                                      f2_pack(d4.x, d4.y));
+          const uint64_t t23 = f2_sub(f2_pack(__uint_as_float(dr[v * 4 + 2]), __uint_as_float(dr[v * 4 + 3])),
+                                      f2_pack(d4.z, d4.w));
+          float a0, a1, a2, a3;
+          f2_unpack(f2_mul(f2_pack(pr[q0], pr[q0 + 1]), t01), a0, a1);
+          f2_unpack(f2_mul(f2_pack(pr[q0 + 2], pr[q0 + 3]), t23), a2, a3);
           dsk[2 * v] = pack2<BF16>(a0, a1);
           dsk[2 * v + 1] = pack2<BF16>(a2, a3);
         }
@@ -480,18 +494,22 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       // 128-byte swizzle -> one TMA reduce-add into the fp32 accumulator (rows
       // past N are clipped by the tensor map).
       constexpr int HALF = D / 2;
+      constexpr int NCH = HALF / 32;
       uint8_t* stage = sDS + g * C::CHUNK;
+      // All of this warpgroup's TMEM columns first, so that the region is released
+      // (dq_drained) before any staging starts.
+      uint32_t qr[NCH][32];
 #pragma unroll
-      for (int c = 0; c < HALF / 32; ++c) {
-        uint32_t qr[32];
-        tmem_ld32(tmem_addr(tbase, lb, C::C_DQ + g * HALF + 32 * c), qr);
-        tmem_wait_ld();
-        reg_fence(qr);
-        if (c == HALF / 32 - 1) {
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&dq_drained);
-        }
+      for (int c = 0; c < NCH; ++c)
+        tmem_ld32(tmem_addr(tbase, lb, C::C_DQ + g * HALF + 32 * c), qr[c]);
+      tmem_wait_ld();
+#pragma unroll
+      for (int c = 0; c < NCH; ++c) reg_fence(qr[c]);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&dq_drained);
+#pragma unroll
+      for (int c = 0; c < NCH; ++c) {
         if (c > 0) {
           if (r == 0) tma_store_wait_read();
           named_bar_sync(wg_bar, 128);
@@ -499,14 +517,14 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 #pragma unroll
         for (int u = 0; u < 8; ++u)
           *reinterpret_cast<uint4*>(stage + r * 128 + ((u ^ (r & 7)) << 4)) =
-              make_uint4(qr[4 * u], qr[4 * u + 1], qr[4 * u + 2], qr[4 * u + 3]);
+              make_uint4(qr[c][4 * u], qr[c][4 * u + 1], qr[c][4 * u + 2], qr[c][4 * u + 3]);
         fence_proxy_async_smem();
         named_bar_sync(wg_bar, 128);
         if (r == 0) {
           tma_reduce_add_3d(&tmdQ, stage, g * HALF + 32 * c, i * 128, bh);
           tma_store_commit();
         }
-        __syncwarp();  // the TMEM loads that follow are warp-collective
+        __syncwarp();
       }
     }
     // All reductions complete before the CTA (and its shared memory) goes away.
