@@ -341,15 +341,11 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           umma_ts(tbase + C::C_DV, tbase + C::C_P(kk >> 2) + (kk & 3) * 8,
                   sdesc_sw128(adO + st * C::TILE + kk * 2048, C::CHUNK, 1024), id_tb,
                   (it > 0 || kk > 0) ? 1u : 0u);
-        // dK += dS^T Q
+        // dQ_i = dS K first (the drain needs only this one; its own TMEM columns when
+        // D = 64: wait for the previous drain), then dK += dS^T Q (A from TMEM, so
+        // the dQ staging that reuses the dS^T tile of shared memory cannot race it).
         if (!mbar_wait(&ds_ready, it & 1, wc, kBSiteMmaDS)) { ok = false; break; }
         tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          umma_ts(tbase + C::C_DK, tbase + C::C_DS(kk >> 2) + (kk & 3) * 8,
-                  sdesc_sw128(aQ + st * C::TILE + kk * 2048, C::CHUNK, 1024), id_tb,
-                  (it > 0 || kk > 0) ? 1u : 0u);
-        // dQ_i = dS K (its own columns when D = 64: wait for the previous drain)
         if (D == 64 && it > 0) {
           if (!mbar_wait(&dq_drained, (it - 1) & 1, wc, kBSiteMmaDrained)) { ok = false; break; }
           tc_fence_after();
@@ -359,9 +355,14 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           umma_ss(tbase + C::C_DQ, sdesc_sw128(aDS + kk * 2048, C::CHUNK, 1024),
                   sdesc_sw128(aK + kk * 2048, C::CHUNK, 1024), id_dq, kk > 0);
         umma_commit(&dq_full);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          umma_ts(tbase + C::C_DK, tbase + C::C_DS(kk >> 2) + (kk & 3) * 8,
+                  sdesc_sw128(aQ + st * C::TILE + kk * 2048, C::CHUNK, 1024), id_tb,
+                  (it > 0 || kk > 0) ? 1u : 0u);
         umma_commit(&qdo_empty[st]);
       }
-      umma_commit(&drain);
+      umma_commit(&drain);  // also tells the compute warps that dK and dV are final
       volatile int no_abort = 0;
       WaitCtl dw{p.status, &no_abort, p.wait_ns};
       mbar_wait(&drain, 0, dw, kBSiteMmaDrain);
@@ -399,12 +400,15 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       // branch per tile, not a compare per element.
       const bool masked = (CAUSAL && i == j) || key >= N;
       const uint64_t sl2x2 = f2_pack(sl2, sl2);
+      uint32_t srr[2][32];
+      tmem_ld32(tmem_addr(tbase, lb, C::C_S + qoff), srr[0]);
+      tmem_ld32(tmem_addr(tbase, lb, C::C_S + qoff + 32), srr[1]);
+      tmem_wait_ld();
+      reg_fence(srr[0]);
+      reg_fence(srr[1]);
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
-        uint32_t sr[32];
-        tmem_ld32(tmem_addr(tbase, lb, C::C_S + qoff + 32 * c), sr);
-        tmem_wait_ld();
-        reg_fence(sr);
+        const uint32_t (&sr)[32] = srr[c];
 #pragma unroll
         for (int v = 0; v < 8; ++v) {
           const float4 l4 = L4[c * 8 + v];
@@ -530,9 +534,10 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     // All reductions complete before the CTA (and its shared memory) goes away.
     if (r == 0) tma_store_wait_all();
     __syncwarp();
+    // dV (warpgroup 0) and dK (warpgroup 1) are final once every MMA has landed.
+    if (ok) ok = named_bar_and(wg_bar, 128, mbar_wait(&drain, 0, wc, kBSiteCmpDQ));
     if (ok) {
-      // dV (warpgroup 0) and dK (warpgroup 1) are final once the last dQ product,
-      // issued after them, has landed.
+      tc_fence_after();
       const uint32_t col = g ? C::C_DK : C::C_DV;
       const float mul = g ? p.scale : 1.0f;
       uint8_t* row = reinterpret_cast<uint8_t*>(g ? p.dK : p.dV) +
