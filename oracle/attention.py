@@ -45,11 +45,13 @@ def _check_shapes(q, k, v):
 
 
 def _scores(q_rows: np.ndarray, k: np.ndarray, row0: int, scale: float,
-            causal: bool) -> tuple[np.ndarray, int]:
+            causal: bool, window: int | None = None) -> tuple[np.ndarray, int]:
     """Scaled scores S = scale * q_rows k^T for query rows row0..row0+len-1.
 
     With ``causal`` the keys after each row's own position are set to -inf and
-    only keys 0..row_last are formed at all.  Returns (S, number of keys used).
+    only keys 0..row_last are formed at all.  With a sliding ``window`` W (causal
+    only) row i also loses the keys before i - W + 1, so that it sees the W most
+    recent keys (itself included).  Returns (S, number of keys used).
     """
     n_rows = q_rows.shape[0]
     n_keys = min(k.shape[0], row0 + n_rows) if causal else k.shape[0]
@@ -58,7 +60,14 @@ def _scores(q_rows: np.ndarray, k: np.ndarray, row0: int, scale: float,
         rows = row0 + np.arange(n_rows)[:, None]
         cols = np.arange(n_keys)[None, :]
         s = np.where(cols > rows, -np.inf, s)
+        if window is not None:
+            s = np.where(cols < rows - window + 1, -np.inf, s)
     return s, n_keys
+
+
+def _check_window(causal: bool, window) -> None:
+    if window is not None and (not causal or int(window) < 1):
+        raise ValueError("a sliding window needs causal=True and window >= 1")
 
 
 def _softmax_rows(s: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
@@ -70,7 +79,7 @@ def _softmax_rows(s: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
 
 
 def attn_fwd_rows_ref(q, k, v, scale: float, causal: bool, bh: int,
-                      rows) -> tuple[np.ndarray, np.ndarray]:
+                      rows, window: int | None = None) -> tuple[np.ndarray, np.ndarray]:
     """O and LSE of selected query rows of one flattened (batch*head) slice.
 
     ``q, k, v`` are [B, H, N, d]; ``bh`` indexes the flattened B*H axis; ``rows``
@@ -80,13 +89,14 @@ def attn_fwd_rows_ref(q, k, v, scale: float, causal: bool, bh: int,
     """
     q, k, v = _f64(q), _f64(k), _f64(v)
     _check_shapes(q, k, v)
+    _check_window(causal, window)
     B, H, N, d = q.shape
     b, h = divmod(int(bh), H)
     rows = np.asarray(rows, dtype=np.int64)
     out = np.empty((rows.size, d))
     lse = np.empty(rows.size)
     for t, r in enumerate(rows):
-        s, nk = _scores(q[b, h, r:r + 1], k[b, h], int(r), scale, causal)
+        s, nk = _scores(q[b, h, r:r + 1], k[b, h], int(r), scale, causal, window)
         p, l = _softmax_rows(s)
         out[t] = (p @ v[b, h, :nk])[0]
         lse[t] = l[0]
@@ -94,13 +104,18 @@ def attn_fwd_rows_ref(q, k, v, scale: float, causal: bool, bh: int,
 
 
 def attn_fwd_ref(q, k, v, scale: float, causal: bool,
-                 row_chunk: int = _ROW_CHUNK) -> tuple[np.ndarray, np.ndarray]:
+                 row_chunk: int = _ROW_CHUNK,
+                 window: int | None = None) -> tuple[np.ndarray, np.ndarray]:
     """Forward attention: O = softmax(scale * Q K^T [causal mask]) V, and LSE.
 
-    Returns (O [B,H,N,d], LSE [B,H,N]) in fp64.
+    ``window`` (causal only) restricts row i to its W most recent keys, the
+    sliding-window attention of "Flash Attention 2: attivarla (llama.cpp,
+    Ollama, vLLM)", section "Modelli con attenzione a finestra scorrevole non
+    standard".  Returns (O [B,H,N,d], LSE [B,H,N]) in fp64.
     """
     q, k, v = _f64(q), _f64(k), _f64(v)
     _check_shapes(q, k, v)
+    _check_window(causal, window)
     B, H, N, d = q.shape
     out = np.empty((B, H, N, d))
     lse = np.empty((B, H, N))
@@ -108,28 +123,29 @@ def attn_fwd_ref(q, k, v, scale: float, causal: bool,
         for h in range(H):
             for r0 in range(0, N, row_chunk):
                 r1 = min(N, r0 + row_chunk)
-                s, nk = _scores(q[b, h, r0:r1], k[b, h], r0, scale, causal)
+                s, nk = _scores(q[b, h, r0:r1], k[b, h], r0, scale, causal, window)
                 p, l = _softmax_rows(s)
                 out[b, h, r0:r1] = p @ v[b, h, :nk]
                 lse[b, h, r0:r1] = l
     return out, lse
 
 
-def attn_probs_ref(q, k, scale: float, causal: bool) -> np.ndarray:
+def attn_probs_ref(q, k, scale: float, causal: bool, window: int | None = None) -> np.ndarray:
     """The full probability matrix P [B,H,N,N] (tiny shapes only; for pins)."""
+    _check_window(causal, window)
     q, k = _f64(q), _f64(k)
     B, H, N, d = q.shape
     p_all = np.zeros((B, H, N, N))
     for b in range(B):
         for h in range(H):
-            s, nk = _scores(q[b, h], k[b, h], 0, scale, causal)
+            s, nk = _scores(q[b, h], k[b, h], 0, scale, causal, window)
             p, _ = _softmax_rows(s)
             p_all[b, h, :, :nk] = p
     return p_all
 
 
 def attn_bwd_ref(q, k, v, do, scale: float, causal: bool,
-                 row_chunk: int = _ROW_CHUNK, heads=None):
+                 row_chunk: int = _ROW_CHUNK, heads=None, window: int | None = None):
     """Gradients of L = sum(O * dO) with respect to Q, K and V (fp64).
 
     The probabilities are recomputed from the scores of each chunk of query
@@ -140,6 +156,7 @@ def attn_bwd_ref(q, k, v, do, scale: float, causal: bool,
     """
     q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
     _check_shapes(q, k, v)
+    _check_window(causal, window)
     if do.shape != q.shape:
         raise ValueError("do must have the shape of q")
     B, H, N, d = q.shape
@@ -153,7 +170,7 @@ def attn_bwd_ref(q, k, v, do, scale: float, causal: bool,
         dv_bh = np.zeros((N, d))
         for r0 in range(0, N, row_chunk):
             r1 = min(N, r0 + row_chunk)
-            s, nk = _scores(q[b, h, r0:r1], k[b, h], r0, scale, causal)
+            s, nk = _scores(q[b, h, r0:r1], k[b, h], r0, scale, causal, window)
             p, _ = _softmax_rows(s)
             do_c = do[b, h, r0:r1]
             dv_bh[:nk] += p.T @ do_c

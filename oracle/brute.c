@@ -18,12 +18,21 @@
  *   dP_ij = sum_c do_ic v_jc
  *   dS_ij = P_ij (dP_ij - sum_l P_il dP_il)
  *   dq_ic = scale sum_j dS_ij k_jc,  dk_jc = scale sum_i dS_ij q_ic
+ * With a sliding window W (causal only; "Flash Attention 2: attivarla", section
+ * "Modelli con attenzione a finestra scorrevole non standard") row i sees only
+ * keys i-W+1..i; brute_set_window(0) turns it off.
  * All arrays are row-major [n][d] doubles.
  */
 #include <math.h>
 #include <stdlib.h>
 
-static int visible(int i, int j, int causal) { return !causal || j <= i; }
+/* window <= 0: no sliding window; otherwise (causal) row i sees keys i-window+1..i */
+static int g_window = 0;
+static int visible(int i, int j, int causal) {
+    if (causal && j > i) return 0;
+    if (causal && g_window > 0 && j < i - g_window + 1) return 0;
+    return 1;
+}
 
 static double score(const double *q, const double *k, int i, int j, int d,
                     double scale) {
@@ -46,6 +55,8 @@ static double row_lse(const double *q, const double *k, int i, int n, int d,
         if (visible(i, j, causal)) z += exp(score(q, k, i, j, d, scale) - m);
     return m + log(z);
 }
+
+void brute_set_window(int window) { g_window = window; }
 
 void brute_attn_fwd(const double *q, const double *k, const double *v,
                     double *o, double *lse, int n, int d, double scale,

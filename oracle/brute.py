@@ -42,6 +42,7 @@ def _load():
                                        ctypes.c_double, ctypes.c_int]
         lib.brute_attn_bwd.argtypes = [dp, dp, dp, dp, dp, dp, dp, ctypes.c_int, ctypes.c_int,
                                        ctypes.c_double, ctypes.c_int]
+        lib.brute_set_window.argtypes = [ctypes.c_int]
         _lib = lib
     return _lib
 
@@ -56,9 +57,10 @@ def _f64(x) -> np.ndarray:
     return np.ascontiguousarray(np.asarray(x, dtype=np.float64))
 
 
-def brute_fwd(q, k, v, scale: float, causal: bool):
+def brute_fwd(q, k, v, scale: float, causal: bool, window: int | None = None):
     """(O, LSE) of [B,H,N,d] inputs by scalar triple loops, fp64."""
     lib = _load()
+    lib.brute_set_window(int(window) if window else 0)
     q, k, v = _f64(q), _f64(k), _f64(v)
     B, H, N, d = q.shape
     o = np.zeros((B, H, N, d))
@@ -74,9 +76,10 @@ def brute_fwd(q, k, v, scale: float, causal: bool):
     return o, lse
 
 
-def brute_bwd(q, k, v, do, scale: float, causal: bool):
+def brute_bwd(q, k, v, do, scale: float, causal: bool, window: int | None = None):
     """(dQ, dK, dV) of [B,H,N,d] inputs by scalar loops, fp64."""
     lib = _load()
+    lib.brute_set_window(int(window) if window else 0)
     q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
     B, H, N, d = q.shape
     dq, dk, dv = (np.zeros((B, H, N, d)) for _ in range(3))

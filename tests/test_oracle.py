@@ -73,6 +73,15 @@ def pin_brute_force(fwd, bwd):
 
 
 def pin_torch_library(fwd, bwd):
+    threads = torch.get_num_threads()
+    torch.set_num_threads(1)  # one summation order on the library side
+    try:
+        _pin_torch_library(fwd, bwd)
+    finally:
+        torch.set_num_threads(threads)
+
+
+def _pin_torch_library(fwd, bwd):
     for i, (B, H, N, d) in enumerate([(2, 3, 37, 16), (1, 2, 64, 32)]):
         for causal in (False, True):
             q, k, v, do = (_rand((B, H, N, d), 100 + 4 * i + j) for j in range(4))
@@ -88,9 +97,9 @@ def pin_torch_library(fwd, bwd):
                                                                   scale=s)
             (to * torch.from_numpy(do)).sum().backward()
             dq, dk, dv = bwd(q, k, v, do, s, causal)
-            _close(dq, tq.grad.numpy(), 1e-10)
-            _close(dk, tk.grad.numpy(), 1e-10)
-            _close(dv, tv.grad.numpy(), 1e-10)
+            _close(dq, tq.grad.numpy(), 1e-9)
+            _close(dk, tk.grad.numpy(), 1e-9)
+            _close(dv, tv.grad.numpy(), 1e-9)
 
 
 def pin_rows_sum_to_one(fwd, bwd):
@@ -205,10 +214,83 @@ def test_oracle_pin(pin):
 
 
 # ----------------------------------------------------------------------------------
+# sliding window ("Flash Attention 2: attivarla", "Modelli con attenzione a finestra
+# scorrevole non standard"): row i sees its W most recent keys i-W+1 .. i
+# ----------------------------------------------------------------------------------
+
+def test_window_matches_brute_force_and_torch():
+    for (B, H, N, d), W in (((1, 2, 33, 8), 5), ((2, 1, 40, 16), 1), ((1, 2, 64, 32), 17)):
+        q, k, v, do = (_rand((B, H, N, d), 200 + N + W + j) for j in range(4))
+        s = 0.4
+        o, lse = oracle.attn_fwd_ref(q, k, v, s, True, window=W)
+        bo, bl = brute_fwd(q, k, v, s, True, window=W)
+        _close(o, bo)
+        _close(lse, bl)
+        g = oracle.attn_bwd_ref(q, k, v, do, s, True, window=W)
+        bg = brute_bwd(q, k, v, do, s, True, window=W)
+        for x, y in zip(g, bg):
+            _close(x, y)
+        # library routine with an explicit boolean mask
+        i = torch.arange(N)[:, None]
+        j = torch.arange(N)[None, :]
+        allowed = (j <= i) & (j > i - W)
+        tq, tk, tv = (torch.tensor(x, requires_grad=True) for x in (q, k, v))
+        to = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, attn_mask=allowed, scale=s)
+        _close(o, to.detach().numpy())
+        (to * torch.from_numpy(do)).sum().backward()
+        _close(g[0], tq.grad.numpy(), 1e-10)
+        _close(g[1], tk.grad.numpy(), 1e-10)
+        _close(g[2], tv.grad.numpy(), 1e-10)
+
+
+def test_window_closed_forms():
+    B, H, N, d = 1, 2, 30, 8
+    q, k, v = (_rand((B, H, N, d), 230 + j) for j in range(3))
+    s = 0.7
+    # W = 1: every row sees only itself
+    o, lse = oracle.attn_fwd_ref(q, k, v, s, True, window=1)
+    _close(o, v)
+    _close(lse, s * np.einsum("bhnc,bhnc->bhn", q, k))
+    # W >= N: plain causal attention
+    for W in (N, N + 7):
+        o2, l2 = oracle.attn_fwd_ref(q, k, v, s, True, window=W)
+        o3, l3 = oracle.attn_fwd_ref(q, k, v, s, True)
+        _close(o2, o3)
+        _close(l2, l3)
+    # Q = 0: O_i is the mean of the W most recent values
+    W = 4
+    o, lse = oracle.attn_fwd_ref(np.zeros_like(q), k, v, 1.0, True, window=W)
+    for i in range(N):
+        lo = max(0, i - W + 1)
+        _close(o[:, :, i], v[:, :, lo:i + 1].mean(axis=2))
+        _close(lse[:, :, i], np.full((B, H), math.log(i + 1 - lo)))
+    with pytest.raises(ValueError):
+        oracle.attn_fwd_ref(q, k, v, s, False, window=3)
+
+
+def test_window_finite_differences():
+    B, H, N, d, W = 1, 1, 6, 4, 3
+    q, k, v, do = (_rand((B, H, N, d), 240 + j) for j in range(4))
+    s, eps = 0.9, 1e-6
+    grads = oracle.attn_bwd_ref(q, k, v, do, s, True, window=W)
+    for which, g in enumerate(grads):
+        num = np.zeros_like(g)
+        for idx in np.ndindex(*g.shape):
+            a = [q.copy(), k.copy(), v.copy()]
+            b = [q.copy(), k.copy(), v.copy()]
+            a[which][idx] += eps
+            b[which][idx] -= eps
+            fp = float((oracle.attn_fwd_ref(*a, s, True, window=W)[0] * do).sum())
+            fm = float((oracle.attn_fwd_ref(*b, s, True, window=W)[0] * do).sum())
+            num[idx] = (fp - fm) / (2 * eps)
+        _close(g, num, 1e-6)
+
+
+# ----------------------------------------------------------------------------------
 # planted mistakes (in copies of the oracle, on the CPU) must fail some pin
 # ----------------------------------------------------------------------------------
 
-def _mut_scores_diag(q_rows, k, row0, scale, causal):
+def _mut_scores_diag(q_rows, k, row0, scale, causal, window=None):
     """Causal mask that also hides the diagonal (j >= i instead of j > i)."""
     n_rows = q_rows.shape[0]
     n_keys = min(k.shape[0], row0 + n_rows) if causal else k.shape[0]
