@@ -180,8 +180,13 @@ int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& 
 
 extern "C" {
 
-int fa2_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, int B, int H,
-            int N, int d, float scale, int causal, int dtype, fa2_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// Shared by fa2_fwd and fa2_fwd_window; window = 0 means no sliding window.
+int fwd_impl(const void* Q, const void* K, const void* V, void* O, float* LSE, int B, int H,
+             int N, int d, float scale, int causal, int window, int dtype, fa2_stream_t stream) {
   if (!Q || !K || !V || !O || !LSE) return FA2_ERR_INVALID_ARG;
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(LSE))
     return FA2_ERR_INVALID_ARG;
@@ -216,6 +221,7 @@ int fa2_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, in
   p.status = st;
   p.wait_ns = wait_ns();
   p.fault = g_fault.load();
+  p.window = window;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const bool bf = dtype == FA2_BF16;
   if (d == 64) {
@@ -226,15 +232,37 @@ int fa2_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, in
   return causal ? launch_fwd<128, false, true>(mq, mk, mv, p, s) : launch_fwd<128, false, false>(mq, mk, mv, p, s);
 }
 
+}  // namespace
+
+extern "C" {
+
+int fa2_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, int B, int H,
+            int N, int d, float scale, int causal, int dtype, fa2_stream_t stream) {
+  return fwd_impl(Q, K, V, O, LSE, B, H, N, d, scale, causal, 0, dtype, stream);
+}
+
+int fa2_fwd_window(const void* Q, const void* K, const void* V, void* O, float* LSE, int B,
+                   int H, int N, int d, float scale, int window, int dtype, fa2_stream_t stream) {
+  if (window < 1) return FA2_ERR_INVALID_ARG;
+  // A window as long as the sequence is plain causal attention.
+  return fwd_impl(Q, K, V, O, LSE, B, H, N, d, scale, 1, window >= N ? 0 : window, dtype,
+                  stream);
+}
+
 size_t fa2_bwd_workspace_size(int B, int H, int N, int d) {
   if (check_sizes(B, H, N, d, 1.0f, 0, FA2_BF16) != FA2_OK) return 0;
   return fa2::bwd_workspace_bytes(static_cast<size_t>(B) * H, N, d);
 }
 
-int fa2_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO,
-            const float* LSE, void* dQ, void* dK, void* dV, void* workspace,
-            size_t workspace_bytes, int B, int H, int N, int d, float scale, int causal,
-            int dtype, fa2_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// Shared by fa2_bwd and fa2_bwd_window; window = 0 means no sliding window.
+int bwd_impl(const void* Q, const void* K, const void* V, const void* O, const void* dO,
+             const float* LSE, void* dQ, void* dK, void* dV, void* workspace,
+             size_t workspace_bytes, int B, int H, int N, int d, float scale, int causal,
+             int window, int dtype, fa2_stream_t stream) {
   if (!Q || !K || !V || !O || !dO || !LSE || !dQ || !dK || !dV) return FA2_ERR_INVALID_ARG;
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(dO) ||
       !aligned16(LSE) || !aligned16(dQ) || !aligned16(dK) || !aligned16(dV))
@@ -265,9 +293,30 @@ int fa2_bwd(const void* Q, const void* K, const void* V, const void* O, const vo
   if (!st) return FA2_ERR_CUDA;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   rc = fa2::launch_bwd(Q, K, V, O, dO, LSE, dQ, dK, dV, workspace, BH, N, d, scale, causal != 0,
-                       dtype == FA2_BF16, st, wait_ns(), s);
+                       dtype == FA2_BF16, st, wait_ns(), s, window);
   if (rc == FA2_OK) g_launches.fetch_add(fa2::kBwdKernelsPerCall);
   return rc;
+}
+
+}  // namespace
+
+extern "C" {
+
+int fa2_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO,
+            const float* LSE, void* dQ, void* dK, void* dV, void* workspace,
+            size_t workspace_bytes, int B, int H, int N, int d, float scale, int causal,
+            int dtype, fa2_stream_t stream) {
+  return bwd_impl(Q, K, V, O, dO, LSE, dQ, dK, dV, workspace, workspace_bytes, B, H, N, d, scale,
+                  causal, 0, dtype, stream);
+}
+
+int fa2_bwd_window(const void* Q, const void* K, const void* V, const void* O, const void* dO,
+                   const float* LSE, void* dQ, void* dK, void* dV, void* workspace,
+                   size_t workspace_bytes, int B, int H, int N, int d, float scale, int window,
+                   int dtype, fa2_stream_t stream) {
+  if (window < 1) return FA2_ERR_INVALID_ARG;
+  return bwd_impl(Q, K, V, O, dO, LSE, dQ, dK, dV, workspace, workspace_bytes, B, H, N, d, scale,
+                  1, window >= N ? 0 : window, dtype, stream);
 }
 
 }  // extern "C"

@@ -139,6 +139,7 @@ struct BwdParams {
   void* dK;           // [BH][N][D] 16-bit
   void* dV;           // [BH][N][D] 16-bit
   int N, Npad, BH, n_kv;
+  int window;         // causal only: query i sees keys i-window+1..i (0 = no window)
   float scale, scale_log2;
   unsigned int* status;
   unsigned long long wait_ns;
@@ -229,7 +230,12 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   const int bh = static_cast<int>(blockIdx.x) % p.BH;
   const int n_q = p.n_kv;
   const int i_begin = CAUSAL ? j : 0;
-  const int n_it = n_q - i_begin;
+  // With a sliding window the last query that sees a key of this tile is
+  // j*128 + 127 + window - 1.
+  const int i_end = (CAUSAL && p.window > 0)
+                        ? min(n_q, (j * 128 + 127 + p.window - 1) / 128 + 1)
+                        : n_q;
+  const int n_it = i_end - i_begin;
 
   WaitCtl wc{p.status, &abort_flag, p.wait_ns};
 
@@ -398,7 +404,9 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       float pr[64];
       // Masking (key after query on the diagonal tile, or key past N) is rare: one
       // branch per tile, not a compare per element.
-      const bool masked = (CAUSAL && i == j) || key >= N;
+      const int win = p.window;
+      const bool masked = (CAUSAL && i == j) || key >= N ||
+                          (CAUSAL && win > 0 && i * 128 + 127 - j * 128 >= win);
       const uint64_t sl2x2 = f2_pack(sl2, sl2);
       uint32_t srr[2][32];
       tmem_ld32(tmem_addr(tbase, lb, C::C_S + qoff), srr[0]);
@@ -429,7 +437,9 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       if (masked) {
 #pragma unroll
         for (int qc = 0; qc < 64; ++qc)
-          if ((CAUSAL && i == j && qoff + qc < r) || key >= N) pr[qc] = 0.f;
+          if ((CAUSAL && i == j && qoff + qc < r) || key >= N ||
+              (CAUSAL && win > 0 && i * 128 + qoff + qc - key >= win))
+            pr[qc] = 0.f;
       }
       {
         uint32_t pk[32];
@@ -580,7 +590,7 @@ bool make_acc_map(CUtensorMap* map, float* base, int BH, int N, int d);
 template <int D, bool BF16, bool CAUSAL>
 int launch_bwd_t(const void* Q, const void* K, const void* V, const void* O, const void* dO,
                  const float* LSE, void* dQ, void* dK, void* dV, void* workspace, int BH, int N,
-                 float scale, unsigned int* status, unsigned long long wait_ns,
+                 float scale, int window, unsigned int* status, unsigned long long wait_ns,
                  cudaStream_t stream) {
   using Cfg = BwdCfg<D>;
   const int Npad = static_cast<int>(bwd_npad(N));
@@ -623,6 +633,7 @@ int launch_bwd_t(const void* Q, const void* K, const void* V, const void* O, con
     bp.n_kv = Npad / 128;
     bp.scale = scale;
     bp.scale_log2 = scale * 1.4426950408889634f;
+    bp.window = window;
     bp.status = status;
     bp.wait_ns = wait_ns;
     const unsigned int grid = static_cast<unsigned int>(bp.n_kv) * static_cast<unsigned int>(BH);
@@ -643,10 +654,10 @@ int launch_bwd_t(const void* Q, const void* K, const void* V, const void* O, con
 inline int launch_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO,
                       const float* LSE, void* dQ, void* dK, void* dV, void* workspace, int BH,
                       int N, int d, float scale, bool causal, bool bf16, unsigned int* status,
-                      unsigned long long wait_ns, cudaStream_t s) {
+                      unsigned long long wait_ns, cudaStream_t s, int window = 0) {
 #define FA2_BWD_CALL(D_, BF_, CA_)                                                          \
   return launch_bwd_t<D_, BF_, CA_>(Q, K, V, O, dO, LSE, dQ, dK, dV, workspace, BH, N, scale, \
-                                    status, wait_ns, s)
+                                    window, status, wait_ns, s)
   if (d == 64) {
     if (bf16) { if (causal) FA2_BWD_CALL(64, true, true); FA2_BWD_CALL(64, true, false); }
     if (causal) FA2_BWD_CALL(64, false, true);

@@ -47,6 +47,7 @@ struct FwdParams {
   unsigned int* status;        // device status word
   unsigned long long wait_ns;  // budget of one bounded wait
   int fault;                   // test hook: 1 = skip the first K load
+  int window;                  // causal only: row i sees keys i-window+1..i (0 = no window)
 };
 
 template <int D>
@@ -110,19 +111,27 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   const int qb = p.n_qblk - 1 - static_cast<int>(blockIdx.x) / p.BH;
   const int bh = static_cast<int>(blockIdx.x) % p.BH;
   const int n_kv_all = (N + C::BN - 1) / C::BN;
-  int row0[2], n_kv[2];
+  // Key tiles [j_lo[t], j_hi[t]) are the ones query tile t needs: all of them,
+  // or (causal) up to its diagonal, and (sliding window) from the tile that holds
+  // the first key its first row still sees.  Tiles past N have an empty range.
+  int row0[2], j_lo[2], j_hi[2];
 #pragma unroll
   for (int t = 0; t < 2; ++t) {
     row0[t] = qb * 256 + t * 128;
+    j_lo[t] = 0;
     if (row0[t] >= N) {
-      n_kv[t] = 0;
+      j_hi[t] = 0;
     } else if (CAUSAL) {
-      n_kv[t] = min(n_kv_all, row0[t] / C::BN + 1);
+      j_hi[t] = min(n_kv_all, row0[t] / C::BN + 1);
+      if (p.window > 0) j_lo[t] = max(0, row0[t] - p.window + 1) / C::BN;
     } else {
-      n_kv[t] = n_kv_all;
+      j_hi[t] = n_kv_all;
     }
   }
-  const int n_kv_max = max(n_kv[0], n_kv[1]);
+  // The CTA walks key tiles j0 .. j1-1; the K/V ring is indexed from j0.
+  const int j0 = (j_hi[1] > 0) ? min(j_lo[0], j_lo[1]) : j_lo[0];
+  const int j1 = max(j_hi[0], j_hi[1]);
+  const int n_steps = j1 - j0;
 
   WaitCtl wc{p.status, &abort_flag, p.wait_ns};
 
@@ -161,29 +170,30 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       tma_prefetch_desc(&tmV);
       const uint64_t keep = policy_evict_last();
       uint32_t q_bytes = 0;
-      for (int t = 0; t < 2; ++t) q_bytes += (n_kv[t] > 0) ? C::TILE : 0;
+      for (int t = 0; t < 2; ++t) q_bytes += (j_hi[t] > 0) ? C::TILE : 0;
       mbar_arrive_expect_tx(&bar_q, q_bytes);
       for (int t = 0; t < 2; ++t) {
-        if (n_kv[t] == 0) continue;
+        if (j_hi[t] == 0) continue;
         for (int c = 0; c < C::KCH; ++c)
           tma_load_3d(sQ + t * C::TILE + c * C::CHUNK, &tmQ, &bar_q, c * 64, row0[t], bh);
       }
       int k_issued = 0, v_issued = 0;  // loads issued so far
       bool ok = true;
-      for (int j = 0; j < n_kv_max && ok; ++j) {
-        const int ks = j % C::KS, vs = j % C::VS;
-        if (j >= C::KS && !mbar_wait(&k_empty[ks], ((j / C::KS) - 1) & 1, wc, kSiteProdKEmpty)) {
+      for (int jj = 0; jj < n_steps && ok; ++jj) {
+        const int j = j0 + jj;  // key tile; jj is its slot count in the rings
+        const int ks = jj % C::KS, vs = jj % C::VS;
+        if (jj >= C::KS && !mbar_wait(&k_empty[ks], ((jj / C::KS) - 1) & 1, wc, kSiteProdKEmpty)) {
           ok = false;
           break;
         }
-        if (!(p.fault == 1 && j == 0)) {
+        if (!(p.fault == 1 && jj == 0)) {
           mbar_arrive_expect_tx(&k_full[ks], C::TILE);
           for (int c = 0; c < C::KCH; ++c)
             tma_load_3d_hint(sK + ks * C::TILE + c * C::CHUNK, &tmK, &k_full[ks], c * 64,
                              j * C::BN, bh, keep);
-          k_issued = j + 1;
+          k_issued = jj + 1;
         }
-        if (j >= C::VS && !mbar_wait(&v_empty[vs], ((j / C::VS) - 1) & 1, wc, kSiteProdVEmpty)) {
+        if (jj >= C::VS && !mbar_wait(&v_empty[vs], ((jj / C::VS) - 1) & 1, wc, kSiteProdVEmpty)) {
           ok = false;
           break;
         }
@@ -191,7 +201,7 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         for (int c = 0; c < C::KCH; ++c)
           tma_load_3d_hint(sV + vs * C::TILE + c * C::CHUNK, &tmV, &v_full[vs], c * 64,
                            j * C::BN, bh, keep);
-        v_issued = j + 1;
+        v_issued = jj + 1;
       }
       if (!ok) {
         // Let every copy already issued land before the CTA exits.
@@ -233,29 +243,36 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       bool ok = mbar_wait(&bar_q, 0, wc, kSiteMmaQ) && mbar_wait(&k_full[0], 0, wc, kSiteMmaK);
       if (ok) {
         tc_fence_after();
-        issue_qk(0, 0);
-        umma_commit(&s_full[0]);
-        if (n_kv[1] > 0) {
-          issue_qk(1, 0);
-          umma_commit(&s_full[1]);
-        }
+        // Tiles whose key range starts at j0 get their first S now.
+        for (int t = 0; t < 2; ++t)
+          if (j_hi[t] > j_lo[t] && j_lo[t] == j0) {
+            issue_qk(t, 0);
+            umma_commit(&s_full[t]);
+          }
         umma_commit(&k_empty[0]);
       }
-      for (int j = 0; j < n_kv_max && ok; ++j) {
-        const int vs = j % C::VS;
-        const int ks1 = (j + 1) % C::KS;
-        const bool has_next = j + 1 < n_kv_max;
+      for (int jj = 0; jj < n_steps && ok; ++jj) {
+        const int j = j0 + jj;
+        const int vs = jj % C::VS;
+        const int ks1 = (jj + 1) % C::KS;
+        const bool has_next = jj + 1 < n_steps;
         bool k_next_ready = false;
-        if (!mbar_wait(&v_full[vs], (j / C::VS) & 1, wc, kSiteMmaV)) { ok = false; break; }
-        auto tile_step = [&](int t, int nkv_t) -> bool {
-          if (j >= nkv_t) return true;
-          if (!mbar_wait(&p_ready[t], j & 1, wc, kSiteMmaP)) return false;
-          tc_fence_after();
-          issue_pv(t, vs, j > 0);
-          umma_commit(&o_done[t]);
-          if (j + 1 < nkv_t) {
+        if (!mbar_wait(&v_full[vs], (jj / C::VS) & 1, wc, kSiteMmaV)) { ok = false; break; }
+        auto tile_step = [&](int t) -> bool {
+          const int lo = t ? j_lo[1] : j_lo[0];
+          const int hi = t ? j_hi[1] : j_hi[0];
+          if (j >= lo && j < hi) {
+            const int step = j - lo;  // this tile's own step count
+            if (!mbar_wait(&p_ready[t], step & 1, wc, kSiteMmaP)) return false;
+            tc_fence_after();
+            issue_pv(t, vs, step > 0);
+            umma_commit(&o_done[t]);
+          }
+          // S for step j + 1 (this tile's next step, or its first when its range
+          // starts there); P of step j in the same columns was consumed above.
+          if (j + 1 >= lo && j + 1 < hi) {
             if (!k_next_ready) {
-              if (!mbar_wait(&k_full[ks1], ((j + 1) / C::KS) & 1, wc, kSiteMmaK)) return false;
+              if (!mbar_wait(&k_full[ks1], ((jj + 1) / C::KS) & 1, wc, kSiteMmaK)) return false;
               tc_fence_after();
               k_next_ready = true;
             }
@@ -264,7 +281,9 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           }
           return true;
         };
-        ok = tile_step(0, n_kv[0]) && tile_step(1, n_kv[1]);
+        ok = tile_step(0) && tile_step(1);
+        if (ok && has_next && !k_next_ready)  // a slot is only released once its load landed
+          ok = mbar_wait(&k_full[ks1], ((jj + 1) / C::KS) & 1, wc, kSiteMmaK);
         if (!ok) break;
         umma_commit(&v_empty[vs]);
         if (has_next) umma_commit(&k_empty[ks1]);
@@ -284,7 +303,8 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     const int wq = warp & 3;      // TMEM lane quadrant
     const int r_loc = wq * 32 + lane;
     const int my_row0 = t ? row0[1] : row0[0];
-    const int my_nkv = t ? n_kv[1] : n_kv[0];
+    const int my_lo = t ? j_lo[1] : j_lo[0];
+    const int my_nkv = (t ? j_hi[1] : j_hi[0]) - my_lo;  // steps of this tile
     const int row = my_row0 + r_loc;
     const uint32_t s_col = t ? C::S_COL1 : C::S_COL0;
     const uint32_t o_col = t ? C::O_COL1 : C::O_COL0;
@@ -293,9 +313,11 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     float m = -INFINITY;  // running max, log2 units of scaled scores
     float l = 0.f;        // running sum of exp2(s * sl2 - m)
     bool ok = my_nkv > 0;
-    for (int j = 0; j < my_nkv && ok; ++j) {
+    const int win = p.window;
+    for (int step = 0; step < my_nkv && ok; ++step) {
+      const int j = my_lo + step;  // key tile of this step
       // Warp-uniform wait: the TMEM loads and stores below are warp-collective.
-      ok = __all_sync(0xffffffffu, mbar_wait(&s_full[t], j & 1, wc, kSiteSoftS));
+      ok = __all_sync(0xffffffffu, mbar_wait(&s_full[t], step & 1, wc, kSiteSoftS));
       if (!ok) break;
       tc_fence_after();
       uint32_t sr[128];
@@ -306,12 +328,15 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       tmem_wait_ld();
       reg_fence(sr);
       const int key0 = j * C::BN;
-      const bool need_mask = (CAUSAL && key0 + C::BN - 1 > my_row0) || (key0 + C::BN > N);
+      // Keys after the row (causal), past N, or before the row's window start.
+      const bool need_mask = (CAUSAL && key0 + C::BN - 1 > my_row0) || (key0 + C::BN > N) ||
+                             (CAUSAL && win > 0 && key0 < my_row0 + 127 - win + 1);
       if (need_mask) {
-        const int lim = CAUSAL ? min(row - key0 + 1, N - key0) : (N - key0);
+        const int hi_lim = CAUSAL ? min(row - key0 + 1, N - key0) : (N - key0);
+        const int lo_lim = (CAUSAL && win > 0) ? row - win + 1 - key0 : 0;
 #pragma unroll
         for (int i = 0; i < 128; ++i)
-          if (i >= lim) sr[i] = __float_as_uint(-INFINITY);
+          if (i >= hi_lim || i < lo_lim) sr[i] = __float_as_uint(-INFINITY);
       }
       float mx[8];
 #pragma unroll
@@ -329,8 +354,8 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       mx[6] = fmaxf(mx[6], mx[7]);
       mx[0] = fmax3(mx[0], mx[3], mx[6]);
       const float m_new = fmaxf(m, mx[0] * sl2);
-      if (j == 0) {
-        m = m_new;
+      if (step == 0) {
+        m = m_new;  // -inf when the window hides this whole tile from the row
       } else {
         // Lazy rescale: the stale maximum is kept unless it fell behind by more
         // than 8 (a factor 256 in the exponentials); the output accumulator is
@@ -340,7 +365,7 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           const float f = need ? ex2_approx(m - m_new) : 1.0f;
           if (need) m = m_new;
           l *= f;
-          ok = __all_sync(0xffffffffu, mbar_wait(&o_done[t], (j - 1) & 1, wc, kSiteSoftO));
+          ok = __all_sync(0xffffffffu, mbar_wait(&o_done[t], (step - 1) & 1, wc, kSiteSoftO));
           if (!ok) break;
           tc_fence_after();
 #pragma unroll
@@ -358,7 +383,9 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       // P = 2^(s * scale * log2 e - m): arguments two at a time (f32x2),
       // exponentials on the MUFU unit (or the polynomial, see kPolyFrom).
       const uint64_t sl2x2 = f2_pack(sl2, sl2);
-      const uint64_t negm2 = f2_pack(-m, -m);
+      // A row that has seen no key yet (m = -inf) gets exp2(-inf) = 0 everywhere.
+      const float neg_m = (m == -INFINITY) ? 0.f : -m;
+      const uint64_t negm2 = f2_pack(neg_m, neg_m);
       uint64_t sum2[4] = {0, 0, 0, 0};
 #pragma unroll
       for (int h = 0; h < 2; ++h) {

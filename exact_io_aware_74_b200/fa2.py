@@ -27,8 +27,9 @@ FA2_FP16 = 0
 FA2_BF16 = 1
 
 # Every symbol include/fa2.h declares.
-EXPORTS = ("fa2_fwd", "fa2_bwd_workspace_size", "fa2_bwd", "fa2_bwd_noalloc",
-           "fa2_get_device_status", "fa2_status_string", "fa2_debug_set", "fa2_launch_count")
+EXPORTS = ("fa2_fwd", "fa2_fwd_window", "fa2_bwd_workspace_size", "fa2_bwd", "fa2_bwd_window",
+           "fa2_bwd_noalloc", "fa2_get_device_status", "fa2_status_string", "fa2_debug_set",
+           "fa2_launch_count")
 
 _lib = None
 
@@ -51,6 +52,10 @@ def load() -> ctypes.CDLL:
     vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
     lib.fa2_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, i, vp]
     lib.fa2_fwd.restype = i
+    lib.fa2_fwd_window.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, i, vp]
+    lib.fa2_fwd_window.restype = i
+    lib.fa2_bwd_window.argtypes = [vp] * 10 + [sz, i, i, i, i, f, i, i, vp]
+    lib.fa2_bwd_window.restype = i
     lib.fa2_bwd_workspace_size.argtypes = [i, i, i, i]
     lib.fa2_bwd_workspace_size.restype = sz
     lib.fa2_bwd.argtypes = [vp] * 10 + [sz, i, i, i, i, f, i, i, vp]
@@ -103,6 +108,26 @@ def fa2_fwd(q, k, v, o, lse, scale: float, causal: bool, stream=None) -> int:
     B, H, N, d = q.shape
     return load().fa2_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d,
                           float(scale), int(bool(causal)), _dtype_code(q), _stream(stream))
+
+
+def fa2_fwd_window(q, k, v, o, lse, scale: float, window: int, stream=None) -> int:
+    """Raw call of the sliding-window forward (causal, ``window`` most recent keys)."""
+    _check_layout(q, k, v, o, lse)
+    B, H, N, d = q.shape
+    return load().fa2_fwd_window(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d,
+                                 float(scale), int(window), _dtype_code(q), _stream(stream))
+
+
+def fa2_bwd_window(q, k, v, o, do, lse, dq, dk, dv, workspace, scale: float, window: int,
+                   stream=None) -> int:
+    """Raw call of the sliding-window backward."""
+    _check_layout(q, k, v, o, do, lse, dq, dk, dv)
+    B, H, N, d = q.shape
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    return load().fa2_bwd_window(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse),
+                                 _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace), ws_bytes, B, H,
+                                 N, d, float(scale), int(window), _dtype_code(q),
+                                 _stream(stream))
 
 
 def fa2_bwd_workspace_size(B: int, H: int, N: int, d: int) -> int:
@@ -159,6 +184,29 @@ def forward(q, k, v, scale: float, causal: bool, stream=None):
     if rc != FA2_OK:
         raise FA2Error(rc, "fa2_fwd")
     return o, lse
+
+
+def forward_window(q, k, v, scale: float, window: int, stream=None):
+    """Allocating wrapper of fa2_fwd_window."""
+    B, H, N, d = q.shape
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    rc = fa2_fwd_window(q, k, v, o, lse, scale, window, stream)
+    if rc != FA2_OK:
+        raise FA2Error(rc, "fa2_fwd_window")
+    return o, lse
+
+
+def backward_window(q, k, v, o, do, lse, scale: float, window: int, stream=None):
+    """Allocating wrapper of fa2_bwd_window."""
+    B, H, N, d = q.shape
+    workspace = torch.empty(fa2_bwd_workspace_size(B, H, N, d), dtype=torch.uint8,
+                            device=q.device)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    rc = fa2_bwd_window(q, k, v, o, do, lse, dq, dk, dv, workspace, scale, window, stream)
+    if rc != FA2_OK:
+        raise FA2Error(rc, "fa2_bwd_window")
+    return dq, dk, dv
 
 
 def backward(q, k, v, o, do, lse, scale: float, causal: bool, workspace=None, stream=None):

@@ -79,6 +79,19 @@ int fa2_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, in
             int N, int d, float scale, int causal, int dtype, fa2_stream_t stream);
 
 /*
+ * Forward pass with a sliding window (local causal attention): query row i sees
+ * keys max(0, i - window + 1) .. i, its ``window`` most recent keys.  Source:
+ * [QL] "Modelli con attenzione a finestra scorrevole non standard" (models with
+ * sliding-window attention, e.g. alternating local and global layers).
+ *
+ *   window : >= 1 (FA2_ERR_INVALID_ARG otherwise); window >= N is plain causal
+ * Other arguments, layouts and errors as for fa2_fwd (causal is implied).  Key
+ * tiles entirely outside a query tile's window are skipped, not masked.
+ */
+int fa2_fwd_window(const void* Q, const void* K, const void* V, void* O, float* LSE, int B,
+                   int H, int N, int d, float scale, int window, int dtype, fa2_stream_t stream);
+
+/*
  * Bytes of device workspace fa2_bwd needs for these sizes (the per-row
  * D = rowsum(dO * O) and a float32 dQ accumulator), a multiple of 256.
  * Returns 0 for sizes fa2_bwd would reject.
@@ -103,6 +116,16 @@ int fa2_bwd(const void* Q, const void* K, const void* V, const void* O, const vo
             const float* LSE, void* dQ, void* dK, void* dV, void* workspace,
             size_t workspace_bytes, int B, int H, int N, int d, float scale, int causal,
             int dtype, fa2_stream_t stream);
+
+/*
+ * Backward of fa2_fwd_window: same window reading as the forward; arguments,
+ * workspace and errors as for fa2_bwd (causal implied).  O and LSE must come
+ * from fa2_fwd_window with the same window.
+ */
+int fa2_bwd_window(const void* Q, const void* K, const void* V, const void* O, const void* dO,
+                   const float* LSE, void* dQ, void* dK, void* dV, void* workspace,
+                   size_t workspace_bytes, int B, int H, int N, int d, float scale, int window,
+                   int dtype, fa2_stream_t stream);
 
 /*
  * Allocation-free backward.  The paper has no counterpart: this entry point

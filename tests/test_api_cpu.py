@@ -114,3 +114,13 @@ def test_binding_fails_loudly_when_library_missing(monkeypatch, tmp_path):
     monkeypatch.setattr(fa2, "LIB_PATH", str(tmp_path / "libfa2.so"))
     with pytest.raises(RuntimeError, match="missing"):
         fa2.load()
+
+
+def test_window_validation_without_device(lib):
+    args = (P, 2 * P, 3 * P, 4 * P, 5 * P, 1, 1, 64, 64, 0.1)
+    assert lib.fa2_fwd_window(*args, 0, 1, None) == fa2.FA2_ERR_INVALID_ARG
+    assert lib.fa2_fwd_window(*args, -5, 1, None) == fa2.FA2_ERR_INVALID_ARG
+    assert lib.fa2_fwd_window(*args[:8], 96, 0.1, 8, 1, None) == fa2.FA2_ERR_UNSUPPORTED
+    ptrs = [P * (i + 1) for i in range(9)]
+    ws = fa2.fa2_bwd_workspace_size(1, 1, 64, 64)
+    assert lib.fa2_bwd_window(*ptrs, 16 * P, ws, 1, 1, 64, 64, 0.1, 0, 1, None) == fa2.FA2_ERR_INVALID_ARG
