@@ -208,13 +208,23 @@ class Step:
                                   dtype=torch.uint8, device=dev)
 
     def fwd(self, stream):
-        _check(self.fa2, self.fa2.fa2_fwd(self.q, self.k, self.v, self.o, self.lse, self.w.scale,
-                                          self.w.causal, stream), "fa2_fwd")
+        if self.w.window:
+            rc = self.fa2.fa2_fwd_window(self.q, self.k, self.v, self.o, self.lse, self.w.scale,
+                                         self.w.window, stream)
+        else:
+            rc = self.fa2.fa2_fwd(self.q, self.k, self.v, self.o, self.lse, self.w.scale,
+                                  self.w.causal, stream)
+        _check(self.fa2, rc, "fa2_fwd")
 
     def bwd(self, stream):
-        _check(self.fa2, self.fa2.fa2_bwd(self.q, self.k, self.v, self.o, self.do, self.lse,
-                                          self.dq, self.dk, self.dv, self.ws, self.w.scale,
-                                          self.w.causal, stream), "fa2_bwd")
+        if self.w.window:
+            rc = self.fa2.fa2_bwd_window(self.q, self.k, self.v, self.o, self.do, self.lse,
+                                         self.dq, self.dk, self.dv, self.ws, self.w.scale,
+                                         self.w.window, stream)
+        else:
+            rc = self.fa2.fa2_bwd(self.q, self.k, self.v, self.o, self.do, self.lse, self.dq,
+                                  self.dk, self.dv, self.ws, self.w.scale, self.w.causal, stream)
+        _check(self.fa2, rc, "fa2_bwd")
 
     def results(self):
         return (self.dq, self.dk, self.dv) if self.w.backward else (self.o, self.lse)
@@ -294,10 +304,11 @@ def cpu_baseline(w, budget_s: float = 12.0) -> dict:
     x = workload_inputs(w, B=1, H=1)
     per_head = w.fwd_flops / (w.B * w.H) + (w.bwd_flops / (w.B * w.H) if w.backward else 0.0)
     done, t0 = 0, time.perf_counter()
+    win = w.window or None
     while True:
-        oracle.attn_fwd_ref(x["q"], x["k"], x["v"], w.scale, w.causal)
+        oracle.attn_fwd_ref(x["q"], x["k"], x["v"], w.scale, w.causal, window=win)
         if w.backward:
-            oracle.attn_bwd_ref(x["q"], x["k"], x["v"], x["do"], w.scale, w.causal)
+            oracle.attn_bwd_ref(x["q"], x["k"], x["v"], x["do"], w.scale, w.causal, window=win)
         done += 1
         el = time.perf_counter() - t0
         if el >= budget_s or done >= w.B * w.H:
@@ -369,7 +380,7 @@ def run_ours(args):
     }
     if not args.no_extras and rank == 0:
         extras = {}
-        for name in (HEADLINE_WORKLOAD, WORKLOAD_ORDER[3], WORKLOAD_ORDER[4]):
+        for name in (HEADLINE_WORKLOAD, WORKLOAD_ORDER[3], WORKLOAD_ORDER[4], WORKLOAD_ORDER[5]):
             ww = WORKLOADS[name]
             it = 10 if ww.N >= 16384 else 20
             _, f_ms, b_ms, _ = time_workload(fa2, ww, it, 3, dev, stream, None)
@@ -415,10 +426,12 @@ def run_reference(args):
     x = workload_inputs(w, B=1, H=1)
     per_head = step_flops(w) / (w.B * w.H)
 
+    win = w.window or None
+
     def one():
-        oracle.attn_fwd_ref(x["q"], x["k"], x["v"], w.scale, w.causal)
+        oracle.attn_fwd_ref(x["q"], x["k"], x["v"], w.scale, w.causal, window=win)
         if w.backward:
-            oracle.attn_bwd_ref(x["q"], x["k"], x["v"], x["do"], w.scale, w.causal)
+            oracle.attn_bwd_ref(x["q"], x["k"], x["v"], x["do"], w.scale, w.causal, window=win)
 
     for _ in range(args.warmup):
         one()

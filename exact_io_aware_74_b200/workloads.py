@@ -45,6 +45,7 @@ class Workload:
     input_scale: float = 1.0
     outlier_frac: float = 0.0
     outlier_mult: float = 8.0
+    window: int = 0  # sliding window (causal only): row i sees its `window` most recent keys
     note: str = field(default="", compare=False)
 
     @property
@@ -53,7 +54,15 @@ class Workload:
 
     @property
     def fwd_flops(self) -> float:
-        """Algorithmic forward FLOPs: two N x N x d products, halved when causal."""
+        """Algorithmic forward FLOPs: two N x N x d products, halved when causal.
+
+        With a sliding window W the products cover the sum over rows of the keys
+        each row sees, min(i + 1, W), instead of N^2 / 2.
+        """
+        if self.window:
+            w, n = min(self.window, self.N), self.N
+            pairs = w * (w + 1) / 2.0 + (n - w) * w
+            return 4.0 * self.B * self.H * self.d * pairs
         f = 4.0 * self.B * self.H * self.N * self.N * self.d
         return f / 2.0 if self.causal else f
 
@@ -80,6 +89,12 @@ WORKLOADS = {
         "fwd_bf16_b1h32_n32768_d128_causal_outliers", 1, 32, 32768, 128, "bf16", True, 4,
         outlier_frac=0.01, outlier_mult=8.0,
         note="long-context causal forward, 1% of key rows x8 per head"),
+    # Not one of the five headline workloads: the sliding-window row, measured on
+    # the training shape with a 1024-key window.
+    "fwdbwd_bf16_b8h16_n4096_d128_window1024": Workload(
+        "fwdbwd_bf16_b8h16_n4096_d128_window1024", 8, 16, 4096, 128, "bf16", True, 5,
+        backward=True, input_scale=0.5, window=1024,
+        note="training shape with a sliding window of 1024 keys"),
 }
 
 WORKLOAD_ORDER = list(WORKLOADS)

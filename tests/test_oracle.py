@@ -463,3 +463,13 @@ def test_exp2_poly3_relative_error_bound():
     rel = np.abs(got / np.exp2(x.astype(np.float32).astype(np.float64)) - 1.0)
     assert rel.max() < 1e-4  # fitted bound 7.5e-5, below the fp16 half-ulp 2.4e-4
     assert 0 < _exp2_poly3_f32(np.array([-np.inf]))[0] < 1e-37  # clamped, not NaN
+
+
+def test_window_flop_count():
+    """Algorithmic FLOPs of a windowed workload: sum over rows of min(i+1, W) keys."""
+    from exact_io_aware_74_b200.workloads import Workload
+    w = Workload("x", 1, 1, 10, 4, "bf16", True, 0, window=3)
+    pairs = sum(min(i + 1, 3) for i in range(10))
+    assert w.fwd_flops == 4 * 4 * pairs
+    full = Workload("y", 1, 1, 10, 4, "bf16", True, 0, window=10)
+    assert full.fwd_flops == Workload("z", 1, 1, 10, 4, "bf16", True, 0).fwd_flops + 4 * 4 * 5

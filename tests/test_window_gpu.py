@@ -87,3 +87,27 @@ def test_window_rejects_bad_window():
     ws = torch.empty(fa2.fa2_bwd_workspace_size(1, 1, 64, 64), dtype=torch.uint8, device="cuda")
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     assert fa2.fa2_bwd_window(q, k, v, o, do, lse, dq, dk, dv, ws, 0.1, -3) == fa2.FA2_ERR_INVALID_ARG
+
+
+@pytest.mark.slow
+def test_window_workload_full_size_sampled():
+    """The measured sliding-window workload at full size: sampled forward rows and
+    one whole head of the backward against the oracle."""
+    from exact_io_aware_74_b200.workloads import WORKLOADS, workload_inputs
+    w = WORKLOADS["fwdbwd_bf16_b8h16_n4096_d128_window1024"]
+    x = workload_inputs(w)
+    q, k, v, do = (x[n].cuda() for n in ("q", "k", "v", "do"))
+    o, lse = fa2.forward_window(q, k, v, w.scale, w.window)
+    dq, dk, dv = fa2.backward_window(q, k, v, o, do, lse, w.scale, w.window)
+    assert fa2.fa2_get_device_status() == (fa2.FA2_OK, 0)
+    rows = [0, 1, 1023, 1024, 1025, 2047, 3000, 4095]
+    bh = w.B * w.H - 1
+    ro, rl = oracle.attn_fwd_rows_ref(x["q"], x["k"], x["v"], w.scale, True, bh, rows,
+                                      window=w.window)
+    b, h = divmod(bh, w.H)
+    assert np.max(np.abs(o[b, h, rows].cpu().double().numpy() - ro)) <= O_TOL["bf16"]
+    assert np.max(np.abs(lse[b, h, rows].cpu().double().numpy() - rl)) <= 1e-3
+    rq, rk, rv = oracle.attn_bwd_ref(x["q"], x["k"], x["v"], x["do"], w.scale, True,
+                                     heads=[bh], window=w.window)
+    for got, ref in ((dq, rq), (dk, rk), (dv, rv)):
+        _check_grad(got[b, h].cpu()[None, None], ref[b, h][None, None])
