@@ -314,6 +314,11 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       constexpr uint32_t id_dq = idesc_f16(128, D, BF16, true, true);      // dQ (A, B MN-major)
       const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aQ = smem_u32(sQ),
                      adO = smem_u32(sdO), aDS = smem_u32(sDS);
+      // Base descriptors; a K step or a ring stage only moves the start address.
+      const uint64_t kK = sdesc_sw128(aK, 16, 1024), kV = sdesc_sw128(aV, 16, 1024);
+      const uint64_t kQ = sdesc_sw128(aQ, 16, 1024), kdO = sdesc_sw128(adO, 16, 1024);
+      const uint64_t mQ = sdesc_sw128(aQ, C::CHUNK, 1024), mdO = sdesc_sw128(adO, C::CHUNK, 1024);
+      const uint64_t mK = sdesc_sw128(aK, C::CHUNK, 1024), mDS = sdesc_sw128(aDS, C::CHUNK, 1024);
       bool ok = mbar_wait(&bar_kv, 0, wc, kBSiteMmaKV);
       for (int it = 0; it < n_it && ok; ++it) {
         const int st = it % C::ST;
@@ -323,8 +328,8 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * C::CHUNK + (kk & 3) * 32;
-          umma_ss(tbase + C::C_S, sdesc_sw128(aK + off, 16, 1024),
-                  sdesc_sw128(aQ + st * C::TILE + off, 16, 1024), id_kk, kk > 0);
+          umma_ss(tbase + C::C_S, sdesc_add(kK, off), sdesc_add(kQ, st * C::TILE + off), id_kk,
+                  kk > 0);
         }
         umma_commit(&s_full);
         // dP^T = V dO^T (its columns hold the previous dQ partial when D = 128)
@@ -335,8 +340,8 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * C::CHUNK + (kk & 3) * 32;
-          umma_ss(tbase + C::C_DP, sdesc_sw128(aV + off, 16, 1024),
-                  sdesc_sw128(adO + st * C::TILE + off, 16, 1024), id_kk, kk > 0);
+          umma_ss(tbase + C::C_DP, sdesc_add(kV, off), sdesc_add(kdO, st * C::TILE + off), id_kk,
+                  kk > 0);
         }
         umma_commit(&dp_full);
         // dV += P^T dO
@@ -345,7 +350,7 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)  // queries 16 kk .. 16 kk + 15: warpgroup kk / 4
           umma_ts(tbase + C::C_DV, tbase + C::C_P(kk >> 2) + (kk & 3) * 8,
-                  sdesc_sw128(adO + st * C::TILE + kk * 2048, C::CHUNK, 1024), id_tb,
+                  sdesc_add(mdO, st * C::TILE + kk * 2048), id_tb,
                   (it > 0 || kk > 0) ? 1u : 0u);
         // dQ_i = dS K first (the drain needs only this one; its own TMEM columns when
         // D = 64: wait for the previous drain), then dK += dS^T Q (A from TMEM, so
@@ -358,13 +363,13 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         }
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          umma_ss(tbase + C::C_DQ, sdesc_sw128(aDS + kk * 2048, C::CHUNK, 1024),
-                  sdesc_sw128(aK + kk * 2048, C::CHUNK, 1024), id_dq, kk > 0);
+          umma_ss(tbase + C::C_DQ, sdesc_add(mDS, kk * 2048), sdesc_add(mK, kk * 2048), id_dq,
+                  kk > 0);
         umma_commit(&dq_full);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
           umma_ts(tbase + C::C_DK, tbase + C::C_DS(kk >> 2) + (kk & 3) * 8,
-                  sdesc_sw128(aQ + st * C::TILE + kk * 2048, C::CHUNK, 1024), id_tb,
+                  sdesc_add(mQ, st * C::TILE + kk * 2048), id_tb,
                   (it > 0 || kk > 0) ? 1u : 0u);
         umma_commit(&qdo_empty[st]);
       }

@@ -23,10 +23,11 @@
 //   warp  9    MMA issuer (tcgen05, one thread)
 //   warps 10-11 idle (they complete the third warpgroup)
 // The kernel is compiled for 168 registers per thread (384 x 168 = 64512); the
-// third warpgroup gives registers back (down to 40) and the two softmax
-// warpgroups take them (up to 232): 2 x 128 x 232 + 128 x 40 = 64512, so the
-// re-split never asks for more than the launch holds.  The host refuses to
-// launch a build whose register count is not 168.
+// third warpgroup gives registers back (down to 56) and the two softmax
+// warpgroups take them (up to 224): 2 x 128 x 224 + 128 x 56 = 64512, so the
+// re-split never asks for more than the launch holds.  (232 / 40 made the MMA
+// issuer spill and measured slower.)  The host refuses to launch a build whose
+// register count is not 168.
 // TMEM (512 columns x 128 lanes, fp32): S_t at column 128 t, O_t at 256 + D t.
 // P_t (16-bit) overwrites the first 64 columns of S_t and feeds the P V MMA
 // straight from TMEM.  The MMA warp alternates between the two query tiles so
@@ -63,8 +64,11 @@ struct FwdCfg {
   static constexpr int SMEM = (QT + KS + VS) * TILE + 1024;
   static constexpr int THREADS = 384;
   static constexpr int LAUNCH_REGS = 168;  // per thread, as compiled (checked on the host)
-  static constexpr int SOFT_REGS = 232;
-  static constexpr int OTHER_REGS = 40;
+#ifndef FA2_FWD_SOFT_REGS
+#define FA2_FWD_SOFT_REGS 224
+#endif
+  static constexpr int SOFT_REGS = FA2_FWD_SOFT_REGS;
+  static constexpr int OTHER_REGS = (THREADS * LAUNCH_REGS - 2 * 128 * SOFT_REGS) / 128 / 8 * 8;
   static_assert(2 * 128 * SOFT_REGS + 128 * OTHER_REGS <= THREADS * LAUNCH_REGS,
                 "register re-split exceeds the launch allocation");
   static constexpr uint32_t S_COL0 = 0, S_COL1 = 128;
@@ -239,16 +243,20 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                   (acc || kk > 0) ? 1u : 0u);
         }
       };
+      const int lo0 = j_lo[0], hi0 = j_hi[0], lo1 = j_lo[1], hi1 = j_hi[1];
 
       bool ok = mbar_wait(&bar_q, 0, wc, kSiteMmaQ) && mbar_wait(&k_full[0], 0, wc, kSiteMmaK);
       if (ok) {
         tc_fence_after();
         // Tiles whose key range starts at j0 get their first S now.
-        for (int t = 0; t < 2; ++t)
-          if (j_hi[t] > j_lo[t] && j_lo[t] == j0) {
-            issue_qk(t, 0);
-            umma_commit(&s_full[t]);
-          }
+        if (hi0 > lo0 && lo0 == j0) {
+          issue_qk(0, 0);
+          umma_commit(&s_full[0]);
+        }
+        if (hi1 > lo1 && lo1 == j0) {
+          issue_qk(1, 0);
+          umma_commit(&s_full[1]);
+        }
         umma_commit(&k_empty[0]);
       }
       for (int jj = 0; jj < n_steps && ok; ++jj) {
@@ -258,9 +266,7 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         const bool has_next = jj + 1 < n_steps;
         bool k_next_ready = false;
         if (!mbar_wait(&v_full[vs], (jj / C::VS) & 1, wc, kSiteMmaV)) { ok = false; break; }
-        auto tile_step = [&](int t) -> bool {
-          const int lo = t ? j_lo[1] : j_lo[0];
-          const int hi = t ? j_hi[1] : j_hi[0];
+        auto tile_step = [&](int t, int lo, int hi) -> bool {
           if (j >= lo && j < hi) {
             const int step = j - lo;  // this tile's own step count
             if (!mbar_wait(&p_ready[t], step & 1, wc, kSiteMmaP)) return false;
@@ -281,7 +287,7 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           }
           return true;
         };
-        ok = tile_step(0) && tile_step(1);
+        ok = tile_step(0, lo0, hi0) && tile_step(1, lo1, hi1);
         if (ok && has_next && !k_next_ready)  // a slot is only released once its load landed
           ok = mbar_wait(&k_full[ks1], ((jj + 1) / C::KS) & 1, wc, kSiteMmaK);
         if (!ok) break;

@@ -355,6 +355,13 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t smem_addr, uint32_t lbo
   return d;
 }
 
+// The same descriptor for an operand ``byte_off`` bytes further on (16-byte
+// multiple).  Shared-memory addresses stay below 2^18, so the 14-bit start
+// address field cannot carry into the next field.
+__device__ __forceinline__ uint64_t sdesc_add(uint64_t desc, uint32_t byte_off) {
+  return desc + static_cast<uint64_t>(byte_off >> 4);
+}
+
 // Instruction descriptor, kind::f16 with fp32 accumulator.
 //   bits 4..5 D format (1 = f32), 7..9 A format, 10..12 B format (0 f16, 1 bf16),
 //   bit 15 A MN-major, bit 16 B MN-major, 17..22 N >> 3, 24..28 M >> 4.
