@@ -45,6 +45,7 @@ closed forms, invariances and central finite differences.
 """
 
 from .attention import (  # noqa: F401
+    attn_fwd_decode_ref,
     attn_fwd_ref,
     attn_fwd_rows_ref,
     attn_bwd_ref,

@@ -182,3 +182,34 @@ def attn_bwd_ref(q, k, v, do, scale: float, causal: bool,
         dk[b, h] = dk_bh
         dv[b, h] = dv_bh
     return dq, dk, dv
+
+
+def attn_fwd_decode_ref(q, k, v, scale: float, causal: bool) -> tuple[np.ndarray, np.ndarray]:
+    """Attention of Nq queries against Nk keys (Nq <= Nk): the decode-like case.
+
+    q is [B,H,Nq,d]; k, v are [B,H,Nk,d].  The queries are the last Nq positions
+    of the sequence, so with ``causal`` query i sees keys 0 .. Nk - Nq + i
+    (bottom-right alignment); without it every key.  This is the inference
+    setting of "Flash Attention spiegata: una guida completa", section
+    "Parallelismo lungo la lunghezza della sequenza" (small batches, long
+    prompts).  Returns (O [B,H,Nq,d], LSE [B,H,Nq]) in fp64.
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    if q.ndim != 4 or k.ndim != 4 or v.shape != k.shape or q.shape[:2] != k.shape[:2] \
+            or q.shape[3] != k.shape[3] or q.shape[2] > k.shape[2]:
+        raise ValueError("q [B,H,Nq,d] and k, v [B,H,Nk,d] with Nq <= Nk")
+    B, H, Nq, d = q.shape
+    Nk = k.shape[2]
+    out = np.empty((B, H, Nq, d))
+    lse = np.empty((B, H, Nq))
+    rows = (Nk - Nq) + np.arange(Nq)[:, None]
+    cols = np.arange(Nk)[None, :]
+    for b in range(B):
+        for h in range(H):
+            s = scale * (q[b, h] @ k[b, h].T)
+            if causal:
+                s = np.where(cols > rows, -np.inf, s)
+            p, l = _softmax_rows(s)
+            out[b, h] = p @ v[b, h]
+            lse[b, h] = l
+    return out, lse

@@ -287,6 +287,42 @@ def test_window_finite_differences():
 
 
 # ----------------------------------------------------------------------------------
+# decode-like attention: Nq queries (the last positions) against Nk keys
+# ----------------------------------------------------------------------------------
+
+def test_decode_is_the_tail_of_full_causal_attention():
+    """Decoding q after a prefix equals the last Nq rows of causal attention over
+    [prefix; q] (both sides of the check use their own code paths)."""
+    B, H, Nk, d = 2, 2, 45, 16
+    for Nq in (1, 3, 45):
+        k, v = _rand((B, H, Nk, d), 300 + Nq), _rand((B, H, Nk, d), 301 + Nq)
+        qfull = _rand((B, H, Nk, d), 302 + Nq)
+        q = qfull[:, :, Nk - Nq:]
+        o, lse = oracle.attn_fwd_decode_ref(q, k, v, 0.3, True)
+        fo, fl = oracle.attn_fwd_ref(qfull, k, v, 0.3, True)
+        _close(o, fo[:, :, Nk - Nq:])
+        _close(lse, fl[:, :, Nk - Nq:])
+        # without the mask it is plain attention of those rows
+        o2, l2 = oracle.attn_fwd_decode_ref(q, k, v, 0.3, False)
+        fo2, fl2 = oracle.attn_fwd_ref(qfull, k, v, 0.3, False)
+        _close(o2, fo2[:, :, Nk - Nq:])
+        _close(l2, fl2[:, :, Nk - Nq:])
+
+
+def test_decode_matches_torch_with_mask():
+    B, H, Nq, Nk, d = 1, 3, 5, 70, 32
+    q, k, v = _rand((B, H, Nq, d), 310), _rand((B, H, Nk, d), 311), _rand((B, H, Nk, d), 312)
+    allowed = torch.arange(Nk)[None, :] <= (Nk - Nq + torch.arange(Nq)[:, None])
+    to = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q), torch.from_numpy(k), torch.from_numpy(v), attn_mask=allowed,
+        scale=0.2)
+    o, _ = oracle.attn_fwd_decode_ref(q, k, v, 0.2, True)
+    _close(o, to.numpy())
+    with pytest.raises(ValueError):
+        oracle.attn_fwd_decode_ref(k, q, q, 0.2, True)  # Nq > Nk
+
+
+# ----------------------------------------------------------------------------------
 # planted mistakes (in copies of the oracle, on the CPU) must fail some pin
 # ----------------------------------------------------------------------------------
 
