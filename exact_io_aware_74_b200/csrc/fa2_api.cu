@@ -12,6 +12,7 @@
 
 #include "../../include/fa2.h"
 #include "fa2_bwd.cuh"
+#include "fa2_decode.cuh"
 #include "fa2_fwd.cuh"
 
 namespace {
@@ -151,7 +152,7 @@ unsigned long long wait_ns() { return static_cast<unsigned long long>(g_wait_ms.
 
 template <int D, bool BF16, bool CAUSAL>
 int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-               const fa2::FwdParams& p, cudaStream_t stream) {
+               const fa2::FwdParams& p, int n_split, cudaStream_t stream) {
   using Cfg = fa2::FwdCfg<D>;
   auto kern = fa2::fa2_fwd_kernel<D, BF16, CAUSAL>;
   // The kernel re-splits its registers between warpgroups; that is only sound
@@ -169,8 +170,20 @@ int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& 
     cudaGetLastError();
     return FA2_ERR_CUDA;
   }
-  const unsigned int grid = static_cast<unsigned int>(p.n_qblk) * static_cast<unsigned int>(p.BH);
+  const dim3 grid(static_cast<unsigned int>(p.n_qblk) * static_cast<unsigned int>(p.BH),
+                  static_cast<unsigned int>(n_split));
   kern<<<grid, Cfg::THREADS, Cfg::SMEM, stream>>>(mq, mk, mv, p);
+  if (cudaGetLastError() != cudaSuccess) return FA2_ERR_CUDA;
+  g_launches.fetch_add(1);
+  return FA2_OK;
+}
+
+template <int D, bool BF16>
+int launch_combine(const float* O_part, const float* LSE_part, void* O, float* LSE,
+                   long long rows, int n_split, cudaStream_t stream) {
+  const unsigned int grid = static_cast<unsigned int>((rows + 7) / 8);
+  fa2::fa2_decode_combine_kernel<D, BF16><<<grid, 256, 0, stream>>>(O_part, LSE_part, O, LSE, rows,
+                                                                  n_split);
   if (cudaGetLastError() != cudaSuccess) return FA2_ERR_CUDA;
   g_launches.fetch_add(1);
   return FA2_OK;
@@ -178,11 +191,60 @@ int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& 
 
 }  // namespace
 
-extern "C" {
-
-}  // extern "C"
-
 namespace {
+
+// Shared by every forward entry point.  Query rows [BH][Nq], key rows [BH][Nk];
+// off = Nk - Nq aligns the causal mask to the bottom right; window = 0 means no
+// sliding window.  n_split = 1: O and LSE are written directly; otherwise the key
+// tiles are cut into n_split stretches of kv_per_split, the partials go to
+// O_part / LSE_part and a second kernel merges them into O and LSE.
+int fwd_core(const void* Q, const void* K, const void* V, void* O, float* LSE, int BH, int Nq,
+             int Nk, int d, float scale, int causal, int window, int dtype, int n_split,
+             int kv_per_split, float* O_part, float* LSE_part, fa2_stream_t stream) {
+  int dev = 0;
+  int rc = check_device(&dev);
+  if (rc != FA2_OK) return rc;
+  unsigned int* st = status_word(dev);
+  if (!st) return FA2_ERR_CUDA;
+
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, Q, BH, Nq, d, dtype) || !make_map(&mk, K, BH, Nk, d, dtype) ||
+      !make_map(&mv, V, BH, Nk, d, dtype))
+    return FA2_ERR_CUDA;
+
+  fa2::FwdParams p{};
+  p.O = O;
+  p.LSE = LSE;
+  p.Nq = Nq;
+  p.Nk = Nk;
+  p.off = Nk - Nq;
+  p.BH = BH;
+  p.n_qblk = (Nq + 255) / 256;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.status = st;
+  p.wait_ns = wait_ns();
+  p.fault = g_fault.load();
+  p.window = window;
+  p.kv_per_split = n_split > 1 ? kv_per_split : 0;
+  p.O_part = O_part;
+  p.LSE_part = LSE_part;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const bool bf = dtype == FA2_BF16;
+  if (d == 64) {
+    if (bf) rc = causal ? launch_fwd<64, true, true>(mq, mk, mv, p, n_split, s) : launch_fwd<64, true, false>(mq, mk, mv, p, n_split, s);
+    else rc = causal ? launch_fwd<64, false, true>(mq, mk, mv, p, n_split, s) : launch_fwd<64, false, false>(mq, mk, mv, p, n_split, s);
+  } else {
+    if (bf) rc = causal ? launch_fwd<128, true, true>(mq, mk, mv, p, n_split, s) : launch_fwd<128, true, false>(mq, mk, mv, p, n_split, s);
+    else rc = causal ? launch_fwd<128, false, true>(mq, mk, mv, p, n_split, s) : launch_fwd<128, false, false>(mq, mk, mv, p, n_split, s);
+  }
+  if (rc != FA2_OK || n_split == 1) return rc;
+  const long long rows = static_cast<long long>(BH) * Nq;
+  if (d == 64)
+    return bf ? launch_combine<64, true>(O_part, LSE_part, O, LSE, rows, n_split, s)
+              : launch_combine<64, false>(O_part, LSE_part, O, LSE, rows, n_split, s);
+  return bf ? launch_combine<128, true>(O_part, LSE_part, O, LSE, rows, n_split, s)
+            : launch_combine<128, false>(O_part, LSE_part, O, LSE, rows, n_split, s);
+}
 
 // Shared by fa2_fwd and fa2_fwd_window; window = 0 means no sliding window.
 int fwd_impl(const void* Q, const void* K, const void* V, void* O, float* LSE, int B, int H,
@@ -200,36 +262,24 @@ int fwd_impl(const void* Q, const void* K, const void* V, void* O, float* LSE, i
       overlaps(LSE, lse_bytes, Q, bytes) || overlaps(LSE, lse_bytes, K, bytes) ||
       overlaps(LSE, lse_bytes, V, bytes))
     return FA2_ERR_INVALID_ARG;
-  int dev = 0;
-  rc = check_device(&dev);
-  if (rc != FA2_OK) return rc;
-  unsigned int* st = status_word(dev);
-  if (!st) return FA2_ERR_CUDA;
+  return fwd_core(Q, K, V, O, LSE, BH, N, N, d, scale, causal, window, dtype, 1, 0, nullptr,
+                  nullptr, stream);
+}
 
-  CUtensorMap mq, mk, mv;
-  if (!make_map(&mq, Q, BH, N, d, dtype) || !make_map(&mk, K, BH, N, d, dtype) ||
-      !make_map(&mv, V, BH, N, d, dtype))
-    return FA2_ERR_CUDA;
+// Key tiles per split when the n_kv key tiles are cut into n_split stretches,
+// and the number of non-empty stretches that gives.
+int kv_tiles_per_split(int n_kv, int n_split) { return (n_kv + n_split - 1) / n_split; }
+int effective_splits(int n_kv, int n_split) {
+  const int per = kv_tiles_per_split(n_kv, n_split);
+  return (n_kv + per - 1) / per;
+}
 
-  fa2::FwdParams p{};
-  p.O = O;
-  p.LSE = LSE;
-  p.N = N;
-  p.BH = BH;
-  p.n_qblk = (N + 255) / 256;
-  p.scale_log2 = scale * 1.4426950408889634f;
-  p.status = st;
-  p.wait_ns = wait_ns();
-  p.fault = g_fault.load();
-  p.window = window;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  const bool bf = dtype == FA2_BF16;
-  if (d == 64) {
-    if (bf) return causal ? launch_fwd<64, true, true>(mq, mk, mv, p, s) : launch_fwd<64, true, false>(mq, mk, mv, p, s);
-    return causal ? launch_fwd<64, false, true>(mq, mk, mv, p, s) : launch_fwd<64, false, false>(mq, mk, mv, p, s);
-  }
-  if (bf) return causal ? launch_fwd<128, true, true>(mq, mk, mv, p, s) : launch_fwd<128, true, false>(mq, mk, mv, p, s);
-  return causal ? launch_fwd<128, false, true>(mq, mk, mv, p, s) : launch_fwd<128, false, false>(mq, mk, mv, p, s);
+constexpr int kMaxSplits = 1024;
+
+// Checks of fa2_fwd_decode's sizes that need no CUDA call.
+int check_decode_sizes(int B, int H, int Nq, int Nk, int d, float scale, int causal, int dtype) {
+  if (Nq < 1 || Nk < Nq) return FA2_ERR_INVALID_ARG;
+  return check_sizes(B, H, Nk, d, scale, causal, dtype);
 }
 
 }  // namespace
@@ -247,6 +297,89 @@ int fa2_fwd_window(const void* Q, const void* K, const void* V, void* O, float* 
   // A window as long as the sequence is plain causal attention.
   return fwd_impl(Q, K, V, O, LSE, B, H, N, d, scale, 1, window >= N ? 0 : window, dtype,
                   stream);
+}
+
+int fa2_fwd_decode_splits(int B, int H, int Nq, int Nk, int d, int sm_count) {
+  if (check_decode_sizes(B, H, Nq, Nk, d, 1.0f, 0, FA2_BF16) != FA2_OK) return 0;
+  if (sm_count <= 0) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sm_count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        sm_count <= 0) {
+      cudaGetLastError();
+      return 0;
+    }
+  }
+  // One forward CTA runs per SM.  A CTA costs its key tiles plus about three
+  // tiles' worth of set-up, pipeline fill and partial-result traffic; the time
+  // is that cost times the number of waves.  Take the cheapest split, the
+  // smallest one on ties.
+  const long long ctas = static_cast<long long>((Nq + 255) / 256) * B * H;
+  const int n_kv = (Nk + 127) / 128;
+  const int max_split = n_kv < kMaxSplits ? n_kv : kMaxSplits;
+  int best = 1;
+  long long best_cost = -1;
+  for (int sp = 1; sp <= max_split; ++sp) {
+    const int eff = effective_splits(n_kv, sp);
+    if (eff != sp) continue;  // same stretches as a smaller split count
+    const long long waves = (ctas * sp + sm_count - 1) / sm_count;
+    const long long cost = waves * (kv_tiles_per_split(n_kv, sp) + 3);
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best = sp;
+    }
+  }
+  return best;
+}
+
+size_t fa2_fwd_decode_workspace_size(int B, int H, int Nq, int Nk, int d, int n_splits) {
+  if (check_decode_sizes(B, H, Nq, Nk, d, 1.0f, 0, FA2_BF16) != FA2_OK) return 0;
+  if (n_splits < 1 || n_splits > kMaxSplits) return 0;
+  const int eff = effective_splits((Nk + 127) / 128, n_splits);
+  if (eff == 1) return 0;
+  return fa2::decode_workspace_bytes(static_cast<size_t>(eff), static_cast<size_t>(B) * H,
+                                     static_cast<size_t>(Nq), d);
+}
+
+int fa2_fwd_decode(const void* Q, const void* K, const void* V, void* O, float* LSE, int B,
+                   int H, int Nq, int Nk, int d, float scale, int causal, int dtype, int n_splits,
+                   void* workspace, size_t workspace_bytes, fa2_stream_t stream) {
+  if (!Q || !K || !V || !O || !LSE) return FA2_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(LSE))
+    return FA2_ERR_INVALID_ARG;
+  int rc = check_decode_sizes(B, H, Nq, Nk, d, scale, causal, dtype);
+  if (rc != FA2_OK) return rc;
+  if (n_splits < 1 || n_splits > kMaxSplits) return FA2_ERR_INVALID_ARG;
+  const int BH = B * H;
+  const size_t q_bytes = static_cast<size_t>(BH) * Nq * d * 2;
+  const size_t kv_bytes = static_cast<size_t>(BH) * Nk * d * 2;
+  const size_t lse_bytes = static_cast<size_t>(BH) * Nq * sizeof(float);
+  if (overlaps(O, q_bytes, Q, q_bytes) || overlaps(O, q_bytes, K, kv_bytes) ||
+      overlaps(O, q_bytes, V, kv_bytes) || overlaps(LSE, lse_bytes, O, q_bytes) ||
+      overlaps(LSE, lse_bytes, Q, q_bytes) || overlaps(LSE, lse_bytes, K, kv_bytes) ||
+      overlaps(LSE, lse_bytes, V, kv_bytes))
+    return FA2_ERR_INVALID_ARG;
+  const int n_kv = (Nk + 127) / 128;
+  const int eff = effective_splits(n_kv, n_splits);
+  float* O_part = nullptr;
+  float* LSE_part = nullptr;
+  if (eff > 1) {
+    const size_t need = fa2::decode_workspace_bytes(static_cast<size_t>(eff),
+                                                    static_cast<size_t>(BH), Nq, d);
+    if (!workspace || workspace_bytes < need ||
+        (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+      return FA2_ERR_WORKSPACE;
+    const void* bufs[5] = {Q, K, V, O, LSE};
+    const size_t buf_bytes[5] = {q_bytes, kv_bytes, kv_bytes, q_bytes, lse_bytes};
+    for (int i = 0; i < 5; ++i)
+      if (overlaps(workspace, need, bufs[i], buf_bytes[i])) return FA2_ERR_WORKSPACE;
+    O_part = static_cast<float*>(workspace);
+    LSE_part = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
+                                        fa2::decode_opart_bytes(static_cast<size_t>(eff),
+                                                                static_cast<size_t>(BH), Nq, d));
+  }
+  return fwd_core(Q, K, V, O, LSE, BH, Nq, Nk, d, scale, causal, 0, dtype, eff,
+                  kv_tiles_per_split(n_kv, n_splits), O_part, LSE_part, stream);
 }
 
 size_t fa2_bwd_workspace_size(int B, int H, int N, int d) {

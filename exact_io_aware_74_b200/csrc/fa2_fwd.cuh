@@ -39,16 +39,26 @@
 namespace fa2 {
 
 struct FwdParams {
-  void* O;                     // [BH][N][D] 16-bit
-  float* LSE;                  // [BH][N]
-  int N;                       // sequence length
+  void* O;                     // [BH][Nq][D] 16-bit (unused when the keys are split)
+  float* LSE;                  // [BH][Nq]            (unused when the keys are split)
+  int Nq;                      // query rows per (batch, head)
+  int Nk;                      // key / value rows per (batch, head)
+  int off;                     // causal only: query row i sees keys <= i + off (Nk - Nq)
   int BH;                      // batch * heads
-  int n_qblk;                  // ceil(N / 256)
+  int n_qblk;                  // ceil(Nq / 256)
   float scale_log2;            // scale * log2(e)
   unsigned int* status;        // device status word
   unsigned long long wait_ns;  // budget of one bounded wait
   int fault;                   // test hook: 1 = skip the first K load
-  int window;                  // causal only: row i sees keys i-window+1..i (0 = no window)
+  int window;                  // causal only: row i sees keys i+off-window+1..i+off (0 = none)
+  // Split keys (blockIdx.y = split): CTA y covers key tiles [y kv_per_split,
+  // (y + 1) kv_per_split) and writes its rows' partial results, normalised by
+  // its own row sums, to O_part [split][BH][Nq][D] and LSE_part [split][BH][Nq]
+  // (float, -inf for a row that sees no key of the split).  kv_per_split = 0:
+  // no split, O and LSE are written directly.
+  int kv_per_split;
+  float* O_part;
+  float* LSE_part;
 };
 
 template <int D>
@@ -109,31 +119,41 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int N = p.N;
+  const int Nq = p.Nq, Nk = p.Nk;
+  const int off = CAUSAL ? p.off : 0;
+  const bool split = p.kv_per_split > 0;
 
   // Heaviest query blocks first (they see the most keys when causal).
   const int qb = p.n_qblk - 1 - static_cast<int>(blockIdx.x) / p.BH;
   const int bh = static_cast<int>(blockIdx.x) % p.BH;
-  const int n_kv_all = (N + C::BN - 1) / C::BN;
+  const int n_kv_all = (Nk + C::BN - 1) / C::BN;
+  // Key tiles of this CTA's split (all of them when the keys are not split).
+  const int s_lo = split ? static_cast<int>(blockIdx.y) * p.kv_per_split : 0;
+  const int s_hi = split ? min(n_kv_all, s_lo + p.kv_per_split) : n_kv_all;
   // Key tiles [j_lo[t], j_hi[t]) are the ones query tile t needs: all of them,
-  // or (causal) up to its diagonal, and (sliding window) from the tile that holds
-  // the first key its first row still sees.  Tiles past N have an empty range.
+  // or (causal) up to the one holding the last key its last row sees, and
+  // (sliding window) from the tile that holds the first key its first row still
+  // sees; then cut to the split.  Tiles past Nq have an empty range.
   int row0[2], j_lo[2], j_hi[2];
 #pragma unroll
   for (int t = 0; t < 2; ++t) {
     row0[t] = qb * 256 + t * 128;
     j_lo[t] = 0;
-    if (row0[t] >= N) {
+    if (row0[t] >= Nq) {
       j_hi[t] = 0;
     } else if (CAUSAL) {
-      j_hi[t] = min(n_kv_all, row0[t] / C::BN + 1);
-      if (p.window > 0) j_lo[t] = max(0, row0[t] - p.window + 1) / C::BN;
+      j_hi[t] = min(n_kv_all, (min(row0[t] + C::BM - 1, Nq - 1) + off) / C::BN + 1);
+      if (p.window > 0) j_lo[t] = max(0, row0[t] + off - p.window + 1) / C::BN;
     } else {
       j_hi[t] = n_kv_all;
     }
+    j_lo[t] = max(j_lo[t], s_lo);
+    j_hi[t] = min(j_hi[t], s_hi);
+    if (j_hi[t] <= j_lo[t]) j_lo[t] = j_hi[t] = 0;  // nothing to do for this tile
   }
+  const bool has0 = j_hi[0] > 0, has1 = j_hi[1] > 0;
   // The CTA walks key tiles j0 .. j1-1; the K/V ring is indexed from j0.
-  const int j0 = (j_hi[1] > 0) ? min(j_lo[0], j_lo[1]) : j_lo[0];
+  const int j0 = has0 ? (has1 ? min(j_lo[0], j_lo[1]) : j_lo[0]) : j_lo[1];
   const int j1 = max(j_hi[0], j_hi[1]);
   const int n_steps = j1 - j0;
 
@@ -175,6 +195,7 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       const uint64_t keep = policy_evict_last();
       uint32_t q_bytes = 0;
       for (int t = 0; t < 2; ++t) q_bytes += (j_hi[t] > 0) ? C::TILE : 0;
+      // (A CTA whose split holds no key any of its rows sees loads nothing.)
       mbar_arrive_expect_tx(&bar_q, q_bytes);
       for (int t = 0; t < 2; ++t) {
         if (j_hi[t] == 0) continue;
@@ -245,7 +266,8 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       };
       const int lo0 = j_lo[0], hi0 = j_hi[0], lo1 = j_lo[1], hi1 = j_hi[1];
 
-      bool ok = mbar_wait(&bar_q, 0, wc, kSiteMmaQ) && mbar_wait(&k_full[0], 0, wc, kSiteMmaK);
+      bool ok = n_steps > 0 && mbar_wait(&bar_q, 0, wc, kSiteMmaQ) &&
+                mbar_wait(&k_full[0], 0, wc, kSiteMmaK);
       if (ok) {
         tc_fence_after();
         // Tiles whose key range starts at j0 get their first S now.
@@ -320,11 +342,19 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     float l = 0.f;        // running sum of exp2(s * sl2 - m)
     bool ok = my_nkv > 0;
     const int win = p.window;
+    // A warp whose 32 rows are all past Nq only keeps the barrier count: its P
+    // rows feed output rows that are never stored.
+    const bool live = my_row0 + wq * 32 < Nq;
     for (int step = 0; step < my_nkv && ok; ++step) {
       const int j = my_lo + step;  // key tile of this step
       // Warp-uniform wait: the TMEM loads and stores below are warp-collective.
       ok = __all_sync(0xffffffffu, mbar_wait(&s_full[t], step & 1, wc, kSiteSoftS));
       if (!ok) break;
+      if (!live) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_ready[t]);
+        continue;
+      }
       tc_fence_after();
       uint32_t sr[128];
 #pragma unroll
@@ -334,12 +364,13 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       tmem_wait_ld();
       reg_fence(sr);
       const int key0 = j * C::BN;
-      // Keys after the row (causal), past N, or before the row's window start.
-      const bool need_mask = (CAUSAL && key0 + C::BN - 1 > my_row0) || (key0 + C::BN > N) ||
-                             (CAUSAL && win > 0 && key0 < my_row0 + 127 - win + 1);
+      // Keys after the row's last one (causal), past Nk, or before the row's
+      // window start.
+      const bool need_mask = (CAUSAL && key0 + C::BN - 1 > my_row0 + off) || (key0 + C::BN > Nk) ||
+                             (CAUSAL && win > 0 && key0 < my_row0 + off + 127 - win + 1);
       if (need_mask) {
-        const int hi_lim = CAUSAL ? min(row - key0 + 1, N - key0) : (N - key0);
-        const int lo_lim = (CAUSAL && win > 0) ? row - win + 1 - key0 : 0;
+        const int hi_lim = CAUSAL ? min(row + off - key0 + 1, Nk - key0) : (Nk - key0);
+        const int lo_lim = (CAUSAL && win > 0) ? row + off - win + 1 - key0 : 0;
 #pragma unroll
         for (int i = 0; i < 128; ++i)
           if (i >= hi_lim || i < lo_lim) sr[i] = __float_as_uint(-INFINITY);
@@ -426,32 +457,59 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_ready[t]);
     }
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&o_done[t], (my_nkv - 1) & 1, wc, kSiteSoftOEnd));
-    if (ok) {
+    if (ok && live)
+      ok = __all_sync(0xffffffffu, mbar_wait(&o_done[t], (my_nkv - 1) & 1, wc, kSiteSoftOEnd));
+    if (ok && live) {
       tc_fence_after();
-      const float inv_l = 1.0f / l;
-      uint8_t* orow = reinterpret_cast<uint8_t*>(p.O) +
-                      (static_cast<size_t>(bh) * N + row) * (D * 2);
+      // A row can see no key of a split (l = 0): it contributes nothing.
+      const float inv_l = (l > 0.f) ? 1.0f / l : 0.f;
+      const float lse = (l > 0.f) ? (m + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+      const size_t orow_idx = static_cast<size_t>(bh) * Nq + row;
+      if (!split) {
+        uint8_t* orow = reinterpret_cast<uint8_t*>(p.O) + orow_idx * (D * 2);
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld32(tmem_addr(tbase, lane_base, o_col + 32 * c), r);
-        tmem_wait_ld();
-        reg_fence(r);
-        uint4 v[4];
-        uint32_t* pv = reinterpret_cast<uint32_t*>(v);
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld32(tmem_addr(tbase, lane_base, o_col + 32 * c), r);
+          tmem_wait_ld();
+          reg_fence(r);
+          uint4 v[4];
+          uint32_t* pv = reinterpret_cast<uint32_t*>(v);
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
-          pv[i] = pack2<BF16>(__uint_as_float(r[2 * i]) * inv_l,
-                              __uint_as_float(r[2 * i + 1]) * inv_l);
-        if (row < N) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + c * 64);
+          for (int i = 0; i < 16; ++i)
+            pv[i] = pack2<BF16>(__uint_as_float(r[2 * i]) * inv_l,
+                                __uint_as_float(r[2 * i + 1]) * inv_l);
+          if (row < Nq) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + c * 64);
 #pragma unroll
-          for (int i = 0; i < 4; ++i) dst[i] = v[i];
+            for (int i = 0; i < 4; ++i) dst[i] = v[i];
+          }
         }
+        if (row < Nq) p.LSE[orow_idx] = lse;
+      } else {
+        const size_t part = static_cast<size_t>(blockIdx.y) * p.BH * Nq + orow_idx;
+        float* orow = p.O_part + part * D;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld32(tmem_addr(tbase, lane_base, o_col + 32 * c), r);
+          tmem_wait_ld();
+          reg_fence(r);
+          if (row < Nq && l > 0.f) {
+            float4* dst = reinterpret_cast<float4*>(orow + c * 32);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              dst[i] = make_float4(__uint_as_float(r[4 * i]) * inv_l, __uint_as_float(r[4 * i + 1]) * inv_l,
+                                   __uint_as_float(r[4 * i + 2]) * inv_l,
+                                   __uint_as_float(r[4 * i + 3]) * inv_l);
+          }
+        }
+        if (row < Nq) p.LSE_part[part] = lse;
       }
-      if (row < N)
-        p.LSE[static_cast<size_t>(bh) * N + row] = (m + __log2f(l)) * 0.69314718055994531f;
+    } else if (split && my_nkv == 0 && row < Nq) {
+      // The split holds no key this tile's rows see.
+      p.LSE_part[static_cast<size_t>(blockIdx.y) * p.BH * Nq + static_cast<size_t>(bh) * Nq + row] =
+          -INFINITY;
     }
   }
 

@@ -27,7 +27,8 @@ FA2_FP16 = 0
 FA2_BF16 = 1
 
 # Every symbol include/fa2.h declares.
-EXPORTS = ("fa2_fwd", "fa2_fwd_window", "fa2_bwd_workspace_size", "fa2_bwd", "fa2_bwd_window",
+EXPORTS = ("fa2_fwd", "fa2_fwd_window", "fa2_fwd_decode_splits", "fa2_fwd_decode_workspace_size",
+           "fa2_fwd_decode", "fa2_bwd_workspace_size", "fa2_bwd", "fa2_bwd_window",
            "fa2_bwd_noalloc", "fa2_get_device_status", "fa2_status_string", "fa2_debug_set",
            "fa2_launch_count")
 
@@ -54,6 +55,12 @@ def load() -> ctypes.CDLL:
     lib.fa2_fwd.restype = i
     lib.fa2_fwd_window.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, i, vp]
     lib.fa2_fwd_window.restype = i
+    lib.fa2_fwd_decode_splits.argtypes = [i, i, i, i, i, i]
+    lib.fa2_fwd_decode_splits.restype = i
+    lib.fa2_fwd_decode_workspace_size.argtypes = [i, i, i, i, i, i]
+    lib.fa2_fwd_decode_workspace_size.restype = sz
+    lib.fa2_fwd_decode.argtypes = [vp] * 5 + [i, i, i, i, i, f, i, i, i, vp, sz, vp]
+    lib.fa2_fwd_decode.restype = i
     lib.fa2_bwd_window.argtypes = [vp] * 10 + [sz, i, i, i, i, f, i, i, vp]
     lib.fa2_bwd_window.restype = i
     lib.fa2_bwd_workspace_size.argtypes = [i, i, i, i]
@@ -116,6 +123,29 @@ def fa2_fwd_window(q, k, v, o, lse, scale: float, window: int, stream=None) -> i
     B, H, N, d = q.shape
     return load().fa2_fwd_window(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d,
                                  float(scale), int(window), _dtype_code(q), _stream(stream))
+
+
+def fa2_fwd_decode_splits(B: int, H: int, Nq: int, Nk: int, d: int, sm_count: int = 0) -> int:
+    """Split count the library picks for these sizes (0: invalid sizes or no device)."""
+    return int(load().fa2_fwd_decode_splits(B, H, Nq, Nk, d, sm_count))
+
+
+def fa2_fwd_decode_workspace_size(B: int, H: int, Nq: int, Nk: int, d: int,
+                                  n_splits: int) -> int:
+    return int(load().fa2_fwd_decode_workspace_size(B, H, Nq, Nk, d, n_splits))
+
+
+def fa2_fwd_decode(q, k, v, o, lse, scale: float, causal: bool, n_splits: int, workspace,
+                   stream=None) -> int:
+    """Raw call: q, o [B,H,Nq,d]; k, v [B,H,Nk,d]; lse [B,H,Nq] float32;
+    ``workspace`` a uint8 CUDA tensor or None.  Returns the status."""
+    _check_layout(q, k, v, o, lse)
+    B, H, Nq, d = q.shape
+    Nk = k.shape[2]
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    return load().fa2_fwd_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Nq, Nk, d,
+                                 float(scale), int(bool(causal)), _dtype_code(q), int(n_splits),
+                                 _ptr(workspace), ws_bytes, _stream(stream))
 
 
 def fa2_bwd_window(q, k, v, o, do, lse, dq, dk, dv, workspace, scale: float, window: int,
@@ -194,6 +224,27 @@ def forward_window(q, k, v, scale: float, window: int, stream=None):
     rc = fa2_fwd_window(q, k, v, o, lse, scale, window, stream)
     if rc != FA2_OK:
         raise FA2Error(rc, "fa2_fwd_window")
+    return o, lse
+
+
+def forward_decode(q, k, v, scale: float, causal: bool, n_splits: int = 0, stream=None):
+    """Allocating wrapper of fa2_fwd_decode: q [B,H,Nq,d] against k, v [B,H,Nk,d].
+
+    ``n_splits`` = 0 takes the library's choice for the current device.
+    """
+    B, H, Nq, d = q.shape
+    Nk = k.shape[2]
+    if n_splits == 0:
+        n_splits = fa2_fwd_decode_splits(B, H, Nq, Nk, d)
+        if n_splits == 0:
+            raise FA2Error(FA2_ERR_INVALID_ARG, "fa2_fwd_decode_splits")
+    ws = fa2_fwd_decode_workspace_size(B, H, Nq, Nk, d, n_splits)
+    workspace = torch.empty(ws, dtype=torch.uint8, device=q.device) if ws else None
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
+    rc = fa2_fwd_decode(q, k, v, o, lse, scale, causal, n_splits, workspace, stream)
+    if rc != FA2_OK:
+        raise FA2Error(rc, "fa2_fwd_decode")
     return o, lse
 
 

@@ -138,6 +138,71 @@ def make_inputs(B: int, H: int, N: int, d: int, dtype: str, seed: int, *,
     return out
 
 
+@dataclass(frozen=True)
+class DecodeWorkload:
+    """Nq query rows (the last Nq positions) against Nk key/value rows."""
+    name: str
+    B: int
+    H: int
+    Nq: int
+    Nk: int
+    d: int
+    dtype: str
+    causal: bool
+    seed: int
+    note: str = field(default="", compare=False)
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.d)
+
+    @property
+    def pairs(self) -> int:
+        """(query, key) pairs one head scores: query i sees Nk - Nq + i + 1 keys when
+        causal (bottom-right alignment), all Nk otherwise."""
+        if not self.causal:
+            return self.Nq * self.Nk
+        return self.Nq * (self.Nk - self.Nq) + self.Nq * (self.Nq + 1) // 2
+
+    @property
+    def fwd_flops(self) -> float:
+        return 4.0 * self.B * self.H * self.d * self.pairs
+
+    @property
+    def hbm_bytes(self) -> int:
+        """Algorithmic HBM bytes of one call: Q, K, V read once, O and LSE written once."""
+        e = 2  # 16-bit elements
+        bh = self.B * self.H
+        return bh * (self.Nq * self.d * e * 2 + self.Nk * self.d * e * 2 + self.Nq * 4)
+
+
+DECODE_WORKLOADS = {
+    # One decode step after the long-context prompt: one new query per head
+    # against a 32768-entry key/value cache (512 MiB of K and V, beyond L2).
+    "decode_bf16_b1h32_nq1_nk32768_d128": DecodeWorkload(
+        "decode_bf16_b1h32_nq1_nk32768_d128", 1, 32, 1, 32768, 128, "bf16", True, 6,
+        note="decode step: 1 query per head against a 32768-key cache"),
+}
+
+
+def make_decode_inputs(B: int, H: int, Nq: int, Nk: int, d: int, dtype: str, seed: int) -> dict:
+    """Seeded host tensors q [B,H,Nq,d] and k, v [B,H,Nk,d] in ``dtype``: the same
+    recipe as ``make_inputs`` (N(0,1), drawn in the order Q, K, V)."""
+    if dtype not in DTYPES:
+        raise ValueError(f"dtype must be one of {sorted(DTYPES)}")
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(seed))
+    q = torch.randn((B, H, Nq, d), generator=g, dtype=torch.float32)
+    k = torch.randn((B, H, Nk, d), generator=g, dtype=torch.float32)
+    v = torch.randn((B, H, Nk, d), generator=g, dtype=torch.float32)
+    t = DTYPES[dtype]
+    return {"q": q.to(t), "k": k.to(t), "v": v.to(t)}
+
+
+def decode_inputs(w: DecodeWorkload) -> dict:
+    return make_decode_inputs(w.B, w.H, w.Nq, w.Nk, w.d, w.dtype, w.seed)
+
+
 def workload_inputs(w: Workload, *, with_do: bool | None = None, B: int | None = None,
                     H: int | None = None) -> dict:
     """Inputs of a named workload (optionally with fewer batches / heads)."""

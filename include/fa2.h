@@ -92,6 +92,54 @@ int fa2_fwd_window(const void* Q, const void* K, const void* V, void* O, float* 
                    int H, int N, int d, float scale, int window, int dtype, fa2_stream_t stream);
 
 /*
+ * Decode-like forward: Nq query rows against Nk >= Nq key/value rows, e.g. one
+ * new token (Nq = 1) against a long cache.  Source: [DC] "Parallelismo lungo la
+ * lunghezza della sequenza" (with small batches and long sequences the batch x
+ * heads grid leaves the GPU idle, so the work is also split along the
+ * sequence).  The queries are the LAST Nq positions of the sequence: with
+ * causal = 1 query i sees keys 0 .. Nk - Nq + i (bottom-right alignment; Nq = Nk
+ * is fa2_fwd's causal mask); with causal = 0 every key.
+ *
+ * The key tiles (128 keys each) are cut into n_splits stretches; each stretch
+ * is one CTA per 256 query rows per (batch, head), writing a float partial
+ * output and log-sum-exp to the workspace, and a second kernel merges them
+ * (M = max_s L_s, O = sum_s e^{L_s - M} O_s / sum_s e^{L_s - M},
+ * LSE = M + ln sum_s e^{L_s - M}).  n_splits = 1 writes O and LSE directly, like
+ * fa2_fwd.
+ *
+ *   Q, O     : [B][H][Nq][d] dtype (in, out)
+ *   K, V     : [B][H][Nk][d] dtype (in)
+ *   LSE      : out, [B][H][Nq] float
+ *   B, H     : >= 1; 1 <= Nq <= Nk; d in {64, 128}; causal in {0, 1}
+ *   n_splits : 1 .. 1024 (FA2_ERR_INVALID_ARG otherwise); counts above the
+ *              number of key tiles act as one tile per split
+ *   workspace: device scratch of at least fa2_fwd_decode_workspace_size()
+ *              bytes, 256-byte aligned, not overlapping any tensor argument
+ *              (FA2_ERR_WORKSPACE otherwise); may be NULL when that size is 0.
+ * Results are bitwise repeatable for a fixed n_splits; different split counts
+ * round differently (within the stated tolerances).
+ */
+int fa2_fwd_decode(const void* Q, const void* K, const void* V, void* O, float* LSE, int B,
+                   int H, int Nq, int Nk, int d, float scale, int causal, int dtype, int n_splits,
+                   void* workspace, size_t workspace_bytes, fa2_stream_t stream);
+
+/*
+ * The split count fa2_fwd_decode would best use for these sizes on a GPU with
+ * ``sm_count`` SMs (<= 0: the current device's count): the one that minimises
+ * waves x (key tiles per CTA + 3), one forward CTA per SM.  Returns 0 for sizes
+ * fa2_fwd_decode rejects, or when sm_count <= 0 and no device can be queried.
+ */
+int fa2_fwd_decode_splits(int B, int H, int Nq, int Nk, int d, int sm_count);
+
+/*
+ * Bytes of workspace fa2_fwd_decode needs with ``n_splits`` (0 when the keys fit
+ * one split, and for sizes or split counts fa2_fwd_decode rejects): float
+ * partial outputs [S][B*H][Nq][d] and log-sum-exps [S][B*H][Nq], S the number of
+ * non-empty stretches, each part padded to 256 bytes.
+ */
+size_t fa2_fwd_decode_workspace_size(int B, int H, int Nq, int Nk, int d, int n_splits);
+
+/*
  * Bytes of device workspace fa2_bwd needs for these sizes (the per-row
  * D = rowsum(dO * O) and a float32 dQ accumulator), a multiple of 256.
  * Returns 0 for sizes fa2_bwd would reject.

@@ -124,3 +124,75 @@ def test_window_validation_without_device(lib):
     ptrs = [P * (i + 1) for i in range(9)]
     ws = fa2.fa2_bwd_workspace_size(1, 1, 64, 64)
     assert lib.fa2_bwd_window(*ptrs, 16 * P, ws, 1, 1, 64, 64, 0.1, 0, 1, None) == fa2.FA2_ERR_INVALID_ARG
+
+
+def _decode(lib, *, q=P, k=2 * P, v=3 * P, o=4 * P, lse=5 * P, B=1, H=1, Nq=1, Nk=1000, d=64,
+            scale=0.1, causal=1, dtype=1, splits=1, ws=None, ws_bytes=0):
+    return lib.fa2_fwd_decode(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal, dtype, splits, ws,
+                              ws_bytes, None)
+
+
+def test_decode_validation_without_device(lib):
+    E = fa2.FA2_ERR_INVALID_ARG
+    assert _decode(lib, q=0) == E
+    assert _decode(lib, Nq=0) == E
+    assert _decode(lib, Nq=1001) == E            # more queries than keys
+    assert _decode(lib, splits=0) == E
+    assert _decode(lib, splits=1025) == E
+    assert _decode(lib, causal=3) == E
+    assert _decode(lib, o=P) == E                 # O aliases Q
+    assert _decode(lib, d=96) == fa2.FA2_ERR_UNSUPPORTED
+    # 1000 keys are 8 key tiles; 3 splits need a workspace
+    assert _decode(lib, splits=3) == fa2.FA2_ERR_WORKSPACE
+    need = fa2.fa2_fwd_decode_workspace_size(1, 1, 1, 1000, 64, 3)
+    assert _decode(lib, splits=3, ws=64 * P, ws_bytes=need - 1) == fa2.FA2_ERR_WORKSPACE
+    assert _decode(lib, splits=3, ws=64 * P + 16, ws_bytes=need) == fa2.FA2_ERR_WORKSPACE
+    # a workspace that overlaps K
+    assert _decode(lib, splits=3, ws=2 * P, ws_bytes=need) == fa2.FA2_ERR_WORKSPACE
+
+
+def test_decode_calls_pass_validation_then_need_a_device(lib):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("these fake pointers are only safe without a device")
+    assert _decode(lib) in (fa2.FA2_ERR_CUDA, fa2.FA2_ERR_ARCH)
+    need = fa2.fa2_fwd_decode_workspace_size(1, 1, 1, 1000, 64, 3)
+    assert _decode(lib, splits=3, ws=64 * P, ws_bytes=need) in (fa2.FA2_ERR_CUDA,
+                                                                  fa2.FA2_ERR_ARCH)
+    assert fa2.fa2_fwd_decode_splits(1, 32, 1, 32768, 128, 0) == 0  # no device to ask
+
+
+def test_decode_workspace_size(lib):
+    # 9 stretches x 32 heads x 1 row: O part 9*32*128*4 = 147456 bytes (256-aligned),
+    # LSE part 9*32*4 = 1152 -> 1280.
+    assert fa2.fa2_fwd_decode_workspace_size(1, 32, 1, 32768, 128, 9) == 147456 + 1280
+    # One split (or keys in one tile) needs none.
+    assert fa2.fa2_fwd_decode_workspace_size(1, 32, 1, 32768, 128, 1) == 0
+    assert fa2.fa2_fwd_decode_workspace_size(2, 2, 5, 128, 64, 7) == 0
+    # 1000 keys = 8 tiles: 3 splits of 3, 3, 2 tiles (3*64*4 = 768 bytes of O part);
+    # 5 splits -> 2 tiles each -> 4 stretches (1024 bytes)
+    assert fa2.fa2_fwd_decode_workspace_size(1, 1, 1, 1000, 64, 3) == 768 + 256
+    assert fa2.fa2_fwd_decode_workspace_size(1, 1, 1, 1000, 64, 5) == 1024 + 256
+    assert fa2.fa2_fwd_decode_workspace_size(1, 1, 1, 1000, 64, 100) == 2048 + 256
+    assert fa2.fa2_fwd_decode_workspace_size(1, 1, 2, 1, 64, 2) == 0  # Nq > Nk
+    assert fa2.fa2_fwd_decode_workspace_size(1, 1, 1, 1000, 64, 0) == 0
+
+
+@pytest.mark.parametrize("shape,expect", [
+    # 32 heads, 1 query, 256 key tiles on 148 SMs: cost = waves x (tiles per CTA + 3);
+    # 4 splits: 1 wave x 67; 8: 2 x 35; 9: 2 x 32 = 64 (best); 13: 3 x 23.
+    ((1, 32, 1, 32768, 128), 9),
+    # 256 heads, 64 key tiles: 1 split: 2 x 67 = 134; 4 splits: 7 x 19 = 133 (best).
+    ((8, 32, 1, 8192, 128), 4),
+    # A full prefill already fills the GPU: 2048 CTAs, 14 x 35 beats 28 x 19.
+    ((8, 16, 4096, 4096, 128), 1),
+    # One key tile: nothing to split.
+    ((1, 1, 1, 100, 64), 1),
+])
+def test_decode_split_choice(lib, shape, expect):
+    assert fa2.fa2_fwd_decode_splits(*shape, 148) == expect
+
+
+def test_decode_split_choice_rejects_bad_sizes(lib):
+    assert fa2.fa2_fwd_decode_splits(1, 1, 5, 4, 64, 148) == 0
+    assert fa2.fa2_fwd_decode_splits(1, 1, 1, 4, 80, 148) == 0

@@ -1,0 +1,135 @@
+"""GPU parity of the decode-like forward (fa2_fwd_decode) against the oracle.
+
+Reading of "Flash Attention spiegata: una guida completa", section "Parallelismo
+lungo la lunghezza della sequenza": Nq query rows are the last Nq positions of a
+sequence of Nk keys, so with the causal mask query i sees keys 0 .. Nk - Nq + i;
+the keys are split across CTAs and the partial results merged by log-sum-exp.
+Tolerances as for the plain forward: O max-abs 2e-2 (bf16) / 5e-3 (fp16), LSE
+1e-3.  Split counts include 1 (direct epilogue), ragged stretches, more splits
+than key tiles, and the library's own choice.
+"""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from exact_io_aware_74_b200 import fa2
+from exact_io_aware_74_b200.workloads import make_decode_inputs, make_inputs
+
+pytestmark = pytest.mark.gpu
+
+O_TOL = {"bf16": 2e-2, "fp16": 5e-3}
+
+
+def _inputs(B, H, Nq, Nk, d, dtype, seed):
+    x = make_decode_inputs(B, H, Nq, Nk, d, dtype, seed)
+    return x["q"], x["k"], x["v"]
+
+
+def _run(q, k, v, scale, causal, n_splits):
+    o, lse = fa2.forward_decode(q.cuda(), k.cuda(), v.cuda(), scale, causal, n_splits)
+    assert fa2.fa2_get_device_status() == (fa2.FA2_OK, 0)
+    return o.cpu(), lse.cpu()
+
+
+def _check(o, lse, ref_o, ref_l, dtype):
+    assert np.all(np.isfinite(o.double().numpy()))
+    assert np.max(np.abs(o.double().numpy() - ref_o)) <= O_TOL[dtype]
+    assert np.max(np.abs(lse.double().numpy() - ref_l)) <= 1e-3
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("Nq,Nk", [(1, 1), (1, 100), (1, 129), (1, 1000), (1, 4097), (7, 7),
+                                   (7, 700), (128, 128), (128, 1000), (129, 300), (300, 2500),
+                                   (513, 1000)])
+@pytest.mark.parametrize("n_splits", [1, 3, 0, 1024])
+def test_decode_bf16(Nq, Nk, d, causal, n_splits):
+    q, k, v = _inputs(1, 2, Nq, Nk, d, "bf16", seed=Nq * 31 + Nk + d)
+    s = 1 / math.sqrt(d)
+    o, lse = _run(q, k, v, s, causal, n_splits)
+    ro, rl = oracle.attn_fwd_decode_ref(q, k, v, s, causal)
+    _check(o, lse, ro, rl, "bf16")
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("Nq,Nk,n_splits", [(1, 3000, 5), (16, 2048, 4), (200, 777, 2)])
+def test_decode_fp16(Nq, Nk, d, n_splits):
+    q, k, v = _inputs(2, 3, Nq, Nk, d, "fp16", seed=7 * Nq + Nk)
+    o, lse = _run(q, k, v, 0.08, True, n_splits)
+    ro, rl = oracle.attn_fwd_decode_ref(q, k, v, 0.08, True)
+    _check(o, lse, ro, rl, "fp16")
+
+
+def test_decode_with_nq_equal_nk_is_the_plain_forward():
+    """Nq = Nk and one split run the same kernel path as fa2_fwd: identical bits."""
+    x = make_inputs(2, 2, 700, 128, "bf16", seed=61)
+    q, k, v = (x[n].cuda() for n in ("q", "k", "v"))
+    for causal in (False, True):
+        o1, l1 = fa2.forward_decode(q, k, v, 0.09, causal, 1)
+        o2, l2 = fa2.forward(q, k, v, 0.09, causal)
+        assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_decode_is_repeatable_and_split_counts_agree():
+    q, k, v = _inputs(2, 4, 3, 5000, 128, "bf16", seed=62)
+    q, k, v = q.cuda(), k.cuda(), v.cuda()
+    o1, l1 = fa2.forward_decode(q, k, v, 0.1, True, 6)
+    o2, l2 = fa2.forward_decode(q, k, v, 0.1, True, 6)
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+    ro, rl = oracle.attn_fwd_decode_ref(q.cpu(), k.cpu(), v.cpu(), 0.1, True)
+    for sp in (1, 2, 6, 13, 40):
+        o, lse = fa2.forward_decode(q, k, v, 0.1, True, sp)
+        _check(o.cpu(), lse.cpu(), ro, rl, "bf16")
+
+
+def test_decode_splits_that_hold_no_visible_key():
+    """Causal with Nq > 1: the last stretch holds keys the first rows do not see, so
+    those rows get an empty partial (-inf) that must drop out of the merge."""
+    q, k, v = _inputs(1, 2, 200, 600, 64, "bf16", seed=63)
+    ro, rl = oracle.attn_fwd_decode_ref(q, k, v, 0.125, True)
+    for sp in (2, 3, 5):
+        o, lse = _run(q, k, v, 0.125, True, sp)
+        _check(o, lse, ro, rl, "bf16")
+
+
+def test_decode_launches_one_or_two_kernels():
+    q, k, v = (t.cuda() for t in _inputs(1, 2, 1, 1000, 64, "bf16", seed=64))
+    c0 = fa2.fa2_launch_count()
+    fa2.forward_decode(q, k, v, 0.1, False, 1)
+    c1 = fa2.fa2_launch_count()
+    fa2.forward_decode(q, k, v, 0.1, False, 4)
+    c2 = fa2.fa2_launch_count()
+    assert (c1 - c0, c2 - c1) == (1, 2)
+
+
+def test_decode_rejects_missing_workspace():
+    q, k, v = (t.cuda() for t in _inputs(1, 1, 1, 1000, 64, "bf16", seed=65))
+    o = torch.empty_like(q)
+    lse = torch.empty((1, 1, 1), dtype=torch.float32, device="cuda")
+    assert fa2.fa2_fwd_decode(q, k, v, o, lse, 0.1, False, 4, None) == fa2.FA2_ERR_WORKSPACE
+    assert fa2.fa2_fwd_decode(q, k, v, o, lse, 0.1, False, 1, None) == fa2.FA2_OK
+    assert fa2.fa2_get_device_status() == (fa2.FA2_OK, 0)
+
+
+def test_decode_split_choice_on_this_device():
+    n = torch.cuda.get_device_properties(0).multi_processor_count
+    assert fa2.fa2_fwd_decode_splits(1, 32, 1, 32768, 128, 0) == \
+        fa2.fa2_fwd_decode_splits(1, 32, 1, 32768, 128, n)
+
+
+@pytest.mark.slow
+def test_decode_workload_full_size_sampled():
+    """The measured decode workload at full size with the library's split choice:
+    every head checked against the oracle (one query row per head)."""
+    from exact_io_aware_74_b200.workloads import DECODE_WORKLOADS, decode_inputs
+    w = DECODE_WORKLOADS["decode_bf16_b1h32_nq1_nk32768_d128"]
+    x = decode_inputs(w)
+    q, k, v = (x[n].cuda() for n in ("q", "k", "v"))
+    o, lse = fa2.forward_decode(q, k, v, w.scale, w.causal)
+    assert fa2.fa2_get_device_status() == (fa2.FA2_OK, 0)
+    ro, rl = oracle.attn_fwd_decode_ref(x["q"], x["k"], x["v"], w.scale, w.causal)
+    _check(o.cpu(), lse.cpu(), ro, rl, "bf16")
