@@ -310,26 +310,18 @@ int fa2_fwd_decode_splits(int B, int H, int Nq, int Nk, int d, int sm_count) {
       return 0;
     }
   }
-  // One forward CTA runs per SM.  A CTA costs its key tiles plus about three
-  // tiles' worth of set-up, pipeline fill and partial-result traffic; the time
-  // is that cost times the number of waves.  Take the cheapest split, the
-  // smallest one on ties.
+  // One forward CTA runs per SM (its TMEM allocation is the whole SM's).  As
+  // many splits as still fit the CTAs in one wave, and at least 4 key tiles per
+  // split: measured on B200, a second wave or shorter stretches cost more in
+  // per-CTA set-up and the merge than they gain in parallelism.
   const long long ctas = static_cast<long long>((Nq + 255) / 256) * B * H;
-  const int n_kv = (Nk + 127) / 128;
-  const int max_split = n_kv < kMaxSplits ? n_kv : kMaxSplits;
-  int best = 1;
-  long long best_cost = -1;
-  for (int sp = 1; sp <= max_split; ++sp) {
-    const int eff = effective_splits(n_kv, sp);
-    if (eff != sp) continue;  // same stretches as a smaller split count
-    const long long waves = (ctas * sp + sm_count - 1) / sm_count;
-    const long long cost = waves * (kv_tiles_per_split(n_kv, sp) + 3);
-    if (best_cost < 0 || cost < best_cost) {
-      best_cost = cost;
-      best = sp;
-    }
-  }
-  return best;
+  const int n_kv = (Nq > 0) ? (Nk + 127) / 128 : 1;
+  long long sp = sm_count / ctas;
+  const long long cap = n_kv / 4;
+  if (sp > cap) sp = cap;
+  if (sp > kMaxSplits) sp = kMaxSplits;
+  if (sp < 1) sp = 1;
+  return static_cast<int>(sp);
 }
 
 size_t fa2_fwd_decode_workspace_size(int B, int H, int Nq, int Nk, int d, int n_splits) {

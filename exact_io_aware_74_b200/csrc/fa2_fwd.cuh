@@ -156,6 +156,8 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   const int j0 = has0 ? (has1 ? min(j_lo[0], j_lo[1]) : j_lo[0]) : j_lo[1];
   const int j1 = max(j_hi[0], j_hi[1]);
   const int n_steps = j1 - j0;
+  // A CTA with one query tile runs it double-buffered (see the MMA issuer).
+  const bool single = !has1;
 
   WaitCtl wc{p.status, &abort_flag, p.wait_ns};
 
@@ -248,18 +250,19 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       constexpr uint32_t id_pv = idesc_f16(128, D, BF16, false, true);
       const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV);
 
-      auto issue_qk = [&](int t, int ks) {
+      // S = Q_t K^T into S buffer b; O_t += P_b V.
+      auto issue_qk = [&](int t, int b, int ks) {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * C::CHUNK + (kk & 3) * 32;
-          umma_ss(tbase + (t ? C::S_COL1 : C::S_COL0), sdesc_sw128(sQa + t * C::TILE + off, 16, 1024),
+          umma_ss(tbase + (b ? C::S_COL1 : C::S_COL0), sdesc_sw128(sQa + t * C::TILE + off, 16, 1024),
                   sdesc_sw128(sKa + ks * C::TILE + off, 16, 1024), id_qk, kk > 0);
         }
       };
-      auto issue_pv = [&](int t, int vs, bool acc) {
+      auto issue_pv = [&](int t, int b, int vs, bool acc) {
 #pragma unroll
         for (int kk = 0; kk < C::BN / 16; ++kk) {
-          umma_ts(tbase + (t ? C::O_COL1 : C::O_COL0), tbase + (t ? C::S_COL1 : C::S_COL0) + kk * 8,
+          umma_ts(tbase + (t ? C::O_COL1 : C::O_COL0), tbase + (b ? C::S_COL1 : C::S_COL0) + kk * 8,
                   sdesc_sw128(sVa + vs * C::TILE + kk * 2048, C::CHUNK, 1024), id_pv,
                   (acc || kk > 0) ? 1u : 0u);
         }
@@ -268,15 +271,50 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 
       bool ok = n_steps > 0 && mbar_wait(&bar_q, 0, wc, kSiteMmaQ) &&
                 mbar_wait(&k_full[0], 0, wc, kSiteMmaK);
+      if (single) {
+        // One query tile: S is double-buffered in the two S column blocks, and
+        // S of step jj + 1 is issued before P of step jj is awaited, so the
+        // softmax of one step overlaps the P V product of the one before.
+        if (ok) {
+          tc_fence_after();
+          issue_qk(0, 0, 0);
+          umma_commit(&s_full[0]);
+          umma_commit(&k_empty[0]);
+        }
+        for (int jj = 0; jj < n_steps && ok; ++jj) {
+          const int b = jj & 1;
+          if (jj + 1 < n_steps) {
+            // Buffer b^1 held P of step jj - 1, consumed by the P V product
+            // issued (in order, before this) in the previous iteration.
+            const int ks1 = (jj + 1) % C::KS;
+            if (!mbar_wait(&k_full[ks1], ((jj + 1) / C::KS) & 1, wc, kSiteMmaK)) { ok = false; break; }
+            tc_fence_after();
+            issue_qk(0, b ^ 1, ks1);
+            umma_commit(&s_full[b ^ 1]);
+            umma_commit(&k_empty[ks1]);
+          }
+          const int vs = jj % C::VS;
+          if (!mbar_wait(&v_full[vs], (jj / C::VS) & 1, wc, kSiteMmaV) ||
+              !mbar_wait(&p_ready[b], (jj >> 1) & 1, wc, kSiteMmaP)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          issue_pv(0, b, vs, jj > 0);
+          umma_commit(&o_done[0]);
+          umma_commit(&v_empty[vs]);
+        }
+        ok = false;  // the two-tile loop below is skipped
+      }
       if (ok) {
         tc_fence_after();
         // Tiles whose key range starts at j0 get their first S now.
         if (hi0 > lo0 && lo0 == j0) {
-          issue_qk(0, 0);
+          issue_qk(0, 0, 0);
           umma_commit(&s_full[0]);
         }
         if (hi1 > lo1 && lo1 == j0) {
-          issue_qk(1, 0);
+          issue_qk(1, 1, 0);
           umma_commit(&s_full[1]);
         }
         umma_commit(&k_empty[0]);
@@ -293,7 +331,7 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             const int step = j - lo;  // this tile's own step count
             if (!mbar_wait(&p_ready[t], step & 1, wc, kSiteMmaP)) return false;
             tc_fence_after();
-            issue_pv(t, vs, step > 0);
+            issue_pv(t, t, vs, step > 0);
             umma_commit(&o_done[t]);
           }
           // S for step j + 1 (this tile's next step, or its first when its range
@@ -304,7 +342,7 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
               tc_fence_after();
               k_next_ready = true;
             }
-            issue_qk(t, ks1);
+            issue_qk(t, t, ks1);
             umma_commit(&s_full[t]);
           }
           return true;
@@ -334,7 +372,6 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     const int my_lo = t ? j_lo[1] : j_lo[0];
     const int my_nkv = (t ? j_hi[1] : j_hi[0]) - my_lo;  // steps of this tile
     const int row = my_row0 + r_loc;
-    const uint32_t s_col = t ? C::S_COL1 : C::S_COL0;
     const uint32_t o_col = t ? C::O_COL1 : C::O_COL0;
     const uint32_t lane_base = static_cast<uint32_t>(wq * 32);
     const float sl2 = p.scale_log2;  // > 0 (checked on the host)
@@ -347,12 +384,17 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     const bool live = my_row0 + wq * 32 < Nq;
     for (int step = 0; step < my_nkv && ok; ++step) {
       const int j = my_lo + step;  // key tile of this step
+      // S buffer of this step and the phase of its barriers: one buffer per
+      // tile, or (one tile in the CTA) the two buffers in turn.
+      const int buf = single ? (step & 1) : t;
+      const uint32_t par = single ? ((step >> 1) & 1) : (step & 1);
+      const uint32_t s_col = buf ? C::S_COL1 : C::S_COL0;
       // Warp-uniform wait: the TMEM loads and stores below are warp-collective.
-      ok = __all_sync(0xffffffffu, mbar_wait(&s_full[t], step & 1, wc, kSiteSoftS));
+      ok = __all_sync(0xffffffffu, mbar_wait(&s_full[buf], par, wc, kSiteSoftS));
       if (!ok) break;
       if (!live) {
         __syncwarp();
-        if (lane == 0) mbar_arrive(&p_ready[t]);
+        if (lane == 0) mbar_arrive(&p_ready[buf]);
         continue;
       }
       tc_fence_after();
@@ -455,7 +497,7 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&p_ready[t]);
+      if (lane == 0) mbar_arrive(&p_ready[buf]);
     }
     if (ok && live)
       ok = __all_sync(0xffffffffu, mbar_wait(&o_done[t], (my_nkv - 1) & 1, wc, kSiteSoftOEnd));

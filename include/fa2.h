@@ -125,8 +125,9 @@ int fa2_fwd_decode(const void* Q, const void* K, const void* V, void* O, float* 
 
 /*
  * The split count fa2_fwd_decode would best use for these sizes on a GPU with
- * ``sm_count`` SMs (<= 0: the current device's count): the one that minimises
- * waves x (key tiles per CTA + 3), one forward CTA per SM.  Returns 0 for sizes
+ * ``sm_count`` SMs (<= 0: the current device's count): as many as keep all CTAs
+ * in one wave (one CTA per SM, ceil(Nq / 256) x B x H CTAs per split), but no
+ * more than one split per 4 key tiles, and at least 1.  Returns 0 for sizes
  * fa2_fwd_decode rejects, or when sm_count <= 0 and no device can be queried.
  */
 int fa2_fwd_decode_splits(int B, int H, int Nq, int Nk, int d, int sm_count);

@@ -179,15 +179,18 @@ def test_decode_workspace_size(lib):
 
 
 @pytest.mark.parametrize("shape,expect", [
-    # 32 heads, 1 query, 256 key tiles on 148 SMs: cost = waves x (tiles per CTA + 3);
-    # 4 splits: 1 wave x 67; 8: 2 x 35; 9: 2 x 32 = 64 (best); 13: 3 x 23.
-    ((1, 32, 1, 32768, 128), 9),
-    # 256 heads, 64 key tiles: 1 split: 2 x 67 = 134; 4 splits: 7 x 19 = 133 (best).
-    ((8, 32, 1, 8192, 128), 4),
-    # A full prefill already fills the GPU: 2048 CTAs, 14 x 35 beats 28 x 19.
+    # 32 CTAs per split on 148 SMs: 4 splits fill one wave (128 CTAs).
+    ((1, 32, 1, 32768, 128), 4),
+    # 256 CTAs already exceed one wave.
+    ((8, 32, 1, 8192, 128), 1),
+    # A full prefill fills the GPU many times over.
     ((8, 16, 4096, 4096, 128), 1),
-    # One key tile: nothing to split.
-    ((1, 1, 1, 100, 64), 1),
+    # One head: 148 would fit, but 256 key tiles allow 64 splits of 4.
+    ((1, 1, 1, 32768, 64), 64),
+    # 300 queries = 2 CTAs per head per split; 8 heads: 9 splits (144 CTAs).
+    ((1, 8, 300, 65536, 128), 9),
+    # Fewer than 8 key tiles: nothing to split.
+    ((1, 1, 1, 700, 64), 1),
 ])
 def test_decode_split_choice(lib, shape, expect):
     assert fa2.fa2_fwd_decode_splits(*shape, 148) == expect
