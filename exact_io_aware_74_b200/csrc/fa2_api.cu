@@ -46,11 +46,6 @@ EncodeTiledFn encode_fn() {
 
 }  // namespace
 
-namespace fa2 {
-bool make_tile_map(CUtensorMap* map, const void* base, int BH, int N, int d, bool bf16);
-bool make_acc_map(CUtensorMap* map, float* base, int BH, int N, int d);
-}  // namespace fa2
-
 namespace {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -104,16 +99,17 @@ unsigned int* status_word(int dev) {
 
 namespace fa2 {
 
-// [BH][N][d] 16-bit tensor viewed as a 3-D TMA map with 128-row x 64-column
+// [BH][N][d] 16-bit tensor viewed as a 3-D TMA map with box_rows x 64-column
 // boxes and 128-byte swizzle; rows past N read as zeros.
-bool make_tile_map(CUtensorMap* map, const void* base, int BH, int N, int d, bool bf16) {
+bool make_tile_map(CUtensorMap* map, const void* base, int BH, int N, int d, bool bf16,
+                   int box_rows) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
   const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
                               static_cast<cuuint64_t>(BH)};
   const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
                                  static_cast<cuuint64_t>(N) * d * 2};
-  const cuuint32_t box[3] = {64, 128, 1};
+  const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
   const cuuint32_t estr[3] = {1, 1, 1};
   const CUtensorMapDataType ty =
       bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
@@ -144,15 +140,17 @@ bool make_acc_map(CUtensorMap* map, float* base, int BH, int N, int d) {
 
 namespace {
 
-bool make_map(CUtensorMap* map, const void* base, int BH, int N, int d, int dtype) {
-  return fa2::make_tile_map(map, base, BH, N, d, dtype == FA2_BF16);
+bool make_map(CUtensorMap* map, const void* base, int BH, int N, int d, int dtype,
+              int box_rows = 128) {
+  return fa2::make_tile_map(map, base, BH, N, d, dtype == FA2_BF16, box_rows);
 }
 
 unsigned long long wait_ns() { return static_cast<unsigned long long>(g_wait_ms.load()) * 1000000ull; }
 
 template <int D, bool BF16, bool CAUSAL>
 int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-               const fa2::FwdParams& p, int n_split, cudaStream_t stream) {
+               const CUtensorMap& mqr, const fa2::FwdParams& p, int n_split,
+               cudaStream_t stream) {
   using Cfg = fa2::FwdCfg<D>;
   auto kern = fa2::fa2_fwd_kernel<D, BF16, CAUSAL>;
   // The kernel re-splits its registers between warpgroups; that is only sound
@@ -172,7 +170,7 @@ int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& 
   }
   const dim3 grid(static_cast<unsigned int>(p.n_qblk) * static_cast<unsigned int>(p.BH),
                   static_cast<unsigned int>(n_split));
-  kern<<<grid, Cfg::THREADS, Cfg::SMEM, stream>>>(mq, mk, mv, p);
+  kern<<<grid, Cfg::THREADS, Cfg::SMEM, stream>>>(mq, mk, mv, mqr, p);
   if (cudaGetLastError() != cudaSuccess) return FA2_ERR_CUDA;
   g_launches.fetch_add(1);
   return FA2_OK;
@@ -195,22 +193,30 @@ namespace {
 
 // Shared by every forward entry point.  Query rows [BH][Nq], key rows [BH][Nk];
 // off = Nk - Nq aligns the causal mask to the bottom right; window = 0 means no
-// sliding window.  n_split = 1: O and LSE are written directly; otherwise the key
-// tiles are cut into n_split stretches of kv_per_split, the partials go to
-// O_part / LSE_part and a second kernel merges them into O and LSE.
+// sliding window.  The key tiles are cut into n_split stretches of kv_per_split
+// and the queries replicated rep times (1, 2 or 4, rep > 1 only for
+// Nq <= 128 / rep); with n_split x rep = 1 O and LSE are written directly,
+// otherwise the n_split x rep partials go to O_part / LSE_part and a second
+// kernel merges them into O and LSE.
 int fwd_core(const void* Q, const void* K, const void* V, void* O, float* LSE, int BH, int Nq,
              int Nk, int d, float scale, int causal, int window, int dtype, int n_split,
-             int kv_per_split, float* O_part, float* LSE_part, fa2_stream_t stream) {
+             int kv_per_split, int rep, float* O_part, float* LSE_part, fa2_stream_t stream) {
   int dev = 0;
   int rc = check_device(&dev);
   if (rc != FA2_OK) return rc;
   unsigned int* st = status_word(dev);
   if (!st) return FA2_ERR_CUDA;
 
-  CUtensorMap mq, mk, mv;
+  CUtensorMap mq, mk, mv, mqr;
   if (!make_map(&mq, Q, BH, Nq, d, dtype) || !make_map(&mk, K, BH, Nk, d, dtype) ||
       !make_map(&mv, V, BH, Nk, d, dtype))
     return FA2_ERR_CUDA;
+  if (rep > 1) {
+    if (!make_map(&mqr, Q, BH, Nq, d, dtype, 128 / rep)) return FA2_ERR_CUDA;
+  } else {
+    mqr = mq;  // not read
+  }
+  const int n_part = n_split * rep;
 
   fa2::FwdParams p{};
   p.O = O;
@@ -226,24 +232,25 @@ int fwd_core(const void* Q, const void* K, const void* V, void* O, float* LSE, i
   p.fault = g_fault.load();
   p.window = window;
   p.kv_per_split = n_split > 1 ? kv_per_split : 0;
-  p.O_part = O_part;
-  p.LSE_part = LSE_part;
+  p.O_part = n_part > 1 ? O_part : nullptr;
+  p.LSE_part = n_part > 1 ? LSE_part : nullptr;
+  p.rep = rep;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const bool bf = dtype == FA2_BF16;
   if (d == 64) {
-    if (bf) rc = causal ? launch_fwd<64, true, true>(mq, mk, mv, p, n_split, s) : launch_fwd<64, true, false>(mq, mk, mv, p, n_split, s);
-    else rc = causal ? launch_fwd<64, false, true>(mq, mk, mv, p, n_split, s) : launch_fwd<64, false, false>(mq, mk, mv, p, n_split, s);
+    if (bf) rc = causal ? launch_fwd<64, true, true>(mq, mk, mv, mqr, p, n_split, s) : launch_fwd<64, true, false>(mq, mk, mv, mqr, p, n_split, s);
+    else rc = causal ? launch_fwd<64, false, true>(mq, mk, mv, mqr, p, n_split, s) : launch_fwd<64, false, false>(mq, mk, mv, mqr, p, n_split, s);
   } else {
-    if (bf) rc = causal ? launch_fwd<128, true, true>(mq, mk, mv, p, n_split, s) : launch_fwd<128, true, false>(mq, mk, mv, p, n_split, s);
-    else rc = causal ? launch_fwd<128, false, true>(mq, mk, mv, p, n_split, s) : launch_fwd<128, false, false>(mq, mk, mv, p, n_split, s);
+    if (bf) rc = causal ? launch_fwd<128, true, true>(mq, mk, mv, mqr, p, n_split, s) : launch_fwd<128, true, false>(mq, mk, mv, mqr, p, n_split, s);
+    else rc = causal ? launch_fwd<128, false, true>(mq, mk, mv, mqr, p, n_split, s) : launch_fwd<128, false, false>(mq, mk, mv, mqr, p, n_split, s);
   }
-  if (rc != FA2_OK || n_split == 1) return rc;
+  if (rc != FA2_OK || n_part == 1) return rc;
   const long long rows = static_cast<long long>(BH) * Nq;
   if (d == 64)
-    return bf ? launch_combine<64, true>(O_part, LSE_part, O, LSE, rows, n_split, s)
-              : launch_combine<64, false>(O_part, LSE_part, O, LSE, rows, n_split, s);
-  return bf ? launch_combine<128, true>(O_part, LSE_part, O, LSE, rows, n_split, s)
-            : launch_combine<128, false>(O_part, LSE_part, O, LSE, rows, n_split, s);
+    return bf ? launch_combine<64, true>(O_part, LSE_part, O, LSE, rows, n_part, s)
+              : launch_combine<64, false>(O_part, LSE_part, O, LSE, rows, n_part, s);
+  return bf ? launch_combine<128, true>(O_part, LSE_part, O, LSE, rows, n_part, s)
+            : launch_combine<128, false>(O_part, LSE_part, O, LSE, rows, n_part, s);
 }
 
 // Shared by fa2_fwd and fa2_fwd_window; window = 0 means no sliding window.
@@ -262,7 +269,7 @@ int fwd_impl(const void* Q, const void* K, const void* V, void* O, float* LSE, i
       overlaps(LSE, lse_bytes, Q, bytes) || overlaps(LSE, lse_bytes, K, bytes) ||
       overlaps(LSE, lse_bytes, V, bytes))
     return FA2_ERR_INVALID_ARG;
-  return fwd_core(Q, K, V, O, LSE, BH, N, N, d, scale, causal, window, dtype, 1, 0, nullptr,
+  return fwd_core(Q, K, V, O, LSE, BH, N, N, d, scale, causal, window, dtype, 1, 0, 1, nullptr,
                   nullptr, stream);
 }
 
@@ -275,6 +282,9 @@ int effective_splits(int n_kv, int n_split) {
 }
 
 constexpr int kMaxSplits = 1024;
+
+// Query copies fa2_fwd_decode uses: 4 for up to 32 queries, 2 for up to 64.
+int decode_rep(int Nq) { return Nq <= 32 ? 4 : (Nq <= 64 ? 2 : 1); }
 
 // Checks of fa2_fwd_decode's sizes that need no CUDA call.
 int check_decode_sizes(int B, int H, int Nq, int Nk, int d, float scale, int causal, int dtype) {
@@ -327,9 +337,9 @@ int fa2_fwd_decode_splits(int B, int H, int Nq, int Nk, int d, int sm_count) {
 size_t fa2_fwd_decode_workspace_size(int B, int H, int Nq, int Nk, int d, int n_splits) {
   if (check_decode_sizes(B, H, Nq, Nk, d, 1.0f, 0, FA2_BF16) != FA2_OK) return 0;
   if (n_splits < 1 || n_splits > kMaxSplits) return 0;
-  const int eff = effective_splits((Nk + 127) / 128, n_splits);
-  if (eff == 1) return 0;
-  return fa2::decode_workspace_bytes(static_cast<size_t>(eff), static_cast<size_t>(B) * H,
+  const int parts = effective_splits((Nk + 127) / 128, n_splits) * decode_rep(Nq);
+  if (parts == 1) return 0;
+  return fa2::decode_workspace_bytes(static_cast<size_t>(parts), static_cast<size_t>(B) * H,
                                      static_cast<size_t>(Nq), d);
 }
 
@@ -353,10 +363,12 @@ int fa2_fwd_decode(const void* Q, const void* K, const void* V, void* O, float* 
     return FA2_ERR_INVALID_ARG;
   const int n_kv = (Nk + 127) / 128;
   const int eff = effective_splits(n_kv, n_splits);
+  const int rep = decode_rep(Nq);
+  const int parts = eff * rep;
   float* O_part = nullptr;
   float* LSE_part = nullptr;
-  if (eff > 1) {
-    const size_t need = fa2::decode_workspace_bytes(static_cast<size_t>(eff),
+  if (parts > 1) {
+    const size_t need = fa2::decode_workspace_bytes(static_cast<size_t>(parts),
                                                     static_cast<size_t>(BH), Nq, d);
     if (!workspace || workspace_bytes < need ||
         (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
@@ -367,11 +379,11 @@ int fa2_fwd_decode(const void* Q, const void* K, const void* V, void* O, float* 
       if (overlaps(workspace, need, bufs[i], buf_bytes[i])) return FA2_ERR_WORKSPACE;
     O_part = static_cast<float*>(workspace);
     LSE_part = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
-                                        fa2::decode_opart_bytes(static_cast<size_t>(eff),
+                                        fa2::decode_opart_bytes(static_cast<size_t>(parts),
                                                                 static_cast<size_t>(BH), Nq, d));
   }
   return fwd_core(Q, K, V, O, LSE, BH, Nq, Nk, d, scale, causal, 0, dtype, eff,
-                  kv_tiles_per_split(n_kv, n_splits), O_part, LSE_part, stream);
+                  kv_tiles_per_split(n_kv, n_splits), rep, O_part, LSE_part, stream);
 }
 
 size_t fa2_bwd_workspace_size(int B, int H, int N, int d) {

@@ -589,7 +589,10 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 // host launcher
 // ------------------------------------------------------------------------------------
 
-bool make_tile_map(CUtensorMap* map, const void* base, int BH, int N, int d, bool bf16);
+// [BH][N][d] 16-bit tensor as a 3-D TMA map, box_rows x 64-column boxes, 128-byte
+// swizzle; fp32 accumulator map with 128 x 32 boxes (both defined with the host API).
+bool make_tile_map(CUtensorMap* map, const void* base, int BH, int N, int d, bool bf16,
+                   int box_rows = 128);
 bool make_acc_map(CUtensorMap* map, float* base, int BH, int N, int d);
 
 template <int D, bool BF16, bool CAUSAL>

@@ -34,6 +34,8 @@
 // that one warpgroup's softmax overlaps the other tile's matrix products.
 #pragma once
 
+#include <type_traits>
+
 #include "ptx.cuh"
 
 namespace fa2 {
@@ -55,10 +57,17 @@ struct FwdParams {
   // (y + 1) kv_per_split) and writes its rows' partial results, normalised by
   // its own row sums, to O_part [split][BH][Nq][D] and LSE_part [split][BH][Nq]
   // (float, -inf for a row that sees no key of the split).  kv_per_split = 0:
-  // no split, O and LSE are written directly.
+  // all key tiles.  O_part = nullptr: O and LSE are written directly.
   int kv_per_split;
   float* O_part;
   float* LSE_part;
+  // Query copies (1, 2 or 4; > 1 only with Nq <= 128 / rep and partial
+  // results): the 128-row Q tile holds rep copies of the Nq <= 128 / rep
+  // queries, loaded through tmQr (boxes of 128 / rep rows), and copy c scores
+  // only key columns [c 128 / rep, (c + 1) 128 / rep) of every key tile, as
+  // partial result blockIdx.y * rep + c.  A lone query then keeps four softmax
+  // warps busy instead of one.
+  int rep;
 };
 
 template <int D>
@@ -103,7 +112,8 @@ enum FwdSite : uint32_t {
 template <int D, bool BF16, bool CAUSAL>
 __global__ void __launch_bounds__(384, 1)
 fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-               const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
+               const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmQr,
+               const FwdParams p) {
   using C = FwdCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -121,7 +131,8 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   const int lane = threadIdx.x & 31;
   const int Nq = p.Nq, Nk = p.Nk;
   const int off = CAUSAL ? p.off : 0;
-  const bool split = p.kv_per_split > 0;
+  const bool split = p.kv_per_split > 0;    // keys cut into stretches (blockIdx.y)
+  const bool partial = p.O_part != nullptr;  // partial results, merged by a second kernel
 
   // Heaviest query blocks first (they see the most keys when causal).
   const int qb = p.n_qblk - 1 - static_cast<int>(blockIdx.x) / p.BH;
@@ -199,10 +210,21 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       for (int t = 0; t < 2; ++t) q_bytes += (j_hi[t] > 0) ? C::TILE : 0;
       // (A CTA whose split holds no key any of its rows sees loads nothing.)
       mbar_arrive_expect_tx(&bar_q, q_bytes);
-      for (int t = 0; t < 2; ++t) {
-        if (j_hi[t] == 0) continue;
-        for (int c = 0; c < C::KCH; ++c)
-          tma_load_3d(sQ + t * C::TILE + c * C::CHUNK, &tmQ, &bar_q, c * 64, row0[t], bh);
+      if (p.rep > 1) {
+        // rep copies of rows 0 .. 128/rep - 1 (tile 0 only), one box each.
+        if (j_hi[0] > 0) {
+          tma_prefetch_desc(&tmQr);
+          const int qr = C::BM / p.rep;
+          for (int r = 0; r < p.rep; ++r)
+            for (int c = 0; c < C::KCH; ++c)
+              tma_load_3d(sQ + c * C::CHUNK + r * qr * 128, &tmQr, &bar_q, c * 64, 0, bh);
+        }
+      } else {
+        for (int t = 0; t < 2; ++t) {
+          if (j_hi[t] == 0) continue;
+          for (int c = 0; c < C::KCH; ++c)
+            tma_load_3d(sQ + t * C::TILE + c * C::CHUNK, &tmQ, &bar_q, c * 64, row0[t], bh);
+        }
       }
       int k_issued = 0, v_issued = 0;  // loads issued so far
       bool ok = true;
@@ -371,7 +393,12 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     const int my_row0 = t ? row0[1] : row0[0];
     const int my_lo = t ? j_lo[1] : j_lo[0];
     const int my_nkv = (t ? j_hi[1] : j_hi[0]) - my_lo;  // steps of this tile
-    const int row = my_row0 + r_loc;
+    // With rep > 1 the tile holds rep copies of its QR = 128 / rep query rows;
+    // copy qcopy (warp-uniform) owns key columns qcopy * 128 / rep onwards.
+    const int rep = p.rep;
+    const int QR = C::BM / rep;
+    const int qcopy = r_loc / QR;
+    const int row = my_row0 + r_loc % QR;
     const uint32_t o_col = t ? C::O_COL1 : C::O_COL0;
     const uint32_t lane_base = static_cast<uint32_t>(wq * 32);
     const float sl2 = p.scale_log2;  // > 0 (checked on the host)
@@ -381,40 +408,34 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     const int win = p.window;
     // A warp whose 32 rows are all past Nq only keeps the barrier count: its P
     // rows feed output rows that are never stored.
-    const bool live = my_row0 + wq * 32 < Nq;
-    for (int step = 0; step < my_nkv && ok; ++step) {
-      const int j = my_lo + step;  // key tile of this step
-      // S buffer of this step and the phase of its barriers: one buffer per
-      // tile, or (one tile in the CTA) the two buffers in turn.
-      const int buf = single ? (step & 1) : t;
-      const uint32_t par = single ? ((step >> 1) & 1) : (step & 1);
-      const uint32_t s_col = buf ? C::S_COL1 : C::S_COL0;
-      // Warp-uniform wait: the TMEM loads and stores below are warp-collective.
-      ok = __all_sync(0xffffffffu, mbar_wait(&s_full[buf], par, wc, kSiteSoftS));
-      if (!ok) break;
-      if (!live) {
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&p_ready[buf]);
-        continue;
-      }
-      tc_fence_after();
-      uint32_t sr[128];
+    const bool live = my_row0 + (wq * 32) % QR < Nq;
+
+    // One step of the online softmax over the NC key columns this warp owns:
+    // S from TMEM, masks, running max (with the lazy output rescale), P back to
+    // TMEM in 16-bit over the first 64 columns of the S buffer -- zeros in the
+    // columns of the other copies -- and the running sum.  False if a wait ran out.
+    auto soft_step = [&](auto nc_tag, int step, uint32_t s_col) -> bool {
+      constexpr int NC = decltype(nc_tag)::value;
+      constexpr int NP = NC / 2;                  // packed 16-bit pairs of P
+      constexpr int G = NP < 32 ? NP : 32;        // pairs per TMEM store
+      const int col0 = qcopy * NC;
+      uint32_t sr[NC];
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
-        tmem_ld32(tmem_addr(tbase, lane_base, s_col + 32 * c),
+      for (int c = 0; c < NC / 32; ++c)
+        tmem_ld32(tmem_addr(tbase, lane_base, s_col + col0 + 32 * c),
                   *reinterpret_cast<uint32_t(*)[32]>(&sr[32 * c]));
       tmem_wait_ld();
       reg_fence(sr);
-      const int key0 = j * C::BN;
+      const int kc0 = (my_lo + step) * C::BN + col0;  // key of column 0 of sr
       // Keys after the row's last one (causal), past Nk, or before the row's
       // window start.
-      const bool need_mask = (CAUSAL && key0 + C::BN - 1 > my_row0 + off) || (key0 + C::BN > Nk) ||
-                             (CAUSAL && win > 0 && key0 < my_row0 + off + 127 - win + 1);
+      const bool need_mask = (CAUSAL && kc0 + NC - 1 > my_row0 + off) || (kc0 + NC > Nk) ||
+                             (CAUSAL && win > 0 && kc0 < my_row0 + off + 127 - win + 1);
       if (need_mask) {
-        const int hi_lim = CAUSAL ? min(row + off - key0 + 1, Nk - key0) : (Nk - key0);
-        const int lo_lim = (CAUSAL && win > 0) ? row + off - win + 1 - key0 : 0;
+        const int hi_lim = CAUSAL ? min(row + off - kc0 + 1, Nk - kc0) : (Nk - kc0);
+        const int lo_lim = (CAUSAL && win > 0) ? row + off - win + 1 - kc0 : 0;
 #pragma unroll
-        for (int i = 0; i < 128; ++i)
+        for (int i = 0; i < NC; ++i)
           if (i >= hi_lim || i < lo_lim) sr[i] = __float_as_uint(-INFINITY);
       }
       float mx[8];
@@ -422,12 +443,12 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       for (int k = 0; k < 8; ++k)
         mx[k] = fmax3(__uint_as_float(sr[k]), __uint_as_float(sr[k + 8]), __uint_as_float(sr[k + 16]));
 #pragma unroll
-      for (int i = 24; i < 120; i += 16)  // elements 24 .. 119
+      for (int i = 24; i + 24 <= NC; i += 16)  // elements 24 .. NC - 9
 #pragma unroll
         for (int k = 0; k < 8; ++k)
           mx[k] = fmax3(mx[k], __uint_as_float(sr[i + k]), __uint_as_float(sr[i + k + 8]));
 #pragma unroll
-      for (int k = 0; k < 8; ++k) mx[k] = fmaxf(mx[k], __uint_as_float(sr[120 + k]));
+      for (int k = 0; k < 8; ++k) mx[k] = fmaxf(mx[k], __uint_as_float(sr[NC - 8 + k]));
       mx[0] = fmax3(mx[0], mx[1], mx[2]);
       mx[3] = fmax3(mx[3], mx[4], mx[5]);
       mx[6] = fmaxf(mx[6], mx[7]);
@@ -444,8 +465,8 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           const float f = need ? ex2_approx(m - m_new) : 1.0f;
           if (need) m = m_new;
           l *= f;
-          ok = __all_sync(0xffffffffu, mbar_wait(&o_done[t], (step - 1) & 1, wc, kSiteSoftO));
-          if (!ok) break;
+          if (!__all_sync(0xffffffffu, mbar_wait(&o_done[t], (step - 1) & 1, wc, kSiteSoftO)))
+            return false;
           tc_fence_after();
 #pragma unroll
           for (int c = 0; c < D / 32; ++c) {
@@ -467,12 +488,12 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       const uint64_t negm2 = f2_pack(neg_m, neg_m);
       uint64_t sum2[4] = {0, 0, 0, 0};
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        uint32_t pk[32];
+      for (int h = 0; h < NP / G; ++h) {
+        uint32_t pk[G];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const uint64_t arg = f2_fma(f2_pack(__uint_as_float(sr[64 * h + 2 * i]),
-                                              __uint_as_float(sr[64 * h + 2 * i + 1])),
+        for (int i = 0; i < G; ++i) {
+          const uint64_t arg = f2_fma(f2_pack(__uint_as_float(sr[2 * G * h + 2 * i]),
+                                              __uint_as_float(sr[2 * G * h + 2 * i + 1])),
                                       sl2x2, negm2);
           float a, b;
           f2_unpack(arg, a, b);
@@ -486,7 +507,20 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           sum2[i & 3] = f2_add(sum2[i & 3], f2_pack(a, b));
           pk[i] = pack2<BF16>(a, b);
         }
-        tmem_st32(tmem_addr(tbase, lane_base, s_col + 32 * h), pk);
+        const uint32_t dst = tmem_addr(tbase, lane_base, s_col + col0 / 2 + G * h);
+        if constexpr (G == 32) tmem_st32(dst, pk); else tmem_st16(dst, pk);
+      }
+      if constexpr (NC < 128) {
+        // The other copies' key columns contribute nothing to this copy's rows.
+        uint32_t zero[NP];
+#pragma unroll
+        for (int i = 0; i < NP; ++i) zero[i] = 0u;
+#pragma unroll
+        for (int b = 0; b < 128 / NC; ++b) {
+          if (b == qcopy) continue;
+          const uint32_t dst = tmem_addr(tbase, lane_base, s_col + b * NP);
+          if constexpr (NP == 32) tmem_st32(dst, zero); else tmem_st16(dst, zero);
+        }
       }
       {
         const uint64_t s01 = f2_add(f2_add(sum2[0], sum2[1]), f2_add(sum2[2], sum2[3]));
@@ -494,8 +528,30 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         f2_unpack(s01, lo, hi);
         l += lo + hi;
       }
-      tmem_wait_st();
-      tc_fence_before();
+      return true;
+    };
+
+    for (int step = 0; step < my_nkv && ok; ++step) {
+      // S buffer of this step and the phase of its barriers: one buffer per
+      // tile, or (one tile in the CTA) the two buffers in turn.
+      const int buf = single ? (step & 1) : t;
+      const uint32_t par = single ? ((step >> 1) & 1) : (step & 1);
+      const uint32_t s_col = buf ? C::S_COL1 : C::S_COL0;
+      // Warp-uniform wait: the TMEM loads and stores below are warp-collective.
+      ok = __all_sync(0xffffffffu, mbar_wait(&s_full[buf], par, wc, kSiteSoftS));
+      if (!ok) break;
+      if (live) {
+        tc_fence_after();
+        if (rep == 4)
+          ok = soft_step(std::integral_constant<int, 32>{}, step, s_col);
+        else if (rep == 2)
+          ok = soft_step(std::integral_constant<int, 64>{}, step, s_col);
+        else
+          ok = soft_step(std::integral_constant<int, 128>{}, step, s_col);
+        if (!ok) break;
+        tmem_wait_st();
+        tc_fence_before();
+      }
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_ready[buf]);
     }
@@ -507,7 +563,7 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       const float inv_l = (l > 0.f) ? 1.0f / l : 0.f;
       const float lse = (l > 0.f) ? (m + __log2f(l)) * 0.69314718055994531f : -INFINITY;
       const size_t orow_idx = static_cast<size_t>(bh) * Nq + row;
-      if (!split) {
+      if (!partial) {
         uint8_t* orow = reinterpret_cast<uint8_t*>(p.O) + orow_idx * (D * 2);
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
@@ -529,7 +585,7 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         }
         if (row < Nq) p.LSE[orow_idx] = lse;
       } else {
-        const size_t part = static_cast<size_t>(blockIdx.y) * p.BH * Nq + orow_idx;
+        const size_t part = static_cast<size_t>(blockIdx.y * rep + qcopy) * p.BH * Nq + orow_idx;
         float* orow = p.O_part + part * D;
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
@@ -548,10 +604,10 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         }
         if (row < Nq) p.LSE_part[part] = lse;
       }
-    } else if (split && my_nkv == 0 && row < Nq) {
+    } else if (partial && my_nkv == 0 && row < Nq) {
       // The split holds no key this tile's rows see.
-      p.LSE_part[static_cast<size_t>(blockIdx.y) * p.BH * Nq + static_cast<size_t>(bh) * Nq + row] =
-          -INFINITY;
+      p.LSE_part[static_cast<size_t>(blockIdx.y * rep + qcopy) * p.BH * Nq +
+                 static_cast<size_t>(bh) * Nq + row] = -INFINITY;
     }
   }
 

@@ -101,11 +101,14 @@ int fa2_fwd_window(const void* Q, const void* K, const void* V, void* O, float* 
  * is fa2_fwd's causal mask); with causal = 0 every key.
  *
  * The key tiles (128 keys each) are cut into n_splits stretches; each stretch
- * is one CTA per 256 query rows per (batch, head), writing a float partial
- * output and log-sum-exp to the workspace, and a second kernel merges them
- * (M = max_s L_s, O = sum_s e^{L_s - M} O_s / sum_s e^{L_s - M},
- * LSE = M + ln sum_s e^{L_s - M}).  n_splits = 1 writes O and LSE directly, like
- * fa2_fwd.
+ * is one CTA per 256 query rows per (batch, head).  With Nq <= 32 (<= 64) the
+ * queries are also replicated 4 (2) times down the CTA's 128-row tile and each
+ * copy scores a quarter (half) of every key tile's columns, so that four
+ * softmax warps share the work of one query.  Each (stretch, copy) writes a
+ * float partial output and log-sum-exp to the workspace and a second kernel
+ * merges them (M = max_s L_s, O = sum_s e^{L_s - M} O_s / sum_s e^{L_s - M},
+ * LSE = M + ln sum_s e^{L_s - M}).  One stretch and Nq > 64 write O and LSE
+ * directly, like fa2_fwd.
  *
  *   Q, O     : [B][H][Nq][d] dtype (in, out)
  *   K, V     : [B][H][Nk][d] dtype (in)
@@ -133,10 +136,11 @@ int fa2_fwd_decode(const void* Q, const void* K, const void* V, void* O, float* 
 int fa2_fwd_decode_splits(int B, int H, int Nq, int Nk, int d, int sm_count);
 
 /*
- * Bytes of workspace fa2_fwd_decode needs with ``n_splits`` (0 when the keys fit
- * one split, and for sizes or split counts fa2_fwd_decode rejects): float
+ * Bytes of workspace fa2_fwd_decode needs with ``n_splits`` (0 when it writes O
+ * and LSE directly, and for sizes or split counts fa2_fwd_decode rejects): float
  * partial outputs [S][B*H][Nq][d] and log-sum-exps [S][B*H][Nq], S the number of
- * non-empty stretches, each part padded to 256 bytes.
+ * non-empty stretches times the query copies (4 for Nq <= 32, 2 for Nq <= 64,
+ * else 1), each part padded to 256 bytes.
  */
 size_t fa2_fwd_decode_workspace_size(int B, int H, int Nq, int Nk, int d, int n_splits);
 

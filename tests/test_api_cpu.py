@@ -142,20 +142,22 @@ def test_decode_validation_without_device(lib):
     assert _decode(lib, causal=3) == E
     assert _decode(lib, o=P) == E                 # O aliases Q
     assert _decode(lib, d=96) == fa2.FA2_ERR_UNSUPPORTED
-    # 1000 keys are 8 key tiles; 3 splits need a workspace
-    assert _decode(lib, splits=3) == fa2.FA2_ERR_WORKSPACE
-    need = fa2.fa2_fwd_decode_workspace_size(1, 1, 1, 1000, 64, 3)
-    assert _decode(lib, splits=3, ws=64 * P, ws_bytes=need - 1) == fa2.FA2_ERR_WORKSPACE
-    assert _decode(lib, splits=3, ws=64 * P + 16, ws_bytes=need) == fa2.FA2_ERR_WORKSPACE
+    # 100 queries, 1000 keys = 8 key tiles: 3 splits need a workspace
+    assert _decode(lib, Nq=100, splits=3) == fa2.FA2_ERR_WORKSPACE
+    need = fa2.fa2_fwd_decode_workspace_size(1, 1, 100, 1000, 64, 3)
+    assert _decode(lib, Nq=100, splits=3, ws=64 * P, ws_bytes=need - 1) == fa2.FA2_ERR_WORKSPACE
+    assert _decode(lib, Nq=100, splits=3, ws=64 * P + 16, ws_bytes=need) == fa2.FA2_ERR_WORKSPACE
     # a workspace that overlaps K
-    assert _decode(lib, splits=3, ws=2 * P, ws_bytes=need) == fa2.FA2_ERR_WORKSPACE
+    assert _decode(lib, Nq=100, splits=3, ws=2 * P, ws_bytes=need) == fa2.FA2_ERR_WORKSPACE
+    # up to 64 queries are replicated across the tile: partials even with one split
+    assert _decode(lib, Nq=1, splits=1) == fa2.FA2_ERR_WORKSPACE
 
 
 def test_decode_calls_pass_validation_then_need_a_device(lib):
     import torch
     if torch.cuda.is_available():
         pytest.skip("these fake pointers are only safe without a device")
-    assert _decode(lib) in (fa2.FA2_ERR_CUDA, fa2.FA2_ERR_ARCH)
+    assert _decode(lib, Nq=100) in (fa2.FA2_ERR_CUDA, fa2.FA2_ERR_ARCH)
     need = fa2.fa2_fwd_decode_workspace_size(1, 1, 1, 1000, 64, 3)
     assert _decode(lib, splits=3, ws=64 * P, ws_bytes=need) in (fa2.FA2_ERR_CUDA,
                                                                   fa2.FA2_ERR_ARCH)
@@ -163,19 +165,24 @@ def test_decode_calls_pass_validation_then_need_a_device(lib):
 
 
 def test_decode_workspace_size(lib):
-    # 9 stretches x 32 heads x 1 row: O part 9*32*128*4 = 147456 bytes (256-aligned),
-    # LSE part 9*32*4 = 1152 -> 1280.
-    assert fa2.fa2_fwd_decode_workspace_size(1, 32, 1, 32768, 128, 9) == 147456 + 1280
-    # One split (or keys in one tile) needs none.
-    assert fa2.fa2_fwd_decode_workspace_size(1, 32, 1, 32768, 128, 1) == 0
-    assert fa2.fa2_fwd_decode_workspace_size(2, 2, 5, 128, 64, 7) == 0
-    # 1000 keys = 8 tiles: 3 splits of 3, 3, 2 tiles (3*64*4 = 768 bytes of O part);
-    # 5 splits -> 2 tiles each -> 4 stretches (1024 bytes)
-    assert fa2.fa2_fwd_decode_workspace_size(1, 1, 1, 1000, 64, 3) == 768 + 256
-    assert fa2.fa2_fwd_decode_workspace_size(1, 1, 1, 1000, 64, 5) == 1024 + 256
-    assert fa2.fa2_fwd_decode_workspace_size(1, 1, 1, 1000, 64, 100) == 2048 + 256
-    assert fa2.fa2_fwd_decode_workspace_size(1, 1, 2, 1, 64, 2) == 0  # Nq > Nk
-    assert fa2.fa2_fwd_decode_workspace_size(1, 1, 1, 1000, 64, 0) == 0
+    ws = fa2.fa2_fwd_decode_workspace_size
+    # 100 queries (no copies): 1000 keys = 8 tiles; 3 splits of 3, 3, 2 tiles:
+    # O part 3*100*64*4 = 76800 bytes (256-aligned), LSE part 1200 -> 1280.
+    assert ws(1, 1, 100, 1000, 64, 3) == 76800 + 1280
+    # 5 splits -> 2 tiles each -> 4 stretches; 100 splits -> 8 stretches of one tile
+    assert ws(1, 1, 100, 1000, 64, 5) == 4 * 25600 + 1792
+    assert ws(1, 1, 100, 1000, 64, 100) == 8 * 25600 + 3328
+    # One split of more than 64 queries needs none.
+    assert ws(1, 32, 100, 32768, 128, 1) == 0
+    # One query: 4 copies per stretch.  9 stretches x 4 copies x 32 heads:
+    # O part 36*32*128*4 = 589824, LSE part 36*32*4 = 4608.
+    assert ws(1, 32, 1, 32768, 128, 9) == 589824 + 4608
+    assert ws(1, 32, 1, 32768, 128, 1) == 4 * 32 * 512 + 512
+    # 40 queries: 2 copies; one key tile, so 7 splits are one stretch:
+    # O part 2*4*40*64*4 = 81920, LSE part 2*4*40*4 = 1280.
+    assert ws(2, 2, 40, 128, 64, 7) == 81920 + 1280
+    assert ws(1, 1, 2, 1, 64, 2) == 0       # Nq > Nk
+    assert ws(1, 1, 1, 1000, 64, 0) == 0    # no split count
 
 
 @pytest.mark.parametrize("shape,expect", [
