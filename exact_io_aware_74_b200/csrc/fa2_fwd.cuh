@@ -32,6 +32,12 @@
 // P_t (16-bit) overwrites the first 64 columns of S_t and feeds the P V MMA
 // straight from TMEM.  The MMA warp alternates between the two query tiles so
 // that one warpgroup's softmax overlaps the other tile's matrix products.
+// A CTA with one query tile (short or decode-like queries) instead uses both S
+// column blocks as a double buffer: S of step j + 1 is computed while the
+// softmax of step j runs.  Decode-like calls may also cut the keys into
+// stretches (one per blockIdx.y) and replicate up to 64 queries down the tile
+// so every softmax warp has rows to work on; both write partial results that
+// fa2_decode.cuh merges.
 #pragma once
 
 #include <type_traits>
@@ -460,6 +466,8 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         // Lazy rescale: the stale maximum is kept unless it fell behind by more
         // than 8 (a factor 256 in the exponentials); the output accumulator is
         // only touched in that case, after the previous P V product landed.
+        // (The product before that one finished before this step's S, which
+        // this warp has seen, so the barrier is at most one phase behind.)
         const bool need = m_new - m > 8.0f;
         if (__any_sync(0xffffffffu, need)) {
           const float f = need ? ex2_approx(m - m_new) : 1.0f;
@@ -555,6 +563,13 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_ready[buf]);
     }
+    // Wait for the last P V product.  A phase-parity wait is only sound while the
+    // barrier is at most one phase behind.  With one tile per CTA, S of the last
+    // step is issued before P V of the step before it, so that product (phase
+    // my_nkv - 2) may still be pending: wait for it first.  (Every earlier one
+    // finished before S of the last step, which this warp has seen.)
+    if (ok && live && single && my_nkv >= 2)
+      ok = __all_sync(0xffffffffu, mbar_wait(&o_done[t], (my_nkv - 2) & 1, wc, kSiteSoftOEnd));
     if (ok && live)
       ok = __all_sync(0xffffffffu, mbar_wait(&o_done[t], (my_nkv - 1) & 1, wc, kSiteSoftOEnd));
     if (ok && live) {

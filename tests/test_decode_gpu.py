@@ -87,6 +87,21 @@ def test_decode_is_repeatable_and_split_counts_agree():
         _check(o.cpu(), lse.cpu(), ro, rl, "bf16")
 
 
+@pytest.mark.parametrize("Nq,Nk,d,sp", [(64, 3000, 128, 6), (64, 3000, 64, 6), (32, 2000, 128, 4),
+                                        (100, 2000, 128, 5), (128, 1000, 64, 2)])
+def test_decode_repeated_runs_stay_correct(Nq, Nk, d, sp):
+    """Several live softmax warps per CTA and few steps per split: the end-of-loop
+    wait for the last P V product once returned early in some runs (O wrong, LSE
+    right), so the check is repeated over many heads."""
+    q, k, v = _inputs(2, 16, Nq, Nk, d, "bf16", seed=66 + Nq + d)
+    ro, rl = oracle.attn_fwd_decode_ref(q, k, v, d ** -0.5, True)
+    q, k, v = q.cuda(), k.cuda(), v.cuda()
+    for _ in range(8):
+        o, lse = fa2.forward_decode(q, k, v, d ** -0.5, True, sp)
+        assert fa2.fa2_get_device_status() == (fa2.FA2_OK, 0)
+        _check(o.cpu(), lse.cpu(), ro, rl, "bf16")
+
+
 def test_decode_splits_that_hold_no_visible_key():
     """Causal with Nq > 1: the last stretch holds keys the first rows do not see, so
     those rows get an empty partial (-inf) that must drop out of the merge."""
