@@ -34,7 +34,8 @@ sys.path.insert(0, ROOT)
 
 import torch  # noqa: E402
 
-from exact_io_aware_74_b200.workloads import WORKLOADS, WORKLOAD_ORDER, workload_inputs  # noqa: E402
+from exact_io_aware_74_b200.workloads import (  # noqa: E402
+    DECODE_WORKLOADS, WORKLOADS, WORKLOAD_ORDER, decode_inputs, workload_inputs)
 
 METRIC = "FA-2 fwd/bwd TFLOP/s (bf16, 1×B200) and % of dense BF16 tensor peak"
 DEFAULT_WORKLOAD = WORKLOAD_ORDER[1]          # forward + backward, bf16, causal, d = 64
@@ -67,7 +68,8 @@ def input_bytes(w) -> int:
 
 
 # Device sources of each C-ABI call's kernels.
-KERNEL_SOURCES = {"fa2_fwd": ("ptx.cuh", "fa2_fwd.cuh"), "fa2_bwd": ("ptx.cuh", "fa2_bwd.cuh")}
+KERNEL_SOURCES = {"fa2_fwd": ("ptx.cuh", "fa2_fwd.cuh"), "fa2_bwd": ("ptx.cuh", "fa2_bwd.cuh"),
+                  "fa2_fwd_decode": ("ptx.cuh", "fa2_fwd.cuh", "fa2_decode.cuh")}
 
 
 def csrc_hash(call: str) -> str:
@@ -292,6 +294,54 @@ def time_e2e(fa2, st, steps, stream):
     return ms, h2d, d2h
 
 
+def time_decode(fa2, w, iters, dev, stream, hbm_peak, peaks_src):
+    """One decode-like call (fa2_fwd_decode, the library's split count) per step:
+    median CUDA-event time, achieved algorithmic HBM GB/s and its roofline."""
+    x = decode_inputs(w)
+    q, k, v = (x[n].to(dev) for n in ("q", "k", "v"))
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.H, w.Nq), dtype=torch.float32, device=dev)
+    splits = fa2.fa2_fwd_decode_splits(w.B, w.H, w.Nq, w.Nk, w.d)
+    if splits < 1:
+        raise RuntimeError("fa2_fwd_decode_splits failed")
+    nws = fa2.fa2_fwd_decode_workspace_size(w.B, w.H, w.Nq, w.Nk, w.d, splits)
+    ws = torch.empty(nws, dtype=torch.uint8, device=dev) if nws else None
+    flush = None
+    if w.hbm_bytes < 2 * L2_BYTES:
+        flush = torch.zeros(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+
+    def call():
+        _check(fa2, fa2.fa2_fwd_decode(q, k, v, o, lse, w.scale, w.causal, splits, ws, stream),
+               "fa2_fwd_decode")
+
+    for _ in range(3):
+        call()
+    torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(iters)]
+    c0 = fa2.fa2_launch_count()
+    with torch.cuda.stream(stream):
+        for i in range(iters):
+            if flush is not None:
+                flush.add_(1)
+            ev[i][0].record(stream)
+            call()
+            ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    launches = (fa2.fa2_launch_count() - c0) // iters
+    rc, site = fa2.fa2_get_device_status(stream)
+    if rc != fa2.FA2_OK:
+        raise RuntimeError(f"device status {fa2.status_string(rc)} at wait site {site}")
+    ms = statistics.median(e[0].elapsed_time(e[1]) for e in ev)
+    gbs = w.hbm_bytes / (ms / 1e3) / 1e9
+    return {"us": round(ms * 1e3, 2), "splits": splits, "launches_per_call": launches,
+            "hbm_bytes": w.hbm_bytes, "tflops": round(w.fwd_flops / ms / 1e9, 2),
+            "roofline": {"bound": "hbm", "kernel": "fa2_fwd_decode (forward + merge)",
+                         "achieved": round(gbs, 1), "peak": hbm_peak, "unit": "GB/s",
+                         "frac": round(gbs / hbm_peak, 4),
+                         "traffic": traffic_from_profiles(f"fa2_fwd_decode:{w.name}"),
+                         "peak_kind": f"HBM copy, {peaks_src}"}}
+
+
 def cpu_baseline(w, budget_s: float = 12.0) -> dict:
     """The oracle as it stands, timed on this host's cores on whole (b, h) slices."""
     import numpy as np  # noqa: F401
@@ -395,6 +445,9 @@ def run_ours(args):
             extras[name] = e
             torch.cuda.empty_cache()
         out["other_workloads"] = extras
+        out["decode"] = {name: time_decode(fa2, dw, 50, dev, stream, peaks["hbm_gbs"], peaks_src)
+                         for name, dw in DECODE_WORKLOADS.items()}
+        torch.cuda.empty_cache()
         out["headline"] = {"workload": HEADLINE_WORKLOAD,
                            "fwd_tflops": extras[HEADLINE_WORKLOAD]["fwd_tflops"],
                            "pct_of_bf16_burst_peak": extras[HEADLINE_WORKLOAD]["fwd_pct_bf16_burst"],

@@ -33,8 +33,8 @@
 // straight from TMEM.  The MMA warp alternates between the two query tiles so
 // that one warpgroup's softmax overlaps the other tile's matrix products.
 // A CTA with one query tile (short or decode-like queries) instead uses both S
-// column blocks as a double buffer: S of step j + 1 is computed while the
-// softmax of step j runs.  Decode-like calls may also cut the keys into
+// column blocks as a double buffer -- S of step j + 1 is computed while the
+// softmax of step j runs -- and its idle second Q slot as one more V stage.  Decode-like calls may also cut the keys into
 // stretches (one per blockIdx.y) and replicate up to 64 queries down the tile
 // so every softmax warp has rows to work on; both write partial results that
 // fa2_decode.cuh merges.
@@ -128,7 +128,7 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   uint8_t* sK = sQ + C::QT * C::TILE;
   uint8_t* sV = sK + C::KS * C::TILE;
 
-  __shared__ uint64_t bar_q, k_full[C::KS], k_empty[C::KS], v_full[C::VS], v_empty[C::VS];
+  __shared__ uint64_t bar_q, k_full[C::KS], k_empty[C::KS], v_full[C::VS + 1], v_empty[C::VS + 1];
   __shared__ uint64_t s_full[2], p_ready[2], o_done[2], drain;
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
@@ -182,7 +182,7 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     abort_flag = 0;
     mbar_init(&bar_q, 1);
     for (int s = 0; s < C::KS; ++s) { mbar_init(&k_full[s], 1); mbar_init(&k_empty[s], 1); }
-    for (int s = 0; s < C::VS; ++s) { mbar_init(&v_full[s], 1); mbar_init(&v_empty[s], 1); }
+    for (int s = 0; s <= C::VS; ++s) { mbar_init(&v_full[s], 1); mbar_init(&v_empty[s], 1); }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&s_full[t], 1);
       mbar_init(&p_ready[t], 4);
@@ -232,31 +232,44 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             tma_load_3d(sQ + t * C::TILE + c * C::CHUNK, &tmQ, &bar_q, c * 64, row0[t], bh);
         }
       }
+      // With one query tile the second Q slot is one more V stage.
+      const int vring = single ? C::VS + 1 : C::VS;
       int k_issued = 0, v_issued = 0;  // loads issued so far
-      bool ok = true;
-      for (int jj = 0; jj < n_steps && ok; ++jj) {
-        const int j = j0 + jj;  // key tile; jj is its slot count in the rings
-        const int ks = jj % C::KS, vs = jj % C::VS;
-        if (jj >= C::KS && !mbar_wait(&k_empty[ks], ((jj / C::KS) - 1) & 1, wc, kSiteProdKEmpty)) {
-          ok = false;
-          break;
-        }
+      auto load_k = [&](int jj) -> bool {
+        const int ks = jj % C::KS;
+        if (jj >= C::KS && !mbar_wait(&k_empty[ks], ((jj / C::KS) - 1) & 1, wc, kSiteProdKEmpty))
+          return false;
         if (!(p.fault == 1 && jj == 0)) {
           mbar_arrive_expect_tx(&k_full[ks], C::TILE);
           for (int c = 0; c < C::KCH; ++c)
             tma_load_3d_hint(sK + ks * C::TILE + c * C::CHUNK, &tmK, &k_full[ks], c * 64,
-                             j * C::BN, bh, keep);
+                             (j0 + jj) * C::BN, bh, keep);
           k_issued = jj + 1;
         }
-        if (jj >= C::VS && !mbar_wait(&v_empty[vs], ((jj / C::VS) - 1) & 1, wc, kSiteProdVEmpty)) {
-          ok = false;
-          break;
-        }
+        return true;
+      };
+      auto load_v = [&](int jj) -> bool {
+        const int vs = jj % vring;
+        if (jj >= vring && !mbar_wait(&v_empty[vs], ((jj / vring) - 1) & 1, wc, kSiteProdVEmpty))
+          return false;
+        uint8_t* dst = vs < C::VS ? sV + vs * C::TILE : sQ + C::TILE;
         mbar_arrive_expect_tx(&v_full[vs], C::TILE);
         for (int c = 0; c < C::KCH; ++c)
-          tma_load_3d_hint(sV + vs * C::TILE + c * C::CHUNK, &tmV, &v_full[vs], c * 64,
-                           j * C::BN, bh, keep);
+          tma_load_3d_hint(dst + c * C::CHUNK, &tmV, &v_full[vs], c * 64, (j0 + jj) * C::BN, bh,
+                           keep);
         v_issued = jj + 1;
+        return true;
+      };
+      // Loads go out in the order the MMA warp consumes them: with one query
+      // tile, K of step jj + 1 (for S) is needed before V of step jj, and a V
+      // slot waiting for its P V product must not hold back the next K.
+      bool ok = true;
+      if (single) {
+        ok = n_steps == 0 || load_k(0);
+        for (int jj = 0; jj < n_steps && ok; ++jj)
+          ok = (jj + 1 >= n_steps || load_k(jj + 1)) && load_v(jj);
+      } else {
+        for (int jj = 0; jj < n_steps && ok; ++jj) ok = load_k(jj) && load_v(jj);
       }
       if (!ok) {
         // Let every copy already issued land before the CTA exits.
@@ -266,8 +279,8 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         for (int jj = max(0, k_issued - C::KS); jj < k_issued; ++jj)
           if (!(p.fault == 1 && jj == 0))
             mbar_wait(&k_full[jj % C::KS], (jj / C::KS) & 1, dw, kSiteProdDrain);
-        for (int jj = max(0, v_issued - C::VS); jj < v_issued; ++jj)
-          mbar_wait(&v_full[jj % C::VS], (jj / C::VS) & 1, dw, kSiteProdDrain);
+        for (int jj = max(0, v_issued - vring); jj < v_issued; ++jj)
+          mbar_wait(&v_full[jj % vring], (jj / vring) & 1, dw, kSiteProdDrain);
       }
     }
     __syncwarp();
@@ -287,12 +300,16 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                   sdesc_sw128(sKa + ks * C::TILE + off, 16, 1024), id_qk, kk > 0);
         }
       };
+      // V ring slot vs: the V stages, then (one query tile) the second Q slot.
+      auto v_addr = [&](int vs) -> uint32_t {
+        return vs < C::VS ? sVa + vs * C::TILE : sQa + C::TILE;
+      };
       auto issue_pv = [&](int t, int b, int vs, bool acc) {
+        const uint32_t va = v_addr(vs);
 #pragma unroll
         for (int kk = 0; kk < C::BN / 16; ++kk) {
           umma_ts(tbase + (t ? C::O_COL1 : C::O_COL0), tbase + (b ? C::S_COL1 : C::S_COL0) + kk * 8,
-                  sdesc_sw128(sVa + vs * C::TILE + kk * 2048, C::CHUNK, 1024), id_pv,
-                  (acc || kk > 0) ? 1u : 0u);
+                  sdesc_sw128(va + kk * 2048, C::CHUNK, 1024), id_pv, (acc || kk > 0) ? 1u : 0u);
         }
       };
       const int lo0 = j_lo[0], hi0 = j_hi[0], lo1 = j_lo[1], hi1 = j_hi[1];
@@ -321,8 +338,9 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             umma_commit(&s_full[b ^ 1]);
             umma_commit(&k_empty[ks1]);
           }
-          const int vs = jj % C::VS;
-          if (!mbar_wait(&v_full[vs], (jj / C::VS) & 1, wc, kSiteMmaV) ||
+          constexpr int VR = C::VS + 1;  // V ring with the second Q slot
+          const int vs = jj % VR;
+          if (!mbar_wait(&v_full[vs], (jj / VR) & 1, wc, kSiteMmaV) ||
               !mbar_wait(&p_ready[b], (jj >> 1) & 1, wc, kSiteMmaP)) {
             ok = false;
             break;

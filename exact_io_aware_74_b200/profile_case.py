@@ -1,9 +1,11 @@
-"""Runs fa2_fwd (and fa2_bwd) a few times on one shape, for profilers.
+"""Runs fa2_fwd (and fa2_bwd), or fa2_fwd_decode, a few times on one shape, for profilers.
 
     python -m exact_io_aware_74_b200.profile_case B H N d causal [reps] [--fwd-only]
+    python -m exact_io_aware_74_b200.profile_case --decode B H Nq Nk d causal [reps] [splits]
 
 Seeded N(0, 1) bf16 inputs; exits non-zero if a call or the device status fails.
-Used to capture Nsight Compute profiles of one kernel on a small case.
+Used to capture Nsight Compute profiles of one kernel on a small case.  With
+--decode, splits = 0 (the default) takes the library's split count.
 """
 
 from __future__ import annotations
@@ -14,10 +16,25 @@ import sys
 import torch
 
 from exact_io_aware_74_b200 import fa2
-from exact_io_aware_74_b200.workloads import make_inputs
+from exact_io_aware_74_b200.workloads import make_decode_inputs, make_inputs
+
+
+def decode(args: list[str]) -> int:
+    B, H, Nq, Nk, d, causal = (int(a) for a in args[:6])
+    reps = int(args[6]) if len(args) > 6 else 2
+    splits = int(args[7]) if len(args) > 7 else 0
+    x = make_decode_inputs(B, H, Nq, Nk, d, "bf16", seed=5)
+    q, k, v = (x[n].cuda() for n in ("q", "k", "v"))
+    for _ in range(reps):
+        fa2.forward_decode(q, k, v, 1.0 / math.sqrt(d), bool(causal), splits)
+    rc, site = fa2.fa2_get_device_status()
+    print(f"status {fa2.status_string(rc)} site {site}")
+    return 0 if rc == fa2.FA2_OK else 1
 
 
 def main(argv: list[str]) -> int:
+    if "--decode" in argv:
+        return decode([a for a in argv if not a.startswith("--")])
     fwd_only = "--fwd-only" in argv
     args = [a for a in argv if not a.startswith("--")]
     B, H, N, d, causal = (int(a) for a in args[:5])
