@@ -147,12 +147,12 @@ bool make_map(CUtensorMap* map, const void* base, int BH, int N, int d, int dtyp
 
 unsigned long long wait_ns() { return static_cast<unsigned long long>(g_wait_ms.load()) * 1000000ull; }
 
-template <int D, bool BF16, bool CAUSAL>
+template <int D, bool BF16, bool CAUSAL, int REP>
 int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                const CUtensorMap& mqr, const fa2::FwdParams& p, int n_split,
                cudaStream_t stream) {
   using Cfg = fa2::FwdCfg<D>;
-  auto kern = fa2::fa2_fwd_kernel<D, BF16, CAUSAL>;
+  auto kern = fa2::fa2_fwd_kernel<D, BF16, CAUSAL, REP>;
   // The kernel re-splits its registers between warpgroups; that is only sound
   // when every thread was launched with exactly Cfg::LAUNCH_REGS registers.
   static const bool regs_ok = [&] {
@@ -174,6 +174,26 @@ int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& 
   if (cudaGetLastError() != cudaSuccess) return FA2_ERR_CUDA;
   g_launches.fetch_add(1);
   return FA2_OK;
+}
+
+// Instantiation of the forward for the runtime flags.
+template <int D>
+int launch_fwd_any(bool bf, bool causal, int rep, const CUtensorMap& mq, const CUtensorMap& mk,
+                   const CUtensorMap& mv, const CUtensorMap& mqr, const fa2::FwdParams& p,
+                   int n_split, cudaStream_t s) {
+#define FA2_FWD_REP(BF, CA)                                                        \
+  switch (rep) {                                                                   \
+    case 4: return launch_fwd<D, BF, CA, 4>(mq, mk, mv, mqr, p, n_split, s);       \
+    case 2: return launch_fwd<D, BF, CA, 2>(mq, mk, mv, mqr, p, n_split, s);       \
+    default: return launch_fwd<D, BF, CA, 1>(mq, mk, mv, mqr, p, n_split, s);      \
+  }
+  if (bf) {
+    if (causal) { FA2_FWD_REP(true, true) }
+    FA2_FWD_REP(true, false)
+  }
+  if (causal) { FA2_FWD_REP(false, true) }
+  FA2_FWD_REP(false, false)
+#undef FA2_FWD_REP
 }
 
 template <int D, bool BF16>
@@ -234,16 +254,10 @@ int fwd_core(const void* Q, const void* K, const void* V, void* O, float* LSE, i
   p.kv_per_split = n_split > 1 ? kv_per_split : 0;
   p.O_part = n_part > 1 ? O_part : nullptr;
   p.LSE_part = n_part > 1 ? LSE_part : nullptr;
-  p.rep = rep;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const bool bf = dtype == FA2_BF16;
-  if (d == 64) {
-    if (bf) rc = causal ? launch_fwd<64, true, true>(mq, mk, mv, mqr, p, n_split, s) : launch_fwd<64, true, false>(mq, mk, mv, mqr, p, n_split, s);
-    else rc = causal ? launch_fwd<64, false, true>(mq, mk, mv, mqr, p, n_split, s) : launch_fwd<64, false, false>(mq, mk, mv, mqr, p, n_split, s);
-  } else {
-    if (bf) rc = causal ? launch_fwd<128, true, true>(mq, mk, mv, mqr, p, n_split, s) : launch_fwd<128, true, false>(mq, mk, mv, mqr, p, n_split, s);
-    else rc = causal ? launch_fwd<128, false, true>(mq, mk, mv, mqr, p, n_split, s) : launch_fwd<128, false, false>(mq, mk, mv, mqr, p, n_split, s);
-  }
+  rc = (d == 64) ? launch_fwd_any<64>(bf, causal != 0, rep, mq, mk, mv, mqr, p, n_split, s)
+                 : launch_fwd_any<128>(bf, causal != 0, rep, mq, mk, mv, mqr, p, n_split, s);
   if (rc != FA2_OK || n_part == 1) return rc;
   const long long rows = static_cast<long long>(BH) * Nq;
   if (d == 64)

@@ -67,13 +67,6 @@ struct FwdParams {
   int kv_per_split;
   float* O_part;
   float* LSE_part;
-  // Query copies (1, 2 or 4; > 1 only with Nq <= 128 / rep and partial
-  // results): the 128-row Q tile holds rep copies of the Nq <= 128 / rep
-  // queries, loaded through tmQr (boxes of 128 / rep rows), and copy c scores
-  // only key columns [c 128 / rep, (c + 1) 128 / rep) of every key tile, as
-  // partial result blockIdx.y * rep + c.  A lone query then keeps four softmax
-  // warps busy instead of one.
-  int rep;
 };
 
 template <int D>
@@ -115,7 +108,12 @@ enum FwdSite : uint32_t {
   kSiteMmaDrain, kSiteSoftS, kSiteSoftO, kSiteSoftOEnd, kSiteProdDrain
 };
 
-template <int D, bool BF16, bool CAUSAL>
+// REP: query copies (1, 2 or 4; > 1 only with Nq <= 128 / REP and partial
+// results).  The 128-row Q tile then holds REP copies of the Nq queries, loaded
+// through tmQr (boxes of 128 / REP rows), and copy c scores only key columns
+// [c 128 / REP, (c + 1) 128 / REP) of every key tile, as partial result
+// blockIdx.y * REP + c: a lone query keeps four softmax warps busy, not one.
+template <int D, bool BF16, bool CAUSAL, int REP>
 __global__ void __launch_bounds__(384, 1)
 fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmQr,
@@ -216,12 +214,12 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       for (int t = 0; t < 2; ++t) q_bytes += (j_hi[t] > 0) ? C::TILE : 0;
       // (A CTA whose split holds no key any of its rows sees loads nothing.)
       mbar_arrive_expect_tx(&bar_q, q_bytes);
-      if (p.rep > 1) {
-        // rep copies of rows 0 .. 128/rep - 1 (tile 0 only), one box each.
+      if constexpr (REP > 1) {
+        // REP copies of rows 0 .. 128/REP - 1 (tile 0 only), one box each.
         if (j_hi[0] > 0) {
           tma_prefetch_desc(&tmQr);
-          const int qr = C::BM / p.rep;
-          for (int r = 0; r < p.rep; ++r)
+          constexpr int qr = C::BM / REP;
+          for (int r = 0; r < REP; ++r)
             for (int c = 0; c < C::KCH; ++c)
               tma_load_3d(sQ + c * C::CHUNK + r * qr * 128, &tmQr, &bar_q, c * 64, 0, bh);
         }
@@ -417,10 +415,9 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     const int my_row0 = t ? row0[1] : row0[0];
     const int my_lo = t ? j_lo[1] : j_lo[0];
     const int my_nkv = (t ? j_hi[1] : j_hi[0]) - my_lo;  // steps of this tile
-    // With rep > 1 the tile holds rep copies of its QR = 128 / rep query rows;
-    // copy qcopy (warp-uniform) owns key columns qcopy * 128 / rep onwards.
-    const int rep = p.rep;
-    const int QR = C::BM / rep;
+    // With REP > 1 the tile holds REP copies of its QR = 128 / REP query rows;
+    // copy qcopy (warp-uniform) owns key columns qcopy * 128 / REP onwards.
+    constexpr int QR = C::BM / REP;
     const int qcopy = r_loc / QR;
     const int row = my_row0 + r_loc % QR;
     const uint32_t o_col = t ? C::O_COL1 : C::O_COL0;
@@ -568,12 +565,7 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       if (!ok) break;
       if (live) {
         tc_fence_after();
-        if (rep == 4)
-          ok = soft_step(std::integral_constant<int, 32>{}, step, s_col);
-        else if (rep == 2)
-          ok = soft_step(std::integral_constant<int, 64>{}, step, s_col);
-        else
-          ok = soft_step(std::integral_constant<int, 128>{}, step, s_col);
+        ok = soft_step(std::integral_constant<int, C::BN / REP>{}, step, s_col);
         if (!ok) break;
         tmem_wait_st();
         tc_fence_before();
@@ -618,7 +610,7 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         }
         if (row < Nq) p.LSE[orow_idx] = lse;
       } else {
-        const size_t part = static_cast<size_t>(blockIdx.y * rep + qcopy) * p.BH * Nq + orow_idx;
+        const size_t part = static_cast<size_t>(blockIdx.y * REP + qcopy) * p.BH * Nq + orow_idx;
         float* orow = p.O_part + part * D;
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
@@ -639,7 +631,7 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       }
     } else if (partial && my_nkv == 0 && row < Nq) {
       // The split holds no key this tile's rows see.
-      p.LSE_part[static_cast<size_t>(blockIdx.y * rep + qcopy) * p.BH * Nq +
+      p.LSE_part[static_cast<size_t>(blockIdx.y * REP + qcopy) * p.BH * Nq +
                  static_cast<size_t>(bh) * Nq + row] = -INFINITY;
     }
   }
