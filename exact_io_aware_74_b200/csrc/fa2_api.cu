@@ -199,10 +199,23 @@ int launch_fwd_any(bool bf, bool causal, int rep, const CUtensorMap& mq, const C
 template <int D, bool BF16>
 int launch_combine(const float* O_part, const float* LSE_part, void* O, float* LSE,
                    long long rows, int n_split, cudaStream_t stream) {
-  const unsigned int grid = static_cast<unsigned int>((rows + 7) / 8);
-  fa2::fa2_decode_combine_kernel<D, BF16><<<grid, 256, 0, stream>>>(O_part, LSE_part, O, LSE, rows,
-                                                                  n_split);
-  if (cudaGetLastError() != cudaSuccess) return FA2_ERR_CUDA;
+  // Programmatic serialisation: the merge may launch while the forward runs and
+  // waits on the device (griddepcontrol.wait) for it to finish.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned int>((rows + 7) / 8));
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, fa2::fa2_decode_combine_kernel<D, BF16>, O_part, LSE_part, O, LSE,
+                         rows, n_split) != cudaSuccess) {
+    cudaGetLastError();
+    return FA2_ERR_CUDA;
+  }
   g_launches.fetch_add(1);
   return FA2_OK;
 }

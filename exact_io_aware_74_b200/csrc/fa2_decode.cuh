@@ -35,12 +35,16 @@ inline size_t decode_workspace_bytes(size_t S, size_t BH, size_t Nq, int D) {
 }
 
 // One warp per output row (bh, i); lane c owns D/32 consecutive columns.
+// Launched behind the forward with programmatic serialisation: it may start
+// while the forward still runs and waits for it before touching the partials.
 template <int D, bool BF16>
 __global__ void __launch_bounds__(256)
 fa2_decode_combine_kernel(const float* __restrict__ O_part, const float* __restrict__ LSE_part,
                           void* __restrict__ O, float* __restrict__ LSE, long long rows,
                           int n_split) {
   constexpr int PER = D / 32;  // columns per lane: 4 (D = 128) or 2 (D = 64)
+  constexpr int U = 8;         // partial rows in flight per lane
+  griddep_wait();
   const long long row = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= rows) return;  // whole warp leaves together
@@ -57,27 +61,38 @@ fa2_decode_combine_kernel(const float* __restrict__ O_part, const float* __restr
   float wsum = 0.f;
   if (M != -INFINITY) {
     for (int s0 = 0; s0 < n_split; s0 += 32) {
-      // Lane c weighs split s0 + c; the weights are then broadcast one by one.
+      // Lane c weighs split s0 + c; the weights are then broadcast, and U
+      // partial rows are loaded before any is used.  A split the row sees no
+      // key of has weight 0 and its (unwritten) partial row is not read.
       const int s = s0 + lane;
       const float L = (s < n_split) ? LSE_part[s * rows + row] : -INFINITY;
       const float w = (L == -INFINITY) ? 0.f : exp2f((L - M) * kLog2e);
       wsum += w;
       const int cnt = min(32, n_split - s0);
-      for (int c = 0; c < cnt; ++c) {
-        const float wc = __shfl_sync(0xffffffffu, w, c);
-        if (wc == 0.f) continue;  // warp-uniform: every lane holds the same wc
-        const float* src = O_part + ((s0 + c) * rows + row) * D + lane * PER;
-        if constexpr (PER == 4) {
-          const float4 v = *reinterpret_cast<const float4*>(src);
-          acc[0] += wc * v.x;
-          acc[1] += wc * v.y;
-          acc[2] += wc * v.z;
-          acc[3] += wc * v.w;
-        } else {
-          const float2 v = *reinterpret_cast<const float2*>(src);
-          acc[0] += wc * v.x;
-          acc[1] += wc * v.y;
+      for (int c0 = 0; c0 < cnt; c0 += U) {
+        float wc[U], v[U][PER];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          const int c = c0 + u;
+          wc[u] = __shfl_sync(0xffffffffu, w, c & 31);
+          if (c >= cnt) wc[u] = 0.f;
+#pragma unroll
+          for (int i = 0; i < PER; ++i) v[u][i] = 0.f;
+          if (wc[u] != 0.f) {  // warp-uniform
+            const float* src = O_part + ((s0 + c) * rows + row) * D + lane * PER;
+            if constexpr (PER == 4) {
+              const float4 t = *reinterpret_cast<const float4*>(src);
+              v[u][0] = t.x; v[u][1] = t.y; v[u][2] = t.z; v[u][3] = t.w;
+            } else {
+              const float2 t = *reinterpret_cast<const float2*>(src);
+              v[u][0] = t.x; v[u][1] = t.y;
+            }
+          }
         }
+#pragma unroll
+        for (int u = 0; u < U; ++u)
+#pragma unroll
+          for (int i = 0; i < PER; ++i) acc[i] = fmaf(wc[u], v[u][i], acc[i]);
       }
     }
 #pragma unroll

@@ -131,6 +131,10 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
 
+  // A merge kernel queued behind this grid (decode-like calls) may launch now:
+  // it waits for this grid's completion before reading anything.
+  griddep_launch_dependents();
+
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int Nq = p.Nq, Nk = p.Nk;

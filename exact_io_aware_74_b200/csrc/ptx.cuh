@@ -228,6 +228,17 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// Programmatic dependent launch.  launch_dependents: this CTA no longer holds
+// back the launch of a grid queued behind it with programmatic serialisation.
+// dep_wait: blocks until the grid this one depends on has completed and its
+// memory writes are visible (returns at once without such a dependency).
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 // ------------------------------------------------------------------------------------
 // tensor memory
 // ------------------------------------------------------------------------------------
