@@ -56,16 +56,27 @@ bool overlaps(const void* a, size_t a_bytes, const void* b, size_t b_bytes) {
   return x < y + b_bytes && y < x + a_bytes;
 }
 
+// Head dims: multiples of 8 (16-byte rows for TMA) up to 256 in the forward and
+// 128 in the backward.
+constexpr int kMaxFwdHeadDim = 256;
+constexpr int kMaxBwdHeadDim = 128;
+
 // Common checks of fa2_fwd / fa2_bwd that need no CUDA call.
-int check_sizes(int B, int H, int N, int d, float scale, int causal, int dtype) {
+int check_sizes(int B, int H, int N, int d, float scale, int causal, int dtype,
+                int max_d = kMaxFwdHeadDim) {
   if (B < 1 || H < 1 || N < 1) return FA2_ERR_INVALID_ARG;
   if (causal != 0 && causal != 1) return FA2_ERR_INVALID_ARG;
   if (dtype != FA2_FP16 && dtype != FA2_BF16) return FA2_ERR_INVALID_ARG;
   if (!std::isfinite(scale) || !(scale > 0.f)) return FA2_ERR_INVALID_ARG;
   if (static_cast<long long>(B) * H > (1ll << 30) || N > (1 << 30)) return FA2_ERR_INVALID_ARG;
-  if (d != 64 && d != 128) return FA2_ERR_UNSUPPORTED;
+  if (d < 8 || d > max_d || d % 8 != 0) return FA2_ERR_UNSUPPORTED;
   return FA2_OK;
 }
+
+// Forward kernel head dim (tile width) for head dim d: the next of 64, 128, 192, 256.
+int fwd_tile_dim(int d) { return d <= 64 ? 64 : (d <= 128 ? 128 : (d <= 192 ? 192 : 256)); }
+// Query rows per forward CTA: two 128-row tiles up to a tile width of 128, one above.
+int fwd_rows_per_cta(int d) { return fwd_tile_dim(d) <= 128 ? 256 : 128; }
 
 // Current device must be compute capability 10.0; returns its ordinal in *dev.
 int check_device(int* dev) {
@@ -198,7 +209,7 @@ int launch_fwd_any(bool bf, bool causal, int rep, const CUtensorMap& mq, const C
 
 template <int D, bool BF16>
 int launch_combine(const float* O_part, const float* LSE_part, void* O, float* LSE,
-                   long long rows, int n_split, cudaStream_t stream) {
+                   long long rows, int n_split, int d, cudaStream_t stream) {
   // Programmatic serialisation: the merge may launch while the forward runs and
   // waits on the device (griddepcontrol.wait) for it to finish.
   cudaLaunchConfig_t cfg = {};
@@ -212,7 +223,7 @@ int launch_combine(const float* O_part, const float* LSE_part, void* O, float* L
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   if (cudaLaunchKernelEx(&cfg, fa2::fa2_decode_combine_kernel<D, BF16>, O_part, LSE_part, O, LSE,
-                         rows, n_split) != cudaSuccess) {
+                         rows, n_split, d) != cudaSuccess) {
     cudaGetLastError();
     return FA2_ERR_CUDA;
   }
@@ -254,11 +265,12 @@ int fwd_core(const void* Q, const void* K, const void* V, void* O, float* LSE, i
   fa2::FwdParams p{};
   p.O = O;
   p.LSE = LSE;
+  p.d = d;
   p.Nq = Nq;
   p.Nk = Nk;
   p.off = Nk - Nq;
   p.BH = BH;
-  p.n_qblk = (Nq + 255) / 256;
+  p.n_qblk = (Nq + fwd_rows_per_cta(d) - 1) / fwd_rows_per_cta(d);
   p.scale_log2 = scale * 1.4426950408889634f;
   p.status = st;
   p.wait_ns = wait_ns();
@@ -269,15 +281,25 @@ int fwd_core(const void* Q, const void* K, const void* V, void* O, float* LSE, i
   p.LSE_part = n_part > 1 ? LSE_part : nullptr;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const bool bf = dtype == FA2_BF16;
-  rc = (d == 64) ? launch_fwd_any<64>(bf, causal != 0, rep, mq, mk, mv, mqr, p, n_split, s)
-                 : launch_fwd_any<128>(bf, causal != 0, rep, mq, mk, mv, mqr, p, n_split, s);
+  const bool ca = causal != 0;
+  switch (fwd_tile_dim(d)) {
+    case 64: rc = launch_fwd_any<64>(bf, ca, rep, mq, mk, mv, mqr, p, n_split, s); break;
+    case 128: rc = launch_fwd_any<128>(bf, ca, rep, mq, mk, mv, mqr, p, n_split, s); break;
+    case 192: rc = launch_fwd_any<192>(bf, ca, rep, mq, mk, mv, mqr, p, n_split, s); break;
+    default: rc = launch_fwd_any<256>(bf, ca, rep, mq, mk, mv, mqr, p, n_split, s); break;
+  }
   if (rc != FA2_OK || n_part == 1) return rc;
   const long long rows = static_cast<long long>(BH) * Nq;
-  if (d == 64)
-    return bf ? launch_combine<64, true>(O_part, LSE_part, O, LSE, rows, n_part, s)
-              : launch_combine<64, false>(O_part, LSE_part, O, LSE, rows, n_part, s);
-  return bf ? launch_combine<128, true>(O_part, LSE_part, O, LSE, rows, n_part, s)
-            : launch_combine<128, false>(O_part, LSE_part, O, LSE, rows, n_part, s);
+#define FA2_COMBINE(D_)                                                                   \
+  return bf ? launch_combine<D_, true>(O_part, LSE_part, O, LSE, rows, n_part, d, s)      \
+            : launch_combine<D_, false>(O_part, LSE_part, O, LSE, rows, n_part, d, s)
+  switch (fwd_tile_dim(d)) {
+    case 64: FA2_COMBINE(64);
+    case 128: FA2_COMBINE(128);
+    case 192: FA2_COMBINE(192);
+    default: FA2_COMBINE(256);
+  }
+#undef FA2_COMBINE
 }
 
 // Shared by fa2_fwd and fa2_fwd_window; window = 0 means no sliding window.
@@ -351,7 +373,8 @@ int fa2_fwd_decode_splits(int B, int H, int Nq, int Nk, int d, int sm_count) {
   // many splits as still fit the CTAs in one wave, and at least 4 key tiles per
   // split: measured on B200, a second wave or shorter stretches cost more in
   // per-CTA set-up and the merge than they gain in parallelism.
-  const long long ctas = static_cast<long long>((Nq + 255) / 256) * B * H;
+  const long long ctas = static_cast<long long>((Nq + fwd_rows_per_cta(d) - 1) /
+                                               fwd_rows_per_cta(d)) * B * H;
   const int n_kv = (Nq > 0) ? (Nk + 127) / 128 : 1;
   long long sp = sm_count / ctas;
   const long long cap = n_kv / 4;
@@ -367,7 +390,7 @@ size_t fa2_fwd_decode_workspace_size(int B, int H, int Nq, int Nk, int d, int n_
   const int parts = effective_splits((Nk + 127) / 128, n_splits) * decode_rep(Nq);
   if (parts == 1) return 0;
   return fa2::decode_workspace_bytes(static_cast<size_t>(parts), static_cast<size_t>(B) * H,
-                                     static_cast<size_t>(Nq), d);
+                                     static_cast<size_t>(Nq), fwd_tile_dim(d));
 }
 
 int fa2_fwd_decode(const void* Q, const void* K, const void* V, void* O, float* LSE, int B,
@@ -396,7 +419,7 @@ int fa2_fwd_decode(const void* Q, const void* K, const void* V, void* O, float* 
   float* LSE_part = nullptr;
   if (parts > 1) {
     const size_t need = fa2::decode_workspace_bytes(static_cast<size_t>(parts),
-                                                    static_cast<size_t>(BH), Nq, d);
+                                                    static_cast<size_t>(BH), Nq, fwd_tile_dim(d));
     if (!workspace || workspace_bytes < need ||
         (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
       return FA2_ERR_WORKSPACE;
@@ -407,14 +430,15 @@ int fa2_fwd_decode(const void* Q, const void* K, const void* V, void* O, float* 
     O_part = static_cast<float*>(workspace);
     LSE_part = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
                                         fa2::decode_opart_bytes(static_cast<size_t>(parts),
-                                                                static_cast<size_t>(BH), Nq, d));
+                                                                static_cast<size_t>(BH), Nq,
+                                                                fwd_tile_dim(d)));
   }
   return fwd_core(Q, K, V, O, LSE, BH, Nq, Nk, d, scale, causal, 0, dtype, eff,
                   kv_tiles_per_split(n_kv, n_splits), rep, O_part, LSE_part, stream);
 }
 
 size_t fa2_bwd_workspace_size(int B, int H, int N, int d) {
-  if (check_sizes(B, H, N, d, 1.0f, 0, FA2_BF16) != FA2_OK) return 0;
+  if (check_sizes(B, H, N, d, 1.0f, 0, FA2_BF16, kMaxBwdHeadDim) != FA2_OK) return 0;
   return fa2::bwd_workspace_bytes(static_cast<size_t>(B) * H, N, d);
 }
 
@@ -431,7 +455,7 @@ int bwd_impl(const void* Q, const void* K, const void* V, const void* O, const v
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(dO) ||
       !aligned16(LSE) || !aligned16(dQ) || !aligned16(dK) || !aligned16(dV))
     return FA2_ERR_INVALID_ARG;
-  int rc = check_sizes(B, H, N, d, scale, causal, dtype);
+  int rc = check_sizes(B, H, N, d, scale, causal, dtype, kMaxBwdHeadDim);
   if (rc != FA2_OK) return rc;
   const int BH = B * H;
   const size_t bytes = static_cast<size_t>(BH) * N * d * 2;
@@ -536,7 +560,7 @@ int fa2_bwd_noalloc(const void* Q, const void* K, const void* V, const void* O, 
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(dO) ||
       !aligned16(LSE) || !aligned16(dQ) || !aligned16(dK) || !aligned16(dV))
     return FA2_ERR_INVALID_ARG;
-  int rc = check_sizes(B, H, N, d, scale, causal, dtype);
+  int rc = check_sizes(B, H, N, d, scale, causal, dtype, kMaxBwdHeadDim);
   if (rc != FA2_OK) return rc;
   const int BH = B * H;
   const size_t bytes = static_cast<size_t>(BH) * N * d * 2;

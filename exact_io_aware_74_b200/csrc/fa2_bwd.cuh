@@ -48,13 +48,17 @@ namespace fa2 {
 
 constexpr int kBwdKernelsPerCall = 3;
 
-// Workspace: D [BH][Npad] f32 | L2 = LSE*log2(e) [BH][Npad] f32 | dQacc [BH][N][d] f32.
+// Workspace: D [BH][Npad] f32 | L2 = LSE*log2(e) [BH][Npad] f32 | dQacc [BH][N][Dt] f32,
+// Dt the kernel's tile head dim (64 or 128).
 inline size_t bwd_npad(int N) { return (static_cast<size_t>(N) + 127) / 128 * 128; }
 inline size_t bwd_rowstat_bytes(size_t BH, int N) {
   return (2 * BH * bwd_npad(N) * 4 + 255) / 256 * 256;
 }
+// Kernel head dim for a head dim d <= 128: the tiles are 64 or 128 columns wide.
+inline int bwd_tile_dim(int d) { return d <= 64 ? 64 : 128; }
 inline size_t bwd_workspace_bytes(size_t BH, int N, int d) {
-  return bwd_rowstat_bytes(BH, N) + (BH * static_cast<size_t>(N) * d * 4 + 255) / 256 * 256;
+  return bwd_rowstat_bytes(BH, N) +
+         (BH * static_cast<size_t>(N) * bwd_tile_dim(d) * 4 + 255) / 256 * 256;
 }
 
 // ------------------------------------------------------------------------------------
@@ -66,7 +70,7 @@ __global__ void __launch_bounds__(256)
 fa2_bwd_pre_kernel(const uint16_t* __restrict__ O, const uint16_t* __restrict__ dO,
                    const float* __restrict__ LSE, float* __restrict__ Dg,
                    float* __restrict__ Lg, float* __restrict__ dQacc, int N, int Npad,
-                   long long total_rows) {
+                   long long total_rows, int d) {
   constexpr int TPR = D / 8;  // threads per row, 8 elements (16 bytes) each
   constexpr int RPB = 256 / TPR;
   const int sub = threadIdx.x % TPR;
@@ -75,8 +79,8 @@ fa2_bwd_pre_kernel(const uint16_t* __restrict__ O, const uint16_t* __restrict__ 
   const long long bh = in_range ? r / Npad : 0;
   const int q = in_range ? static_cast<int>(r % Npad) : N;
   float acc = 0.f;
-  if (q < N) {
-    const size_t off = (static_cast<size_t>(bh) * N + q) * D + sub * 8;
+  if (q < N && sub * 8 < d) {  // O, dO rows have d (a multiple of 8) columns
+    const size_t off = (static_cast<size_t>(bh) * N + q) * d + sub * 8;
     const uint4 a = *reinterpret_cast<const uint4*>(O + off);
     const uint4 b = *reinterpret_cast<const uint4*>(dO + off);
     const uint32_t* pa = reinterpret_cast<const uint32_t*>(&a);
@@ -96,7 +100,9 @@ fa2_bwd_pre_kernel(const uint16_t* __restrict__ O, const uint16_t* __restrict__ 
       acc = fmaf(a0, b0, acc);
       acc = fmaf(a1, b1, acc);
     }
-    float4* z = reinterpret_cast<float4*>(dQacc + off);
+  }
+  if (q < N) {  // the accumulator has D columns, the padding included
+    float4* z = reinterpret_cast<float4*>(dQacc + (static_cast<size_t>(bh) * N + q) * D + sub * 8);
     z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
     z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
   }
@@ -115,9 +121,14 @@ fa2_bwd_pre_kernel(const uint16_t* __restrict__ O, const uint16_t* __restrict__ 
 template <bool BF16>
 __global__ void __launch_bounds__(256)
 fa2_bwd_dq_kernel(const float* __restrict__ dQacc, uint16_t* __restrict__ dQ, float scale,
-                  long long n8) {
+                  long long n8, int D, int d) {
+  // Thread i converts 8 accumulator columns (group i % (D/8) of row i / (D/8));
+  // groups past the head dim d are padding and are dropped.
   const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (i >= n8) return;
+  const long long row = i / (D / 8);
+  const int g = static_cast<int>(i % (D / 8));
+  if (g * 8 >= d) return;
   const float4 a = reinterpret_cast<const float4*>(dQacc)[2 * i];
   const float4 b = reinterpret_cast<const float4*>(dQacc)[2 * i + 1];
   uint4 out;
@@ -125,7 +136,7 @@ fa2_bwd_dq_kernel(const float* __restrict__ dQacc, uint16_t* __restrict__ dQ, fl
   out.y = pack2<BF16>(a.z * scale, a.w * scale);
   out.z = pack2<BF16>(b.x * scale, b.y * scale);
   out.w = pack2<BF16>(b.z * scale, b.w * scale);
-  reinterpret_cast<uint4*>(dQ)[i] = out;
+  *reinterpret_cast<uint4*>(dQ + row * d + g * 8) = out;
 }
 
 // ------------------------------------------------------------------------------------
@@ -135,9 +146,10 @@ fa2_bwd_dq_kernel(const float* __restrict__ dQacc, uint16_t* __restrict__ dQ, fl
 struct BwdParams {
   const float* Dg;    // [BH][Npad]
   const float* Lg;    // [BH][Npad]
-  float* dQacc;       // [BH][N][D]
-  void* dK;           // [BH][N][D] 16-bit
-  void* dV;           // [BH][N][D] 16-bit
+  float* dQacc;       // [BH][N][D] (D columns, the padding included)
+  void* dK;           // [BH][N][d] 16-bit
+  void* dV;           // [BH][N][d] 16-bit
+  int d;              // head dim (multiple of 8, <= D); tile columns past d are zero fill
   int N, Npad, BH, n_kv;
   int window;         // causal only: query i sees keys i-window+1..i (0 = no window)
   float scale, scale_log2;
@@ -555,8 +567,9 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       tc_fence_after();
       const uint32_t col = g ? C::C_DK : C::C_DV;
       const float mul = g ? p.scale : 1.0f;
+      const int d = p.d;
       uint8_t* row = reinterpret_cast<uint8_t*>(g ? p.dK : p.dV) +
-                     (static_cast<size_t>(bh) * N + key) * (D * 2);
+                     (static_cast<size_t>(bh) * N + key) * (d * 2);
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t rr[32];
@@ -571,7 +584,8 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         if (key < N) {
           uint4* dst4 = reinterpret_cast<uint4*>(row + c * 64);
 #pragma unroll
-          for (int e = 0; e < 4; ++e) dst4[e] = v[e];
+          for (int e = 0; e < 4; ++e)
+            if (c * 32 + 8 * e < d) dst4[e] = v[e];  // 8 columns per store; d % 8 == 0
         }
       }
     }
@@ -598,7 +612,7 @@ bool make_acc_map(CUtensorMap* map, float* base, int BH, int N, int d);
 template <int D, bool BF16, bool CAUSAL>
 int launch_bwd_t(const void* Q, const void* K, const void* V, const void* O, const void* dO,
                  const float* LSE, void* dQ, void* dK, void* dV, void* workspace, int BH, int N,
-                 float scale, int window, unsigned int* status, unsigned long long wait_ns,
+                 int d, float scale, int window, unsigned int* status, unsigned long long wait_ns,
                  cudaStream_t stream) {
   using Cfg = BwdCfg<D>;
   const int Npad = static_cast<int>(bwd_npad(N));
@@ -607,8 +621,8 @@ int launch_bwd_t(const void* Q, const void* K, const void* V, const void* O, con
   float* dQacc = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
                                           bwd_rowstat_bytes(static_cast<size_t>(BH), N));
   CUtensorMap mq, mk, mv, mdo, mdq;
-  if (!make_tile_map(&mq, Q, BH, N, D, BF16) || !make_tile_map(&mk, K, BH, N, D, BF16) ||
-      !make_tile_map(&mv, V, BH, N, D, BF16) || !make_tile_map(&mdo, dO, BH, N, D, BF16) ||
+  if (!make_tile_map(&mq, Q, BH, N, d, BF16) || !make_tile_map(&mk, K, BH, N, d, BF16) ||
+      !make_tile_map(&mv, V, BH, N, d, BF16) || !make_tile_map(&mdo, dO, BH, N, d, BF16) ||
       !make_acc_map(&mdq, dQacc, BH, N, D))
     return 4;  // FA2_ERR_CUDA
   // 1. preprocess
@@ -618,7 +632,7 @@ int launch_bwd_t(const void* Q, const void* K, const void* V, const void* O, con
     const unsigned int grid = static_cast<unsigned int>((rows + RPB - 1) / RPB);
     fa2_bwd_pre_kernel<D, BF16><<<grid, 256, 0, stream>>>(
         static_cast<const uint16_t*>(O), static_cast<const uint16_t*>(dO), LSE, Dg, Lg, dQacc, N,
-        Npad, rows);
+        Npad, rows, d);
     if (cudaGetLastError() != cudaSuccess) return 4;
   }
   // 2. main
@@ -635,6 +649,7 @@ int launch_bwd_t(const void* Q, const void* K, const void* V, const void* O, con
     bp.dQacc = dQacc;
     bp.dK = dK;
     bp.dV = dV;
+    bp.d = d;
     bp.N = N;
     bp.Npad = Npad;
     bp.BH = BH;
@@ -653,7 +668,7 @@ int launch_bwd_t(const void* Q, const void* K, const void* V, const void* O, con
     const long long n8 = static_cast<long long>(BH) * N * D / 8;
     const unsigned int grid = static_cast<unsigned int>((n8 + 255) / 256);
     fa2_bwd_dq_kernel<BF16><<<grid, 256, 0, stream>>>(dQacc, static_cast<uint16_t*>(dQ), scale,
-                                                      n8);
+                                                      n8, D, d);
     if (cudaGetLastError() != cudaSuccess) return 4;
   }
   return 0;
@@ -663,10 +678,10 @@ inline int launch_bwd(const void* Q, const void* K, const void* V, const void* O
                       const float* LSE, void* dQ, void* dK, void* dV, void* workspace, int BH,
                       int N, int d, float scale, bool causal, bool bf16, unsigned int* status,
                       unsigned long long wait_ns, cudaStream_t s, int window = 0) {
-#define FA2_BWD_CALL(D_, BF_, CA_)                                                          \
-  return launch_bwd_t<D_, BF_, CA_>(Q, K, V, O, dO, LSE, dQ, dK, dV, workspace, BH, N, scale, \
+#define FA2_BWD_CALL(D_, BF_, CA_)                                                             \
+  return launch_bwd_t<D_, BF_, CA_>(Q, K, V, O, dO, LSE, dQ, dK, dV, workspace, BH, N, d, scale, \
                                     window, status, wait_ns, s)
-  if (d == 64) {
+  if (d <= 64) {
     if (bf16) { if (causal) FA2_BWD_CALL(64, true, true); FA2_BWD_CALL(64, true, false); }
     if (causal) FA2_BWD_CALL(64, false, true);
     FA2_BWD_CALL(64, false, false);

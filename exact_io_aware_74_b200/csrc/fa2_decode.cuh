@@ -34,15 +34,16 @@ inline size_t decode_workspace_bytes(size_t S, size_t BH, size_t Nq, int D) {
   return decode_opart_bytes(S, BH, Nq, D) + (S * BH * Nq * 4 + 255) / 256 * 256;
 }
 
-// One warp per output row (bh, i); lane c owns D/32 consecutive columns.
+// One warp per output row (bh, i); lane c owns D/32 consecutive columns of the
+// D-column partials and writes those below the head dim d (a multiple of 8).
 // Launched behind the forward with programmatic serialisation: it may start
 // while the forward still runs and waits for it before touching the partials.
 template <int D, bool BF16>
 __global__ void __launch_bounds__(256)
 fa2_decode_combine_kernel(const float* __restrict__ O_part, const float* __restrict__ LSE_part,
                           void* __restrict__ O, float* __restrict__ LSE, long long rows,
-                          int n_split) {
-  constexpr int PER = D / 32;  // columns per lane: 4 (D = 128) or 2 (D = 64)
+                          int n_split, int d) {
+  constexpr int PER = D / 32;  // columns per lane: 2, 4, 6 or 8
   constexpr int U = 8;         // partial rows in flight per lane
   griddep_wait();
   const long long row = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
@@ -80,12 +81,11 @@ fa2_decode_combine_kernel(const float* __restrict__ O_part, const float* __restr
           for (int i = 0; i < PER; ++i) v[u][i] = 0.f;
           if (wc[u] != 0.f) {  // warp-uniform
             const float* src = O_part + ((s0 + c) * rows + row) * D + lane * PER;
-            if constexpr (PER == 4) {
-              const float4 t = *reinterpret_cast<const float4*>(src);
-              v[u][0] = t.x; v[u][1] = t.y; v[u][2] = t.z; v[u][3] = t.w;
-            } else {
-              const float2 t = *reinterpret_cast<const float2*>(src);
-              v[u][0] = t.x; v[u][1] = t.y;
+#pragma unroll
+            for (int i = 0; i < PER / 2; ++i) {  // 8-byte aligned pairs
+              const float2 t = reinterpret_cast<const float2*>(src)[i];
+              v[u][2 * i] = t.x;
+              v[u][2 * i + 1] = t.y;
             }
           }
         }
@@ -102,11 +102,10 @@ fa2_decode_combine_kernel(const float* __restrict__ O_part, const float* __restr
   uint32_t packed[PER / 2];
 #pragma unroll
   for (int i = 0; i < PER / 2; ++i) packed[i] = pack2<BF16>(acc[2 * i] * inv, acc[2 * i + 1] * inv);
-  uint8_t* dst = static_cast<uint8_t*>(O) + (row * D + lane * PER) * 2;
-  if constexpr (PER == 4)
-    *reinterpret_cast<uint2*>(dst) = make_uint2(packed[0], packed[1]);
-  else
-    *reinterpret_cast<uint32_t*>(dst) = packed[0];
+  uint32_t* dst = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(O) + (row * d + lane * PER) * 2);
+#pragma unroll
+  for (int i = 0; i < PER / 2; ++i)
+    if (lane * PER + 2 * i < d) dst[i] = packed[i];  // d is even: whole pairs
   if (lane == 0) LSE[row] = (wsum > 0.f) ? M + logf(wsum) : -INFINITY;
 }
 

@@ -47,13 +47,15 @@
 namespace fa2 {
 
 struct FwdParams {
-  void* O;                     // [BH][Nq][D] 16-bit (unused when the keys are split)
+  void* O;                     // [BH][Nq][d] 16-bit (unused when the keys are split)
   float* LSE;                  // [BH][Nq]            (unused when the keys are split)
+  int d;                       // head dim, a multiple of 8, D - 64 < d <= D (columns past d
+                               // of the tiles are TMA zero fill and are never stored)
   int Nq;                      // query rows per (batch, head)
   int Nk;                      // key / value rows per (batch, head)
   int off;                     // causal only: query row i sees keys <= i + off (Nk - Nq)
   int BH;                      // batch * heads
-  int n_qblk;                  // ceil(Nq / 256)
+  int n_qblk;                  // ceil(Nq / (128 QT)): query blocks per (batch, head)
   float scale_log2;            // scale * log2(e)
   unsigned int* status;        // device status word
   unsigned long long wait_ns;  // budget of one bounded wait
@@ -61,7 +63,8 @@ struct FwdParams {
   int window;                  // causal only: row i sees keys i+off-window+1..i+off (0 = none)
   // Split keys (blockIdx.y = split): CTA y covers key tiles [y kv_per_split,
   // (y + 1) kv_per_split) and writes its rows' partial results, normalised by
-  // its own row sums, to O_part [split][BH][Nq][D] and LSE_part [split][BH][Nq]
+  // its own row sums, to O_part [split][BH][Nq][D] (D columns, the padding
+  // included) and LSE_part [split][BH][Nq]
   // (float, -inf for a row that sees no key of the split).  kv_per_split = 0:
   // all key tiles.  O_part = nullptr: O and LSE are written directly.
   int kv_per_split;
@@ -71,15 +74,23 @@ struct FwdParams {
 
 template <int D>
 struct FwdCfg {
+  static_assert(D == 64 || D == 128 || D == 192 || D == 256, "tile head dims");
   static constexpr int BM = 128;                  // query rows per tile
   static constexpr int BN = 128;                  // keys per tile
-  static constexpr int QT = 2;                    // query tiles per CTA
+  // Query tiles per CTA: two (ping-pong) up to D = 128; one above, where two
+  // D-column output accumulators and two S blocks would exceed TMEM's 512
+  // columns (S double buffer 256 + O D <= 512 still fits).
+  static constexpr int QT = (D <= 128) ? 2 : 1;
   static constexpr int KCH = D / 64;              // 128-byte swizzle chunks along d
   static constexpr int CHUNK = 128 * 128;         // bytes of one 128-row x 64-col chunk
   static constexpr int TILE = 128 * D * 2;        // bytes of one 128-row tile
-  static constexpr int KS = (D == 64) ? 4 : 2;    // K ring stages
-  static constexpr int VS = (D == 64) ? 4 : 2;    // V ring stages
+  // K and V ring stages within 227 KB of shared memory.
+  static constexpr int KS = (D == 64) ? 4 : (D == 256 ? 1 : 2);
+  static constexpr int VS = (D == 64) ? 4 : (D == 128 ? 2 : 1);
+  // With one query tile in the CTA, the second Q slot (if any) is one more V stage.
+  static constexpr int VX = (QT == 2) ? 1 : 0;
   static constexpr int SMEM = (QT + KS + VS) * TILE + 1024;
+  static_assert(SMEM <= 227 * 1024, "shared memory");
   static constexpr int THREADS = 384;
   static constexpr int LAUNCH_REGS = 168;  // per thread, as compiled (checked on the host)
 #ifndef FA2_FWD_SOFT_REGS
@@ -126,7 +137,8 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   uint8_t* sK = sQ + C::QT * C::TILE;
   uint8_t* sV = sK + C::KS * C::TILE;
 
-  __shared__ uint64_t bar_q, k_full[C::KS], k_empty[C::KS], v_full[C::VS + 1], v_empty[C::VS + 1];
+  __shared__ uint64_t bar_q, k_full[C::KS], k_empty[C::KS], v_full[C::VS + C::VX],
+      v_empty[C::VS + C::VX];
   __shared__ uint64_t s_full[2], p_ready[2], o_done[2], drain;
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
@@ -156,9 +168,9 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   int row0[2], j_lo[2], j_hi[2];
 #pragma unroll
   for (int t = 0; t < 2; ++t) {
-    row0[t] = qb * 256 + t * 128;
+    row0[t] = qb * (C::QT * C::BM) + t * C::BM;
     j_lo[t] = 0;
-    if (row0[t] >= Nq) {
+    if (row0[t] >= Nq || t >= C::QT) {
       j_hi[t] = 0;
     } else if (CAUSAL) {
       j_hi[t] = min(n_kv_all, (min(row0[t] + C::BM - 1, Nq - 1) + off) / C::BN + 1);
@@ -176,7 +188,7 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   const int j1 = max(j_hi[0], j_hi[1]);
   const int n_steps = j1 - j0;
   // A CTA with one query tile runs it double-buffered (see the MMA issuer).
-  const bool single = !has1;
+  const bool single = C::QT == 1 || !has1;
 
   WaitCtl wc{p.status, &abort_flag, p.wait_ns};
 
@@ -184,7 +196,7 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     abort_flag = 0;
     mbar_init(&bar_q, 1);
     for (int s = 0; s < C::KS; ++s) { mbar_init(&k_full[s], 1); mbar_init(&k_empty[s], 1); }
-    for (int s = 0; s <= C::VS; ++s) { mbar_init(&v_full[s], 1); mbar_init(&v_empty[s], 1); }
+    for (int s = 0; s < C::VS + C::VX; ++s) { mbar_init(&v_full[s], 1); mbar_init(&v_empty[s], 1); }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&s_full[t], 1);
       mbar_init(&p_ready[t], 4);
@@ -234,8 +246,8 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             tma_load_3d(sQ + t * C::TILE + c * C::CHUNK, &tmQ, &bar_q, c * 64, row0[t], bh);
         }
       }
-      // With one query tile the second Q slot is one more V stage.
-      const int vring = single ? C::VS + 1 : C::VS;
+      // With one query tile the second Q slot (if any) is one more V stage.
+      const int vring = single ? C::VS + C::VX : C::VS;
       int k_issued = 0, v_issued = 0;  // loads issued so far
       auto load_k = [&](int jj) -> bool {
         const int ks = jj % C::KS;
@@ -340,7 +352,7 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             umma_commit(&s_full[b ^ 1]);
             umma_commit(&k_empty[ks1]);
           }
-          constexpr int VR = C::VS + 1;  // V ring with the second Q slot
+          constexpr int VR = C::VS + C::VX;  // V ring with the second Q slot
           const int vs = jj % VR;
           if (!mbar_wait(&v_full[vs], (jj / VR) & 1, wc, kSiteMmaV) ||
               !mbar_wait(&p_ready[b], (jj >> 1) & 1, wc, kSiteMmaP)) {
@@ -593,7 +605,8 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       const float lse = (l > 0.f) ? (m + __log2f(l)) * 0.69314718055994531f : -INFINITY;
       const size_t orow_idx = static_cast<size_t>(bh) * Nq + row;
       if (!partial) {
-        uint8_t* orow = reinterpret_cast<uint8_t*>(p.O) + orow_idx * (D * 2);
+        const int d = p.d;
+        uint8_t* orow = reinterpret_cast<uint8_t*>(p.O) + orow_idx * (d * 2);
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t r[32];
@@ -609,7 +622,8 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           if (row < Nq) {
             uint4* dst = reinterpret_cast<uint4*>(orow + c * 64);
 #pragma unroll
-            for (int i = 0; i < 4; ++i) dst[i] = v[i];
+            for (int i = 0; i < 4; ++i)
+              if (c * 32 + 8 * i < d) dst[i] = v[i];  // 8 columns per store; d % 8 == 0
           }
         }
         if (row < Nq) p.LSE[orow_idx] = lse;
@@ -633,8 +647,9 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         }
         if (row < Nq) p.LSE_part[part] = lse;
       }
-    } else if (partial && my_nkv == 0 && row < Nq) {
-      // The split holds no key this tile's rows see.
+    } else if (partial && my_nkv == 0 && row < Nq && t < C::QT) {
+      // The split holds no key this tile's rows see.  (With one query tile per
+      // CTA, the second warpgroup's rows belong to the next CTA: it writes nothing.)
       p.LSE_part[static_cast<size_t>(blockIdx.y * REP + qcopy) * p.BH * Nq +
                  static_cast<size_t>(bh) * Nq + row] = -INFINITY;
     }

@@ -57,8 +57,10 @@ P = 1 << 20  # a fake, 16-byte aligned "device pointer": never dereferenced on t
     ((P, P, P, 2 * P, 3 * P, 1, 1, 64, 64, float("nan"), 0, 1), fa2.FA2_ERR_INVALID_ARG),
     ((P, P, P, 2 * P, 3 * P, 1, 1, 64, 64, -0.5, 0, 1), fa2.FA2_ERR_INVALID_ARG),  # scale <= 0
     ((P, P, P, P, 3 * P, 1, 1, 64, 64, 0.1, 0, 1), fa2.FA2_ERR_INVALID_ARG),     # O aliases Q
-    ((P, P, P, 2 * P, 3 * P, 1, 1, 64, 96, 0.1, 0, 1), fa2.FA2_ERR_UNSUPPORTED),  # d = 96
-    ((P, P, P, 2 * P, 3 * P, 1, 1, 64, 256, 0.1, 0, 1), fa2.FA2_ERR_UNSUPPORTED),
+    ((P, P, P, 2 * P, 3 * P, 1, 1, 64, 100, 0.1, 0, 1), fa2.FA2_ERR_UNSUPPORTED),  # d % 8 != 0
+    ((P, P, P, 2 * P, 3 * P, 1, 1, 64, 264, 0.1, 0, 1), fa2.FA2_ERR_UNSUPPORTED),  # d > 256
+    ((P, P, P, 2 * P, 3 * P, 1, 1, 64, 0, 0.1, 0, 1), fa2.FA2_ERR_UNSUPPORTED),
+    ((P, P, P, 2 * P, 3 * P, 1, 1, 64, 4, 0.1, 0, 1), fa2.FA2_ERR_UNSUPPORTED),
 ])
 def test_fwd_validation_without_device(lib, args, expect):
     assert lib.fa2_fwd(*args, None) == expect
@@ -84,7 +86,11 @@ def test_bwd_validation_without_device(lib):
     assert ws > 0 and ws % 256 == 0
     # D and LSE*log2(e) padded to 128 rows per head, then the fp32 dQ accumulator
     assert ws >= 2 * 3 * 1000 * 128 * 4
-    assert fa2.fa2_bwd_workspace_size(2, 3, 1000, 96) == 0
+    assert fa2.fa2_bwd_workspace_size(2, 3, 1000, 100) == 0  # d % 8 != 0
+    assert fa2.fa2_bwd_workspace_size(2, 3, 1000, 136) == 0  # backward head dims end at 128
+    # d = 96 runs on 128-wide tiles: the fp32 dQ accumulator has 128 columns
+    assert fa2.fa2_bwd_workspace_size(2, 3, 1000, 96) == fa2.fa2_bwd_workspace_size(2, 3, 1000, 128)
+    assert fa2.fa2_bwd_workspace_size(2, 3, 1000, 8) == fa2.fa2_bwd_workspace_size(2, 3, 1000, 64)
     ptrs = [P * (i + 1) for i in range(9)]
     # workspace too small
     rc = lib.fa2_bwd(*ptrs, 16 * P, 256, 1, 1, 64, 64, 0.1, 0, 1, None)
@@ -120,7 +126,7 @@ def test_window_validation_without_device(lib):
     args = (P, 2 * P, 3 * P, 4 * P, 5 * P, 1, 1, 64, 64, 0.1)
     assert lib.fa2_fwd_window(*args, 0, 1, None) == fa2.FA2_ERR_INVALID_ARG
     assert lib.fa2_fwd_window(*args, -5, 1, None) == fa2.FA2_ERR_INVALID_ARG
-    assert lib.fa2_fwd_window(*args[:8], 96, 0.1, 8, 1, None) == fa2.FA2_ERR_UNSUPPORTED
+    assert lib.fa2_fwd_window(*args[:8], 100, 0.1, 8, 1, None) == fa2.FA2_ERR_UNSUPPORTED
     ptrs = [P * (i + 1) for i in range(9)]
     ws = fa2.fa2_bwd_workspace_size(1, 1, 64, 64)
     assert lib.fa2_bwd_window(*ptrs, 16 * P, ws, 1, 1, 64, 64, 0.1, 0, 1, None) == fa2.FA2_ERR_INVALID_ARG
@@ -141,7 +147,8 @@ def test_decode_validation_without_device(lib):
     assert _decode(lib, splits=1025) == E
     assert _decode(lib, causal=3) == E
     assert _decode(lib, o=P) == E                 # O aliases Q
-    assert _decode(lib, d=96) == fa2.FA2_ERR_UNSUPPORTED
+    assert _decode(lib, d=100) == fa2.FA2_ERR_UNSUPPORTED
+    assert _decode(lib, d=264) == fa2.FA2_ERR_UNSUPPORTED
     # 100 queries, 1000 keys = 8 key tiles: 3 splits need a workspace
     assert _decode(lib, Nq=100, splits=3) == fa2.FA2_ERR_WORKSPACE
     need = fa2.fa2_fwd_decode_workspace_size(1, 1, 100, 1000, 64, 3)
@@ -203,6 +210,25 @@ def test_decode_split_choice(lib, shape, expect):
     assert fa2.fa2_fwd_decode_splits(*shape, 148) == expect
 
 
+def test_head_dims_pick_tile_widths(lib):
+    """Head dims up to 256 in multiples of 8: the decode partials are padded to the
+    tile width (64, 128, 192 or 256 columns), and above 128 a CTA holds one
+    128-row query tile, so a split has twice the CTAs."""
+    ws = fa2.fa2_fwd_decode_workspace_size
+    for d, tile in ((8, 64), (64, 64), (72, 128), (128, 128), (136, 192), (192, 192),
+                    (200, 256), (256, 256)):
+        assert ws(1, 1, 100, 1000, d, 2) == 2 * 100 * tile * 4 + 1024, d
+    # 300 queries: 2 CTAs per head per split at d <= 128, 3 above
+    assert fa2.fa2_fwd_decode_splits(1, 8, 300, 65536, 128, 148) == 9
+    assert fa2.fa2_fwd_decode_splits(1, 8, 300, 65536, 256, 148) == 6
+
+
+def test_bwd_rejects_head_dims_above_128(lib):
+    ptrs = [P * (i + 1) for i in range(9)]
+    assert lib.fa2_bwd(*ptrs, 16 * P, 1 << 30, 1, 1, 64, 192, 0.1, 0, 1, None) == \
+        fa2.FA2_ERR_UNSUPPORTED
+
+
 def test_decode_split_choice_rejects_bad_sizes(lib):
     assert fa2.fa2_fwd_decode_splits(1, 1, 5, 4, 64, 148) == 0
-    assert fa2.fa2_fwd_decode_splits(1, 1, 1, 4, 80, 148) == 0
+    assert fa2.fa2_fwd_decode_splits(1, 1, 1, 4, 84, 148) == 0

@@ -191,7 +191,7 @@ def test_fwd_rejects_bad_arguments_on_device():
     before = fa2.fa2_launch_count()
     lib = fa2.load()
     assert lib.fa2_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
-                       1, 1, 64, 96, 0.1, 0, fa2.FA2_BF16, None) == fa2.FA2_ERR_UNSUPPORTED
+                       1, 1, 64, 100, 0.1, 0, fa2.FA2_BF16, None) == fa2.FA2_ERR_UNSUPPORTED
     assert lib.fa2_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), q.data_ptr(), lse.data_ptr(),
                        1, 1, 64, 64, 0.1, 0, fa2.FA2_BF16, None) == fa2.FA2_ERR_INVALID_ARG
     assert fa2.fa2_launch_count() == before
