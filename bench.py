@@ -430,7 +430,7 @@ def run_ours(args):
     }
     if not args.no_extras and rank == 0:
         extras = {}
-        for name in (HEADLINE_WORKLOAD, WORKLOAD_ORDER[3], WORKLOAD_ORDER[4], WORKLOAD_ORDER[5]):
+        for name in WORKLOAD_ORDER[2:]:  # every workload but the small fp16 and the bench step
             ww = WORKLOADS[name]
             it = 10 if ww.N >= 16384 else 20
             _, f_ms, b_ms, _ = time_workload(fa2, ww, it, 3, dev, stream, None)

@@ -95,6 +95,14 @@ WORKLOADS = {
         "fwdbwd_bf16_b8h16_n4096_d128_window1024", 8, 16, 4096, 128, "bf16", True, 5,
         backward=True, input_scale=0.5, window=1024,
         note="training shape with a sliding window of 1024 keys"),
+    # Head dims other than 64 / 128: the headline shape at d = 96 (forward and
+    # backward, 128-wide tiles) and the forward at d = 256 (one query tile per CTA).
+    "fwdbwd_bf16_b2h32_n8192_d96": Workload(
+        "fwdbwd_bf16_b2h32_n8192_d96", 2, 32, 8192, 96, "bf16", False, 7, backward=True,
+        note="headline shape at head dim 96"),
+    "fwd_bf16_b2h16_n8192_d256": Workload(
+        "fwd_bf16_b2h16_n8192_d256", 2, 16, 8192, 256, "bf16", False, 8,
+        note="forward at head dim 256"),
 }
 
 WORKLOAD_ORDER = list(WORKLOADS)

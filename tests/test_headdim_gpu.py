@@ -144,3 +144,30 @@ def test_bwd_rejects_head_dims_above_128():
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     ws = torch.empty(1 << 20, dtype=torch.uint8, device="cuda")
     assert fa2.fa2_bwd(q, k, v, o, do, lse, dq, dk, dv, ws, 0.1, False) == fa2.FA2_ERR_UNSUPPORTED
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name", ["fwdbwd_bf16_b2h32_n8192_d96", "fwd_bf16_b2h16_n8192_d256"])
+def test_headdim_workloads_full_size_sampled(name):
+    """The measured head-dim workloads at full size: sampled forward rows of the
+    last head against the oracle, and (d = 96) that head's whole backward."""
+    from exact_io_aware_74_b200.workloads import WORKLOADS, workload_inputs
+    w = WORKLOADS[name]
+    x = workload_inputs(w)
+    q, k, v = (x[n].cuda() for n in ("q", "k", "v"))
+    o, lse = fa2.forward(q, k, v, w.scale, w.causal)
+    assert fa2.fa2_get_device_status() == (fa2.FA2_OK, 0)
+    bh = w.B * w.H - 1
+    b, h = divmod(bh, w.H)
+    rows = [0, 1, 127, 128, 4095, 4096, 8190, 8191]
+    ro, rl = oracle.attn_fwd_rows_ref(x["q"], x["k"], x["v"], w.scale, w.causal, bh, rows)
+    assert np.max(np.abs(o[b, h, rows].cpu().double().numpy() - ro)) <= O_TOL["bf16"]
+    assert np.max(np.abs(lse[b, h, rows].cpu().double().numpy() - rl)) <= 1e-3
+    if w.backward:
+        do = x["do"].cuda()
+        dq, dk, dv = fa2.backward(q, k, v, o, do, lse, w.scale, w.causal)
+        assert fa2.fa2_get_device_status() == (fa2.FA2_OK, 0)
+        rq, rk, rv = oracle.attn_bwd_ref(x["q"], x["k"], x["v"], x["do"], w.scale, w.causal,
+                                         heads=[bh])
+        for got, ref in ((dq, rq), (dk, rk), (dv, rv)):
+            _grad_check(got[b, h][None, None], ref[b, h][None, None])
