@@ -130,6 +130,23 @@ bool make_tile_map(CUtensorMap* map, const void* base, int BH, int N, int d, boo
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// [BH][N][d] 8-bit tensor as a 3-D TMA map with 128-row x 128-column boxes and
+// 128-byte swizzle; columns past d and rows past N read as zeros.
+bool make_u8_map(CUtensorMap* map, const void* base, int BH, int N, int d) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
+                              static_cast<cuuint64_t>(BH)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d),
+                                 static_cast<cuuint64_t>(N) * d};
+  const cuuint32_t box[3] = {128, 128, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // fp32 [BH][N][d] accumulator as a 3-D TMA map with 128-row x 32-column boxes
 // and 128-byte swizzle, for tiled reduce-adds; rows past N are clipped.
 bool make_acc_map(CUtensorMap* map, float* base, int BH, int N, int d) {
@@ -158,12 +175,12 @@ bool make_map(CUtensorMap* map, const void* base, int BH, int N, int d, int dtyp
 
 unsigned long long wait_ns() { return static_cast<unsigned long long>(g_wait_ms.load()) * 1000000ull; }
 
-template <int D, bool BF16, bool CAUSAL, int REP>
+template <int D, bool BF16, bool CAUSAL, int REP, bool F8 = false>
 int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                const CUtensorMap& mqr, const fa2::FwdParams& p, int n_split,
                cudaStream_t stream) {
-  using Cfg = fa2::FwdCfg<D>;
-  auto kern = fa2::fa2_fwd_kernel<D, BF16, CAUSAL, REP>;
+  using Cfg = fa2::FwdCfg<D, F8>;
+  auto kern = fa2::fa2_fwd_kernel<D, BF16, CAUSAL, REP, F8>;
   // The kernel re-splits its registers between warpgroups; that is only sound
   // when every thread was launched with exactly Cfg::LAUNCH_REGS registers.
   static const bool regs_ok = [&] {
@@ -435,6 +452,57 @@ int fa2_fwd_decode(const void* Q, const void* K, const void* V, void* O, float* 
   }
   return fwd_core(Q, K, V, O, LSE, BH, Nq, Nk, d, scale, causal, 0, dtype, eff,
                   kv_tiles_per_split(n_kv, n_splits), rep, O_part, LSE_part, stream);
+}
+
+int fa2_fwd_fp8(const void* Q, const void* K, const void* V, void* O, float* LSE, int B, int H,
+                int N, int d, float scale, int causal, float q_scale, float k_scale,
+                float v_scale, fa2_stream_t stream) {
+  if (!Q || !K || !V || !O || !LSE) return FA2_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(LSE))
+    return FA2_ERR_INVALID_ARG;
+  for (float f : {q_scale, k_scale, v_scale})
+    if (!std::isfinite(f) || !(f > 0.f)) return FA2_ERR_INVALID_ARG;
+  int rc = check_sizes(B, H, N, 64, scale, causal, FA2_BF16);
+  if (rc != FA2_OK) return rc;
+  if (d < 16 || d > 128 || d % 16 != 0) return FA2_ERR_UNSUPPORTED;
+  const float sl2 = scale * q_scale * k_scale * 1.4426950408889634f;
+  if (!std::isfinite(sl2) || !(sl2 > 0.f)) return FA2_ERR_INVALID_ARG;
+  const int BH = B * H;
+  const size_t in_bytes = static_cast<size_t>(BH) * N * d;  // one byte per element
+  const size_t o_bytes = in_bytes * 2;
+  const size_t lse_bytes = static_cast<size_t>(BH) * N * sizeof(float);
+  if (overlaps(O, o_bytes, Q, in_bytes) || overlaps(O, o_bytes, K, in_bytes) ||
+      overlaps(O, o_bytes, V, in_bytes) || overlaps(LSE, lse_bytes, O, o_bytes) ||
+      overlaps(LSE, lse_bytes, Q, in_bytes) || overlaps(LSE, lse_bytes, K, in_bytes) ||
+      overlaps(LSE, lse_bytes, V, in_bytes))
+    return FA2_ERR_INVALID_ARG;
+  int dev = 0;
+  rc = check_device(&dev);
+  if (rc != FA2_OK) return rc;
+  unsigned int* st = status_word(dev);
+  if (!st) return FA2_ERR_CUDA;
+  CUtensorMap mq, mk, mv;
+  if (!fa2::make_u8_map(&mq, Q, BH, N, d) || !fa2::make_u8_map(&mk, K, BH, N, d) ||
+      !fa2::make_u8_map(&mv, V, BH, N, d))
+    return FA2_ERR_CUDA;
+  fa2::FwdParams p{};
+  p.O = O;
+  p.LSE = LSE;
+  p.d = d;
+  p.Nq = N;
+  p.Nk = N;
+  p.off = 0;
+  p.BH = BH;
+  p.n_qblk = (N + 255) / 256;
+  p.scale_log2 = sl2;
+  p.status = st;
+  p.wait_ns = wait_ns();
+  p.fault = g_fault.load();
+  p.window = 0;
+  p.o_scale = v_scale;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  return causal ? launch_fwd<128, true, true, 1, true>(mq, mk, mv, mq, p, 1, s)
+                : launch_fwd<128, true, false, 1, true>(mq, mk, mv, mq, p, 1, s);
 }
 
 size_t fa2_bwd_workspace_size(int B, int H, int N, int d) {

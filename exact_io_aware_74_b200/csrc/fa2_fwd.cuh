@@ -61,6 +61,7 @@ struct FwdParams {
   unsigned long long wait_ns;  // budget of one bounded wait
   int fault;                   // test hook: 1 = skip the first K load
   int window;                  // causal only: row i sees keys i+off-window+1..i+off (0 = none)
+  float o_scale;               // 8-bit inputs: the scale of V, applied with 1/l
   // Split keys (blockIdx.y = split): CTA y covers key tiles [y kv_per_split,
   // (y + 1) kv_per_split) and writes its rows' partial results, normalised by
   // its own row sums, to O_part [split][BH][Nq][D] (D columns, the padding
@@ -72,21 +73,26 @@ struct FwdParams {
   float* LSE_part;
 };
 
-template <int D>
+template <int D, bool F8 = false>
 struct FwdCfg {
   static_assert(D == 64 || D == 128 || D == 192 || D == 256, "tile head dims");
+  static_assert(!F8 || D == 128, "8-bit inputs use 128-byte tiles");
+  static constexpr int ESZ = F8 ? 1 : 2;          // bytes per Q/K/V element
+  static constexpr int KE = 32 / ESZ;             // K elements per MMA instruction (32 bytes)
+  static constexpr int CHUNK_COLS = 128 / ESZ;    // elements per 128-byte swizzle row
   static constexpr int BM = 128;                  // query rows per tile
   static constexpr int BN = 128;                  // keys per tile
   // Query tiles per CTA: two (ping-pong) up to D = 128; one above, where two
   // D-column output accumulators and two S blocks would exceed TMEM's 512
   // columns (S double buffer 256 + O D <= 512 still fits).
   static constexpr int QT = (D <= 128) ? 2 : 1;
-  static constexpr int KCH = D / 64;              // 128-byte swizzle chunks along d
-  static constexpr int CHUNK = 128 * 128;         // bytes of one 128-row x 64-col chunk
-  static constexpr int TILE = 128 * D * 2;        // bytes of one 128-row tile
-  // K and V ring stages within 227 KB of shared memory.
-  static constexpr int KS = (D == 64) ? 4 : (D == 256 ? 1 : 2);
-  static constexpr int VS = (D == 64) ? 4 : (D == 128 ? 2 : 1);
+  static constexpr int KCH = D * ESZ / 128;       // 128-byte swizzle chunks along d
+  static constexpr int CHUNK = 128 * 128;         // bytes of one 128-row x 128-byte chunk
+  static constexpr int TILE = 128 * D * ESZ;      // bytes of one 128-row tile
+  // K and V ring stages within 227 KB of shared memory (by tile size: 16, 32,
+  // 48 or 64 KB).
+  static constexpr int KS = (TILE == 16384) ? 4 : (TILE == 65536 ? 1 : 2);
+  static constexpr int VS = (TILE == 16384) ? 4 : (TILE == 32768 ? 2 : 1);
   // With one query tile in the CTA, the second Q slot (if any) is one more V stage.
   static constexpr int VX = (QT == 2) ? 1 : 0;
   static constexpr int SMEM = (QT + KS + VS) * TILE + 1024;
@@ -119,17 +125,22 @@ enum FwdSite : uint32_t {
   kSiteMmaDrain, kSiteSoftS, kSiteSoftO, kSiteSoftOEnd, kSiteProdDrain
 };
 
+// F8: Q, K, V are E4M3 bytes (D = 128-byte tiles, REP = 1), the products are
+// kind::f8f6f4 MMAs, P is rounded to E4M3 for P V, and O is bf16 (BF16 = true);
+// the per-tensor scales of Q and K are folded into scale_log2 and that of V into
+// o_scale.
 // REP: query copies (1, 2 or 4; > 1 only with Nq <= 128 / REP and partial
 // results).  The 128-row Q tile then holds REP copies of the Nq queries, loaded
 // through tmQr (boxes of 128 / REP rows), and copy c scores only key columns
 // [c 128 / REP, (c + 1) 128 / REP) of every key tile, as partial result
 // blockIdx.y * REP + c: a lone query keeps four softmax warps busy, not one.
-template <int D, bool BF16, bool CAUSAL, int REP>
+template <int D, bool BF16, bool CAUSAL, int REP, bool F8 = false>
 __global__ void __launch_bounds__(384, 1)
 fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmQr,
                const FwdParams p) {
-  using C = FwdCfg<D>;
+  static_assert(!F8 || (BF16 && REP == 1), "8-bit inputs: bf16 output, no query copies");
+  using C = FwdCfg<D, F8>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -237,13 +248,13 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           constexpr int qr = C::BM / REP;
           for (int r = 0; r < REP; ++r)
             for (int c = 0; c < C::KCH; ++c)
-              tma_load_3d(sQ + c * C::CHUNK + r * qr * 128, &tmQr, &bar_q, c * 64, 0, bh);
+              tma_load_3d(sQ + c * C::CHUNK + r * qr * 128, &tmQr, &bar_q, c * C::CHUNK_COLS, 0, bh);
         }
       } else {
         for (int t = 0; t < 2; ++t) {
           if (j_hi[t] == 0) continue;
           for (int c = 0; c < C::KCH; ++c)
-            tma_load_3d(sQ + t * C::TILE + c * C::CHUNK, &tmQ, &bar_q, c * 64, row0[t], bh);
+            tma_load_3d(sQ + t * C::TILE + c * C::CHUNK, &tmQ, &bar_q, c * C::CHUNK_COLS, row0[t], bh);
         }
       }
       // With one query tile the second Q slot (if any) is one more V stage.
@@ -269,7 +280,7 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         uint8_t* dst = vs < C::VS ? sV + vs * C::TILE : sQ + C::TILE;
         mbar_arrive_expect_tx(&v_full[vs], C::TILE);
         for (int c = 0; c < C::KCH; ++c)
-          tma_load_3d_hint(dst + c * C::CHUNK, &tmV, &v_full[vs], c * 64, (j0 + jj) * C::BN, bh,
+          tma_load_3d_hint(dst + c * C::CHUNK, &tmV, &v_full[vs], c * C::CHUNK_COLS, (j0 + jj) * C::BN, bh,
                            keep);
         v_issued = jj + 1;
         return true;
@@ -301,29 +312,40 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   } else if (warp == 9) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t id_qk = idesc_f16(128, 128, BF16, false, false);
-      constexpr uint32_t id_pv = idesc_f16(128, D, BF16, false, true);
+      constexpr uint32_t id_qk =
+          F8 ? idesc_e4m3(128, 128, false, false) : idesc_f16(128, 128, BF16, false, false);
+      constexpr uint32_t id_pv =
+          F8 ? idesc_e4m3(128, D, false, true) : idesc_f16(128, D, BF16, false, true);
       const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV);
 
       // S = Q_t K^T into S buffer b; O_t += P_b V.
+      // K steps of 32 bytes: 4 per 128-byte swizzle row, then the next chunk.
       auto issue_qk = [&](int t, int b, int ks) {
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
+        for (int kk = 0; kk < D / C::KE; ++kk) {
           const uint32_t off = (kk >> 2) * C::CHUNK + (kk & 3) * 32;
-          umma_ss(tbase + (b ? C::S_COL1 : C::S_COL0), sdesc_sw128(sQa + t * C::TILE + off, 16, 1024),
-                  sdesc_sw128(sKa + ks * C::TILE + off, 16, 1024), id_qk, kk > 0);
+          const uint32_t dt = tbase + (b ? C::S_COL1 : C::S_COL0);
+          const uint64_t da = sdesc_sw128(sQa + t * C::TILE + off, 16, 1024);
+          const uint64_t db = sdesc_sw128(sKa + ks * C::TILE + off, 16, 1024);
+          if constexpr (F8) umma_ss_f8(dt, da, db, id_qk, kk > 0);
+          else umma_ss(dt, da, db, id_qk, kk > 0);
         }
       };
       // V ring slot vs: the V stages, then (one query tile) the second Q slot.
       auto v_addr = [&](int vs) -> uint32_t {
         return vs < C::VS ? sVa + vs * C::TILE : sQa + C::TILE;
       };
+      // P from TMEM (8 columns = 32 bytes of keys per step), V MN-major: a step
+      // of KE keys advances KE rows of 128 bytes.
       auto issue_pv = [&](int t, int b, int vs, bool acc) {
         const uint32_t va = v_addr(vs);
 #pragma unroll
-        for (int kk = 0; kk < C::BN / 16; ++kk) {
-          umma_ts(tbase + (t ? C::O_COL1 : C::O_COL0), tbase + (b ? C::S_COL1 : C::S_COL0) + kk * 8,
-                  sdesc_sw128(va + kk * 2048, C::CHUNK, 1024), id_pv, (acc || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < C::BN / C::KE; ++kk) {
+          const uint32_t dt = tbase + (t ? C::O_COL1 : C::O_COL0);
+          const uint32_t at = tbase + (b ? C::S_COL1 : C::S_COL0) + kk * 8;
+          const uint64_t db = sdesc_sw128(va + kk * C::KE * 128, C::CHUNK, 1024);
+          if constexpr (F8) umma_ts_f8(dt, at, db, id_pv, (acc || kk > 0) ? 1u : 0u);
+          else umma_ts(dt, at, db, id_pv, (acc || kk > 0) ? 1u : 0u);
         }
       };
       const int lo0 = j_lo[0], hi0 = j_hi[0], lo1 = j_lo[1], hi1 = j_hi[1];
@@ -453,8 +475,9 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     // columns of the other copies -- and the running sum.  False if a wait ran out.
     auto soft_step = [&](auto nc_tag, int step, uint32_t s_col) -> bool {
       constexpr int NC = decltype(nc_tag)::value;
-      constexpr int NP = NC / 2;                  // packed 16-bit pairs of P
-      constexpr int G = NP < 32 ? NP : 32;        // pairs per TMEM store
+      constexpr int EPC = 4 / C::ESZ;             // P values per 32-bit TMEM column
+      constexpr int NP = NC / EPC;                // packed columns of P
+      constexpr int G = NP < 32 ? NP : 32;        // columns per TMEM store
       const int col0 = qcopy * NC;
       uint32_t sr[NC];
 #pragma unroll
@@ -531,22 +554,30 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         uint32_t pk[G];
 #pragma unroll
         for (int i = 0; i < G; ++i) {
-          const uint64_t arg = f2_fma(f2_pack(__uint_as_float(sr[2 * G * h + 2 * i]),
-                                              __uint_as_float(sr[2 * G * h + 2 * i + 1])),
-                                      sl2x2, negm2);
-          float a, b;
-          f2_unpack(arg, a, b);
-          if ((i & 3) >= kPolyFrom) {
-            a = exp2_poly3(a);
-            b = exp2_poly3(b);
-          } else {
-            a = ex2_approx(a);
-            b = ex2_approx(b);
+          float e[EPC];
+#pragma unroll
+          for (int q = 0; q < EPC / 2; ++q) {
+            const int k = EPC * (G * h + i) + 2 * q;  // first of the pair in sr
+            const int pi = (EPC / 2) * i + q;         // pair count within the store
+            const uint64_t arg = f2_fma(
+                f2_pack(__uint_as_float(sr[k]), __uint_as_float(sr[k + 1])), sl2x2, negm2);
+            float a, b;
+            f2_unpack(arg, a, b);
+            if ((pi & 3) >= kPolyFrom) {
+              a = exp2_poly3(a);
+              b = exp2_poly3(b);
+            } else {
+              a = ex2_approx(a);
+              b = ex2_approx(b);
+            }
+            sum2[pi & 3] = f2_add(sum2[pi & 3], f2_pack(a, b));
+            e[2 * q] = a;
+            e[2 * q + 1] = b;
           }
-          sum2[i & 3] = f2_add(sum2[i & 3], f2_pack(a, b));
-          pk[i] = pack2<BF16>(a, b);
+          if constexpr (F8) pk[i] = pack4_e4m3(e[0], e[1], e[2], e[3]);
+          else pk[i] = pack2<BF16>(e[0], e[1]);
         }
-        const uint32_t dst = tmem_addr(tbase, lane_base, s_col + col0 / 2 + G * h);
+        const uint32_t dst = tmem_addr(tbase, lane_base, s_col + col0 / EPC + G * h);
         if constexpr (G == 32) tmem_st32(dst, pk); else tmem_st16(dst, pk);
       }
       if constexpr (NC < 128) {
@@ -601,7 +632,8 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     if (ok && live) {
       tc_fence_after();
       // A row can see no key of a split (l = 0): it contributes nothing.
-      const float inv_l = (l > 0.f) ? 1.0f / l : 0.f;
+      // (8-bit inputs: the scale of V is applied here, once per output element.)
+      const float inv_l = (l > 0.f) ? (F8 ? p.o_scale : 1.0f) / l : 0.f;
       const float lse = (l > 0.f) ? (m + __log2f(l)) * 0.69314718055994531f : -INFINITY;
       const size_t orow_idx = static_cast<size_t>(bh) * Nq + row;
       if (!partial) {

@@ -27,7 +27,7 @@ FA2_FP16 = 0
 FA2_BF16 = 1
 
 # Every symbol include/fa2.h declares.
-EXPORTS = ("fa2_fwd", "fa2_fwd_window", "fa2_fwd_decode_splits", "fa2_fwd_decode_workspace_size",
+EXPORTS = ("fa2_fwd", "fa2_fwd_window", "fa2_fwd_fp8", "fa2_fwd_decode_splits", "fa2_fwd_decode_workspace_size",
            "fa2_fwd_decode", "fa2_bwd_workspace_size", "fa2_bwd", "fa2_bwd_window",
            "fa2_bwd_noalloc", "fa2_get_device_status", "fa2_status_string", "fa2_debug_set",
            "fa2_launch_count")
@@ -55,6 +55,8 @@ def load() -> ctypes.CDLL:
     lib.fa2_fwd.restype = i
     lib.fa2_fwd_window.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, i, vp]
     lib.fa2_fwd_window.restype = i
+    lib.fa2_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, f, f, f, vp]
+    lib.fa2_fwd_fp8.restype = i
     lib.fa2_fwd_decode_splits.argtypes = [i, i, i, i, i, i]
     lib.fa2_fwd_decode_splits.restype = i
     lib.fa2_fwd_decode_workspace_size.argtypes = [i, i, i, i, i, i]
@@ -123,6 +125,21 @@ def fa2_fwd_window(q, k, v, o, lse, scale: float, window: int, stream=None) -> i
     B, H, N, d = q.shape
     return load().fa2_fwd_window(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d,
                                  float(scale), int(window), _dtype_code(q), _stream(stream))
+
+
+def fa2_fwd_fp8(q, k, v, o, lse, scale: float, causal: bool, q_scale: float, k_scale: float,
+                v_scale: float, stream=None) -> int:
+    """Raw call: q, k, v [B,H,N,d] float8_e4m3fn; o [B,H,N,d] bfloat16; lse float32."""
+    _check_layout(q, k, v, o, lse)
+    for t in (q, k, v):
+        if t.dtype != torch.float8_e4m3fn:
+            raise TypeError("q, k, v must be float8_e4m3fn")
+    if o.dtype != torch.bfloat16:
+        raise TypeError("o must be bfloat16")
+    B, H, N, d = q.shape
+    return load().fa2_fwd_fp8(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d,
+                              float(scale), int(bool(causal)), float(q_scale), float(k_scale),
+                              float(v_scale), _stream(stream))
 
 
 def fa2_fwd_decode_splits(B: int, H: int, Nq: int, Nk: int, d: int, sm_count: int = 0) -> int:
@@ -213,6 +230,18 @@ def forward(q, k, v, scale: float, causal: bool, stream=None):
     rc = fa2_fwd(q, k, v, o, lse, scale, causal, stream)
     if rc != FA2_OK:
         raise FA2Error(rc, "fa2_fwd")
+    return o, lse
+
+
+def forward_fp8(q, k, v, scale: float, causal: bool, q_scale: float, k_scale: float,
+                v_scale: float, stream=None):
+    """Allocating wrapper of fa2_fwd_fp8: bf16 O and float32 LSE."""
+    B, H, N, d = q.shape
+    o = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=q.device)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    rc = fa2_fwd_fp8(q, k, v, o, lse, scale, causal, q_scale, k_scale, v_scale, stream)
+    if rc != FA2_OK:
+        raise FA2Error(rc, "fa2_fwd_fp8")
     return o, lse
 
 

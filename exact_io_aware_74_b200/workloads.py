@@ -105,6 +105,14 @@ WORKLOADS = {
         note="forward at head dim 256"),
 }
 
+# 8-bit forward (E4M3 Q, K, V; bf16 O) on the headline shape.  Inputs from
+# make_fp8_inputs; FLOPs counted as for the 16-bit forward.
+FP8_WORKLOADS = {
+    "fwd_e4m3_b2h32_n8192_d128": Workload(
+        "fwd_e4m3_b2h32_n8192_d128", 2, 32, 8192, 128, "e4m3", False, 9,
+        note="headline shape with E4M3 inputs"),
+}
+
 WORKLOAD_ORDER = list(WORKLOADS)
 
 
@@ -209,6 +217,22 @@ def make_decode_inputs(B: int, H: int, Nq: int, Nk: int, d: int, dtype: str, see
 
 def decode_inputs(w: DecodeWorkload) -> dict:
     return make_decode_inputs(w.B, w.H, w.Nq, w.Nk, w.d, w.dtype, w.seed)
+
+
+def make_fp8_inputs(B: int, H: int, N: int, d: int, seed: int, amp: float = 16.0) -> dict:
+    """Seeded E4M3 inputs: N(0, 1) draws (Q, K, V in that order) times ``amp`` (a
+    power of two, so that small values keep their precision and |x| stays far
+    below 448), cast to torch.float8_e4m3fn (round to nearest even).  The real
+    values are the codes times ``scale`` = 1 / amp, returned for each tensor."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(seed))
+    shape = (B, H, N, d)
+    out = {}
+    for name in ("q", "k", "v"):
+        x = torch.randn(shape, generator=g, dtype=torch.float32) * amp
+        out[name] = x.to(torch.float8_e4m3fn)
+    out["scale"] = 1.0 / amp
+    return out
 
 
 def workload_inputs(w: Workload, *, with_do: bool | None = None, B: int | None = None,

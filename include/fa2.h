@@ -145,6 +145,26 @@ int fa2_fwd_decode_splits(int B, int H, int Nq, int Nk, int d, int sm_count);
 size_t fa2_fwd_decode_workspace_size(int B, int H, int Nq, int Nk, int d, int n_splits);
 
 /*
+ * Forward pass with 8-bit (E4M3) inputs.  Source: [DC] FlashAttention-3 section
+ * (FP8 attention: 8-bit floating point for the two matrix products).
+ *
+ *   Q, K, V : in,  [B][H][N][d] E4M3 bytes (1 sign, 4 exponent bits with bias 7,
+ *             3 mantissa bits, no infinities), holding the real values
+ *             q_scale * Q, k_scale * K, v_scale * V respectively
+ *   O       : out, [B][H][N][d] bf16, softmax(scale * (q_scale Q)(k_scale K)^T) (v_scale V)
+ *   LSE     : out, [B][H][N] float, in units of the scaled scores
+ *   d       : a multiple of 16 from 16 to 128 (FA2_ERR_UNSUPPORTED otherwise)
+ *   q_scale, k_scale, v_scale : finite and > 0 (per-tensor dequantisation scales)
+ * Both products run on the 8-bit tensor cores (tcgen05 kind::f8f6f4) with fp32
+ * accumulation; the probabilities P are rounded to E4M3 (relative error <= 2^-4,
+ * absolute <= 2^-10 below 2^-6) before P V, and the row sums use the unrounded
+ * values.  causal, B, H, N, scale and the errors as for fa2_fwd.
+ */
+int fa2_fwd_fp8(const void* Q, const void* K, const void* V, void* O, float* LSE, int B, int H,
+                int N, int d, float scale, int causal, float q_scale, float k_scale,
+                float v_scale, fa2_stream_t stream);
+
+/*
  * Bytes of device workspace fa2_bwd needs for these sizes (the per-row
  * D = rowsum(dO * O) and a float32 dQ accumulator), a multiple of 256.
  * Returns 0 for sizes fa2_bwd would reject.

@@ -46,6 +46,8 @@ closed forms, invariances and central finite differences.
 
 from .attention import (  # noqa: F401
     attn_fwd_decode_ref,
+    attn_fwd_fp8_ref,
+    e4m3_decode,
     attn_fwd_ref,
     attn_fwd_rows_ref,
     attn_bwd_ref,

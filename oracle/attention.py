@@ -213,3 +213,33 @@ def attn_fwd_decode_ref(q, k, v, scale: float, causal: bool) -> tuple[np.ndarray
             out[b, h] = p @ v[b, h]
             lse[b, h] = l
     return out, lse
+
+
+def e4m3_decode(codes) -> np.ndarray:
+    """Real values of E4M3 bytes (uint8 array), from the format's definition.
+
+    One sign bit, four exponent bits with bias 7 and three mantissa bits:
+    exponent 0 holds subnormals m/8 * 2^-6; otherwise (1 + m/8) * 2^(e - 7);
+    the pattern with every exponent and mantissa bit set is NaN (there are no
+    infinities, so the largest finite magnitude is 1.75 * 2^8 = 448).  This is
+    the 8-bit floating point that "Flash Attention spiegata: una guida
+    completa", FlashAttention-3 section, names for FP8 attention.
+    """
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = (c & 0x7).astype(np.float64)
+    mag = np.where(e == 0, m / 8.0 * 2.0 ** -6, (1.0 + m / 8.0) * np.exp2(e.astype(np.float64) - 7))
+    mag = np.where((e == 15) & (c & 0x7 == 7), np.nan, mag)
+    return sign * mag
+
+
+def attn_fwd_fp8_ref(q8, k8, v8, scale: float, causal: bool, q_scale: float, k_scale: float,
+                     v_scale: float) -> tuple[np.ndarray, np.ndarray]:
+    """Attention of E4M3 inputs: the plain definition applied to their real values
+    q_scale * Q, k_scale * K, v_scale * V (q8, k8, v8: uint8 codes [B,H,N,d]).
+    Returns (O, LSE) in fp64."""
+    q = e4m3_decode(q8) * q_scale
+    k = e4m3_decode(k8) * k_scale
+    v = e4m3_decode(v8) * v_scale
+    return attn_fwd_ref(q, k, v, scale, causal)

@@ -19,7 +19,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 def _header_functions():
     src = open(os.path.join(ROOT, "include", "fa2.h")).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return sorted(set(re.findall(r"\b(fa2_[a-z_]+)\s*\(", src)))
+    return sorted(set(re.findall(r"\b(fa2_[a-z0-9_]+)\s*\(", src)))
 
 
 @pytest.fixture(scope="module")
@@ -232,3 +232,23 @@ def test_bwd_rejects_head_dims_above_128(lib):
 def test_decode_split_choice_rejects_bad_sizes(lib):
     assert fa2.fa2_fwd_decode_splits(1, 1, 5, 4, 64, 148) == 0
     assert fa2.fa2_fwd_decode_splits(1, 1, 1, 4, 84, 148) == 0
+
+
+def test_fp8_validation_without_device(lib):
+    def call(q=P, o=4 * P, N=64, d=64, scale=0.1, causal=0, qs=1.0, ks=1.0, vs=1.0):
+        return lib.fa2_fwd_fp8(q, 2 * P, 3 * P, o, 5 * P, 1, 1, N, d, scale, causal, qs, ks, vs,
+                               None)
+    E = fa2.FA2_ERR_INVALID_ARG
+    assert call(q=0) == E
+    assert call(causal=2) == E
+    assert call(qs=0.0) == E
+    assert call(vs=float("inf")) == E
+    assert call(ks=-1.0) == E
+    assert call(scale=float("nan")) == E
+    assert call(o=P) == E                       # O overlaps Q
+    for d in (8, 24, 100, 144, 256):
+        assert call(d=d) == fa2.FA2_ERR_UNSUPPORTED, d
+    import torch
+    if not torch.cuda.is_available():
+        for d in (16, 64, 128):
+            assert call(d=d) in (fa2.FA2_ERR_CUDA, fa2.FA2_ERR_ARCH)

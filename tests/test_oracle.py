@@ -509,3 +509,55 @@ def test_window_flop_count():
     assert w.fwd_flops == 4 * 4 * pairs
     full = Workload("y", 1, 1, 10, 4, "bf16", True, 0, window=10)
     assert full.fwd_flops == Workload("z", 1, 1, 10, 4, "bf16", True, 0).fwd_flops + 4 * 4 * 5
+
+
+# ------------------------------------------------------------------------------------
+# 8-bit inputs: E4M3 decoding ("Flash Attention spiegata", FlashAttention-3 section)
+# ------------------------------------------------------------------------------------
+
+def test_e4m3_decode_anchor_values():
+    """Values fixed by the format: bias 7, three mantissa bits, no infinities."""
+    d = oracle.e4m3_decode(np.array([0x00, 0x80, 0x01, 0x07, 0x08, 0x38, 0x39, 0x3F, 0x40,
+                                     0x77, 0x7E, 0xFE, 0xB8], dtype=np.uint8))
+    expect = [0.0, -0.0, 2.0 ** -9, 7 * 2.0 ** -9, 2.0 ** -6, 1.0, 1.125, 1.875, 2.0,
+              240.0, 448.0, -448.0, -1.0]
+    assert np.array_equal(d, expect)
+    assert np.signbit(d[1])
+    assert np.isnan(oracle.e4m3_decode(np.array([0x7F, 0xFF], dtype=np.uint8))).all()
+
+
+def test_e4m3_decode_matches_torch_on_every_code():
+    codes = np.arange(256, dtype=np.uint8)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).double().numpy()
+    assert np.array_equal(oracle.e4m3_decode(codes), ref, equal_nan=True)
+
+
+def test_e4m3_decode_is_monotone_over_positive_codes():
+    v = oracle.e4m3_decode(np.arange(0x00, 0x7F, dtype=np.uint8))  # 0 .. 448
+    assert np.all(np.diff(v) > 0)
+
+
+def test_fp8_ref_is_attention_of_the_real_values():
+    """The 8-bit reference equals the scalar brute force on the decoded, scaled
+    inputs (codes drawn at random, scales powers of two)."""
+    from exact_io_aware_74_b200.workloads import make_fp8_inputs
+    x = make_fp8_inputs(1, 2, 19, 16, seed=3)
+    codes = {n: x[n].view(torch.uint8).numpy() for n in ("q", "k", "v")}
+    s = x["scale"]
+    for causal in (False, True):
+        o, lse = oracle.attn_fwd_fp8_ref(codes["q"], codes["k"], codes["v"], 0.25, causal,
+                                         s, s, 2 * s)
+        real = {n: oracle.e4m3_decode(codes[n]) * (2 * s if n == "v" else s) for n in codes}
+        bo, bl = brute_fwd(real["q"], real["k"], real["v"], 0.25, causal)
+        _close(o, bo)
+        _close(lse, bl)
+
+
+def test_fp8_inputs_recipe():
+    from exact_io_aware_74_b200.workloads import make_fp8_inputs
+    x = make_fp8_inputs(1, 1, 64, 32, seed=11)
+    assert x["q"].dtype == torch.float8_e4m3fn and x["scale"] == 1 / 16
+    g = torch.Generator().manual_seed(11)
+    q = torch.randn((1, 1, 64, 32), generator=g) * 16
+    assert torch.equal(x["q"].view(torch.uint8), q.to(torch.float8_e4m3fn).view(torch.uint8))
+    assert float(x["q"].float().abs().max()) < 448
