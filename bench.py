@@ -35,7 +35,8 @@ sys.path.insert(0, ROOT)
 import torch  # noqa: E402
 
 from exact_io_aware_74_b200.workloads import (  # noqa: E402
-    DECODE_WORKLOADS, WORKLOADS, WORKLOAD_ORDER, decode_inputs, workload_inputs)
+    DECODE_WORKLOADS, FP8_WORKLOADS, WORKLOADS, WORKLOAD_ORDER, decode_inputs, make_fp8_inputs,
+    workload_inputs)
 
 METRIC = "FA-2 fwd/bwd TFLOP/s (bf16, 1×B200) and % of dense BF16 tensor peak"
 DEFAULT_WORKLOAD = WORKLOAD_ORDER[1]          # forward + backward, bf16, causal, d = 64
@@ -342,6 +343,48 @@ def time_decode(fa2, w, iters, dev, stream, hbm_peak, peaks_src):
                          "peak_kind": f"HBM copy, {peaks_src}"}}
 
 
+# Nominal dense 8-bit / 16-bit tensor throughput on B200 (4.5 / 2.25 PFLOP/s): the
+# 8-bit roofline is the measured 16-bit peak times this ratio.
+FP8_OVER_BF16 = 2.0
+
+
+def time_fp8(fa2, w, iters, dev, stream, bf16_peak, peaks_src):
+    """fa2_fwd_fp8 on an E4M3 workload: median CUDA-event time per call, algorithmic
+    TFLOP/s and the fraction of the 8-bit tensor peak."""
+    x = make_fp8_inputs(w.B, w.H, w.N, w.d, seed=w.seed)
+    s = x["scale"]
+    q, k, v = (x[n].to(dev) for n in ("q", "k", "v"))
+    o = torch.empty((w.B, w.H, w.N, w.d), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
+
+    def call():
+        _check(fa2, fa2.fa2_fwd_fp8(q, k, v, o, lse, w.scale, w.causal, s, s, s, stream),
+               "fa2_fwd_fp8")
+
+    for _ in range(3):
+        call()
+    torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(iters)]
+    with torch.cuda.stream(stream):
+        for i in range(iters):
+            ev[i][0].record(stream)
+            call()
+            ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    rc, site = fa2.fa2_get_device_status(stream)
+    if rc != fa2.FA2_OK:
+        raise RuntimeError(f"device status {fa2.status_string(rc)} at wait site {site}")
+    ms = statistics.median(e[0].elapsed_time(e[1]) for e in ev)
+    tf = w.fwd_flops / ms / 1e9
+    peak = bf16_peak * FP8_OVER_BF16
+    return {"fwd_ms": round(ms, 4), "fwd_tflops": round(tf, 1),
+            "roofline": {"bound": "tensor", "kernel": "fa2_fwd_kernel (E4M3)",
+                         "achieved": round(tf, 1), "peak": peak, "unit": "TFLOP/s",
+                         "frac": round(tf / peak, 4),
+                         "peak_kind": f"bf16 burst x {FP8_OVER_BF16} (nominal e4m3/bf16), "
+                                      f"{peaks_src}"}}
+
+
 def cpu_baseline(w, budget_s: float = 12.0) -> dict:
     """The oracle as it stands, timed on this host's cores on whole (b, h) slices."""
     import numpy as np  # noqa: F401
@@ -447,6 +490,8 @@ def run_ours(args):
         out["other_workloads"] = extras
         out["decode"] = {name: time_decode(fa2, dw, 50, dev, stream, peaks["hbm_gbs"], peaks_src)
                          for name, dw in DECODE_WORKLOADS.items()}
+        out["fp8"] = {name: time_fp8(fa2, fw, 20, dev, stream, peaks["bf16_tflops"], peaks_src)
+                      for name, fw in FP8_WORKLOADS.items()}
         torch.cuda.empty_cache()
         out["headline"] = {"workload": HEADLINE_WORKLOAD,
                            "fwd_tflops": extras[HEADLINE_WORKLOAD]["fwd_tflops"],
