@@ -2,6 +2,7 @@
 
     python -m exact_io_aware_74_b200.profile_case B H N d causal [reps] [--fwd-only]
     python -m exact_io_aware_74_b200.profile_case --decode B H Nq Nk d causal [reps] [splits]
+    python -m exact_io_aware_74_b200.profile_case --fp8 B H N d causal [reps]
 
 Seeded N(0, 1) bf16 inputs; exits non-zero if a call or the device status fails.
 Used to capture Nsight Compute profiles of one kernel on a small case.  With
@@ -16,7 +17,7 @@ import sys
 import torch
 
 from exact_io_aware_74_b200 import fa2
-from exact_io_aware_74_b200.workloads import make_decode_inputs, make_inputs
+from exact_io_aware_74_b200.workloads import make_decode_inputs, make_fp8_inputs, make_inputs
 
 
 def decode(args: list[str]) -> int:
@@ -32,9 +33,24 @@ def decode(args: list[str]) -> int:
     return 0 if rc == fa2.FA2_OK else 1
 
 
+def fp8(args: list[str]) -> int:
+    B, H, N, d, causal = (int(a) for a in args[:5])
+    reps = int(args[5]) if len(args) > 5 else 2
+    x = make_fp8_inputs(B, H, N, d, seed=5)
+    q, k, v = (x[n].cuda() for n in ("q", "k", "v"))
+    s = x["scale"]
+    for _ in range(reps):
+        fa2.forward_fp8(q, k, v, 1.0 / math.sqrt(d), bool(causal), s, s, s)
+    rc, site = fa2.fa2_get_device_status()
+    print(f"status {fa2.status_string(rc)} site {site}")
+    return 0 if rc == fa2.FA2_OK else 1
+
+
 def main(argv: list[str]) -> int:
     if "--decode" in argv:
         return decode([a for a in argv if not a.startswith("--")])
+    if "--fp8" in argv:
+        return fp8([a for a in argv if not a.startswith("--")])
     fwd_only = "--fwd-only" in argv
     args = [a for a in argv if not a.startswith("--")]
     B, H, N, d, causal = (int(a) for a in args[:5])
