@@ -118,6 +118,12 @@ struct FwdCfg {
 #define FA2_POLY_FROM 4
 #endif
 constexpr int kPolyFrom = FA2_POLY_FROM;
+// The same split for 8-bit inputs, whose matrix products take half the tensor
+// time, leaving the exponential unit the busiest pipe.
+#ifndef FA2_POLY_FROM_F8
+#define FA2_POLY_FROM_F8 4
+#endif
+constexpr int kPolyFromF8 = FA2_POLY_FROM_F8;
 
 // Wait-site ids reported through the status word.
 enum FwdSite : uint32_t {
@@ -563,7 +569,7 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                 f2_pack(__uint_as_float(sr[k]), __uint_as_float(sr[k + 1])), sl2x2, negm2);
             float a, b;
             f2_unpack(arg, a, b);
-            if ((pi & 3) >= kPolyFrom) {
+            if ((pi & 3) >= (F8 ? kPolyFromF8 : kPolyFrom)) {
               a = exp2_poly3(a);
               b = exp2_poly3(b);
             } else {
