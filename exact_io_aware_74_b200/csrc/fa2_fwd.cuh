@@ -23,11 +23,11 @@
 //   warp  9    MMA issuer (tcgen05, one thread)
 //   warps 10-11 idle (they complete the third warpgroup)
 // The kernel is compiled for 168 registers per thread (384 x 168 = 64512); the
-// third warpgroup gives registers back (down to 56) and the two softmax
-// warpgroups take them (up to 224): 2 x 128 x 224 + 128 x 56 = 64512, so the
-// re-split never asks for more than the launch holds.  (232 / 40 made the MMA
-// issuer spill and measured slower.)  The host refuses to launch a build whose
-// register count is not 168.
+// third warpgroup gives registers back (down to 72) and the two softmax
+// warpgroups take them (up to 216): 2 x 128 x 216 + 128 x 72 = 64512, so the
+// re-split never asks for more than the launch holds.  (232 / 40 and 224 / 56
+// made the MMA issuer spill.)  The host refuses to launch a build whose register
+// count is not 168.
 // TMEM (512 columns x 128 lanes, fp32): S_t at column 128 t, O_t at 256 + D t.
 // P_t (16-bit) overwrites the first 64 columns of S_t and feeds the P V MMA
 // straight from TMEM.  The MMA warp alternates between the two query tiles so
@@ -100,7 +100,7 @@ struct FwdCfg {
   static constexpr int THREADS = 384;
   static constexpr int LAUNCH_REGS = 168;  // per thread, as compiled (checked on the host)
 #ifndef FA2_FWD_SOFT_REGS
-#define FA2_FWD_SOFT_REGS 224
+#define FA2_FWD_SOFT_REGS 216
 #endif
   static constexpr int SOFT_REGS = FA2_FWD_SOFT_REGS;
   static constexpr int OTHER_REGS = (THREADS * LAUNCH_REGS - 2 * 128 * SOFT_REGS) / 128 / 8 * 8;
@@ -108,6 +108,10 @@ struct FwdCfg {
                 "register re-split exceeds the launch allocation");
   static constexpr uint32_t S_COL0 = 0, S_COL1 = 128;
   static constexpr uint32_t O_COL0 = 256, O_COL1 = 256 + D;
+  // D = 64 with two query tiles: each tile's P has its own 64 columns after the
+  // two O blocks, so the S block is free as soon as the softmax has read it.
+  static constexpr bool SEP_P = (D == 64);
+  static constexpr uint32_t P_COL0 = 384, P_COL1 = 448;
 };
 
 // Pairs i of a score row with (i & 3) >= kPolyFrom take the polynomial exp2
@@ -156,7 +160,7 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 
   __shared__ uint64_t bar_q, k_full[C::KS], k_empty[C::KS], v_full[C::VS + C::VX],
       v_empty[C::VS + C::VX];
-  __shared__ uint64_t s_full[2], p_ready[2], o_done[2], drain;
+  __shared__ uint64_t s_full[2], s_free[2], p_ready[2], o_done[2], drain;
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
 
@@ -206,6 +210,8 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   const int n_steps = j1 - j0;
   // A CTA with one query tile runs it double-buffered (see the MMA issuer).
   const bool single = C::QT == 1 || !has1;
+  // Two query tiles at D = 64: P in its own columns, S(j + 1) issued once S(j) is read.
+  const bool sep = C::SEP_P && !single;
 
   WaitCtl wc{p.status, &abort_flag, p.wait_ns};
 
@@ -216,6 +222,7 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     for (int s = 0; s < C::VS + C::VX; ++s) { mbar_init(&v_full[s], 1); mbar_init(&v_empty[s], 1); }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&s_full[t], 1);
+      mbar_init(&s_free[t], 4);
       mbar_init(&p_ready[t], 4);
       mbar_init(&o_done[t], 1);
     }
@@ -343,12 +350,12 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       };
       // P from TMEM (8 columns = 32 bytes of keys per step), V MN-major: a step
       // of KE keys advances KE rows of 128 bytes.
-      auto issue_pv = [&](int t, int b, int vs, bool acc) {
+      auto issue_pv = [&](int t, uint32_t a_col, int vs, bool acc) {
         const uint32_t va = v_addr(vs);
 #pragma unroll
         for (int kk = 0; kk < C::BN / C::KE; ++kk) {
           const uint32_t dt = tbase + (t ? C::O_COL1 : C::O_COL0);
-          const uint32_t at = tbase + (b ? C::S_COL1 : C::S_COL0) + kk * 8;
+          const uint32_t at = tbase + a_col + kk * 8;
           const uint64_t db = sdesc_sw128(va + kk * C::KE * 128, C::CHUNK, 1024);
           if constexpr (F8) umma_ts_f8(dt, at, db, id_pv, (acc || kk > 0) ? 1u : 0u);
           else umma_ts(dt, at, db, id_pv, (acc || kk > 0) ? 1u : 0u);
@@ -388,7 +395,7 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             break;
           }
           tc_fence_after();
-          issue_pv(0, b, vs, jj > 0);
+          issue_pv(0, b ? C::S_COL1 : C::S_COL0, vs, jj > 0);
           umma_commit(&o_done[0]);
           umma_commit(&v_empty[vs]);
         }
@@ -414,17 +421,15 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         const bool has_next = jj + 1 < n_steps;
         bool k_next_ready = false;
         if (!mbar_wait(&v_full[vs], (jj / C::VS) & 1, wc, kSiteMmaV)) { ok = false; break; }
-        auto tile_step = [&](int t, int lo, int hi) -> bool {
-          if (j >= lo && j < hi) {
-            const int step = j - lo;  // this tile's own step count
-            if (!mbar_wait(&p_ready[t], step & 1, wc, kSiteMmaP)) return false;
-            tc_fence_after();
-            issue_pv(t, t, vs, step > 0);
-            umma_commit(&o_done[t]);
-          }
+        auto next_s = [&](int t, int lo, int hi) -> bool {
           // S for step j + 1 (this tile's next step, or its first when its range
-          // starts there); P of step j in the same columns was consumed above.
+          // starts there).
           if (j + 1 >= lo && j + 1 < hi) {
+            if (sep && j >= lo) {
+              // The S block still holds S of step j until the softmax has read it.
+              if (!mbar_wait(&s_free[t], (j - lo) & 1, wc, kSiteMmaP)) return false;
+              tc_fence_after();
+            }
             if (!k_next_ready) {
               if (!mbar_wait(&k_full[ks1], ((jj + 1) / C::KS) & 1, wc, kSiteMmaK)) return false;
               tc_fence_after();
@@ -435,7 +440,24 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           }
           return true;
         };
-        ok = tile_step(0, lo0, hi0) && tile_step(1, lo1, hi1);
+        auto pv = [&](int t, int lo, int hi) -> bool {
+          if (j >= lo && j < hi) {
+            const int step = j - lo;  // this tile's own step count
+            if (!mbar_wait(&p_ready[t], step & 1, wc, kSiteMmaP)) return false;
+            tc_fence_after();
+            const uint32_t a_col = sep ? (t ? C::P_COL1 : C::P_COL0) : (t ? C::S_COL1 : C::S_COL0);
+            issue_pv(t, a_col, vs, step > 0);
+            umma_commit(&o_done[t]);
+          }
+          return true;
+        };
+        if (sep) {
+          // Both tiles' next S as soon as their scores are read, then the P V products.
+          ok = next_s(0, lo0, hi0) && next_s(1, lo1, hi1) && pv(0, lo0, hi0) && pv(1, lo1, hi1);
+        } else {
+          // P of step j sits in the S block: P V first, then the next S over it.
+          ok = pv(0, lo0, hi0) && next_s(0, lo0, hi0) && pv(1, lo1, hi1) && next_s(1, lo1, hi1);
+        }
         if (ok && has_next && !k_next_ready)  // a slot is only released once its load landed
           ok = mbar_wait(&k_full[ks1], ((jj + 1) / C::KS) & 1, wc, kSiteMmaK);
         if (!ok) break;
@@ -492,6 +514,11 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                   *reinterpret_cast<uint32_t(*)[32]>(&sr[32 * c]));
       tmem_wait_ld();
       reg_fence(sr);
+      if (sep) {  // the S block may now take the next scores
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s_free[t]);
+      }
       const int kc0 = (my_lo + step) * C::BN + col0;  // key of column 0 of sr
       // Keys after the row's last one (causal), past Nk, or before the row's
       // window start.
@@ -555,6 +582,13 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       const float neg_m = (m == -INFINITY) ? 0.f : -m;
       const uint64_t negm2 = f2_pack(neg_m, neg_m);
       uint64_t sum2[4] = {0, 0, 0, 0};
+      // With its own P columns the previous P V product may still be reading them.
+      if (sep && step > 0) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&o_done[t], (step - 1) & 1, wc, kSiteSoftO)))
+          return false;
+        tc_fence_after();
+      }
+      const uint32_t p_col = sep ? (t ? C::P_COL1 : C::P_COL0) : s_col;
 #pragma unroll
       for (int h = 0; h < NP / G; ++h) {
         uint32_t pk[G];
@@ -583,7 +617,7 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           if constexpr (F8) pk[i] = pack4_e4m3(e[0], e[1], e[2], e[3]);
           else pk[i] = pack2<BF16>(e[0], e[1]);
         }
-        const uint32_t dst = tmem_addr(tbase, lane_base, s_col + col0 / EPC + G * h);
+        const uint32_t dst = tmem_addr(tbase, lane_base, p_col + col0 / EPC + G * h);
         if constexpr (G == 32) tmem_st32(dst, pk); else tmem_st16(dst, pk);
       }
       if constexpr (NC < 128) {
@@ -622,6 +656,16 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         if (!ok) break;
         tmem_wait_st();
         tc_fence_before();
+      } else if (sep) {
+        // Keep the barrier counts: S read; and, like the live warps (which wait
+        // for the previous P V product before writing P), arrive for this step's
+        // P only once the previous step's P was complete and consumed.
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s_free[t]);
+        if (step > 0) {
+          ok = __all_sync(0xffffffffu, mbar_wait(&o_done[t], (step - 1) & 1, wc, kSiteSoftO));
+          if (!ok) break;
+        }
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_ready[buf]);
