@@ -48,6 +48,14 @@ namespace fa2 {
 
 constexpr int kBwdKernelsPerCall = 3;
 
+// Groups of four probabilities v (of eight per 32 queries) with (v & 3) >=
+// kBwdPolyFrom take the FMA-pipe exp2 polynomial instead of the MUFU unit
+// (4: none).
+#ifndef FA2_BWD_POLY_FROM
+#define FA2_BWD_POLY_FROM 4
+#endif
+constexpr int kBwdPolyFrom = FA2_BWD_POLY_FROM;
+
 // Workspace: D [BH][Npad] f32 | L2 = LSE*log2(e) [BH][Npad] f32 | dQacc [BH][N][Dt] f32,
 // Dt the kernel's tile head dim (64 or 128).
 inline size_t bwd_npad(int N) { return (static_cast<size_t>(N) + 127) / 128 * 128; }
@@ -445,10 +453,17 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           f2_unpack(a01, x0, x1);
           f2_unpack(a23, x2, x3);
           const int q0 = c * 32 + v * 4;
-          pr[q0 + 0] = ex2_approx(x0);
-          pr[q0 + 1] = ex2_approx(x1);
-          pr[q0 + 2] = ex2_approx(x2);
-          pr[q0 + 3] = ex2_approx(x3);
+          if ((v & 3) >= kBwdPolyFrom) {  // FMA-pipe exp2 for this group of four
+            pr[q0 + 0] = exp2_poly3(x0);
+            pr[q0 + 1] = exp2_poly3(x1);
+            pr[q0 + 2] = exp2_poly3(x2);
+            pr[q0 + 3] = exp2_poly3(x3);
+          } else {
+            pr[q0 + 0] = ex2_approx(x0);
+            pr[q0 + 1] = ex2_approx(x1);
+            pr[q0 + 2] = ex2_approx(x2);
+            pr[q0 + 3] = ex2_approx(x3);
+          }
         }
       }
       if (masked) {
