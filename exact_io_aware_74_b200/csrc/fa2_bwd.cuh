@@ -81,6 +81,11 @@ fa2_bwd_pre_kernel(const uint16_t* __restrict__ O, const uint16_t* __restrict__ 
                    long long total_rows, int d) {
   constexpr int TPR = D / 8;  // threads per row, 8 elements (16 bytes) each
   constexpr int RPB = 256 / TPR;
+  // Launched behind the caller's previous kernel (the forward, typically) with
+  // programmatic serialisation: let the main kernel start its set-up, then wait
+  // for O and LSE.
+  griddep_launch_dependents();
+  griddep_wait();
   const int sub = threadIdx.x % TPR;
   const long long r = static_cast<long long>(blockIdx.x) * RPB + threadIdx.x / TPR;
   const bool in_range = r < total_rows;  // no early exit: the shuffle below is warp-wide
@@ -132,6 +137,7 @@ fa2_bwd_dq_kernel(const float* __restrict__ dQacc, uint16_t* __restrict__ dQ, fl
                   long long n8, int D, int d) {
   // Thread i converts 8 accumulator columns (group i % (D/8) of row i / (D/8));
   // groups past the head dim d are padding and are dropped.
+  griddep_wait();  // the main kernel's reductions are complete and visible
   const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (i >= n8) return;
   const long long row = i / (D / 8);
@@ -221,6 +227,9 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     if (threadIdx.x == 0) atomicCAS(p.status, 0u, 4u | (kBSiteAlign << 8));
     return;
   }
+  // The dQ finalisation queued behind this grid may launch now; it waits for
+  // this grid to complete before reading the accumulator.
+  griddep_launch_dependents();
   uint8_t* smem = smem_raw;
   uint8_t* sK = smem;
   uint8_t* sV = sK + C::TILE;
@@ -294,6 +303,9 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         tma_load_3d(sV + c * C::CHUNK, &tmV, &bar_kv, c * 64, j * 128, bh);
       }
       const uint64_t keep = policy_evict_last();
+      // K and V do not depend on the preprocess; the L, D rows (and the zeroed
+      // dQ accumulator the compute warps add into) do.
+      griddep_wait();
       int issued = 0;
       bool ok = true;
       for (int it = 0; it < n_it; ++it) {
@@ -401,6 +413,7 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     __syncwarp();
   } else {
     // ------------------------------------------------------------------ compute
+    griddep_wait();  // the accumulator this role adds into was zeroed by the preprocess
     const int g = warp >> 2;                   // warpgroup: query columns 64 g .. 64 g + 63
     const int wq = warp & 3;                   // TMEM lane quadrant
     const int r = wq * 32 + lane;              // key row (P^T, dS^T) / query row (dQ)
@@ -624,6 +637,27 @@ bool make_tile_map(CUtensorMap* map, const void* base, int BH, int N, int d, boo
                    int box_rows = 128);
 bool make_acc_map(CUtensorMap* map, float* base, int BH, int N, int d);
 
+// Launch with programmatic stream serialisation: the kernel may start while the
+// previous kernel on the stream finishes; it waits (griddepcontrol.wait) before
+// touching that kernel's results.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, int smem,
+                       cudaStream_t stream, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+  if (e != cudaSuccess) cudaGetLastError();
+  return e;
+}
+
 template <int D, bool BF16, bool CAUSAL>
 int launch_bwd_t(const void* Q, const void* K, const void* V, const void* O, const void* dO,
                  const float* LSE, void* dQ, void* dK, void* dV, void* workspace, int BH, int N,
@@ -645,10 +679,10 @@ int launch_bwd_t(const void* Q, const void* K, const void* V, const void* O, con
     const long long rows = static_cast<long long>(BH) * Npad;
     constexpr int RPB = 256 / (D / 8);
     const unsigned int grid = static_cast<unsigned int>((rows + RPB - 1) / RPB);
-    fa2_bwd_pre_kernel<D, BF16><<<grid, 256, 0, stream>>>(
-        static_cast<const uint16_t*>(O), static_cast<const uint16_t*>(dO), LSE, Dg, Lg, dQacc, N,
-        Npad, rows, d);
-    if (cudaGetLastError() != cudaSuccess) return 4;
+    if (launch_pdl(fa2_bwd_pre_kernel<D, BF16>, dim3(grid), dim3(256), 0, stream,
+                   static_cast<const uint16_t*>(O), static_cast<const uint16_t*>(dO), LSE, Dg, Lg,
+                   dQacc, N, Npad, rows, d) != cudaSuccess)
+      return 4;
   }
   // 2. main
   {
@@ -675,16 +709,17 @@ int launch_bwd_t(const void* Q, const void* K, const void* V, const void* O, con
     bp.status = status;
     bp.wait_ns = wait_ns;
     const unsigned int grid = static_cast<unsigned int>(bp.n_kv) * static_cast<unsigned int>(BH);
-    kern<<<grid, Cfg::THREADS, Cfg::SMEM, stream>>>(mq, mk, mv, mdo, mdq, bp);
-    if (cudaGetLastError() != cudaSuccess) return 4;
+    if (launch_pdl(kern, dim3(grid), dim3(Cfg::THREADS), Cfg::SMEM, stream, mq, mk, mv, mdo, mdq,
+                   bp) != cudaSuccess)
+      return 4;
   }
   // 3. dQ finalise
   {
     const long long n8 = static_cast<long long>(BH) * N * D / 8;
     const unsigned int grid = static_cast<unsigned int>((n8 + 255) / 256);
-    fa2_bwd_dq_kernel<BF16><<<grid, 256, 0, stream>>>(dQacc, static_cast<uint16_t*>(dQ), scale,
-                                                      n8, D, d);
-    if (cudaGetLastError() != cudaSuccess) return 4;
+    if (launch_pdl(fa2_bwd_dq_kernel<BF16>, dim3(grid), dim3(256), 0, stream, dQacc,
+                   static_cast<uint16_t*>(dQ), scale, n8, D, d) != cudaSuccess)
+      return 4;
   }
   return 0;
 }
