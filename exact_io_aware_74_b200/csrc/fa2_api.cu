@@ -278,6 +278,9 @@ int fwd_core(const void* Q, const void* K, const void* V, void* O, float* LSE, i
     mqr = mq;  // not read
   }
   const int n_part = n_split * rep;
+  // One CTA per (query block, batch*head) in x, one per key stretch in y.
+  const long long n_qblk = (Nq + fwd_rows_per_cta(d) - 1) / fwd_rows_per_cta(d);
+  if (n_qblk * BH > 0x7fffffffll || n_split > 65535) return FA2_ERR_INVALID_ARG;
 
   fa2::FwdParams p{};
   p.O = O;
@@ -287,7 +290,7 @@ int fwd_core(const void* Q, const void* K, const void* V, void* O, float* LSE, i
   p.Nk = Nk;
   p.off = Nk - Nq;
   p.BH = BH;
-  p.n_qblk = (Nq + fwd_rows_per_cta(d) - 1) / fwd_rows_per_cta(d);
+  p.n_qblk = static_cast<int>(n_qblk);
   p.scale_log2 = scale * 1.4426950408889634f;
   p.status = st;
   p.wait_ns = wait_ns();

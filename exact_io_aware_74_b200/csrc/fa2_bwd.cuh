@@ -665,6 +665,7 @@ int launch_bwd_t(const void* Q, const void* K, const void* V, const void* O, con
                  cudaStream_t stream) {
   using Cfg = BwdCfg<D>;
   const int Npad = static_cast<int>(bwd_npad(N));
+  if (static_cast<long long>(Npad / 128) * BH > 0x7fffffffll) return 1;  // FA2_ERR_INVALID_ARG
   float* Dg = static_cast<float*>(workspace);
   float* Lg = Dg + static_cast<size_t>(BH) * Npad;
   float* dQacc = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
