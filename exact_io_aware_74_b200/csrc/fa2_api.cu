@@ -496,6 +496,7 @@ int fa2_fwd_fp8(const void* Q, const void* K, const void* V, void* O, float* LSE
   p.Nk = N;
   p.off = 0;
   p.BH = BH;
+  if (static_cast<long long>((N + 255) / 256) * BH > 0x7fffffffll) return FA2_ERR_INVALID_ARG;
   p.n_qblk = (N + 255) / 256;
   p.scale_log2 = sl2;
   p.status = st;
