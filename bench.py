@@ -63,6 +63,22 @@ def step_flops(w) -> float:
     return w.fwd_flops + (w.bwd_flops if w.backward else 0.0)
 
 
+# NVIDIA's published dense (no 2:4 sparsity) bf16 tensor throughput of one B200.
+DATASHEET_BF16_TFLOPS = 2250.0
+
+
+def fwd_bytes(w) -> int:
+    """Algorithmic HBM bytes of one forward: Q, K, V read once, O written once (16-bit),
+    LSE written (fp32)."""
+    return w.B * w.H * w.N * (4 * w.d * 2 + 4)
+
+
+def bwd_bytes(w) -> int:
+    """Algorithmic HBM bytes of one backward: Q, K, V, O, dO read and dQ, dK, dV written
+    once (16-bit), LSE read (fp32)."""
+    return w.B * w.H * w.N * (8 * w.d * 2 + 4)
+
+
 def input_bytes(w) -> int:
     n = w.B * w.H * w.N * w.d * 2
     return n * (4 if w.backward else 3)
@@ -459,7 +475,11 @@ def run_ours(args):
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
         "pct_of_peak": {"bf16_burst": round(100 * value / world / peaks["bf16_tflops"], 1),
                         "bf16_sustained": round(100 * value / world / peak, 1),
+                        "datasheet_dense_bf16": round(100 * value / world / DATASHEET_BF16_TFLOPS, 1),
                         "source": peaks_src},
+        "calls_gbs": {"fa2_fwd": round(fwd_bytes(w) / statistics.mean(fwd_ms) / 1e6, 1),
+                      **({"fa2_bwd": round(bwd_bytes(w) / statistics.mean(bwd_ms) / 1e6, 1)}
+                         if w.backward else {})},
         "calls_ms": {k: round(v[0], 5) for k, v in calls.items()},
         "roofline": {"bound": "tensor", "kernel": dom_label, "achieved": round(achieved, 1),
                      "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
@@ -475,18 +495,32 @@ def run_ours(args):
         extras = {}
         for name in WORKLOAD_ORDER[2:]:  # every workload but the small fp16 and the bench step
             ww = WORKLOADS[name]
-            it = 10 if ww.N >= 16384 else 20
-            _, f_ms, b_ms, _ = time_workload(fa2, ww, it, 3, dev, stream, None)
+            _, f_ms, b_ms, _ = time_workload(fa2, ww, 20, 3, dev, stream, None)
             fm = statistics.median(f_ms)
             e = {"fwd_ms": round(fm, 4), "fwd_tflops": round(ww.fwd_flops / fm / 1e9, 1),
-                 "fwd_pct_bf16_burst": round(100 * ww.fwd_flops / fm / 1e9 / peaks["bf16_tflops"], 1)}
+                 "fwd_pct_bf16_burst": round(100 * ww.fwd_flops / fm / 1e9 / peaks["bf16_tflops"], 1),
+                 "fwd_pct_bf16_sustained": round(
+                     100 * ww.fwd_flops / fm / 1e9 / peaks["bf16_tflops_sustained"], 1),
+                 "fwd_pct_datasheet": round(100 * ww.fwd_flops / fm / 1e9 / DATASHEET_BF16_TFLOPS, 1),
+                 "fwd_gbs": round(fwd_bytes(ww) / fm / 1e6, 1)}
             if ww.backward:
                 bm = statistics.median(b_ms)
                 e.update({"bwd_ms": round(bm, 4), "bwd_tflops": round(ww.bwd_flops / bm / 1e9, 1),
                           "bwd_pct_bf16_burst": round(
-                              100 * ww.bwd_flops / bm / 1e9 / peaks["bf16_tflops"], 1)})
+                              100 * ww.bwd_flops / bm / 1e9 / peaks["bf16_tflops"], 1),
+                          "bwd_gbs": round(bwd_bytes(ww) / bm / 1e6, 1)})
             extras[name] = e
             torch.cuda.empty_cache()
+        # The small fp16 forward is latency-bound: microseconds and bytes per second.
+        w1 = WORKLOADS[WORKLOAD_ORDER[0]]
+        flush1 = torch.zeros(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+        _, f_ms, _, _ = time_workload(fa2, w1, 50, 5, dev, stream, flush1)
+        fm = statistics.median(f_ms)
+        out["small"] = {"workload": w1.name, "fwd_us": round(fm * 1e3, 2),
+                        "fwd_gbs": round(fwd_bytes(w1) / fm / 1e6, 1),
+                        "fwd_tflops": round(w1.fwd_flops / fm / 1e9, 3),
+                        "note": "launch/latency-bound: 129 KiB of traffic, one CTA per head"}
+        del flush1
         out["other_workloads"] = extras
         out["decode"] = {name: time_decode(fa2, dw, 50, dev, stream, peaks["hbm_gbs"], peaks_src)
                          for name, dw in DECODE_WORKLOADS.items()}
@@ -496,6 +530,9 @@ def run_ours(args):
         out["headline"] = {"workload": HEADLINE_WORKLOAD,
                            "fwd_tflops": extras[HEADLINE_WORKLOAD]["fwd_tflops"],
                            "pct_of_bf16_burst_peak": extras[HEADLINE_WORKLOAD]["fwd_pct_bf16_burst"],
+                           "pct_of_bf16_sustained_peak":
+                               extras[HEADLINE_WORKLOAD]["fwd_pct_bf16_sustained"],
+                           "pct_of_datasheet_dense_bf16": extras[HEADLINE_WORKLOAD]["fwd_pct_datasheet"],
                            "target_pct": 60.0}
     if rank == 0 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(w)
