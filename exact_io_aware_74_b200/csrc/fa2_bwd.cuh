@@ -182,18 +182,11 @@ struct BwdCfg {
   static constexpr int CTRL_BYTES = 256;              // barriers, TMEM address, abort flag
   // No alignment slack: the dynamic region must start 1024-byte aligned (checked).
   static constexpr int SMEM = (2 + 2 * ST) * TILE + DS_BYTES + LD_BYTES + CTRL_BYTES;
-  // Compute warpgroups: each owns QPW query columns of every step.  Four at
-  // D = 64 (halving each warpgroup's exponential and dS work per step), two at
-  // D = 128 (where the registers of 576 threads would not suffice).  Warpgroups 0
-  // and 1 also drain the dQ partial, D / 2 head columns each.
-  static constexpr int NWG = (D == 64) ? 4 : 2;
-  static constexpr int QPW = 128 / NWG;
-  static constexpr int NDR = 2;
-  static constexpr int THREADS = NWG * 128 + 64;  // + TMA producer and MMA warps
+  static constexpr int THREADS = 320;
   static constexpr uint32_t C_S = 0, C_DP = 128;
-  // packed P^T / dS^T of warpgroup g: columns QPW g + (0 | QPW / 2) .. + QPW / 2 - 1
-  __host__ __device__ static constexpr uint32_t C_P(int g) { return QPW * g; }
-  __host__ __device__ static constexpr uint32_t C_DS(int g) { return QPW * g + QPW / 2; }
+  // packed P^T / dS^T of warpgroup g: columns 64 g + (0 | 32) .. + 31
+  __host__ __device__ static constexpr uint32_t C_P(int g) { return 64u * g; }
+  __host__ __device__ static constexpr uint32_t C_DS(int g) { return 64u * g + 32u; }
   static constexpr uint32_t C_DV = 256, C_DK = 256 + D;
   static constexpr uint32_t C_DQ = (D == 128) ? 128 : 384;
 };
@@ -203,7 +196,7 @@ struct BwdCfg {
 template <int ST>
 struct BwdCtrl {
   uint64_t bar_kv, qdo_full[ST], qdo_empty[ST];
-  uint64_t s_full, dp_full, p_ready, ds_ready, dq_full, dq_drained, drain, stage_free;
+  uint64_t s_full, dp_full, p_ready, ds_ready, dq_full, dq_drained, drain;
   uint32_t tmem_slot;
   int abort_flag;
 };
@@ -223,7 +216,7 @@ enum BwdSite : uint32_t {
 };
 
 template <int D, bool BF16, bool CAUSAL>
-__global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
+__global__ void __launch_bounds__(320, 1)
 fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
                const __grid_constant__ CUtensorMap tmdQ, const BwdParams p) {
@@ -256,7 +249,6 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   uint64_t& dq_full = ctl.dq_full;
   uint64_t& dq_drained = ctl.dq_drained;
   uint64_t& drain = ctl.drain;
-  uint64_t& stage_free = ctl.stage_free;
   uint32_t& tmem_slot = ctl.tmem_slot;
   int& abort_flag = ctl.abort_flag;
 
@@ -282,12 +274,11 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     for (int s = 0; s < C::ST; ++s) { mbar_init(&qdo_full[s], 1); mbar_init(&qdo_empty[s], 1); }
     mbar_init(&s_full, 1);
     mbar_init(&dp_full, 1);
-    mbar_init(&p_ready, C::NWG * 4);
-    mbar_init(&ds_ready, C::NWG * 4);
+    mbar_init(&p_ready, 8);
+    mbar_init(&ds_ready, 8);
     mbar_init(&dq_full, 1);
-    mbar_init(&dq_drained, C::NDR * 4);
+    mbar_init(&dq_drained, 8);
     mbar_init(&drain, 1);
-    mbar_init(&stage_free, C::NDR);
     fence_mbar_init();
   }
   if (warp == 0) {
@@ -299,7 +290,7 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   tc_fence_after();
   const uint32_t tbase = tmem_slot;
 
-  if (warp == C::NWG * 4) {
+  if (warp == 8) {
     // ------------------------------------------------------------------ producer
     if (lane == 0) {
       tma_prefetch_desc(&tmQ);
@@ -347,7 +338,7 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       mbar_wait(&bar_kv, 0, dw, kBSiteProdDrain);
     }
     __syncwarp();
-  } else if (warp == C::NWG * 4 + 1) {
+  } else if (warp == 9) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t id_kk = idesc_f16(128, 128, BF16, false, false);  // S^T, dP^T
@@ -388,11 +379,9 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         // dV += P^T dO
         if (!mbar_wait(&p_ready, it & 1, wc, kBSiteMmaP)) { ok = false; break; }
         tc_fence_after();
-        // queries 16 kk .. 16 kk + 15 belong to warpgroup kk / KPW, packed 8 columns each
-        constexpr int KPW = C::QPW / 16;
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          umma_ts(tbase + C::C_DV, tbase + C::C_P(kk / KPW) + (kk % KPW) * 8,
+        for (int kk = 0; kk < 8; ++kk)  // queries 16 kk .. 16 kk + 15: warpgroup kk / 4
+          umma_ts(tbase + C::C_DV, tbase + C::C_P(kk >> 2) + (kk & 3) * 8,
                   sdesc_add(mdO, st * C::TILE + kk * 2048), id_tb,
                   (it > 0 || kk > 0) ? 1u : 0u);
         // dQ_i = dS K first (the drain needs only this one; its own TMEM columns when
@@ -411,7 +400,7 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         umma_commit(&dq_full);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          umma_ts(tbase + C::C_DK, tbase + C::C_DS(kk / KPW) + (kk % KPW) * 8,
+          umma_ts(tbase + C::C_DK, tbase + C::C_DS(kk >> 2) + (kk & 3) * 8,
                   sdesc_add(mQ, st * C::TILE + kk * 2048), id_tb,
                   (it > 0 || kk > 0) ? 1u : 0u);
         umma_commit(&qdo_empty[st]);
@@ -425,16 +414,13 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   } else {
     // ------------------------------------------------------------------ compute
     griddep_wait();  // the accumulator this role adds into was zeroed by the preprocess
-    const int g = warp >> 2;                   // warpgroup: query columns QPW g .. QPW g + QPW - 1
+    const int g = warp >> 2;                   // warpgroup: query columns 64 g .. 64 g + 63
     const int wq = warp & 3;                   // TMEM lane quadrant
     const int r = wq * 32 + lane;              // key row (P^T, dS^T) / query row (dQ)
     const int key = j * 128 + r;
     const uint32_t lb = static_cast<uint32_t>(wq * 32);
     const float sl2 = p.scale_log2;
-    constexpr int QPW = C::QPW;
-    constexpr int NCQ = QPW / 32;              // 32-column TMEM chunks of this warpgroup
-    const int qoff = QPW * g;
-    const bool drains = g < C::NDR;            // this warpgroup moves dQ partials
+    const int qoff = 64 * g;
     const uint32_t wg_bar = 1 + g;             // named barrier of this warpgroup
     bool ok = true;
     for (int it = 0; it < n_it && ok; ++it) {
@@ -453,21 +439,21 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       tc_fence_after();
       // P^T (this warpgroup's 64 query columns): exp2(S^T * scale * log2e - LSE * log2e),
       // zero where the key comes after the query or lies past N.
-      float pr[QPW];
+      float pr[64];
       // Masking (key after query on the diagonal tile, or key past N) is rare: one
       // branch per tile, not a compare per element.
       const int win = p.window;
       const bool masked = (CAUSAL && i == j) || key >= N ||
                           (CAUSAL && win > 0 && i * 128 + 127 - j * 128 >= win);
       const uint64_t sl2x2 = f2_pack(sl2, sl2);
-      uint32_t srr[NCQ][32];
-#pragma unroll
-      for (int c = 0; c < NCQ; ++c) tmem_ld32(tmem_addr(tbase, lb, C::C_S + qoff + 32 * c), srr[c]);
+      uint32_t srr[2][32];
+      tmem_ld32(tmem_addr(tbase, lb, C::C_S + qoff), srr[0]);
+      tmem_ld32(tmem_addr(tbase, lb, C::C_S + qoff + 32), srr[1]);
       tmem_wait_ld();
+      reg_fence(srr[0]);
+      reg_fence(srr[1]);
 #pragma unroll
-      for (int c = 0; c < NCQ; ++c) reg_fence(srr[c]);
-#pragma unroll
-      for (int c = 0; c < NCQ; ++c) {
+      for (int c = 0; c < 2; ++c) {
         const uint32_t (&sr)[32] = srr[c];
 #pragma unroll
         for (int v = 0; v < 8; ++v) {
@@ -495,17 +481,16 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       }
       if (masked) {
 #pragma unroll
-        for (int qc = 0; qc < QPW; ++qc)
+        for (int qc = 0; qc < 64; ++qc)
           if ((CAUSAL && i == j && qoff + qc < r) || key >= N ||
               (CAUSAL && win > 0 && i * 128 + qoff + qc - key >= win))
             pr[qc] = 0.f;
       }
       {
-        uint32_t pk[QPW / 2];
+        uint32_t pk[32];
 #pragma unroll
-        for (int e = 0; e < QPW / 2; ++e) pk[e] = pack2<BF16>(pr[2 * e], pr[2 * e + 1]);
-        if constexpr (QPW == 64) tmem_st32(tmem_addr(tbase, lb, C::C_P(g)), pk);
-        else tmem_st16(tmem_addr(tbase, lb, C::C_P(g)), pk);
+        for (int e = 0; e < 32; ++e) pk[e] = pack2<BF16>(pr[2 * e], pr[2 * e + 1]);
+        tmem_st32(tmem_addr(tbase, lb, C::C_P(g)), pk);
       }
       tmem_wait_st();
       tc_fence_before();
@@ -519,17 +504,13 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       if (!ok) break;
       tc_fence_after();
       if (it > 0) {
-        // The dS^T chunks of shared memory doubled as the staging tiles of the
-        // previous dQ reduces: those bulk copies must have finished reading them.
-        if (drains && r == 0) {
-          tma_store_wait_read();
-          mbar_arrive(&stage_free);
-        }
-        ok = named_bar_and(wg_bar, 128, mbar_wait(&stage_free, (it - 1) & 1, wc, kBSiteCmpDP));
-        if (!ok) break;
+        // This warpgroup's dS^T chunk doubled as the staging tile of the previous
+        // dQ reduce: that bulk copy must have finished reading it.
+        if (r == 0) tma_store_wait_read();
+        named_bar_sync(wg_bar, 128);
       }
 #pragma unroll
-      for (int c = 0; c < NCQ; ++c) {
+      for (int c = 0; c < 2; ++c) {
         uint32_t dr[32];
         tmem_ld32(tmem_addr(tbase, lb, C::C_DP + qoff + 32 * c), dr);
         tmem_wait_ld();
@@ -554,10 +535,7 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         for (int uu = 0; uu < 4; ++uu) {
           const int u = c * 4 + uu;
           const uint4 val = make_uint4(dsk[4 * uu], dsk[4 * uu + 1], dsk[4 * uu + 2], dsk[4 * uu + 3]);
-          // query qoff + 32 c + 8 uu: chunk of 64 queries, 16-byte unit within it
-          const int q = qoff + 32 * c + 8 * uu;
-          *reinterpret_cast<uint4*>(sDS + (q >> 6) * C::CHUNK + r * 128 +
-                                    ((((q & 63) >> 3) ^ (r & 7)) << 4)) = val;
+          *reinterpret_cast<uint4*>(sDS + g * C::CHUNK + r * 128 + ((u ^ (r & 7)) << 4)) = val;
         }
       }
       fence_proxy_async_smem();
@@ -565,17 +543,16 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&ds_ready);
-      if (!drains) continue;
       // dQ partial: query row r, head columns g D/2 .. (g+1) D/2 - 1 -> fp32 accumulator
       ok = named_bar_and(wg_bar, 128, mbar_wait(&dq_full, it & 1, wc, kBSiteCmpDQ));
       if (!ok) break;
       tc_fence_after();
       // dQ partial, head columns g D/2 .. (g+1) D/2 - 1, 32 at a time: TMEM ->
-      // dS^T chunk g of shared memory (free: the dQ product that read it has
-      // completed), laid out as a 128-row x 32-float tile with 128-byte swizzle
-      // -> one TMA reduce-add into the fp32 accumulator (rows past N are clipped
-      // by the tensor map).
-      constexpr int HALF = D / C::NDR;
+      // this warpgroup's dS^T chunk of shared memory (free: the dQ product that
+      // read it has completed), laid out as a 128-row x 32-float tile with
+      // 128-byte swizzle -> one TMA reduce-add into the fp32 accumulator (rows
+      // past N are clipped by the tensor map).
+      constexpr int HALF = D / 2;
       constexpr int NCH = HALF / 32;
       uint8_t* stage = sDS + g * C::CHUNK;
       // All of this warpgroup's TMEM columns first, so that the region is released
@@ -612,21 +589,17 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     // All reductions complete before the CTA (and its shared memory) goes away.
     if (r == 0) tma_store_wait_all();
     __syncwarp();
-    // dV (even warpgroups) and dK (odd ones) are final once every MMA has landed;
-    // with four warpgroups each writes half of the head columns.
+    // dV (warpgroup 0) and dK (warpgroup 1) are final once every MMA has landed.
     if (ok) ok = named_bar_and(wg_bar, 128, mbar_wait(&drain, 0, wc, kBSiteCmpDQ));
     if (ok) {
       tc_fence_after();
-      const bool is_dk = (g & 1) != 0;
-      const uint32_t col = is_dk ? C::C_DK : C::C_DV;
-      const float mul = is_dk ? p.scale : 1.0f;
-      constexpr int CPW = (D / 32) / (C::NWG / 2);  // 32-column chunks per warpgroup
-      const int c_begin = (g >> 1) * CPW;
+      const uint32_t col = g ? C::C_DK : C::C_DV;
+      const float mul = g ? p.scale : 1.0f;
       const int d = p.d;
-      uint8_t* row = reinterpret_cast<uint8_t*>(is_dk ? p.dK : p.dV) +
+      uint8_t* row = reinterpret_cast<uint8_t*>(g ? p.dK : p.dV) +
                      (static_cast<size_t>(bh) * N + key) * (d * 2);
 #pragma unroll
-      for (int c = c_begin; c < c_begin + CPW; ++c) {
+      for (int c = 0; c < D / 32; ++c) {
         uint32_t rr[32];
         tmem_ld32(tmem_addr(tbase, lb, col + 32 * c), rr);
         tmem_wait_ld();
