@@ -160,7 +160,7 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 
   __shared__ uint64_t bar_q, k_full[C::KS], k_empty[C::KS], v_full[C::VS + C::VX],
       v_empty[C::VS + C::VX];
-  __shared__ uint64_t s_full[2], s_free[2], p_half[2], p_ready[2], o_done[2], drain;
+  __shared__ uint64_t s_full[2], s_free[2], p_ready[2], o_done[2], drain;
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
 
@@ -223,7 +223,6 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     for (int t = 0; t < 2; ++t) {
       mbar_init(&s_full[t], 1);
       mbar_init(&s_free[t], 4);
-      mbar_init(&p_half[t], 4);
       mbar_init(&p_ready[t], 4);
       mbar_init(&o_done[t], 1);
     }
@@ -351,12 +350,10 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       };
       // P from TMEM (8 columns = 32 bytes of keys per step), V MN-major: a step
       // of KE keys advances KE rows of 128 bytes.
-      // P's first half (keys 0-63) can be consumed before its second half is written.
-      constexpr int KSTEPS = C::BN / C::KE;
-      auto issue_pv = [&](int t, uint32_t a_col, int vs, bool acc, int kk0, int kk1) {
+      auto issue_pv = [&](int t, uint32_t a_col, int vs, bool acc) {
         const uint32_t va = v_addr(vs);
 #pragma unroll
-        for (int kk = kk0; kk < kk1; ++kk) {
+        for (int kk = 0; kk < C::BN / C::KE; ++kk) {
           const uint32_t dt = tbase + (t ? C::O_COL1 : C::O_COL0);
           const uint32_t at = tbase + a_col + kk * 8;
           const uint64_t db = sdesc_sw128(va + kk * C::KE * 128, C::CHUNK, 1024);
@@ -393,18 +390,12 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           constexpr int VR = C::VS + C::VX;  // V ring with the second Q slot
           const int vs = jj % VR;
           if (!mbar_wait(&v_full[vs], (jj / VR) & 1, wc, kSiteMmaV) ||
-              !mbar_wait(&p_half[b], (jj >> 1) & 1, wc, kSiteMmaP)) {
+              !mbar_wait(&p_ready[b], (jj >> 1) & 1, wc, kSiteMmaP)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          issue_pv(0, b ? C::S_COL1 : C::S_COL0, vs, jj > 0, 0, KSTEPS / 2);
-          if (!mbar_wait(&p_ready[b], (jj >> 1) & 1, wc, kSiteMmaP)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          issue_pv(0, b ? C::S_COL1 : C::S_COL0, vs, true, KSTEPS / 2, KSTEPS);
+          issue_pv(0, b ? C::S_COL1 : C::S_COL0, vs, jj > 0);
           umma_commit(&o_done[0]);
           umma_commit(&v_empty[vs]);
         }
@@ -452,13 +443,10 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         auto pv = [&](int t, int lo, int hi) -> bool {
           if (j >= lo && j < hi) {
             const int step = j - lo;  // this tile's own step count
-            const uint32_t a_col = sep ? (t ? C::P_COL1 : C::P_COL0) : (t ? C::S_COL1 : C::S_COL0);
-            if (!mbar_wait(&p_half[t], step & 1, wc, kSiteMmaP)) return false;
-            tc_fence_after();
-            issue_pv(t, a_col, vs, step > 0, 0, KSTEPS / 2);
             if (!mbar_wait(&p_ready[t], step & 1, wc, kSiteMmaP)) return false;
             tc_fence_after();
-            issue_pv(t, a_col, vs, true, KSTEPS / 2, KSTEPS);
+            const uint32_t a_col = sep ? (t ? C::P_COL1 : C::P_COL0) : (t ? C::S_COL1 : C::S_COL0);
+            issue_pv(t, a_col, vs, step > 0);
             umma_commit(&o_done[t]);
           }
           return true;
@@ -509,15 +497,11 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     // rows feed output rows that are never stored.
     const bool live = my_row0 + (wq * 32) % QR < Nq;
 
-    // 16-bit P of one query copy is stored in two 64-key pieces: the first is
-    // signalled (p_half) as soon as it is in TMEM.  Otherwise both signals come
-    // together at the end of the step.
-    constexpr bool kSplitP = !F8 && REP == 1;
     // One step of the online softmax over the NC key columns this warp owns:
     // S from TMEM, masks, running max (with the lazy output rescale), P back to
     // TMEM in 16-bit over the first 64 columns of the S buffer -- zeros in the
     // columns of the other copies -- and the running sum.  False if a wait ran out.
-    auto soft_step = [&](auto nc_tag, int step, uint32_t s_col, int buf) -> bool {
+    auto soft_step = [&](auto nc_tag, int step, uint32_t s_col) -> bool {
       constexpr int NC = decltype(nc_tag)::value;
       constexpr int EPC = 4 / C::ESZ;             // P values per 32-bit TMEM column
       constexpr int NP = NC / EPC;                // packed columns of P
@@ -635,14 +619,6 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         }
         const uint32_t dst = tmem_addr(tbase, lane_base, p_col + col0 / EPC + G * h);
         if constexpr (G == 32) tmem_st32(dst, pk); else tmem_st16(dst, pk);
-        if constexpr (kSplitP) {
-          if (h == 0) {  // keys 0-63 of P are in TMEM: the first half of P V may start
-            tmem_wait_st();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&p_half[buf]);
-          }
-        }
       }
       if constexpr (NC < 128) {
         // The other copies' key columns contribute nothing to this copy's rows.
@@ -676,7 +652,7 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       if (!ok) break;
       if (live) {
         tc_fence_after();
-        ok = soft_step(std::integral_constant<int, C::BN / REP>{}, step, s_col, buf);
+        ok = soft_step(std::integral_constant<int, C::BN / REP>{}, step, s_col);
         if (!ok) break;
         tmem_wait_st();
         tc_fence_before();
@@ -692,10 +668,7 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         }
       }
       __syncwarp();
-      if (lane == 0) {
-        if (!kSplitP || !live) mbar_arrive(&p_half[buf]);
-        mbar_arrive(&p_ready[buf]);
-      }
+      if (lane == 0) mbar_arrive(&p_ready[buf]);
     }
     // Wait for the last P V product.  A phase-parity wait is only sound while the
     // barrier is at most one phase behind.  With one tile per CTA, S of the last
