@@ -89,13 +89,27 @@ KERNEL_SOURCES = {"fa2_fwd": ("ptx.cuh", "fa2_fwd.cuh"), "fa2_bwd": ("ptx.cuh", 
                   "fa2_fwd_decode": ("ptx.cuh", "fa2_fwd.cuh", "fa2_decode.cuh")}
 
 
+def _code_only(src: str) -> str:
+    """C++ source without comments and blank lines: edits to comments alone do not
+    change the kernels a traffic record was taken from."""
+    import re
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    out = []
+    for line in src.splitlines():
+        # drop // comments (the kernels have no "//" inside string literals)
+        line = line.split("//", 1)[0].rstrip()
+        if line:
+            out.append(line)
+    return "\n".join(out)
+
+
 def csrc_hash(call: str) -> str:
-    """Hash of the device source files of one call's kernels."""
+    """Hash of the code (comments aside) of the device source files of one call's kernels."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "exact_io_aware_74_b200", "csrc")
     for name in KERNEL_SOURCES[call]:
-        with open(os.path.join(csrc, name), "rb") as f:
-            h.update(name.encode() + f.read())
+        with open(os.path.join(csrc, name), encoding="utf-8") as f:
+            h.update(name.encode() + _code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 

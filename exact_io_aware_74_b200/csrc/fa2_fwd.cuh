@@ -9,8 +9,8 @@
 //   принципы работы": (1) fewer non-matmul operations -- here the running
 //   maximum is only applied to the output when it grows by more than 2^8, and
 //   the 1/l normalisation happens once at the end; (2) parallelism over the
-//   sequence -- every CTA owns 256 query rows of one (batch, head); (3) work
-//   split across warps so that softmax statistics never go through shared
+//   sequence -- every CTA owns up to 256 query rows of one (batch, head); (3)
+//   work split across warps so that softmax statistics never go through shared
 //   memory -- here one thread owns one query row, read straight from TMEM.
 //   "Flash Attention spiegata", "Specializzazione dei warp" and "TMA":
 //   producer and consumer warps and asynchronous tile copies (Hopper-era prior
@@ -28,16 +28,24 @@
 // re-split never asks for more than the launch holds.  (232 / 40 and 224 / 56
 // made the MMA issuer spill.)  The host refuses to launch a build whose register
 // count is not 168.
+//
 // TMEM (512 columns x 128 lanes, fp32): S_t at column 128 t, O_t at 256 + D t.
 // P_t (16-bit) overwrites the first 64 columns of S_t and feeds the P V MMA
 // straight from TMEM.  The MMA warp alternates between the two query tiles so
-// that one warpgroup's softmax overlaps the other tile's matrix products.
-// A CTA with one query tile (short or decode-like queries) instead uses both S
-// column blocks as a double buffer -- S of step j + 1 is computed while the
-// softmax of step j runs -- and its idle second Q slot as one more V stage.  Decode-like calls may also cut the keys into
+// that one warpgroup's softmax overlaps the other tile's matrix products.  At
+// D = 64 the two P have columns of their own (384 and 448), so S of step j + 1
+// is computed as soon as the softmax has read S of step j.
+//
+// A CTA with one query tile -- short or decode-like queries, and every CTA at
+// tile widths D = 192 / 256, where two D-column accumulators would not fit TMEM
+// -- instead uses both S column blocks as a double buffer (S of step j + 1 is
+// computed while the softmax of step j runs) and its idle second Q slot, if
+// any, as one more V stage.  Decode-like calls may also cut the keys into
 // stretches (one per blockIdx.y) and replicate up to 64 queries down the tile
 // so every softmax warp has rows to work on; both write partial results that
-// fa2_decode.cuh merges.
+// fa2_decode.cuh merges.  With 8-bit inputs (F8) the tiles are 128 bytes wide,
+// the products are kind::f8f6f4 MMAs and P is rounded to E4M3, four per TMEM
+// column.
 #pragma once
 
 #include <type_traits>
@@ -49,7 +57,8 @@ namespace fa2 {
 struct FwdParams {
   void* O;                     // [BH][Nq][d] 16-bit (unused when the keys are split)
   float* LSE;                  // [BH][Nq]            (unused when the keys are split)
-  int d;                       // head dim, a multiple of 8, D - 64 < d <= D (columns past d
+  int d;                       // head dim: 16-bit inputs D - 64 < d <= D, a multiple of 8;
+                               // 8-bit inputs a multiple of 16 up to 128 (columns past d
                                // of the tiles are TMA zero fill and are never stored)
   int Nq;                      // query rows per (batch, head)
   int Nk;                      // key / value rows per (batch, head)
