@@ -553,7 +553,7 @@ int bwd_impl(const void* Q, const void* K, const void* V, const void* O, const v
   if (!st) return FA2_ERR_CUDA;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   rc = fa2::launch_bwd(Q, K, V, O, dO, LSE, dQ, dK, dV, workspace, BH, N, d, scale, causal != 0,
-                       dtype == FA2_BF16, st, wait_ns(), s, window);
+                       dtype == FA2_BF16, st, wait_ns(), s, window, g_fault.load());
   if (rc == FA2_OK) g_launches.fetch_add(fa2::kBwdKernelsPerCall);
   return rc;
 }
@@ -660,7 +660,7 @@ int fa2_bwd_noalloc(const void* Q, const void* K, const void* V, const void* O, 
   if (!st) st = reinterpret_cast<unsigned int*>(base);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   rc = fa2::launch_bwd(Q, K, V, O, dO, LSE, dQ, dK, dV, base + kNoAllocStatusBytes, BH, N, d,
-                       scale, causal != 0, dtype == FA2_BF16, st, wait_ns(), s);
+                       scale, causal != 0, dtype == FA2_BF16, st, wait_ns(), s, 0, g_fault.load());
   if (rc == FA2_OK) g_launches.fetch_add(fa2::kBwdKernelsPerCall);
   return rc;
 }

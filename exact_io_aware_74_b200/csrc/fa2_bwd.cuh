@@ -169,6 +169,7 @@ struct BwdParams {
   float scale, scale_log2;
   unsigned int* status;
   unsigned long long wait_ns;
+  int fault;          // test hook: 1 = skip the K, V load (a consumer's wait runs out)
 };
 
 template <int D>
@@ -297,10 +298,12 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
       tma_prefetch_desc(&tmdO);
-      mbar_arrive_expect_tx(&bar_kv, 2 * C::TILE);
-      for (int c = 0; c < C::KCH; ++c) {
-        tma_load_3d(sK + c * C::CHUNK, &tmK, &bar_kv, c * 64, j * 128, bh);
-        tma_load_3d(sV + c * C::CHUNK, &tmV, &bar_kv, c * 64, j * 128, bh);
+      if (p.fault != 1) {
+        mbar_arrive_expect_tx(&bar_kv, 2 * C::TILE);
+        for (int c = 0; c < C::KCH; ++c) {
+          tma_load_3d(sK + c * C::CHUNK, &tmK, &bar_kv, c * 64, j * 128, bh);
+          tma_load_3d(sV + c * C::CHUNK, &tmV, &bar_kv, c * 64, j * 128, bh);
+        }
       }
       const uint64_t keep = policy_evict_last();
       // K and V do not depend on the preprocess; the L, D rows (and the zeroed
@@ -334,8 +337,9 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         for (int it = max(0, issued - C::ST); it < issued; ++it)
           mbar_wait(&qdo_full[it % C::ST], (it / C::ST) & 1, dw, kBSiteProdDrain);
       }
-      // K and V always land before exit, even on an aborted run.
-      mbar_wait(&bar_kv, 0, dw, kBSiteProdDrain);
+      // K and V always land before exit, even on an aborted run (unless the test
+      // hook skipped them: then nothing is in flight).
+      if (p.fault != 1) mbar_wait(&bar_kv, 0, dw, kBSiteProdDrain);
     }
     __syncwarp();
   } else if (warp == 9) {
@@ -662,7 +666,7 @@ template <int D, bool BF16, bool CAUSAL>
 int launch_bwd_t(const void* Q, const void* K, const void* V, const void* O, const void* dO,
                  const float* LSE, void* dQ, void* dK, void* dV, void* workspace, int BH, int N,
                  int d, float scale, int window, unsigned int* status, unsigned long long wait_ns,
-                 cudaStream_t stream) {
+                 int fault, cudaStream_t stream) {
   using Cfg = BwdCfg<D>;
   const int Npad = static_cast<int>(bwd_npad(N));
   if (static_cast<long long>(Npad / 128) * BH > 0x7fffffffll) return 1;  // FA2_ERR_INVALID_ARG
@@ -709,6 +713,7 @@ int launch_bwd_t(const void* Q, const void* K, const void* V, const void* O, con
     bp.window = window;
     bp.status = status;
     bp.wait_ns = wait_ns;
+    bp.fault = fault;
     const unsigned int grid = static_cast<unsigned int>(bp.n_kv) * static_cast<unsigned int>(BH);
     if (launch_pdl(kern, dim3(grid), dim3(Cfg::THREADS), Cfg::SMEM, stream, mq, mk, mv, mdo, mdq,
                    bp) != cudaSuccess)
@@ -728,10 +733,11 @@ int launch_bwd_t(const void* Q, const void* K, const void* V, const void* O, con
 inline int launch_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO,
                       const float* LSE, void* dQ, void* dK, void* dV, void* workspace, int BH,
                       int N, int d, float scale, bool causal, bool bf16, unsigned int* status,
-                      unsigned long long wait_ns, cudaStream_t s, int window = 0) {
+                      unsigned long long wait_ns, cudaStream_t s, int window = 0,
+                      int fault = 0) {
 #define FA2_BWD_CALL(D_, BF_, CA_)                                                             \
   return launch_bwd_t<D_, BF_, CA_>(Q, K, V, O, dO, LSE, dQ, dK, dV, workspace, BH, N, d, scale, \
-                                    window, status, wait_ns, s)
+                                    window, status, wait_ns, fault, s)
   if (d <= 64) {
     if (bf16) { if (causal) FA2_BWD_CALL(64, true, true); FA2_BWD_CALL(64, true, false); }
     if (causal) FA2_BWD_CALL(64, false, true);

@@ -243,9 +243,10 @@ const char* fa2_status_string(int status);
 /*
  * Test hook.  ``wait_limit_ms`` sets the wall-clock budget of every bounded
  * in-kernel wait (0 restores the default of 2000 ms).  ``fault`` = 1 makes the
- * next forward launches skip their first K-tile load, so a consumer's wait
- * runs out and the timeout path is exercised without any GPU fault; 0 turns it
- * off.  Not for production use.
+ * next forward launches skip their first K-tile load and the next backward
+ * launches skip their K and V load, so a consumer's wait runs out and the
+ * timeout path is exercised without any GPU fault; 0 turns it off.  Not for
+ * production use.
  */
 void fa2_debug_set(int fault, unsigned int wait_limit_ms);
 
