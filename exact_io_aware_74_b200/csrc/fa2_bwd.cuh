@@ -42,6 +42,8 @@
 
 #include <cuda_fp16.h>
 
+#include <atomic>
+
 #include "ptx.cuh"
 
 namespace fa2 {
@@ -641,6 +643,27 @@ bool make_tile_map(CUtensorMap* map, const void* base, int BH, int N, int d, boo
                    int box_rows = 128);
 bool make_acc_map(CUtensorMap* map, float* base, int BH, int N, int d);
 
+// Raises a kernel's dynamic shared memory limit once per device (the attribute is
+// host state, set before the first launch on each device, not per call).
+template <typename Kern>
+bool set_smem_once(Kern kern, int smem) {
+  constexpr int kDevs = 64;
+  static std::atomic<bool> done[kDevs];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kDevs) {
+    cudaGetLastError();
+    return false;
+  }
+  if (done[dev].load(std::memory_order_acquire)) return true;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+      cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  done[dev].store(true, std::memory_order_release);
+  return true;
+}
+
 // Launch with programmatic stream serialisation: the kernel may start while the
 // previous kernel on the stream finishes; it waits (griddepcontrol.wait) before
 // touching that kernel's results.
@@ -692,11 +715,7 @@ int launch_bwd_t(const void* Q, const void* K, const void* V, const void* O, con
   // 2. main
   {
     auto kern = fa2_bwd_kernel<D, BF16, CAUSAL>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM) !=
-        cudaSuccess) {
-      cudaGetLastError();
-      return 4;
-    }
+    if (!set_smem_once(kern, Cfg::SMEM)) return 4;
     BwdParams bp{};
     bp.Dg = Dg;
     bp.Lg = Lg;
