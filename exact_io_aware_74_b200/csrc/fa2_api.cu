@@ -191,7 +191,8 @@ int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& 
     cudaGetLastError();
     return FA2_ERR_CUDA;
   }
-  if (!fa2::set_smem_once(kern, Cfg::SMEM)) return FA2_ERR_CUDA;
+  static std::atomic<bool> smem_set[fa2::kSmemFlagDevices];  // this instantiation's flags
+  if (!fa2::set_smem_once(kern, Cfg::SMEM, smem_set)) return FA2_ERR_CUDA;
   const dim3 grid(static_cast<unsigned int>(p.n_qblk) * static_cast<unsigned int>(p.BH),
                   static_cast<unsigned int>(n_split));
   kern<<<grid, Cfg::THREADS, Cfg::SMEM, stream>>>(mq, mk, mv, mqr, p);

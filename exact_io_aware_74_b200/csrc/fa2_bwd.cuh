@@ -644,13 +644,13 @@ bool make_tile_map(CUtensorMap* map, const void* base, int BH, int N, int d, boo
 bool make_acc_map(CUtensorMap* map, float* base, int BH, int N, int d);
 
 // Raises a kernel's dynamic shared memory limit once per device (the attribute is
-// host state, set before the first launch on each device, not per call).
+// host state, set before the first launch on each device, not per call).  Every
+// kernel instantiation passes flags of its own (a static array in its launcher).
+constexpr int kSmemFlagDevices = 64;
 template <typename Kern>
-bool set_smem_once(Kern kern, int smem) {
-  constexpr int kDevs = 64;
-  static std::atomic<bool> done[kDevs];
+bool set_smem_once(Kern kern, int smem, std::atomic<bool> (&done)[kSmemFlagDevices]) {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kDevs) {
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kSmemFlagDevices) {
     cudaGetLastError();
     return false;
   }
@@ -715,7 +715,8 @@ int launch_bwd_t(const void* Q, const void* K, const void* V, const void* O, con
   // 2. main
   {
     auto kern = fa2_bwd_kernel<D, BF16, CAUSAL>;
-    if (!set_smem_once(kern, Cfg::SMEM)) return 4;
+    static std::atomic<bool> smem_set[kSmemFlagDevices];  // this instantiation's flags
+    if (!set_smem_once(kern, Cfg::SMEM, smem_set)) return 4;
     BwdParams bp{};
     bp.Dg = Dg;
     bp.Lg = Lg;
