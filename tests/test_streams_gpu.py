@@ -103,7 +103,7 @@ def test_cuda_graph_capture_replays_forward_backward_and_decode():
         outs = _fwd_bwd(q, k, v, do, s, ws)
         assert fa2.fa2_fwd_decode(qd, kd, vd, od, lsed, 0.1, True, sp, wsd, s) == fa2.FA2_OK
     for _ in range(3):
-        for t in outs + [od, lsed]:
+        for t in list(outs) + [od, lsed]:
             t.zero_()
         g.replay()
         torch.cuda.synchronize()
