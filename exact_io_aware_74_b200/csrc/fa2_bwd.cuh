@@ -179,11 +179,7 @@ struct BwdCfg {
   static constexpr int KCH = D / 64;
   static constexpr int CHUNK = 128 * 128;
   static constexpr int TILE = 128 * D * 2;
-#ifndef FA2_BWD_ST64
-#define FA2_BWD_ST64 2
-#endif
-  // (Q, dO) ring stages: 231.7 KB of shared memory at D = 128 leave room for two.
-  static constexpr int ST = (D == 64) ? FA2_BWD_ST64 : 2;
+  static constexpr int ST = 2;                 // (Q, dO) ring stages
   static constexpr int DS_BYTES = 128 * 128 * 2;
   static constexpr int LD_BYTES = ST * 2 * 128 * 4;  // LSE*log2e and D rows of each stage
   static constexpr int CTRL_BYTES = 256;              // barriers, TMEM address, abort flag
