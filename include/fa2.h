@@ -33,8 +33,10 @@
  *   - The return value reports argument validation and launch only; the kernels
  *     run asynchronously.  Failures inside a kernel (a bounded wait that ran out)
  *     are reported by fa2_get_device_status().
- *   - Head dims 64 and 128 are supported; any other d returns
- *     FA2_ERR_UNSUPPORTED and launches nothing (no silent fallback).
+ *   - Head dims: any multiple of 8 from 8 to 256 in the forward calls
+ *     (fa2_fwd, fa2_fwd_window, fa2_fwd_decode), from 8 to 128 in the backward
+ *     calls, and any multiple of 16 up to 128 in fa2_fwd_fp8.  Any other d
+ *     returns FA2_ERR_UNSUPPORTED and launches nothing (no silent fallback).
  *   - Only compute capability 10.0 devices (B200, sm_100a) are supported;
  *     others return FA2_ERR_ARCH.
  *   - The library allocates one small device status word per device on first
@@ -55,7 +57,7 @@ typedef struct CUstream_st* fa2_stream_t;
 typedef enum {
   FA2_OK = 0,
   FA2_ERR_INVALID_ARG = 1, /* null / misaligned pointer, bad size, flag or scale */
-  FA2_ERR_UNSUPPORTED = 2, /* head dim other than 64 or 128 */
+  FA2_ERR_UNSUPPORTED = 2, /* head dim the call does not support */
   FA2_ERR_ARCH = 3,        /* current device is not compute capability 10.0 */
   FA2_ERR_CUDA = 4,        /* a CUDA runtime / driver call failed */
   FA2_ERR_TIMEOUT = 5,     /* a bounded in-kernel wait ran out (device status) */
@@ -71,7 +73,8 @@ typedef enum { FA2_FP16 = 0, FA2_BF16 = 1 } fa2_dtype;
  *   Q, K, V : in,  [B][H][N][d] dtype
  *   O       : out, [B][H][N][d] dtype, O_i = sum_j softmax_j(S_i) V_j
  *   LSE     : out, [B][H][N] float (natural log, scaled-score units)
- *   B, H, N : >= 1; d in {64, 128}; scale finite; causal in {0, 1};
+ *   B, H, N : >= 1; d a multiple of 8 up to 256; scale finite and > 0;
+ *             causal in {0, 1};
  *   dtype   : FA2_FP16 or FA2_BF16
  * O must not overlap Q, K or V.  Results are bitwise repeatable run to run.
  */
@@ -113,7 +116,7 @@ int fa2_fwd_window(const void* Q, const void* K, const void* V, void* O, float* 
  *   Q, O     : [B][H][Nq][d] dtype (in, out)
  *   K, V     : [B][H][Nk][d] dtype (in)
  *   LSE      : out, [B][H][Nq] float
- *   B, H     : >= 1; 1 <= Nq <= Nk; d in {64, 128}; causal in {0, 1}
+ *   B, H     : >= 1; 1 <= Nq <= Nk; d a multiple of 8 up to 256; causal in {0, 1}
  *   n_splits : 1 .. 1024 (FA2_ERR_INVALID_ARG otherwise); counts above the
  *              number of key tiles act as one tile per split
  *   workspace: device scratch of at least fa2_fwd_decode_workspace_size()
@@ -179,6 +182,7 @@ size_t fa2_bwd_workspace_size(int B, int H, int N, int d);
  *   Q, K, V, O, dO : in,  [B][H][N][d] dtype (O and LSE as fa2_fwd wrote them)
  *   LSE            : in,  [B][H][N] float
  *   dQ, dK, dV     : out, [B][H][N][d] dtype
+ *   d              : a multiple of 8 up to 128 (FA2_ERR_UNSUPPORTED otherwise)
  *   workspace      : scratch of at least fa2_bwd_workspace_size() bytes,
  *                    256-byte aligned, owned by the caller; its contents on
  *                    entry do not matter and on return are unspecified
