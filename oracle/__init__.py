@@ -37,7 +37,13 @@ is the plainest one):
 * LSE_i: natural log of sum_j exp(S_ij) over the unmasked keys of row i, in
   units of the scaled scores S = scale * Q K^T;
 * backward of the loss L with dL/dO = dO: dV = P^T dO, dP = dO V^T,
-  D_i = sum_j P_ij dP_ij, dS = P * (dP - D), dQ = scale dS K, dK = scale dS^T Q.
+  D_i = sum_j P_ij dP_ij, dS = P * (dP - D), dQ = scale dS K, dK = scale dS^T Q;
+* sliding window W (causal only): query i sees keys i - W + 1 .. i;
+* decode-like attention (``attn_fwd_decode_ref``): the Nq <= Nk queries are the
+  last Nq positions, so with the causal mask query i sees keys 0 .. Nk - Nq + i;
+* 8-bit inputs (``attn_fwd_fp8_ref``): E4M3 codes (bias 7, three mantissa bits,
+  no infinities; ``e4m3_decode`` follows the format's definition) times a
+  per-tensor scale, then the plain definition above.
 
 Every function is pinned by ``tests/test_oracle.py`` against things other than
 itself: the scalar brute force, PyTorch's fp64 CPU attention and autograd,
