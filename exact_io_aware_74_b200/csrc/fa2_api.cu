@@ -24,6 +24,7 @@ std::mutex g_mu;
 unsigned int* g_status[kMaxDevices] = {};  // one device word per device, lazily allocated
 std::atomic<int> g_fault{0};
 std::atomic<unsigned int> g_wait_ms{kDefaultWaitMs};
+std::atomic<int> g_bwd_ctas{0};  // test hook: cap on the backward grid (0 = one CTA per SM)
 std::atomic<unsigned long long> g_launches{0};
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -550,7 +551,8 @@ int bwd_impl(const void* Q, const void* K, const void* V, const void* O, const v
   if (!st) return FA2_ERR_CUDA;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   rc = fa2::launch_bwd(Q, K, V, O, dO, LSE, dQ, dK, dV, workspace, BH, N, d, scale, causal != 0,
-                       dtype == FA2_BF16, st, wait_ns(), s, window, g_fault.load());
+                       dtype == FA2_BF16, st, wait_ns(), s, window, g_fault.load(),
+                       g_bwd_ctas.load());
   if (rc == FA2_OK) g_launches.fetch_add(fa2::kBwdKernelsPerCall);
   return rc;
 }
@@ -657,7 +659,8 @@ int fa2_bwd_noalloc(const void* Q, const void* K, const void* V, const void* O, 
   if (!st) st = reinterpret_cast<unsigned int*>(base);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   rc = fa2::launch_bwd(Q, K, V, O, dO, LSE, dQ, dK, dV, base + kNoAllocStatusBytes, BH, N, d,
-                       scale, causal != 0, dtype == FA2_BF16, st, wait_ns(), s, 0, g_fault.load());
+                       scale, causal != 0, dtype == FA2_BF16, st, wait_ns(), s, 0, g_fault.load(),
+                       g_bwd_ctas.load());
   if (rc == FA2_OK) g_launches.fetch_add(fa2::kBwdKernelsPerCall);
   return rc;
 }
@@ -698,6 +701,8 @@ void fa2_debug_set(int fault, unsigned int wait_limit_ms) {
   g_fault.store(fault == 1 ? 1 : 0);
   g_wait_ms.store(wait_limit_ms == 0 ? kDefaultWaitMs : wait_limit_ms);
 }
+
+void fa2_debug_set_bwd_grid(int max_ctas) { g_bwd_ctas.store(max_ctas > 0 ? max_ctas : 0); }
 
 unsigned long long fa2_launch_count(void) { return g_launches.load(); }
 

@@ -42,6 +42,7 @@
 
 #include <cuda_fp16.h>
 
+#include <algorithm>
 #include <atomic>
 
 #include "ptx.cuh"
@@ -180,11 +181,15 @@ struct BwdCfg {
   static constexpr int CHUNK = 128 * 128;
   static constexpr int TILE = 128 * D * 2;
   static constexpr int ST = 2;                 // (Q, dO) ring stages
+  // K/V buffers: a CTA runs several key tiles in turn.  At D = 64 the next tile's
+  // K and V load into a buffer of their own while the current tile runs; at
+  // D = 128 there is room for one, reloaded once the tile's last product has read it.
+  static constexpr int KVB = (D == 64) ? 2 : 1;
   static constexpr int DS_BYTES = 128 * 128 * 2;
   static constexpr int LD_BYTES = ST * 2 * 128 * 4;  // LSE*log2e and D rows of each stage
   static constexpr int CTRL_BYTES = 256;              // barriers, TMEM address, abort flag
   // No alignment slack: the dynamic region must start 1024-byte aligned (checked).
-  static constexpr int SMEM = (2 + 2 * ST) * TILE + DS_BYTES + LD_BYTES + CTRL_BYTES;
+  static constexpr int SMEM = (2 * KVB + 2 * ST) * TILE + DS_BYTES + LD_BYTES + CTRL_BYTES;
   static constexpr int THREADS = 320;
   static constexpr uint32_t C_S = 0, C_DP = 128;
   // packed P^T / dS^T of warpgroup g: columns 64 g + (0 | 32) .. + 31
@@ -198,8 +203,8 @@ struct BwdCfg {
 // so that the 1024-byte aligned tiles start at the base of the window).
 template <int ST>
 struct BwdCtrl {
-  uint64_t bar_kv, qdo_full[ST], qdo_empty[ST];
-  uint64_t s_full, dp_full, p_ready, ds_ready, dq_full, dq_drained, drain;
+  uint64_t bar_kv[2], kv_empty[2], acc_free, qdo_full[ST], qdo_empty[ST];
+  uint64_t s_full, dp_full, p_ready, ds_ready, dq_full, dq_drained, drain, fin;
   uint32_t tmem_slot;
   int abort_flag;
 };
@@ -215,7 +220,8 @@ __device__ __forceinline__ void bulk_load_1d(void* smem_dst, const void* gmem_sr
 
 enum BwdSite : uint32_t {
   kBSiteAlign = 31, kBSiteProdEmpty = 32, kBSiteMmaKV, kBSiteMmaQ, kBSiteMmaDrained, kBSiteMmaP, kBSiteMmaDS,
-  kBSiteMmaDrain, kBSiteCmpQ, kBSiteCmpS, kBSiteCmpDP, kBSiteCmpDQ, kBSiteProdDrain
+  kBSiteMmaDrain, kBSiteCmpQ, kBSiteCmpS, kBSiteCmpDP, kBSiteCmpDQ, kBSiteProdDrain, kBSiteMmaAcc,
+  kBSiteProdKV
 };
 
 template <int D, bool BF16, bool CAUSAL>
@@ -234,15 +240,17 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   // this grid to complete before reading the accumulator.
   griddep_launch_dependents();
   uint8_t* smem = smem_raw;
-  uint8_t* sK = smem;
-  uint8_t* sV = sK + C::TILE;
-  uint8_t* sQ = sV + C::TILE;                // ST tiles
+  uint8_t* sK = smem;                        // KVB tiles
+  uint8_t* sV = sK + C::KVB * C::TILE;       // KVB tiles
+  uint8_t* sQ = sV + C::KVB * C::TILE;       // ST tiles
   uint8_t* sdO = sQ + C::ST * C::TILE;       // ST tiles
   uint8_t* sDS = sdO + C::ST * C::TILE;      // dS^T, MN-major for the dQ product
   float* sLD = reinterpret_cast<float*>(sDS + C::DS_BYTES);  // [ST][2][128]: L, D
   BwdCtrl<C::ST>& ctl = *reinterpret_cast<BwdCtrl<C::ST>*>(sDS + C::DS_BYTES + C::LD_BYTES);
   static_assert(sizeof(BwdCtrl<C::ST>) <= C::CTRL_BYTES, "control block too large");
-  uint64_t& bar_kv = ctl.bar_kv;
+  uint64_t* bar_kv = ctl.bar_kv;
+  uint64_t* kv_empty = ctl.kv_empty;
+  uint64_t& acc_free = ctl.acc_free;
   uint64_t* qdo_full = ctl.qdo_full;
   uint64_t* qdo_empty = ctl.qdo_empty;
   uint64_t& s_full = ctl.s_full;
@@ -252,28 +260,49 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   uint64_t& dq_full = ctl.dq_full;
   uint64_t& dq_drained = ctl.dq_drained;
   uint64_t& drain = ctl.drain;
+  uint64_t& fin = ctl.fin;
   uint32_t& tmem_slot = ctl.tmem_slot;
   int& abort_flag = ctl.abort_flag;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int N = p.N;
-  const int j = static_cast<int>(blockIdx.x) / p.BH;   // key tile (heaviest first when causal)
-  const int bh = static_cast<int>(blockIdx.x) % p.BH;
   const int n_q = p.n_kv;
-  const int i_begin = CAUSAL ? j : 0;
-  // With a sliding window the last query that sees a key of this tile is
-  // j*128 + 127 + window - 1.
-  const int i_end = (CAUSAL && p.window > 0)
-                        ? min(n_q, (j * 128 + 127 + p.window - 1) / 128 + 1)
-                        : n_q;
-  const int n_it = i_end - i_begin;
+  // Tile scheduler.  Key tiles t = j * BH + bh are listed heaviest first (causal:
+  // key tile j is seen by query tiles j .. n - 1, so the work falls with j).  The
+  // grid has at most one CTA per SM, and CTA c runs tiles c, 2G - 1 - c, 2G + c,
+  // 4G - 1 - c, ... of the list (G CTAs: a snake over it), so that every CTA gets
+  // about the same number of query steps and pays its set-up once.
+  // (The helpers below copy what they need from p: capturing the kernel parameter
+  // itself would take its address and copy it to local memory.)
+  const int G = static_cast<int>(gridDim.x);
+  const int cta = static_cast<int>(blockIdx.x);
+  const int BH = p.BH;
+  const int win = p.window;
+  const int T = n_q * BH;
+  auto tile_of = [=](int k) {
+    const int t = k * G + ((k & 1) ? G - 1 - cta : cta);
+    return t < T ? t : -1;
+  };
+  // Query tiles that see key tile j: from j on when causal, and with a sliding
+  // window up to the last query that sees its last key, j*128 + 127 + window - 1.
+  auto q_begin = [](int j) { return CAUSAL ? j : 0; };
+  auto q_end = [=](int j) {
+    return (CAUSAL && win > 0) ? min(n_q, (j * 128 + 127 + win - 1) / 128 + 1) : n_q;
+  };
+  // bar_kv[b] and kv_empty[b] complete once per tile that uses buffer b: the
+  // phase parity of tile k's turn on its buffer.
+  auto kv_par = [](int k) { return static_cast<uint32_t>((C::KVB == 2 ? (k >> 1) : k) & 1); };
 
   WaitCtl wc{p.status, &abort_flag, p.wait_ns};
 
   if (threadIdx.x == 0) {
     abort_flag = 0;
-    mbar_init(&bar_kv, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&bar_kv[b], 1);
+      mbar_init(&kv_empty[b], 1);
+    }
+    mbar_init(&acc_free, 8);
     for (int s = 0; s < C::ST; ++s) { mbar_init(&qdo_full[s], 1); mbar_init(&qdo_empty[s], 1); }
     mbar_init(&s_full, 1);
     mbar_init(&dp_full, 1);
@@ -282,6 +311,7 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     mbar_init(&dq_full, 1);
     mbar_init(&dq_drained, 8);
     mbar_init(&drain, 1);
+    mbar_init(&fin, 1);
     fence_mbar_init();
   }
   if (warp == 0) {
@@ -300,48 +330,83 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
       tma_prefetch_desc(&tmdO);
-      if (p.fault != 1) {
-        mbar_arrive_expect_tx(&bar_kv, 2 * C::TILE);
+      int last_kv0 = -1, last_kv1 = -1;  // the last of the CTA's tiles whose K, V went to buffer 0, 1
+      // K and V of the CTA's tile k into its buffer (the test hook skips them: a
+      // consumer's wait then runs out).
+      const bool skip_kv = p.fault == 1;
+      auto load_kv = [&](int k) {
+        if (skip_kv) return;
+        const int t = tile_of(k);
+        const int b = k % C::KVB;
+        const int row = (t / BH) * 128, bh = t % BH;
+        mbar_arrive_expect_tx(&bar_kv[b], 2 * C::TILE);
         for (int c = 0; c < C::KCH; ++c) {
-          tma_load_3d(sK + c * C::CHUNK, &tmK, &bar_kv, c * 64, j * 128, bh);
-          tma_load_3d(sV + c * C::CHUNK, &tmV, &bar_kv, c * 64, j * 128, bh);
+          tma_load_3d(sK + b * C::TILE + c * C::CHUNK, &tmK, &bar_kv[b], c * 64, row, bh);
+          tma_load_3d(sV + b * C::TILE + c * C::CHUNK, &tmV, &bar_kv[b], c * 64, row, bh);
         }
-      }
+        if (b == 0) last_kv0 = k; else last_kv1 = k;
+      };
+      // K and V do not depend on the preprocess: the first tiles' go out at once.
+      // The L, D rows (and the zeroed dQ accumulator the compute warps add into) do.
+      load_kv(0);
+      if (C::KVB == 2 && tile_of(1) >= 0) load_kv(1);
       const uint64_t keep = policy_evict_last();
-      // K and V do not depend on the preprocess; the L, D rows (and the zeroed
-      // dQ accumulator the compute warps add into) do.
       griddep_wait();
-      int issued = 0;
+      int gs = 0;  // query steps issued so far (ring slot and phase)
       bool ok = true;
-      for (int it = 0; it < n_it; ++it) {
-        const int st = it % C::ST;
-        if (it >= C::ST &&
-            !mbar_wait(&qdo_empty[st], ((it / C::ST) - 1) & 1, wc, kBSiteProdEmpty)) {
-          ok = false;
-          break;
+      for (int k = 0; ok; ++k) {
+        const int t = tile_of(k);
+        if (t < 0) break;
+        const int bh = t % p.BH;
+        const int i0 = q_begin(t / p.BH), n_it = q_end(t / p.BH) - i0;
+        for (int it = 0; it < n_it; ++it) {
+          const int st = gs % C::ST;
+          if (gs >= C::ST &&
+              !mbar_wait(&qdo_empty[st], ((gs / C::ST) - 1) & 1, wc, kBSiteProdEmpty)) {
+            ok = false;
+            break;
+          }
+          const int row = (i0 + it) * 128;
+          mbar_arrive_expect_tx(&qdo_full[st], 2 * C::TILE + 2 * 512);
+          const size_t stat = static_cast<size_t>(bh) * p.Npad + row;
+          bulk_load_1d(sLD + st * 256, p.Lg + stat, 512, &qdo_full[st]);
+          bulk_load_1d(sLD + st * 256 + 128, p.Dg + stat, 512, &qdo_full[st]);
+          for (int c = 0; c < C::KCH; ++c) {
+            tma_load_3d_hint(sQ + st * C::TILE + c * C::CHUNK, &tmQ, &qdo_full[st], c * 64, row,
+                             bh, keep);
+            tma_load_3d_hint(sdO + st * C::TILE + c * C::CHUNK, &tmdO, &qdo_full[st], c * 64,
+                             row, bh, keep);
+          }
+          ++gs;
+          // The next K, V load.  Two buffers: tile k + 1's, a step or two into tile
+          // k, once tile k - 1 has released the buffer.  One buffer: tile k's own,
+          // right after its first (Q, dO) load, once tile k - 1's last product has
+          // read the buffer.
+          int nk = -1;
+          if (C::KVB == 2) {
+            if (k >= 1 && it == min(C::ST, n_it - 1) && tile_of(k + 1) >= 0) nk = k + 1;
+          } else if (k >= 1 && it == 0) {
+            nk = k;
+          }
+          if (nk >= 0) {
+            if (!mbar_wait(&kv_empty[nk % C::KVB], kv_par(nk - C::KVB), wc, kBSiteProdKV)) {
+              ok = false;
+              break;
+            }
+            load_kv(nk);
+          }
         }
-        const int row = (i_begin + it) * 128;
-        mbar_arrive_expect_tx(&qdo_full[st], 2 * C::TILE + 2 * 512);
-        const size_t stat = static_cast<size_t>(bh) * p.Npad + row;
-        bulk_load_1d(sLD + st * 256, p.Lg + stat, 512, &qdo_full[st]);
-        bulk_load_1d(sLD + st * 256 + 128, p.Dg + stat, 512, &qdo_full[st]);
-        for (int c = 0; c < C::KCH; ++c) {
-          tma_load_3d_hint(sQ + st * C::TILE + c * C::CHUNK, &tmQ, &qdo_full[st], c * 64, row,
-                           bh, keep);
-          tma_load_3d_hint(sdO + st * C::TILE + c * C::CHUNK, &tmdO, &qdo_full[st], c * 64,
-                           row, bh, keep);
-        }
-        issued = it + 1;
       }
       volatile int no_abort = 0;
       WaitCtl dw{p.status, &no_abort, 100000000ull};
       if (!ok) {
-        for (int it = max(0, issued - C::ST); it < issued; ++it)
-          mbar_wait(&qdo_full[it % C::ST], (it / C::ST) & 1, dw, kBSiteProdDrain);
+        for (int q = max(0, gs - C::ST); q < gs; ++q)
+          mbar_wait(&qdo_full[q % C::ST], (q / C::ST) & 1, dw, kBSiteProdDrain);
       }
-      // K and V always land before exit, even on an aborted run (unless the test
-      // hook skipped them: then nothing is in flight).
-      if (p.fault != 1) mbar_wait(&bar_kv, 0, dw, kBSiteProdDrain);
+      // Every K, V load lands before exit, even on an aborted run (one at most is
+      // in flight per buffer: a reload waits for the previous one to be consumed).
+      if (last_kv0 >= 0) mbar_wait(&bar_kv[0], kv_par(last_kv0), dw, kBSiteProdDrain);
+      if (last_kv1 >= 0) mbar_wait(&bar_kv[1], kv_par(last_kv1), dw, kBSiteProdDrain);
     }
     __syncwarp();
   } else if (warp == 9) {
@@ -352,69 +417,90 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       constexpr uint32_t id_dq = idesc_f16(128, D, BF16, true, true);      // dQ (A, B MN-major)
       const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aQ = smem_u32(sQ),
                      adO = smem_u32(sdO), aDS = smem_u32(sDS);
-      // Base descriptors; a K step or a ring stage only moves the start address.
+      // Base descriptors; a K step, a ring stage or a K/V buffer only moves the
+      // start address.
       const uint64_t kK = sdesc_sw128(aK, 16, 1024), kV = sdesc_sw128(aV, 16, 1024);
       const uint64_t kQ = sdesc_sw128(aQ, 16, 1024), kdO = sdesc_sw128(adO, 16, 1024);
       const uint64_t mQ = sdesc_sw128(aQ, C::CHUNK, 1024), mdO = sdesc_sw128(adO, C::CHUNK, 1024);
       const uint64_t mK = sdesc_sw128(aK, C::CHUNK, 1024), mDS = sdesc_sw128(aDS, C::CHUNK, 1024);
-      bool ok = mbar_wait(&bar_kv, 0, wc, kBSiteMmaKV);
-      for (int it = 0; it < n_it && ok; ++it) {
-        const int st = it % C::ST;
-        if (!mbar_wait(&qdo_full[st], (it / C::ST) & 1, wc, kBSiteMmaQ)) { ok = false; break; }
-        tc_fence_after();
-        // S^T = K Q^T
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::CHUNK + (kk & 3) * 32;
-          umma_ss(tbase + C::C_S, sdesc_add(kK, off), sdesc_add(kQ, st * C::TILE + off), id_kk,
-                  kk > 0);
-        }
-        umma_commit(&s_full);
-        // dP^T = V dO^T (its columns hold the previous dQ partial when D = 128)
-        if (D == 128 && it > 0) {
-          if (!mbar_wait(&dq_drained, (it - 1) & 1, wc, kBSiteMmaDrained)) { ok = false; break; }
+      bool ok = true;
+      int gs = 0;  // query steps so far
+      for (int k = 0; ok; ++k) {
+        const int t = tile_of(k);
+        if (t < 0) break;
+        const int n_it = q_end(t / p.BH) - q_begin(t / p.BH);
+        const int b = k % C::KVB;
+        const uint32_t kvo = static_cast<uint32_t>(b * C::TILE);  // this tile's K, V buffer
+        if (!mbar_wait(&bar_kv[b], kv_par(k), wc, kBSiteMmaKV)) { ok = false; break; }
+        for (int it = 0; it < n_it; ++it, ++gs) {
+          const int st = gs % C::ST;
+          if (!mbar_wait(&qdo_full[st], (gs / C::ST) & 1, wc, kBSiteMmaQ)) { ok = false; break; }
           tc_fence_after();
-        }
+          // S^T = K Q^T
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::CHUNK + (kk & 3) * 32;
-          umma_ss(tbase + C::C_DP, sdesc_add(kV, off), sdesc_add(kdO, st * C::TILE + off), id_kk,
-                  kk > 0);
-        }
-        umma_commit(&dp_full);
-        // dV += P^T dO
-        if (!mbar_wait(&p_ready, it & 1, wc, kBSiteMmaP)) { ok = false; break; }
-        tc_fence_after();
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * C::CHUNK + (kk & 3) * 32;
+            umma_ss(tbase + C::C_S, sdesc_add(kK, kvo + off), sdesc_add(kQ, st * C::TILE + off),
+                    id_kk, kk > 0);
+          }
+          umma_commit(&s_full);
+          // dP^T = V dO^T (its columns hold the previous dQ partial when D = 128)
+          if (D == 128 && gs > 0) {
+            if (!mbar_wait(&dq_drained, (gs - 1) & 1, wc, kBSiteMmaDrained)) { ok = false; break; }
+            tc_fence_after();
+          }
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)  // queries 16 kk .. 16 kk + 15: warpgroup kk / 4
-          umma_ts(tbase + C::C_DV, tbase + C::C_P(kk >> 2) + (kk & 3) * 8,
-                  sdesc_add(mdO, st * C::TILE + kk * 2048), id_tb,
-                  (it > 0 || kk > 0) ? 1u : 0u);
-        // dQ_i = dS K first (the drain needs only this one; its own TMEM columns when
-        // D = 64: wait for the previous drain), then dK += dS^T Q (A from TMEM, so
-        // the dQ staging that reuses the dS^T tile of shared memory cannot race it).
-        if (!mbar_wait(&ds_ready, it & 1, wc, kBSiteMmaDS)) { ok = false; break; }
-        tc_fence_after();
-        if (D == 64 && it > 0) {
-          if (!mbar_wait(&dq_drained, (it - 1) & 1, wc, kBSiteMmaDrained)) { ok = false; break; }
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * C::CHUNK + (kk & 3) * 32;
+            umma_ss(tbase + C::C_DP, sdesc_add(kV, kvo + off), sdesc_add(kdO, st * C::TILE + off),
+                    id_kk, kk > 0);
+          }
+          umma_commit(&dp_full);
+          // dV += P^T dO
+          if (!mbar_wait(&p_ready, gs & 1, wc, kBSiteMmaP)) { ok = false; break; }
           tc_fence_after();
+          if (k > 0 && it == 0) {
+            // A tile's first dV and dK products overwrite the accumulators: the
+            // previous tile's epilogue must have read them out.
+            if (!mbar_wait(&acc_free, (k - 1) & 1, wc, kBSiteMmaAcc)) { ok = false; break; }
+            tc_fence_after();
+          }
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)  // queries 16 kk .. 16 kk + 15: warpgroup kk / 4
+            umma_ts(tbase + C::C_DV, tbase + C::C_P(kk >> 2) + (kk & 3) * 8,
+                    sdesc_add(mdO, st * C::TILE + kk * 2048), id_tb,
+                    (it > 0 || kk > 0) ? 1u : 0u);
+          // dQ_i = dS K first (the drain needs only this one; its own TMEM columns
+          // when D = 64: wait for the previous drain), then dK += dS^T Q (A from
+          // TMEM, so the dQ staging that reuses the dS^T tile of shared memory
+          // cannot race it).
+          if (!mbar_wait(&ds_ready, gs & 1, wc, kBSiteMmaDS)) { ok = false; break; }
+          tc_fence_after();
+          if (D == 64 && gs > 0) {
+            if (!mbar_wait(&dq_drained, (gs - 1) & 1, wc, kBSiteMmaDrained)) { ok = false; break; }
+            tc_fence_after();
+          }
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            umma_ss(tbase + C::C_DQ, sdesc_add(mDS, kk * 2048), sdesc_add(mK, kvo + kk * 2048),
+                    id_dq, kk > 0);
+          umma_commit(&dq_full);
+          // The tile's K, V have been read for the last time: release the buffer.
+          if (it == n_it - 1) umma_commit(&kv_empty[b]);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            umma_ts(tbase + C::C_DK, tbase + C::C_DS(kk >> 2) + (kk & 3) * 8,
+                    sdesc_add(mQ, st * C::TILE + kk * 2048), id_tb,
+                    (it > 0 || kk > 0) ? 1u : 0u);
+          umma_commit(&qdo_empty[st]);
         }
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          umma_ss(tbase + C::C_DQ, sdesc_add(mDS, kk * 2048), sdesc_add(mK, kk * 2048), id_dq,
-                  kk > 0);
-        umma_commit(&dq_full);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          umma_ts(tbase + C::C_DK, tbase + C::C_DS(kk >> 2) + (kk & 3) * 8,
-                  sdesc_add(mQ, st * C::TILE + kk * 2048), id_tb,
-                  (it > 0 || kk > 0) ? 1u : 0u);
-        umma_commit(&qdo_empty[st]);
+        if (!ok) break;
+        umma_commit(&drain);  // the tile's dK and dV are final once this lands
       }
-      umma_commit(&drain);  // also tells the compute warps that dK and dV are final
+      umma_commit(&fin);  // every product issued has landed once this does
       volatile int no_abort = 0;
       WaitCtl dw{p.status, &no_abort, p.wait_ns};
-      mbar_wait(&drain, 0, dw, kBSiteMmaDrain);
+      mbar_wait(&fin, 0, dw, kBSiteMmaDrain);
     }
     __syncwarp();
   } else {
@@ -423,206 +509,221 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     const int g = warp >> 2;                   // warpgroup: query columns 64 g .. 64 g + 63
     const int wq = warp & 3;                   // TMEM lane quadrant
     const int r = wq * 32 + lane;              // key row (P^T, dS^T) / query row (dQ)
-    const int key = j * 128 + r;
     const uint32_t lb = static_cast<uint32_t>(wq * 32);
     const float sl2 = p.scale_log2;
     const int qoff = 64 * g;
     const uint32_t wg_bar = 1 + g;             // named barrier of this warpgroup
     bool ok = true;
-    for (int it = 0; it < n_it && ok; ++it) {
-      const int i = i_begin + it;
-      const int st = it % C::ST;
-      // This tile's LSE*log2e and D rows arrive in shared memory with Q_i and dO_i.
-      const float4* L4 = reinterpret_cast<const float4*>(sLD + st * 256 + qoff);
-      const float4* D4 = reinterpret_cast<const float4*>(sLD + st * 256 + 128 + qoff);
-      // Every wait of a compute warpgroup ends in a warpgroup-wide vote, so that all
-      // of its 128 threads leave together on a timeout (the named barriers below
-      // have no time limit and must never be left waiting).
-      ok = named_bar_and(wg_bar, 128, mbar_wait(&qdo_full[st], (it / C::ST) & 1, wc, kBSiteCmpQ));
-      if (!ok) break;
-      ok = named_bar_and(wg_bar, 128, mbar_wait(&s_full, it & 1, wc, kBSiteCmpS));
-      if (!ok) break;
-      tc_fence_after();
-      // P^T (this warpgroup's 64 query columns): exp2(S^T * scale * log2e - LSE * log2e),
-      // zero where the key comes after the query or lies past N.
-      float pr[64];
-      // Masking (key after query on the diagonal tile, or key past N) is rare: one
-      // branch per tile, not a compare per element.
-      const int win = p.window;
-      const bool masked = (CAUSAL && i == j) || key >= N ||
-                          (CAUSAL && win > 0 && i * 128 + 127 - j * 128 >= win);
-      const uint64_t sl2x2 = f2_pack(sl2, sl2);
-      uint32_t srr[2][32];
-      tmem_ld32(tmem_addr(tbase, lb, C::C_S + qoff), srr[0]);
-      tmem_ld32(tmem_addr(tbase, lb, C::C_S + qoff + 32), srr[1]);
-      tmem_wait_ld();
-      reg_fence(srr[0]);
-      reg_fence(srr[1]);
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        const uint32_t (&sr)[32] = srr[c];
-#pragma unroll
-        for (int v = 0; v < 8; ++v) {
-          const float4 l4 = L4[c * 8 + v];
-          const uint64_t a01 = f2_fma(f2_pack(__uint_as_float(sr[v * 4]), __uint_as_float(sr[v * 4 + 1])),
-                                      sl2x2, f2_pack(-l4.x, -l4.y));
-          const uint64_t a23 = f2_fma(f2_pack(__uint_as_float(sr[v * 4 + 2]), __uint_as_float(sr[v * 4 + 3])),
-                                      sl2x2, f2_pack(-l4.z, -l4.w));
-          float x0, x1, x2, x3;
-          f2_unpack(a01, x0, x1);
-          f2_unpack(a23, x2, x3);
-          const int q0 = c * 32 + v * 4;
-          if ((v & 3) >= kBwdPolyFrom) {  // FMA-pipe exp2 for this group of four
-            pr[q0 + 0] = exp2_poly3(x0);
-            pr[q0 + 1] = exp2_poly3(x1);
-            pr[q0 + 2] = exp2_poly3(x2);
-            pr[q0 + 3] = exp2_poly3(x3);
-          } else {
-            pr[q0 + 0] = ex2_approx(x0);
-            pr[q0 + 1] = ex2_approx(x1);
-            pr[q0 + 2] = ex2_approx(x2);
-            pr[q0 + 3] = ex2_approx(x3);
+    int gs = 0;  // query steps so far
+    for (int k = 0; ok; ++k) {
+      const int t = tile_of(k);
+      if (t < 0) break;
+      const int j = t / p.BH, bh = t % p.BH;
+      const int key = j * 128 + r;
+      const int i_begin = q_begin(j);
+      const int n_it = q_end(j) - i_begin;
+      for (int it = 0; it < n_it && ok; ++it, ++gs) {
+        const int i = i_begin + it;
+        const int st = gs % C::ST;
+        // This tile's LSE*log2e and D rows arrive in shared memory with Q_i and dO_i.
+        const float4* L4 = reinterpret_cast<const float4*>(sLD + st * 256 + qoff);
+        const float4* D4 = reinterpret_cast<const float4*>(sLD + st * 256 + 128 + qoff);
+        // Every wait of a compute warpgroup ends in a warpgroup-wide vote, so that all
+        // of its 128 threads leave together on a timeout (the named barriers below
+        // have no time limit and must never be left waiting).
+        ok = named_bar_and(wg_bar, 128, mbar_wait(&qdo_full[st], (gs / C::ST) & 1, wc, kBSiteCmpQ));
+        if (!ok) break;
+        ok = named_bar_and(wg_bar, 128, mbar_wait(&s_full, gs & 1, wc, kBSiteCmpS));
+        if (!ok) break;
+        tc_fence_after();
+        // P^T (this warpgroup's 64 query columns): exp2(S^T * scale * log2e - LSE * log2e),
+        // zero where the key comes after the query or lies past N.
+        float pr[64];
+        // Masking (key after query on the diagonal tile, or key past N) is rare: one
+        // branch per tile, not a compare per element.
+        const bool masked = (CAUSAL && i == j) || key >= N ||
+                            (CAUSAL && win > 0 && i * 128 + 127 - j * 128 >= win);
+        const uint64_t sl2x2 = f2_pack(sl2, sl2);
+        uint32_t srr[2][32];
+        tmem_ld32(tmem_addr(tbase, lb, C::C_S + qoff), srr[0]);
+        tmem_ld32(tmem_addr(tbase, lb, C::C_S + qoff + 32), srr[1]);
+        tmem_wait_ld();
+        reg_fence(srr[0]);
+        reg_fence(srr[1]);
+  #pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          const uint32_t (&sr)[32] = srr[c];
+  #pragma unroll
+          for (int v = 0; v < 8; ++v) {
+            const float4 l4 = L4[c * 8 + v];
+            const uint64_t a01 = f2_fma(f2_pack(__uint_as_float(sr[v * 4]), __uint_as_float(sr[v * 4 + 1])),
+                                        sl2x2, f2_pack(-l4.x, -l4.y));
+            const uint64_t a23 = f2_fma(f2_pack(__uint_as_float(sr[v * 4 + 2]), __uint_as_float(sr[v * 4 + 3])),
+                                        sl2x2, f2_pack(-l4.z, -l4.w));
+            float x0, x1, x2, x3;
+            f2_unpack(a01, x0, x1);
+            f2_unpack(a23, x2, x3);
+            const int q0 = c * 32 + v * 4;
+            if ((v & 3) >= kBwdPolyFrom) {  // FMA-pipe exp2 for this group of four
+              pr[q0 + 0] = exp2_poly3(x0);
+              pr[q0 + 1] = exp2_poly3(x1);
+              pr[q0 + 2] = exp2_poly3(x2);
+              pr[q0 + 3] = exp2_poly3(x3);
+            } else {
+              pr[q0 + 0] = ex2_approx(x0);
+              pr[q0 + 1] = ex2_approx(x1);
+              pr[q0 + 2] = ex2_approx(x2);
+              pr[q0 + 3] = ex2_approx(x3);
+            }
           }
         }
-      }
-      if (masked) {
-#pragma unroll
-        for (int qc = 0; qc < 64; ++qc)
-          if ((CAUSAL && i == j && qoff + qc < r) || key >= N ||
-              (CAUSAL && win > 0 && i * 128 + qoff + qc - key >= win))
-            pr[qc] = 0.f;
-      }
-      {
-        uint32_t pk[32];
-#pragma unroll
-        for (int e = 0; e < 32; ++e) pk[e] = pack2<BF16>(pr[2 * e], pr[2 * e + 1]);
-        tmem_st32(tmem_addr(tbase, lb, C::C_P(g)), pk);
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&p_ready);
-      // dS^T = P^T * (dP^T - D), 32 queries at a time, written to TMEM (A operand
-      // of dK) and to shared memory (A operand of dQ).  The shared copy is
-      // MN-major with 128-byte swizzle: chunk g holds queries 64 g .. 64 g + 63 of
-      // every key row; 16-byte unit u of row r sits at unit u ^ (r % 8).
-      ok = named_bar_and(wg_bar, 128, mbar_wait(&dp_full, it & 1, wc, kBSiteCmpDP));
-      if (!ok) break;
-      tc_fence_after();
-      if (it > 0) {
-        // This warpgroup's dS^T chunk doubled as the staging tile of the previous
-        // dQ reduce: that bulk copy must have finished reading it.
-        if (r == 0) tma_store_wait_read();
-        named_bar_sync(wg_bar, 128);
-      }
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        uint32_t dr[32];
-        tmem_ld32(tmem_addr(tbase, lb, C::C_DP + qoff + 32 * c), dr);
-        tmem_wait_ld();
-        reg_fence(dr);
-        uint32_t dsk[16];
-#pragma unroll
-        for (int v = 0; v < 8; ++v) {
-          const float4 d4 = D4[c * 8 + v];
-          const int q0 = c * 32 + v * 4;
-          const uint64_t t01 = f2_sub(f2_pack(__uint_as_float(dr[v * 4]), __uint_as_float(dr[v * 4 + 1])),
-                                      f2_pack(d4.x, d4.y));
-          const uint64_t t23 = f2_sub(f2_pack(__uint_as_float(dr[v * 4 + 2]), __uint_as_float(dr[v * 4 + 3])),
-                                      f2_pack(d4.z, d4.w));
-          float a0, a1, a2, a3;
-          f2_unpack(f2_mul(f2_pack(pr[q0], pr[q0 + 1]), t01), a0, a1);
-          f2_unpack(f2_mul(f2_pack(pr[q0 + 2], pr[q0 + 3]), t23), a2, a3);
-          dsk[2 * v] = pack2<BF16>(a0, a1);
-          dsk[2 * v + 1] = pack2<BF16>(a2, a3);
+        if (masked) {
+  #pragma unroll
+          for (int qc = 0; qc < 64; ++qc)
+            if ((CAUSAL && i == j && qoff + qc < r) || key >= N ||
+                (CAUSAL && win > 0 && i * 128 + qoff + qc - key >= win))
+              pr[qc] = 0.f;
         }
-        tmem_st16(tmem_addr(tbase, lb, C::C_DS(g) + 16 * c), dsk);
-#pragma unroll
-        for (int uu = 0; uu < 4; ++uu) {
-          const int u = c * 4 + uu;
-          const uint4 val = make_uint4(dsk[4 * uu], dsk[4 * uu + 1], dsk[4 * uu + 2], dsk[4 * uu + 3]);
-          *reinterpret_cast<uint4*>(sDS + g * C::CHUNK + r * 128 + ((u ^ (r & 7)) << 4)) = val;
+        {
+          uint32_t pk[32];
+  #pragma unroll
+          for (int e = 0; e < 32; ++e) pk[e] = pack2<BF16>(pr[2 * e], pr[2 * e + 1]);
+          tmem_st32(tmem_addr(tbase, lb, C::C_P(g)), pk);
         }
-      }
-      fence_proxy_async_smem();
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&ds_ready);
-      // dQ partial: query row r, head columns g D/2 .. (g+1) D/2 - 1 -> fp32 accumulator
-      ok = named_bar_and(wg_bar, 128, mbar_wait(&dq_full, it & 1, wc, kBSiteCmpDQ));
-      if (!ok) break;
-      tc_fence_after();
-      // dQ partial, head columns g D/2 .. (g+1) D/2 - 1, 32 at a time: TMEM ->
-      // this warpgroup's dS^T chunk of shared memory (free: the dQ product that
-      // read it has completed), laid out as a 128-row x 32-float tile with
-      // 128-byte swizzle -> one TMA reduce-add into the fp32 accumulator (rows
-      // past N are clipped by the tensor map).
-      constexpr int HALF = D / 2;
-      constexpr int NCH = HALF / 32;
-      uint8_t* stage = sDS + g * C::CHUNK;
-      // All of this warpgroup's TMEM columns first, so that the region is released
-      // (dq_drained) before any staging starts.
-      uint32_t qr[NCH][32];
-#pragma unroll
-      for (int c = 0; c < NCH; ++c)
-        tmem_ld32(tmem_addr(tbase, lb, C::C_DQ + g * HALF + 32 * c), qr[c]);
-      tmem_wait_ld();
-#pragma unroll
-      for (int c = 0; c < NCH; ++c) reg_fence(qr[c]);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&dq_drained);
-#pragma unroll
-      for (int c = 0; c < NCH; ++c) {
-        if (c > 0) {
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_ready);
+        // dS^T = P^T * (dP^T - D), 32 queries at a time, written to TMEM (A operand
+        // of dK) and to shared memory (A operand of dQ).  The shared copy is
+        // MN-major with 128-byte swizzle: chunk g holds queries 64 g .. 64 g + 63 of
+        // every key row; 16-byte unit u of row r sits at unit u ^ (r % 8).
+        ok = named_bar_and(wg_bar, 128, mbar_wait(&dp_full, gs & 1, wc, kBSiteCmpDP));
+        if (!ok) break;
+        tc_fence_after();
+        if (gs > 0) {
+          // This warpgroup's dS^T chunk doubled as the staging tile of the previous
+          // dQ reduce: that bulk copy must have finished reading it.
           if (r == 0) tma_store_wait_read();
           named_bar_sync(wg_bar, 128);
         }
-#pragma unroll
-        for (int u = 0; u < 8; ++u)
-          *reinterpret_cast<uint4*>(stage + r * 128 + ((u ^ (r & 7)) << 4)) =
-              make_uint4(qr[c][4 * u], qr[c][4 * u + 1], qr[c][4 * u + 2], qr[c][4 * u + 3]);
-        fence_proxy_async_smem();
-        named_bar_sync(wg_bar, 128);
-        if (r == 0) {
-          tma_reduce_add_3d(&tmdQ, stage, g * HALF + 32 * c, i * 128, bh);
-          tma_store_commit();
+  #pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          uint32_t dr[32];
+          tmem_ld32(tmem_addr(tbase, lb, C::C_DP + qoff + 32 * c), dr);
+          tmem_wait_ld();
+          reg_fence(dr);
+          uint32_t dsk[16];
+  #pragma unroll
+          for (int v = 0; v < 8; ++v) {
+            const float4 d4 = D4[c * 8 + v];
+            const int q0 = c * 32 + v * 4;
+            const uint64_t t01 = f2_sub(f2_pack(__uint_as_float(dr[v * 4]), __uint_as_float(dr[v * 4 + 1])),
+                                        f2_pack(d4.x, d4.y));
+            const uint64_t t23 = f2_sub(f2_pack(__uint_as_float(dr[v * 4 + 2]), __uint_as_float(dr[v * 4 + 3])),
+                                        f2_pack(d4.z, d4.w));
+            float a0, a1, a2, a3;
+            f2_unpack(f2_mul(f2_pack(pr[q0], pr[q0 + 1]), t01), a0, a1);
+            f2_unpack(f2_mul(f2_pack(pr[q0 + 2], pr[q0 + 3]), t23), a2, a3);
+            dsk[2 * v] = pack2<BF16>(a0, a1);
+            dsk[2 * v + 1] = pack2<BF16>(a2, a3);
+          }
+          tmem_st16(tmem_addr(tbase, lb, C::C_DS(g) + 16 * c), dsk);
+  #pragma unroll
+          for (int uu = 0; uu < 4; ++uu) {
+            const int u = c * 4 + uu;
+            const uint4 val = make_uint4(dsk[4 * uu], dsk[4 * uu + 1], dsk[4 * uu + 2], dsk[4 * uu + 3]);
+            *reinterpret_cast<uint4*>(sDS + g * C::CHUNK + r * 128 + ((u ^ (r & 7)) << 4)) = val;
+          }
         }
+        fence_proxy_async_smem();
+        tmem_wait_st();
+        tc_fence_before();
         __syncwarp();
+        if (lane == 0) mbar_arrive(&ds_ready);
+        // dQ partial: query row r, head columns g D/2 .. (g+1) D/2 - 1 -> fp32 accumulator
+        ok = named_bar_and(wg_bar, 128, mbar_wait(&dq_full, gs & 1, wc, kBSiteCmpDQ));
+        if (!ok) break;
+        tc_fence_after();
+        // dQ partial, head columns g D/2 .. (g+1) D/2 - 1, 32 at a time: TMEM ->
+        // this warpgroup's dS^T chunk of shared memory (free: the dQ product that
+        // read it has completed), laid out as a 128-row x 32-float tile with
+        // 128-byte swizzle -> one TMA reduce-add into the fp32 accumulator (rows
+        // past N are clipped by the tensor map).
+        constexpr int HALF = D / 2;
+        constexpr int NCH = HALF / 32;
+        uint8_t* stage = sDS + g * C::CHUNK;
+        // All of this warpgroup's TMEM columns first, so that the region is released
+        // (dq_drained) before any staging starts.
+        uint32_t qr[NCH][32];
+  #pragma unroll
+        for (int c = 0; c < NCH; ++c)
+          tmem_ld32(tmem_addr(tbase, lb, C::C_DQ + g * HALF + 32 * c), qr[c]);
+        tmem_wait_ld();
+  #pragma unroll
+        for (int c = 0; c < NCH; ++c) reg_fence(qr[c]);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&dq_drained);
+  #pragma unroll
+        for (int c = 0; c < NCH; ++c) {
+          if (c > 0) {
+            if (r == 0) tma_store_wait_read();
+            named_bar_sync(wg_bar, 128);
+          }
+  #pragma unroll
+          for (int u = 0; u < 8; ++u)
+            *reinterpret_cast<uint4*>(stage + r * 128 + ((u ^ (r & 7)) << 4)) =
+                make_uint4(qr[c][4 * u], qr[c][4 * u + 1], qr[c][4 * u + 2], qr[c][4 * u + 3]);
+          fence_proxy_async_smem();
+          named_bar_sync(wg_bar, 128);
+          if (r == 0) {
+            tma_reduce_add_3d(&tmdQ, stage, g * HALF + 32 * c, i * 128, bh);
+            tma_store_commit();
+          }
+          __syncwarp();
+        }
       }
-    }
-    // All reductions complete before the CTA (and its shared memory) goes away.
-    if (r == 0) tma_store_wait_all();
-    __syncwarp();
-    // dV (warpgroup 0) and dK (warpgroup 1) are final once every MMA has landed.
-    if (ok) ok = named_bar_and(wg_bar, 128, mbar_wait(&drain, 0, wc, kBSiteCmpDQ));
-    if (ok) {
+      if (!ok) break;
+      // dV (warpgroup 0) and dK (warpgroup 1) of the tile are final once its
+      // products have landed: read them out of TMEM, hand the columns to the next
+      // tile's products, then store them.
+      ok = named_bar_and(wg_bar, 128, mbar_wait(&drain, k & 1, wc, kBSiteCmpDQ));
+      if (!ok) break;
       tc_fence_after();
       const uint32_t col = g ? C::C_DK : C::C_DV;
       const float mul = g ? p.scale : 1.0f;
-      const int d = p.d;
-      uint8_t* row = reinterpret_cast<uint8_t*>(g ? p.dK : p.dV) +
-                     (static_cast<size_t>(bh) * N + key) * (d * 2);
+      uint4 v[D / 32][4];
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t rr[32];
         tmem_ld32(tmem_addr(tbase, lb, col + 32 * c), rr);
         tmem_wait_ld();
         reg_fence(rr);
-        uint4 v[4];
-        uint32_t* pv = reinterpret_cast<uint32_t*>(v);
+        uint32_t* pv = reinterpret_cast<uint32_t*>(v[c]);
 #pragma unroll
         for (int e = 0; e < 16; ++e)
           pv[e] = pack2<BF16>(__uint_as_float(rr[2 * e]) * mul, __uint_as_float(rr[2 * e + 1]) * mul);
-        if (key < N) {
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_free);
+      if (key < N) {
+        const int d = p.d;
+        uint8_t* row = reinterpret_cast<uint8_t*>(g ? p.dK : p.dV) +
+                       (static_cast<size_t>(bh) * N + key) * (d * 2);
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
           uint4* dst4 = reinterpret_cast<uint4*>(row + c * 64);
 #pragma unroll
           for (int e = 0; e < 4; ++e)
-            if (c * 32 + 8 * e < d) dst4[e] = v[e];  // 8 columns per store; d % 8 == 0
+            if (c * 32 + 8 * e < d) dst4[e] = v[c][e];  // 8 columns per store; d % 8 == 0
         }
       }
     }
+    // All reductions complete before the CTA (and its shared memory) goes away.
+    if (r == 0) tma_store_wait_all();
+    __syncwarp();
   }
 
   tc_fence_before();
@@ -689,10 +790,11 @@ template <int D, bool BF16, bool CAUSAL>
 int launch_bwd_t(const void* Q, const void* K, const void* V, const void* O, const void* dO,
                  const float* LSE, void* dQ, void* dK, void* dV, void* workspace, int BH, int N,
                  int d, float scale, int window, unsigned int* status, unsigned long long wait_ns,
-                 int fault, cudaStream_t stream) {
+                 int fault, int max_ctas, cudaStream_t stream) {
   using Cfg = BwdCfg<D>;
   const int Npad = static_cast<int>(bwd_npad(N));
-  if (static_cast<long long>(Npad / 128) * BH > 0x7fffffffll) return 1;  // FA2_ERR_INVALID_ARG
+  // The tile list (key tiles x heads) is indexed with 32-bit ints in the kernel.
+  if (static_cast<long long>(Npad / 128) * BH > (1ll << 30)) return 1;  // FA2_ERR_INVALID_ARG
   float* Dg = static_cast<float*>(workspace);
   float* Lg = Dg + static_cast<size_t>(BH) * Npad;
   float* dQacc = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
@@ -734,7 +836,18 @@ int launch_bwd_t(const void* Q, const void* K, const void* V, const void* O, con
     bp.status = status;
     bp.wait_ns = wait_ns;
     bp.fault = fault;
-    const unsigned int grid = static_cast<unsigned int>(bp.n_kv) * static_cast<unsigned int>(BH);
+    // Persistent grid: one CTA per SM at most (the kernel's shared memory and TMEM
+    // admit one per SM), each running its share of the tile list.
+    int dev = 0, n_sm = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        n_sm <= 0) {
+      cudaGetLastError();
+      return 4;
+    }
+    long long ctas = std::min(static_cast<long long>(bp.n_kv) * BH, static_cast<long long>(n_sm));
+    if (max_ctas > 0) ctas = std::min(ctas, static_cast<long long>(max_ctas));
+    const unsigned int grid = static_cast<unsigned int>(ctas);
     if (launch_pdl(kern, dim3(grid), dim3(Cfg::THREADS), Cfg::SMEM, stream, mq, mk, mv, mdo, mdq,
                    bp) != cudaSuccess)
       return 4;
@@ -754,10 +867,10 @@ inline int launch_bwd(const void* Q, const void* K, const void* V, const void* O
                       const float* LSE, void* dQ, void* dK, void* dV, void* workspace, int BH,
                       int N, int d, float scale, bool causal, bool bf16, unsigned int* status,
                       unsigned long long wait_ns, cudaStream_t s, int window = 0,
-                      int fault = 0) {
+                      int fault = 0, int max_ctas = 0) {
 #define FA2_BWD_CALL(D_, BF_, CA_)                                                             \
   return launch_bwd_t<D_, BF_, CA_>(Q, K, V, O, dO, LSE, dQ, dK, dV, workspace, BH, N, d, scale, \
-                                    window, status, wait_ns, fault, s)
+                                    window, status, wait_ns, fault, max_ctas, s)
   if (d <= 64) {
     if (bf16) { if (causal) FA2_BWD_CALL(64, true, true); FA2_BWD_CALL(64, true, false); }
     if (causal) FA2_BWD_CALL(64, false, true);

@@ -254,6 +254,13 @@ const char* fa2_status_string(int status);
  */
 void fa2_debug_set(int fault, unsigned int wait_limit_ms);
 
+/*
+ * Test hook.  Caps the backward's persistent grid at ``max_ctas`` CTAs (0, the
+ * default, restores one CTA per SM), so that small problems run several key tiles
+ * per CTA.  Results do not depend on it.  Not for production use.
+ */
+void fa2_debug_set_bwd_grid(int max_ctas);
+
 /* Number of kernels this library has launched in this process (all devices). */
 unsigned long long fa2_launch_count(void);
 
