@@ -346,12 +346,14 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         }
         if (b == 0) last_kv0 = k; else last_kv1 = k;
       };
-      // K and V do not depend on the preprocess: the first tiles' go out at once.
-      // The L, D rows (and the zeroed dQ accumulator the compute warps add into) do.
-      load_kv(0);
-      if (C::KVB == 2 && tile_of(1) >= 0) load_kv(1);
+      // Nothing is read before the wait for the preprocess grid: its completion
+      // also covers the kernels before it, one of which (the caller's, launched
+      // with an early trigger) may still be writing K or V.  The L, D rows and the
+      // zeroed dQ accumulator come from the preprocess itself.
       const uint64_t keep = policy_evict_last();
       griddep_wait();
+      load_kv(0);
+      if (C::KVB == 2 && tile_of(1) >= 0) load_kv(1);
       int gs = 0;  // query steps issued so far (ring slot and phase)
       bool ok = true;
       for (int k = 0; ok; ++k) {
