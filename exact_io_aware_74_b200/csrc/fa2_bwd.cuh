@@ -192,9 +192,19 @@ struct BwdCfg {
   static constexpr int SMEM = (2 * KVB + 2 * ST) * TILE + DS_BYTES + LD_BYTES + CTRL_BYTES;
   static constexpr int THREADS = 320;
   static constexpr uint32_t C_S = 0, C_DP = 128;
-  // packed P^T / dS^T of warpgroup g: columns 64 g + (0 | 32) .. + 31
-  __host__ __device__ static constexpr uint32_t C_P(int g) { return 64u * g; }
-  __host__ __device__ static constexpr uint32_t C_DS(int g) { return 64u * g + 32u; }
+  // Software-pipelined steps (D = 64, where TMEM has room): packed P^T of warpgroup
+  // g in columns 448 + 32 g .. + 31 (free at D = 64), packed dS^T in its own dP^T
+  // columns 128 + 64 g .. + 31, so the score columns are free as soon as the scores
+  // have been read and the next step's scores can be computed during this step's
+  // dS.  Otherwise (D = 128, no free columns) P^T and dS^T of warpgroup g sit in
+  // its score columns, 64 g + (0 | 32) .. + 31.
+  static constexpr bool PIPE = (D == 64);
+  __host__ __device__ static constexpr uint32_t C_P(int g) {
+    return PIPE ? 448u + 32u * g : 64u * g;
+  }
+  __host__ __device__ static constexpr uint32_t C_DS(int g) {
+    return PIPE ? C_DP + 64u * g : 64u * g + 32u;
+  }
   static constexpr uint32_t C_DV = 256, C_DK = 256 + D;
   static constexpr uint32_t C_DQ = (D == 128) ? 128 : 384;
 };
@@ -425,76 +435,124 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       const uint64_t kQ = sdesc_sw128(aQ, 16, 1024), kdO = sdesc_sw128(adO, 16, 1024);
       const uint64_t mQ = sdesc_sw128(aQ, C::CHUNK, 1024), mdO = sdesc_sw128(adO, C::CHUNK, 1024);
       const uint64_t mK = sdesc_sw128(aK, C::CHUNK, 1024), mDS = sdesc_sw128(aDS, C::CHUNK, 1024);
+      // The products of a step; `st` is its ring slot, `kvo` the tile's K/V buffer.
+      auto mma_s = [&](int st, uint32_t kvo) {  // S^T = K Q^T
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * C::CHUNK + (kk & 3) * 32;
+          umma_ss(tbase + C::C_S, sdesc_add(kK, kvo + off), sdesc_add(kQ, st * C::TILE + off),
+                  id_kk, kk > 0);
+        }
+        umma_commit(&s_full);
+      };
+      auto mma_dp = [&](int st, uint32_t kvo) {  // dP^T = V dO^T
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * C::CHUNK + (kk & 3) * 32;
+          umma_ss(tbase + C::C_DP, sdesc_add(kV, kvo + off), sdesc_add(kdO, st * C::TILE + off),
+                  id_kk, kk > 0);
+        }
+        umma_commit(&dp_full);
+      };
+      auto mma_dv = [&](int st, bool first) {  // dV += P^T dO (queries 16 kk ..: warpgroup kk / 4)
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          umma_ts(tbase + C::C_DV, tbase + C::C_P(kk >> 2) + (kk & 3) * 8,
+                  sdesc_add(mdO, st * C::TILE + kk * 2048), id_tb, (!first || kk > 0) ? 1u : 0u);
+      };
+      auto mma_dq = [&](uint32_t kvo) {  // dQ_i = dS K
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          umma_ss(tbase + C::C_DQ, sdesc_add(mDS, kk * 2048), sdesc_add(mK, kvo + kk * 2048),
+                  id_dq, kk > 0);
+        umma_commit(&dq_full);
+      };
+      auto mma_dk = [&](int st, bool first) {  // dK += dS^T Q; the step's last read of Q, dO
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          umma_ts(tbase + C::C_DK, tbase + C::C_DS(kk >> 2) + (kk & 3) * 8,
+                  sdesc_add(mQ, st * C::TILE + kk * 2048), id_tb, (!first || kk > 0) ? 1u : 0u);
+        umma_commit(&qdo_empty[st]);
+      };
       bool ok = true;
       int gs = 0;  // query steps so far
       for (int k = 0; ok; ++k) {
         const int t = tile_of(k);
         if (t < 0) break;
-        const int n_it = q_end(t / p.BH) - q_begin(t / p.BH);
+        const int n_it = q_end(t / BH) - q_begin(t / BH);
         const int b = k % C::KVB;
         const uint32_t kvo = static_cast<uint32_t>(b * C::TILE);  // this tile's K, V buffer
         if (!mbar_wait(&bar_kv[b], kv_par(k), wc, kBSiteMmaKV)) { ok = false; break; }
-        for (int it = 0; it < n_it; ++it, ++gs) {
-          const int st = gs % C::ST;
-          if (!mbar_wait(&qdo_full[st], (gs / C::ST) & 1, wc, kBSiteMmaQ)) { ok = false; break; }
+        if constexpr (C::PIPE) {
+          // Step g + 1's scores go out once the compute warps have read step g's
+          // (p_ready), so that they overlap step g's dS; step g + 1's dP^T follows
+          // step g's dK, whose dS^T operand sits in the dP^T columns.
+          if (!mbar_wait(&qdo_full[gs % C::ST], (gs / C::ST) & 1, wc, kBSiteMmaQ)) { ok = false; break; }
           tc_fence_after();
-          // S^T = K Q^T
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * C::CHUNK + (kk & 3) * 32;
-            umma_ss(tbase + C::C_S, sdesc_add(kK, kvo + off), sdesc_add(kQ, st * C::TILE + off),
-                    id_kk, kk > 0);
-          }
-          umma_commit(&s_full);
-          // dP^T = V dO^T (its columns hold the previous dQ partial when D = 128)
-          if (D == 128 && gs > 0) {
-            if (!mbar_wait(&dq_drained, (gs - 1) & 1, wc, kBSiteMmaDrained)) { ok = false; break; }
+          mma_s(gs % C::ST, kvo);
+          mma_dp(gs % C::ST, kvo);
+          for (int it = 0; it < n_it; ++it, ++gs) {
+            const int st = gs % C::ST;
+            if (!mbar_wait(&p_ready, gs & 1, wc, kBSiteMmaP)) { ok = false; break; }
             tc_fence_after();
-          }
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * C::CHUNK + (kk & 3) * 32;
-            umma_ss(tbase + C::C_DP, sdesc_add(kV, kvo + off), sdesc_add(kdO, st * C::TILE + off),
-                    id_kk, kk > 0);
-          }
-          umma_commit(&dp_full);
-          // dV += P^T dO
-          if (!mbar_wait(&p_ready, gs & 1, wc, kBSiteMmaP)) { ok = false; break; }
-          tc_fence_after();
-          if (k > 0 && it == 0) {
-            // A tile's first dV and dK products overwrite the accumulators: the
-            // previous tile's epilogue must have read them out.
-            if (!mbar_wait(&acc_free, (k - 1) & 1, wc, kBSiteMmaAcc)) { ok = false; break; }
+            if (k > 0 && it == 0) {
+              // A tile's first dV and dK products overwrite the accumulators: the
+              // previous tile's epilogue must have read them out.
+              if (!mbar_wait(&acc_free, (k - 1) & 1, wc, kBSiteMmaAcc)) { ok = false; break; }
+              tc_fence_after();
+            }
+            mma_dv(st, it == 0);
+            if (it + 1 < n_it) {
+              const int st1 = (gs + 1) % C::ST;
+              if (!mbar_wait(&qdo_full[st1], ((gs + 1) / C::ST) & 1, wc, kBSiteMmaQ)) { ok = false; break; }
+              tc_fence_after();
+              mma_s(st1, kvo);
+            }
+            if (!mbar_wait(&ds_ready, gs & 1, wc, kBSiteMmaDS)) { ok = false; break; }
             tc_fence_after();
+            if (gs > 0) {  // the dQ columns hold the previous partial until drained
+              if (!mbar_wait(&dq_drained, (gs - 1) & 1, wc, kBSiteMmaDrained)) { ok = false; break; }
+              tc_fence_after();
+            }
+            mma_dq(kvo);
+            // The tile's K, V have been read for the last time: release the buffer.
+            if (it == n_it - 1) umma_commit(&kv_empty[b]);
+            mma_dk(st, it == 0);
+            if (it + 1 < n_it) mma_dp((gs + 1) % C::ST, kvo);
           }
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)  // queries 16 kk .. 16 kk + 15: warpgroup kk / 4
-            umma_ts(tbase + C::C_DV, tbase + C::C_P(kk >> 2) + (kk & 3) * 8,
-                    sdesc_add(mdO, st * C::TILE + kk * 2048), id_tb,
-                    (it > 0 || kk > 0) ? 1u : 0u);
-          // dQ_i = dS K first (the drain needs only this one; its own TMEM columns
-          // when D = 64: wait for the previous drain), then dK += dS^T Q (A from
-          // TMEM, so the dQ staging that reuses the dS^T tile of shared memory
-          // cannot race it).
-          if (!mbar_wait(&ds_ready, gs & 1, wc, kBSiteMmaDS)) { ok = false; break; }
-          tc_fence_after();
-          if (D == 64 && gs > 0) {
-            if (!mbar_wait(&dq_drained, (gs - 1) & 1, wc, kBSiteMmaDrained)) { ok = false; break; }
+        } else {
+          for (int it = 0; it < n_it; ++it, ++gs) {
+            const int st = gs % C::ST;
+            if (!mbar_wait(&qdo_full[st], (gs / C::ST) & 1, wc, kBSiteMmaQ)) { ok = false; break; }
             tc_fence_after();
+            mma_s(st, kvo);
+            // dP^T's columns hold the previous dQ partial (D = 128) until drained.
+            if (C::C_DQ == C::C_DP && gs > 0) {
+              if (!mbar_wait(&dq_drained, (gs - 1) & 1, wc, kBSiteMmaDrained)) { ok = false; break; }
+              tc_fence_after();
+            }
+            mma_dp(st, kvo);
+            if (!mbar_wait(&p_ready, gs & 1, wc, kBSiteMmaP)) { ok = false; break; }
+            tc_fence_after();
+            if (k > 0 && it == 0) {
+              if (!mbar_wait(&acc_free, (k - 1) & 1, wc, kBSiteMmaAcc)) { ok = false; break; }
+              tc_fence_after();
+            }
+            mma_dv(st, it == 0);
+            // dQ_i = dS K first (the drain needs only this one; with its own TMEM
+            // columns, wait for the previous drain), then dK += dS^T Q (A from TMEM,
+            // so the dQ staging that reuses the dS^T tile of shared memory cannot
+            // race it).
+            if (!mbar_wait(&ds_ready, gs & 1, wc, kBSiteMmaDS)) { ok = false; break; }
+            tc_fence_after();
+            if (C::C_DQ != C::C_DP && gs > 0) {
+              if (!mbar_wait(&dq_drained, (gs - 1) & 1, wc, kBSiteMmaDrained)) { ok = false; break; }
+              tc_fence_after();
+            }
+            mma_dq(kvo);
+            if (it == n_it - 1) umma_commit(&kv_empty[b]);
+            mma_dk(st, it == 0);
           }
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            umma_ss(tbase + C::C_DQ, sdesc_add(mDS, kk * 2048), sdesc_add(mK, kvo + kk * 2048),
-                    id_dq, kk > 0);
-          umma_commit(&dq_full);
-          // The tile's K, V have been read for the last time: release the buffer.
-          if (it == n_it - 1) umma_commit(&kv_empty[b]);
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            umma_ts(tbase + C::C_DK, tbase + C::C_DS(kk >> 2) + (kk & 3) * 8,
-                    sdesc_add(mQ, st * C::TILE + kk * 2048), id_tb,
-                    (it > 0 || kk > 0) ? 1u : 0u);
-          umma_commit(&qdo_empty[st]);
         }
         if (!ok) break;
         umma_commit(&drain);  // the tile's dK and dV are final once this lands
@@ -517,6 +575,7 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     const uint32_t wg_bar = 1 + g;             // named barrier of this warpgroup
     bool ok = true;
     int gs = 0;  // query steps so far
+    float pr[64];  // this warpgroup's P^T of a step, from its P stage to its dS stage
     for (int k = 0; ok; ++k) {
       const int t = tile_of(k);
       if (t < 0) break;
@@ -524,27 +583,24 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       const int key = j * 128 + r;
       const int i_begin = q_begin(j);
       const int n_it = q_end(j) - i_begin;
-      for (int it = 0; it < n_it && ok; ++it, ++gs) {
-        const int i = i_begin + it;
-        const int st = gs % C::ST;
-        // This tile's LSE*log2e and D rows arrive in shared memory with Q_i and dO_i.
-        const float4* L4 = reinterpret_cast<const float4*>(sLD + st * 256 + qoff);
-        const float4* D4 = reinterpret_cast<const float4*>(sLD + st * 256 + 128 + qoff);
-        // Every wait of a compute warpgroup ends in a warpgroup-wide vote, so that all
-        // of its 128 threads leave together on a timeout (the named barriers below
-        // have no time limit and must never be left waiting).
-        ok = named_bar_and(wg_bar, 128, mbar_wait(&qdo_full[st], (gs / C::ST) & 1, wc, kBSiteCmpQ));
-        if (!ok) break;
-        ok = named_bar_and(wg_bar, 128, mbar_wait(&s_full, gs & 1, wc, kBSiteCmpS));
-        if (!ok) break;
+      // The three stages of query step gp (query tile ip).  Every wait of a compute
+      // warpgroup ends in a warpgroup-wide vote, so that all of its 128 threads
+      // leave together on a timeout (the named barriers have no time limit and must
+      // never be left waiting).
+      auto stage_p = [&](int gp, int ip) -> bool {
+        const int stp = gp % C::ST;
+        // The tile's LSE*log2e and D rows arrive in shared memory with Q_i and dO_i.
+        const float4* L4 = reinterpret_cast<const float4*>(sLD + stp * 256 + qoff);
+        if (!named_bar_and(wg_bar, 128, mbar_wait(&qdo_full[stp], (gp / C::ST) & 1, wc, kBSiteCmpQ)))
+          return false;
+        if (!named_bar_and(wg_bar, 128, mbar_wait(&s_full, gp & 1, wc, kBSiteCmpS))) return false;
         tc_fence_after();
         // P^T (this warpgroup's 64 query columns): exp2(S^T * scale * log2e - LSE * log2e),
         // zero where the key comes after the query or lies past N.
-        float pr[64];
         // Masking (key after query on the diagonal tile, or key past N) is rare: one
         // branch per tile, not a compare per element.
-        const bool masked = (CAUSAL && i == j) || key >= N ||
-                            (CAUSAL && win > 0 && i * 128 + 127 - j * 128 >= win);
+        const bool masked = (CAUSAL && ip == j) || key >= N ||
+                            (CAUSAL && win > 0 && ip * 128 + 127 - j * 128 >= win);
         const uint64_t sl2x2 = f2_pack(sl2, sl2);
         uint32_t srr[2][32];
         tmem_ld32(tmem_addr(tbase, lb, C::C_S + qoff), srr[0]);
@@ -552,10 +608,10 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         tmem_wait_ld();
         reg_fence(srr[0]);
         reg_fence(srr[1]);
-  #pragma unroll
+#pragma unroll
         for (int c = 0; c < 2; ++c) {
           const uint32_t (&sr)[32] = srr[c];
-  #pragma unroll
+#pragma unroll
           for (int v = 0; v < 8; ++v) {
             const float4 l4 = L4[c * 8 + v];
             const uint64_t a01 = f2_fma(f2_pack(__uint_as_float(sr[v * 4]), __uint_as_float(sr[v * 4 + 1])),
@@ -580,15 +636,15 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           }
         }
         if (masked) {
-  #pragma unroll
+#pragma unroll
           for (int qc = 0; qc < 64; ++qc)
-            if ((CAUSAL && i == j && qoff + qc < r) || key >= N ||
-                (CAUSAL && win > 0 && i * 128 + qoff + qc - key >= win))
+            if ((CAUSAL && ip == j && qoff + qc < r) || key >= N ||
+                (CAUSAL && win > 0 && ip * 128 + qoff + qc - key >= win))
               pr[qc] = 0.f;
         }
         {
           uint32_t pk[32];
-  #pragma unroll
+#pragma unroll
           for (int e = 0; e < 32; ++e) pk[e] = pack2<BF16>(pr[2 * e], pr[2 * e + 1]);
           tmem_st32(tmem_addr(tbase, lb, C::C_P(g)), pk);
         }
@@ -596,27 +652,30 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&p_ready);
-        // dS^T = P^T * (dP^T - D), 32 queries at a time, written to TMEM (A operand
-        // of dK) and to shared memory (A operand of dQ).  The shared copy is
-        // MN-major with 128-byte swizzle: chunk g holds queries 64 g .. 64 g + 63 of
-        // every key row; 16-byte unit u of row r sits at unit u ^ (r % 8).
-        ok = named_bar_and(wg_bar, 128, mbar_wait(&dp_full, gs & 1, wc, kBSiteCmpDP));
-        if (!ok) break;
+        return true;
+      };
+      // dS^T = P^T * (dP^T - D), 32 queries at a time, written to TMEM (A operand
+      // of dK) and to shared memory (A operand of dQ).  The shared copy is
+      // MN-major with 128-byte swizzle: chunk g holds queries 64 g .. 64 g + 63 of
+      // every key row; 16-byte unit u of row r sits at unit u ^ (r % 8).
+      auto stage_ds = [&](int gd) -> bool {
+        const float4* D4 = reinterpret_cast<const float4*>(sLD + (gd % C::ST) * 256 + 128 + qoff);
+        if (!named_bar_and(wg_bar, 128, mbar_wait(&dp_full, gd & 1, wc, kBSiteCmpDP))) return false;
         tc_fence_after();
-        if (gs > 0) {
+        if (gd > 0) {
           // This warpgroup's dS^T chunk doubled as the staging tile of the previous
           // dQ reduce: that bulk copy must have finished reading it.
           if (r == 0) tma_store_wait_read();
           named_bar_sync(wg_bar, 128);
         }
-  #pragma unroll
+#pragma unroll
         for (int c = 0; c < 2; ++c) {
           uint32_t dr[32];
           tmem_ld32(tmem_addr(tbase, lb, C::C_DP + qoff + 32 * c), dr);
           tmem_wait_ld();
           reg_fence(dr);
           uint32_t dsk[16];
-  #pragma unroll
+#pragma unroll
           for (int v = 0; v < 8; ++v) {
             const float4 d4 = D4[c * 8 + v];
             const int q0 = c * 32 + v * 4;
@@ -631,7 +690,7 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             dsk[2 * v + 1] = pack2<BF16>(a2, a3);
           }
           tmem_st16(tmem_addr(tbase, lb, C::C_DS(g) + 16 * c), dsk);
-  #pragma unroll
+#pragma unroll
           for (int uu = 0; uu < 4; ++uu) {
             const int u = c * 4 + uu;
             const uint4 val = make_uint4(dsk[4 * uu], dsk[4 * uu + 1], dsk[4 * uu + 2], dsk[4 * uu + 3]);
@@ -643,9 +702,10 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&ds_ready);
-        // dQ partial: query row r, head columns g D/2 .. (g+1) D/2 - 1 -> fp32 accumulator
-        ok = named_bar_and(wg_bar, 128, mbar_wait(&dq_full, gs & 1, wc, kBSiteCmpDQ));
-        if (!ok) break;
+        return true;
+      };
+      auto stage_dq = [&](int gq, int iq) -> bool {
+        if (!named_bar_and(wg_bar, 128, mbar_wait(&dq_full, gq & 1, wc, kBSiteCmpDQ))) return false;
         tc_fence_after();
         // dQ partial, head columns g D/2 .. (g+1) D/2 - 1, 32 at a time: TMEM ->
         // this warpgroup's dS^T chunk of shared memory (free: the dQ product that
@@ -655,37 +715,88 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         constexpr int HALF = D / 2;
         constexpr int NCH = HALF / 32;
         uint8_t* stage = sDS + g * C::CHUNK;
-        // All of this warpgroup's TMEM columns first, so that the region is released
-        // (dq_drained) before any staging starts.
-        uint32_t qr[NCH][32];
-  #pragma unroll
-        for (int c = 0; c < NCH; ++c)
-          tmem_ld32(tmem_addr(tbase, lb, C::C_DQ + g * HALF + 32 * c), qr[c]);
-        tmem_wait_ld();
-  #pragma unroll
-        for (int c = 0; c < NCH; ++c) reg_fence(qr[c]);
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&dq_drained);
-  #pragma unroll
-        for (int c = 0; c < NCH; ++c) {
-          if (c > 0) {
-            if (r == 0) tma_store_wait_read();
-            named_bar_sync(wg_bar, 128);
+        if constexpr (C::PIPE) {
+          // One 32-column tile, 16 columns at a time: the next step's P^T is live
+          // beside it.  The columns are released once both halves are read.
+          static_assert(NCH == 1, "pipelined steps assume D = 64");
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            uint32_t q16[16];
+            tmem_ld16(tmem_addr(tbase, lb, C::C_DQ + g * HALF + 16 * h), q16);
+            tmem_wait_ld();
+            reg_fence(q16);
+            if (h == 1) {
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&dq_drained);
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+              *reinterpret_cast<uint4*>(stage + r * 128 + (((4 * h + u) ^ (r & 7)) << 4)) =
+                  make_uint4(q16[4 * u], q16[4 * u + 1], q16[4 * u + 2], q16[4 * u + 3]);
           }
-  #pragma unroll
-          for (int u = 0; u < 8; ++u)
-            *reinterpret_cast<uint4*>(stage + r * 128 + ((u ^ (r & 7)) << 4)) =
-                make_uint4(qr[c][4 * u], qr[c][4 * u + 1], qr[c][4 * u + 2], qr[c][4 * u + 3]);
           fence_proxy_async_smem();
           named_bar_sync(wg_bar, 128);
           if (r == 0) {
-            tma_reduce_add_3d(&tmdQ, stage, g * HALF + 32 * c, i * 128, bh);
+            tma_reduce_add_3d(&tmdQ, stage, g * HALF, iq * 128, bh);
             tma_store_commit();
           }
           __syncwarp();
+        } else {
+          // All of this warpgroup's TMEM columns first, so that the region is released
+          // (dq_drained) before any staging starts.
+          uint32_t qr[NCH][32];
+#pragma unroll
+          for (int c = 0; c < NCH; ++c)
+            tmem_ld32(tmem_addr(tbase, lb, C::C_DQ + g * HALF + 32 * c), qr[c]);
+          tmem_wait_ld();
+#pragma unroll
+          for (int c = 0; c < NCH; ++c) reg_fence(qr[c]);
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&dq_drained);
+#pragma unroll
+          for (int c = 0; c < NCH; ++c) {
+            if (c > 0) {
+              if (r == 0) tma_store_wait_read();
+              named_bar_sync(wg_bar, 128);
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+              *reinterpret_cast<uint4*>(stage + r * 128 + ((u ^ (r & 7)) << 4)) =
+                  make_uint4(qr[c][4 * u], qr[c][4 * u + 1], qr[c][4 * u + 2], qr[c][4 * u + 3]);
+            fence_proxy_async_smem();
+            named_bar_sync(wg_bar, 128);
+            if (r == 0) {
+              tma_reduce_add_3d(&tmdQ, stage, g * HALF + 32 * c, iq * 128, bh);
+              tma_store_commit();
+            }
+            __syncwarp();
+          }
         }
+        return true;
+      };
+      // Plain order: P, dS, dQ drain of each step.  Pipelined (C::PIPE): P of step
+      // i + 1 between dS and the dQ drain of step i, so that step i's dQ product and
+      // step i + 1's dP product run while the softmax works.
+      const int g0 = gs;
+      if constexpr (C::PIPE) ok = stage_p(g0, i_begin);
+      for (int it = 0; it < n_it && ok; ++it) {
+        if constexpr (!C::PIPE) {
+          ok = stage_p(g0 + it, i_begin + it);
+          if (!ok) break;
+        }
+        ok = stage_ds(g0 + it);
+        if (!ok) break;
+        if constexpr (C::PIPE) {
+          if (it + 1 < n_it) {
+            ok = stage_p(g0 + it + 1, i_begin + it + 1);
+            if (!ok) break;
+          }
+        }
+        ok = stage_dq(g0 + it, i_begin + it);
       }
+      gs = g0 + n_it;
       if (!ok) break;
       // dV (warpgroup 0) and dK (warpgroup 1) of the tile are final once its
       // products have landed: read them out of TMEM, hand the columns to the next
