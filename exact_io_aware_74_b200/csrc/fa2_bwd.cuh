@@ -576,6 +576,237 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     bool ok = true;
     int gs = 0;  // query steps so far
     float pr[64];  // this warpgroup's P^T of a step, from its P stage to its dS stage
+    // The three stages of query step gp (query tile ip of key tile j).  Every wait
+    // of a compute warpgroup ends in a warpgroup-wide vote, so that all of its 128
+    // threads leave together on a timeout (the named barriers have no time limit and
+    // must never be left waiting).
+    auto stage_p = [&](int gp, int ip, int j, int key) -> bool {
+      const int stp = gp % C::ST;
+      // The tile's LSE*log2e and D rows arrive in shared memory with Q_i and dO_i.
+      const float4* L4 = reinterpret_cast<const float4*>(sLD + stp * 256 + qoff);
+      if (!named_bar_and(wg_bar, 128, mbar_wait(&qdo_full[stp], (gp / C::ST) & 1, wc, kBSiteCmpQ)))
+        return false;
+      if (!named_bar_and(wg_bar, 128, mbar_wait(&s_full, gp & 1, wc, kBSiteCmpS))) return false;
+      tc_fence_after();
+      // P^T (this warpgroup's 64 query columns): exp2(S^T * scale * log2e - LSE * log2e),
+      // zero where the key comes after the query or lies past N.
+      // Masking (key after query on the diagonal tile, or key past N) is rare: one
+      // branch per tile, not a compare per element.
+      const bool masked = (CAUSAL && ip == j) || key >= N ||
+                          (CAUSAL && win > 0 && ip * 128 + 127 - j * 128 >= win);
+      const uint64_t sl2x2 = f2_pack(sl2, sl2);
+      uint32_t srr[2][32];
+      tmem_ld32(tmem_addr(tbase, lb, C::C_S + qoff), srr[0]);
+      tmem_ld32(tmem_addr(tbase, lb, C::C_S + qoff + 32), srr[1]);
+      tmem_wait_ld();
+      reg_fence(srr[0]);
+      reg_fence(srr[1]);
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        const uint32_t (&sr)[32] = srr[c];
+#pragma unroll
+        for (int v = 0; v < 8; ++v) {
+          const float4 l4 = L4[c * 8 + v];
+          const uint64_t a01 = f2_fma(f2_pack(__uint_as_float(sr[v * 4]), __uint_as_float(sr[v * 4 + 1])),
+                                      sl2x2, f2_pack(-l4.x, -l4.y));
+          const uint64_t a23 = f2_fma(f2_pack(__uint_as_float(sr[v * 4 + 2]), __uint_as_float(sr[v * 4 + 3])),
+                                      sl2x2, f2_pack(-l4.z, -l4.w));
+          float x0, x1, x2, x3;
+          f2_unpack(a01, x0, x1);
+          f2_unpack(a23, x2, x3);
+          const int q0 = c * 32 + v * 4;
+          if ((v & 3) >= kBwdPolyFrom) {  // FMA-pipe exp2 for this group of four
+            pr[q0 + 0] = exp2_poly3(x0);
+            pr[q0 + 1] = exp2_poly3(x1);
+            pr[q0 + 2] = exp2_poly3(x2);
+            pr[q0 + 3] = exp2_poly3(x3);
+          } else {
+            pr[q0 + 0] = ex2_approx(x0);
+            pr[q0 + 1] = ex2_approx(x1);
+            pr[q0 + 2] = ex2_approx(x2);
+            pr[q0 + 3] = ex2_approx(x3);
+          }
+        }
+      }
+      if (masked) {
+#pragma unroll
+        for (int qc = 0; qc < 64; ++qc)
+          if ((CAUSAL && ip == j && qoff + qc < r) || key >= N ||
+              (CAUSAL && win > 0 && ip * 128 + qoff + qc - key >= win))
+            pr[qc] = 0.f;
+      }
+      {
+        uint32_t pk[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) pk[e] = pack2<BF16>(pr[2 * e], pr[2 * e + 1]);
+        tmem_st32(tmem_addr(tbase, lb, C::C_P(g)), pk);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_ready);
+      return true;
+    };
+    // dS^T = P^T * (dP^T - D), 32 queries at a time, written to TMEM (A operand
+    // of dK) and to shared memory (A operand of dQ).  The shared copy is
+    // MN-major with 128-byte swizzle: chunk g holds queries 64 g .. 64 g + 63 of
+    // every key row; 16-byte unit u of row r sits at unit u ^ (r % 8).
+    auto stage_ds = [&](int gd) -> bool {
+      const float4* D4 = reinterpret_cast<const float4*>(sLD + (gd % C::ST) * 256 + 128 + qoff);
+      if (!named_bar_and(wg_bar, 128, mbar_wait(&dp_full, gd & 1, wc, kBSiteCmpDP))) return false;
+      tc_fence_after();
+      if (gd > 0) {
+        // This warpgroup's dS^T chunk doubled as the staging tile of the previous
+        // dQ reduce: that bulk copy must have finished reading it.
+        if (r == 0) tma_store_wait_read();
+        named_bar_sync(wg_bar, 128);
+      }
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        uint32_t dr[32];
+        tmem_ld32(tmem_addr(tbase, lb, C::C_DP + qoff + 32 * c), dr);
+        tmem_wait_ld();
+        reg_fence(dr);
+        uint32_t dsk[16];
+#pragma unroll
+        for (int v = 0; v < 8; ++v) {
+          const float4 d4 = D4[c * 8 + v];
+          const int q0 = c * 32 + v * 4;
+          const uint64_t t01 = f2_sub(f2_pack(__uint_as_float(dr[v * 4]), __uint_as_float(dr[v * 4 + 1])),
+                                      f2_pack(d4.x, d4.y));
+          const uint64_t t23 = f2_sub(f2_pack(__uint_as_float(dr[v * 4 + 2]), __uint_as_float(dr[v * 4 + 3])),
+                                      f2_pack(d4.z, d4.w));
+          float a0, a1, a2, a3;
+          f2_unpack(f2_mul(f2_pack(pr[q0], pr[q0 + 1]), t01), a0, a1);
+          f2_unpack(f2_mul(f2_pack(pr[q0 + 2], pr[q0 + 3]), t23), a2, a3);
+          dsk[2 * v] = pack2<BF16>(a0, a1);
+          dsk[2 * v + 1] = pack2<BF16>(a2, a3);
+        }
+        tmem_st16(tmem_addr(tbase, lb, C::C_DS(g) + 16 * c), dsk);
+#pragma unroll
+        for (int uu = 0; uu < 4; ++uu) {
+          const int u = c * 4 + uu;
+          const uint4 val = make_uint4(dsk[4 * uu], dsk[4 * uu + 1], dsk[4 * uu + 2], dsk[4 * uu + 3]);
+          *reinterpret_cast<uint4*>(sDS + g * C::CHUNK + r * 128 + ((u ^ (r & 7)) << 4)) = val;
+        }
+      }
+      fence_proxy_async_smem();
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ds_ready);
+      return true;
+    };
+    auto stage_dq = [&](int gq, int iq, int bh) -> bool {
+      if (!named_bar_and(wg_bar, 128, mbar_wait(&dq_full, gq & 1, wc, kBSiteCmpDQ))) return false;
+      tc_fence_after();
+      // dQ partial, head columns g D/2 .. (g+1) D/2 - 1, 32 at a time: TMEM ->
+      // this warpgroup's dS^T chunk of shared memory (free: the dQ product that
+      // read it has completed), laid out as a 128-row x 32-float tile with
+      // 128-byte swizzle -> one TMA reduce-add into the fp32 accumulator (rows
+      // past N are clipped by the tensor map).
+      constexpr int HALF = D / 2;
+      constexpr int NCH = HALF / 32;
+      uint8_t* stage = sDS + g * C::CHUNK;
+      if constexpr (C::PIPE) {
+        // One 32-column tile, 16 columns at a time: the next step's P^T is live
+        // beside it.  The columns are released once both halves are read.
+        static_assert(NCH == 1, "pipelined steps assume D = 64");
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t q16[16];
+          tmem_ld16(tmem_addr(tbase, lb, C::C_DQ + g * HALF + 16 * h), q16);
+          tmem_wait_ld();
+          reg_fence(q16);
+          if (h == 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&dq_drained);
+          }
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+            *reinterpret_cast<uint4*>(stage + r * 128 + (((4 * h + u) ^ (r & 7)) << 4)) =
+                make_uint4(q16[4 * u], q16[4 * u + 1], q16[4 * u + 2], q16[4 * u + 3]);
+        }
+        fence_proxy_async_smem();
+        named_bar_sync(wg_bar, 128);
+        if (r == 0) {
+          tma_reduce_add_3d(&tmdQ, stage, g * HALF, iq * 128, bh);
+          tma_store_commit();
+        }
+        __syncwarp();
+      } else {
+        // All of this warpgroup's TMEM columns first, so that the region is released
+        // (dq_drained) before any staging starts.
+        uint32_t qr[NCH][32];
+#pragma unroll
+        for (int c = 0; c < NCH; ++c)
+          tmem_ld32(tmem_addr(tbase, lb, C::C_DQ + g * HALF + 32 * c), qr[c]);
+        tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < NCH; ++c) reg_fence(qr[c]);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&dq_drained);
+#pragma unroll
+        for (int c = 0; c < NCH; ++c) {
+          if (c > 0) {
+            if (r == 0) tma_store_wait_read();
+            named_bar_sync(wg_bar, 128);
+          }
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+            *reinterpret_cast<uint4*>(stage + r * 128 + ((u ^ (r & 7)) << 4)) =
+                make_uint4(qr[c][4 * u], qr[c][4 * u + 1], qr[c][4 * u + 2], qr[c][4 * u + 3]);
+          fence_proxy_async_smem();
+          named_bar_sync(wg_bar, 128);
+          if (r == 0) {
+            tma_reduce_add_3d(&tmdQ, stage, g * HALF + 32 * c, iq * 128, bh);
+            tma_store_commit();
+          }
+          __syncwarp();
+        }
+      }
+      return true;
+    };
+    // dV (warpgroup 0) and dK (warpgroup 1) of the tile are final once its
+    // products have landed: read them out of TMEM, hand the columns to the next
+    // tile's products, then store them.
+    auto epilogue = [&](int k, int key, int bh) -> bool {
+      if (!named_bar_and(wg_bar, 128, mbar_wait(&drain, k & 1, wc, kBSiteCmpDQ))) return false;
+      tc_fence_after();
+      const uint32_t col = g ? C::C_DK : C::C_DV;
+      const float mul = g ? p.scale : 1.0f;
+      const int d = p.d;
+      uint8_t* row = reinterpret_cast<uint8_t*>(g ? p.dK : p.dV) +
+                     (static_cast<size_t>(bh) * N + key) * (d * 2);
+      // 32 columns at a time: TMEM -> 16-bit -> global (stores do not wait), the
+      // columns handed back once the last chunk is in registers.
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t rr[32];
+        tmem_ld32(tmem_addr(tbase, lb, col + 32 * c), rr);
+        tmem_wait_ld();
+        reg_fence(rr);
+        if (c == D / 32 - 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&acc_free);
+        }
+        uint4 v[4];
+        uint32_t* pv = reinterpret_cast<uint32_t*>(v);
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          pv[e] = pack2<BF16>(__uint_as_float(rr[2 * e]) * mul, __uint_as_float(rr[2 * e + 1]) * mul);
+        if (key < N) {
+          uint4* dst4 = reinterpret_cast<uint4*>(row + c * 64);
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            if (c * 32 + 8 * e < d) dst4[e] = v[e];  // 8 columns per store; d % 8 == 0
+        }
+      }
+      return true;
+    };
     for (int k = 0; ok; ++k) {
       const int t = tile_of(k);
       if (t < 0) break;
@@ -583,256 +814,29 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       const int key = j * 128 + r;
       const int i_begin = q_begin(j);
       const int n_it = q_end(j) - i_begin;
-      // The three stages of query step gp (query tile ip).  Every wait of a compute
-      // warpgroup ends in a warpgroup-wide vote, so that all of its 128 threads
-      // leave together on a timeout (the named barriers have no time limit and must
-      // never be left waiting).
-      auto stage_p = [&](int gp, int ip) -> bool {
-        const int stp = gp % C::ST;
-        // The tile's LSE*log2e and D rows arrive in shared memory with Q_i and dO_i.
-        const float4* L4 = reinterpret_cast<const float4*>(sLD + stp * 256 + qoff);
-        if (!named_bar_and(wg_bar, 128, mbar_wait(&qdo_full[stp], (gp / C::ST) & 1, wc, kBSiteCmpQ)))
-          return false;
-        if (!named_bar_and(wg_bar, 128, mbar_wait(&s_full, gp & 1, wc, kBSiteCmpS))) return false;
-        tc_fence_after();
-        // P^T (this warpgroup's 64 query columns): exp2(S^T * scale * log2e - LSE * log2e),
-        // zero where the key comes after the query or lies past N.
-        // Masking (key after query on the diagonal tile, or key past N) is rare: one
-        // branch per tile, not a compare per element.
-        const bool masked = (CAUSAL && ip == j) || key >= N ||
-                            (CAUSAL && win > 0 && ip * 128 + 127 - j * 128 >= win);
-        const uint64_t sl2x2 = f2_pack(sl2, sl2);
-        uint32_t srr[2][32];
-        tmem_ld32(tmem_addr(tbase, lb, C::C_S + qoff), srr[0]);
-        tmem_ld32(tmem_addr(tbase, lb, C::C_S + qoff + 32), srr[1]);
-        tmem_wait_ld();
-        reg_fence(srr[0]);
-        reg_fence(srr[1]);
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          const uint32_t (&sr)[32] = srr[c];
-#pragma unroll
-          for (int v = 0; v < 8; ++v) {
-            const float4 l4 = L4[c * 8 + v];
-            const uint64_t a01 = f2_fma(f2_pack(__uint_as_float(sr[v * 4]), __uint_as_float(sr[v * 4 + 1])),
-                                        sl2x2, f2_pack(-l4.x, -l4.y));
-            const uint64_t a23 = f2_fma(f2_pack(__uint_as_float(sr[v * 4 + 2]), __uint_as_float(sr[v * 4 + 3])),
-                                        sl2x2, f2_pack(-l4.z, -l4.w));
-            float x0, x1, x2, x3;
-            f2_unpack(a01, x0, x1);
-            f2_unpack(a23, x2, x3);
-            const int q0 = c * 32 + v * 4;
-            if ((v & 3) >= kBwdPolyFrom) {  // FMA-pipe exp2 for this group of four
-              pr[q0 + 0] = exp2_poly3(x0);
-              pr[q0 + 1] = exp2_poly3(x1);
-              pr[q0 + 2] = exp2_poly3(x2);
-              pr[q0 + 3] = exp2_poly3(x3);
-            } else {
-              pr[q0 + 0] = ex2_approx(x0);
-              pr[q0 + 1] = ex2_approx(x1);
-              pr[q0 + 2] = ex2_approx(x2);
-              pr[q0 + 3] = ex2_approx(x3);
-            }
-          }
-        }
-        if (masked) {
-#pragma unroll
-          for (int qc = 0; qc < 64; ++qc)
-            if ((CAUSAL && ip == j && qoff + qc < r) || key >= N ||
-                (CAUSAL && win > 0 && ip * 128 + qoff + qc - key >= win))
-              pr[qc] = 0.f;
-        }
-        {
-          uint32_t pk[32];
-#pragma unroll
-          for (int e = 0; e < 32; ++e) pk[e] = pack2<BF16>(pr[2 * e], pr[2 * e + 1]);
-          tmem_st32(tmem_addr(tbase, lb, C::C_P(g)), pk);
-        }
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&p_ready);
-        return true;
-      };
-      // dS^T = P^T * (dP^T - D), 32 queries at a time, written to TMEM (A operand
-      // of dK) and to shared memory (A operand of dQ).  The shared copy is
-      // MN-major with 128-byte swizzle: chunk g holds queries 64 g .. 64 g + 63 of
-      // every key row; 16-byte unit u of row r sits at unit u ^ (r % 8).
-      auto stage_ds = [&](int gd) -> bool {
-        const float4* D4 = reinterpret_cast<const float4*>(sLD + (gd % C::ST) * 256 + 128 + qoff);
-        if (!named_bar_and(wg_bar, 128, mbar_wait(&dp_full, gd & 1, wc, kBSiteCmpDP))) return false;
-        tc_fence_after();
-        if (gd > 0) {
-          // This warpgroup's dS^T chunk doubled as the staging tile of the previous
-          // dQ reduce: that bulk copy must have finished reading it.
-          if (r == 0) tma_store_wait_read();
-          named_bar_sync(wg_bar, 128);
-        }
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          uint32_t dr[32];
-          tmem_ld32(tmem_addr(tbase, lb, C::C_DP + qoff + 32 * c), dr);
-          tmem_wait_ld();
-          reg_fence(dr);
-          uint32_t dsk[16];
-#pragma unroll
-          for (int v = 0; v < 8; ++v) {
-            const float4 d4 = D4[c * 8 + v];
-            const int q0 = c * 32 + v * 4;
-            const uint64_t t01 = f2_sub(f2_pack(__uint_as_float(dr[v * 4]), __uint_as_float(dr[v * 4 + 1])),
-                                        f2_pack(d4.x, d4.y));
-            const uint64_t t23 = f2_sub(f2_pack(__uint_as_float(dr[v * 4 + 2]), __uint_as_float(dr[v * 4 + 3])),
-                                        f2_pack(d4.z, d4.w));
-            float a0, a1, a2, a3;
-            f2_unpack(f2_mul(f2_pack(pr[q0], pr[q0 + 1]), t01), a0, a1);
-            f2_unpack(f2_mul(f2_pack(pr[q0 + 2], pr[q0 + 3]), t23), a2, a3);
-            dsk[2 * v] = pack2<BF16>(a0, a1);
-            dsk[2 * v + 1] = pack2<BF16>(a2, a3);
-          }
-          tmem_st16(tmem_addr(tbase, lb, C::C_DS(g) + 16 * c), dsk);
-#pragma unroll
-          for (int uu = 0; uu < 4; ++uu) {
-            const int u = c * 4 + uu;
-            const uint4 val = make_uint4(dsk[4 * uu], dsk[4 * uu + 1], dsk[4 * uu + 2], dsk[4 * uu + 3]);
-            *reinterpret_cast<uint4*>(sDS + g * C::CHUNK + r * 128 + ((u ^ (r & 7)) << 4)) = val;
-          }
-        }
-        fence_proxy_async_smem();
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&ds_ready);
-        return true;
-      };
-      auto stage_dq = [&](int gq, int iq) -> bool {
-        if (!named_bar_and(wg_bar, 128, mbar_wait(&dq_full, gq & 1, wc, kBSiteCmpDQ))) return false;
-        tc_fence_after();
-        // dQ partial, head columns g D/2 .. (g+1) D/2 - 1, 32 at a time: TMEM ->
-        // this warpgroup's dS^T chunk of shared memory (free: the dQ product that
-        // read it has completed), laid out as a 128-row x 32-float tile with
-        // 128-byte swizzle -> one TMA reduce-add into the fp32 accumulator (rows
-        // past N are clipped by the tensor map).
-        constexpr int HALF = D / 2;
-        constexpr int NCH = HALF / 32;
-        uint8_t* stage = sDS + g * C::CHUNK;
-        if constexpr (C::PIPE) {
-          // One 32-column tile, 16 columns at a time: the next step's P^T is live
-          // beside it.  The columns are released once both halves are read.
-          static_assert(NCH == 1, "pipelined steps assume D = 64");
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            uint32_t q16[16];
-            tmem_ld16(tmem_addr(tbase, lb, C::C_DQ + g * HALF + 16 * h), q16);
-            tmem_wait_ld();
-            reg_fence(q16);
-            if (h == 1) {
-              tc_fence_before();
-              __syncwarp();
-              if (lane == 0) mbar_arrive(&dq_drained);
-            }
-#pragma unroll
-            for (int u = 0; u < 4; ++u)
-              *reinterpret_cast<uint4*>(stage + r * 128 + (((4 * h + u) ^ (r & 7)) << 4)) =
-                  make_uint4(q16[4 * u], q16[4 * u + 1], q16[4 * u + 2], q16[4 * u + 3]);
-          }
-          fence_proxy_async_smem();
-          named_bar_sync(wg_bar, 128);
-          if (r == 0) {
-            tma_reduce_add_3d(&tmdQ, stage, g * HALF, iq * 128, bh);
-            tma_store_commit();
-          }
-          __syncwarp();
-        } else {
-          // All of this warpgroup's TMEM columns first, so that the region is released
-          // (dq_drained) before any staging starts.
-          uint32_t qr[NCH][32];
-#pragma unroll
-          for (int c = 0; c < NCH; ++c)
-            tmem_ld32(tmem_addr(tbase, lb, C::C_DQ + g * HALF + 32 * c), qr[c]);
-          tmem_wait_ld();
-#pragma unroll
-          for (int c = 0; c < NCH; ++c) reg_fence(qr[c]);
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&dq_drained);
-#pragma unroll
-          for (int c = 0; c < NCH; ++c) {
-            if (c > 0) {
-              if (r == 0) tma_store_wait_read();
-              named_bar_sync(wg_bar, 128);
-            }
-#pragma unroll
-            for (int u = 0; u < 8; ++u)
-              *reinterpret_cast<uint4*>(stage + r * 128 + ((u ^ (r & 7)) << 4)) =
-                  make_uint4(qr[c][4 * u], qr[c][4 * u + 1], qr[c][4 * u + 2], qr[c][4 * u + 3]);
-            fence_proxy_async_smem();
-            named_bar_sync(wg_bar, 128);
-            if (r == 0) {
-              tma_reduce_add_3d(&tmdQ, stage, g * HALF + 32 * c, iq * 128, bh);
-              tma_store_commit();
-            }
-            __syncwarp();
-          }
-        }
-        return true;
-      };
       // Plain order: P, dS, dQ drain of each step.  Pipelined (C::PIPE): P of step
       // i + 1 between dS and the dQ drain of step i, so that step i's dQ product and
       // step i + 1's dP product run while the softmax works.
       const int g0 = gs;
-      if constexpr (C::PIPE) ok = stage_p(g0, i_begin);
+      if constexpr (C::PIPE) ok = stage_p(g0, i_begin, j, key);
       for (int it = 0; it < n_it && ok; ++it) {
         if constexpr (!C::PIPE) {
-          ok = stage_p(g0 + it, i_begin + it);
+          ok = stage_p(g0 + it, i_begin + it, j, key);
           if (!ok) break;
         }
         ok = stage_ds(g0 + it);
         if (!ok) break;
         if constexpr (C::PIPE) {
           if (it + 1 < n_it) {
-            ok = stage_p(g0 + it + 1, i_begin + it + 1);
+            ok = stage_p(g0 + it + 1, i_begin + it + 1, j, key);
             if (!ok) break;
           }
         }
-        ok = stage_dq(g0 + it, i_begin + it);
+        ok = stage_dq(g0 + it, i_begin + it, bh);
       }
       gs = g0 + n_it;
       if (!ok) break;
-      // dV (warpgroup 0) and dK (warpgroup 1) of the tile are final once its
-      // products have landed: read them out of TMEM, hand the columns to the next
-      // tile's products, then store them.
-      ok = named_bar_and(wg_bar, 128, mbar_wait(&drain, k & 1, wc, kBSiteCmpDQ));
-      if (!ok) break;
-      tc_fence_after();
-      const uint32_t col = g ? C::C_DK : C::C_DV;
-      const float mul = g ? p.scale : 1.0f;
-      uint4 v[D / 32][4];
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t rr[32];
-        tmem_ld32(tmem_addr(tbase, lb, col + 32 * c), rr);
-        tmem_wait_ld();
-        reg_fence(rr);
-        uint32_t* pv = reinterpret_cast<uint32_t*>(v[c]);
-#pragma unroll
-        for (int e = 0; e < 16; ++e)
-          pv[e] = pack2<BF16>(__uint_as_float(rr[2 * e]) * mul, __uint_as_float(rr[2 * e + 1]) * mul);
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&acc_free);
-      if (key < N) {
-        const int d = p.d;
-        uint8_t* row = reinterpret_cast<uint8_t*>(g ? p.dK : p.dV) +
-                       (static_cast<size_t>(bh) * N + key) * (d * 2);
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint4* dst4 = reinterpret_cast<uint4*>(row + c * 64);
-#pragma unroll
-          for (int e = 0; e < 4; ++e)
-            if (c * 32 + 8 * e < d) dst4[e] = v[c][e];  // 8 columns per store; d % 8 == 0
-        }
-      }
+      ok = epilogue(k, key, bh);
     }
     // All reductions complete before the CTA (and its shared memory) goes away.
     if (r == 0) tma_store_wait_all();
