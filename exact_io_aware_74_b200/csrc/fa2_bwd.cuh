@@ -8,12 +8,15 @@
 //   dV = P^T dO,  dP = dO V^T,  D_i = sum_c dO_ic O_ic,
 //   dS = P * (dP - D),  dQ = scale dS K,  dK = scale dS^T Q.
 //
-// Three kernels per call, all on the caller's stream:
+// Three kernels per call, all on the caller's stream, chained by programmatic
+// dependent launch (each reads nothing before its griddepcontrol.wait):
 //   1. fa2_bwd_pre_kernel  : D and LSE * log2(e) per query row (padded to a
 //                            multiple of 128 rows), and a zeroed fp32 dQ
 //                            accumulator;
-//   2. fa2_bwd_kernel      : one CTA per (128-key tile, batch*head); loops over
-//                            the query tiles that see those keys;
+//   2. fa2_bwd_kernel      : persistent, at most one CTA per SM.  The key tiles
+//                            (128 keys, batch*head) are listed heaviest first and
+//                            dealt to the CTAs in snake order; each tile loops
+//                            over the query tiles that see its keys;
 //   3. fa2_bwd_dq_kernel   : dQ = scale * accumulator, rounded to 16 bits.
 //
 // Main kernel, CTA layout (320 threads):
@@ -21,17 +24,23 @@
 //             row r of the tile for the query columns 64 g .. 64 g + 63 of P^T
 //             and dS^T, and query row r of the current query tile for the head
 //             columns g D/2 .. (g+1) D/2 - 1 when it moves the dQ partial from
-//             TMEM to the fp32 accumulator (vector atomics).  Splitting every
-//             row between the two warpgroups halves the per-tile chain
-//             P^T -> dS^T -> dQ drain that the products wait on;
-//   warp  8   TMA producer: K_j and V_j once, then a 2-stage ring of (Q_i, dO_i);
+//             TMEM through shared memory into the fp32 accumulator (one TMA
+//             reduce-add per 128 x 32 tile).  Splitting every row between the
+//             two warpgroups halves the per-step chain P^T -> dS^T -> dQ drain
+//             that the products wait on;
+//   warp  8   TMA producer: K_j and V_j per tile (two buffers at D = 64, the next
+//             tile's loaded during the current one), a 2-stage ring of (Q_i, dO_i)
+//             and the tile's LSE / D rows, across the CTA's tiles;
 //   warp  9   tcgen05 MMA issuer (one thread).
-// TMEM (fp32 columns): S^T [0,128), warpgroup g's query columns at [64 g, 64 g + 64);
-// each warpgroup packs its P^T (16-bit pairs) into [64 g, 64 g + 32) and its dS^T
-// into [64 g + 32, 64 g + 64) -- inside its own score columns, which it has fully
-// read by then, never the other warpgroup's; dP^T [128,256); dV [256,256+D);
-// dK [256+D,256+2D); the dQ partial reuses [128,256) when D = 128 and has
-// [384,448) when D = 64.
+// TMEM (fp32 columns), D = 128: S^T [0,128), warpgroup g's query columns at
+// [64 g, 64 g + 64); each warpgroup packs its P^T (16-bit pairs) into
+// [64 g, 64 g + 32) and its dS^T into [64 g + 32, 64 g + 64) -- inside its own
+// score columns, which it has fully read by then, never the other warpgroup's;
+// dP^T [128,256), also the dQ partial; dV [256,384); dK [384,512).
+// D = 64: S^T [0,128); dP^T [128,256) with warpgroup g's packed dS^T written over
+// its own dP^T columns [128 + 64 g, + 32); dV [256,320); dK [320,384); dQ
+// [384,448); packed P^T of warpgroup g at [448 + 32 g, + 32).  The score columns
+// are then free once read, and the steps are software-pipelined (BwdCfg::PIPE).
 // Products (M = 128 rows of the first operand, K = 16 per instruction):
 //   S^T  = K_j  Q_i^T   (A = K smem K-major, B = Q smem K-major)
 //   dP^T = V_j  dO_i^T  (A = V smem K-major, B = dO smem K-major)
