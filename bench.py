@@ -13,7 +13,7 @@ Multi-GPU (under torchrun): every rank runs an independent replica of the same
 workload (the attention of every (batch, head) is independent; no collective sits
 on the data path), so scaling is weak.
 
-``--impl reference`` times the CPU fp64 oracle (the reference arm of this build)
+``--impl reference`` times the CPU fp64 oracle (the reference arm)
 on a bounded sample of the same workload, on rank 0 only.
 """
 
