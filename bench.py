@@ -170,7 +170,7 @@ class ClockSampler:
             self._nv = pynvml
             self._h = pynvml.nvmlDeviceGetHandleByIndex(self.index)
             self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
-        except Exception as e:  # pragma: no cover - depends on the box
+        except Exception as e:  # pragma: no cover - depends on the host (NVML present or not)
             self.error = repr(e)
             return self
         self._thread = threading.Thread(target=self._run, daemon=True)
