@@ -25,6 +25,7 @@ unsigned int* g_status[kMaxDevices] = {};  // one device word per device, lazily
 std::atomic<int> g_fault{0};
 std::atomic<unsigned int> g_wait_ms{kDefaultWaitMs};
 std::atomic<int> g_bwd_ctas{0};  // test hook: cap on the backward grid (0 = one CTA per SM)
+std::atomic<int> g_fwd_tiles{0};  // test hook: forward query tiles per CTA (0 = chosen, 1, 2)
 std::atomic<unsigned long long> g_launches{0};
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -176,12 +177,12 @@ bool make_map(CUtensorMap* map, const void* base, int BH, int N, int d, int dtyp
 
 unsigned long long wait_ns() { return static_cast<unsigned long long>(g_wait_ms.load()) * 1000000ull; }
 
-template <int D, bool BF16, bool CAUSAL, int REP, bool F8 = false>
+template <int D, bool BF16, bool CAUSAL, int REP, bool F8 = false, bool ONE = false>
 int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                const CUtensorMap& mqr, const fa2::FwdParams& p, int n_split,
                cudaStream_t stream) {
-  using Cfg = fa2::FwdCfg<D, F8>;
-  auto kern = fa2::fa2_fwd_kernel<D, BF16, CAUSAL, REP, F8>;
+  using Cfg = fa2::FwdCfg<D, F8, ONE>;
+  auto kern = fa2::fa2_fwd_kernel<D, BF16, CAUSAL, REP, F8, ONE>;
   // The kernel re-splits its registers between warpgroups; that is only sound
   // when every thread was launched with exactly Cfg::LAUNCH_REGS registers.
   static const bool regs_ok = [&] {
@@ -202,11 +203,23 @@ int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& 
   return FA2_OK;
 }
 
-// Instantiation of the forward for the runtime flags.
+// Instantiation of the forward for the runtime flags (one: one query tile per
+// CTA at D <= 128, plain calls only).
 template <int D>
-int launch_fwd_any(bool bf, bool causal, int rep, const CUtensorMap& mq, const CUtensorMap& mk,
-                   const CUtensorMap& mv, const CUtensorMap& mqr, const fa2::FwdParams& p,
-                   int n_split, cudaStream_t s) {
+int launch_fwd_any(bool bf, bool causal, int rep, bool one, const CUtensorMap& mq,
+                   const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mqr,
+                   const fa2::FwdParams& p, int n_split, cudaStream_t s) {
+  if constexpr (D <= 128) {
+    if (one) {
+      if (rep != 1 || n_split != 1) return FA2_ERR_INVALID_ARG;
+      if (bf) {
+        return causal ? launch_fwd<D, true, true, 1, false, true>(mq, mk, mv, mqr, p, 1, s)
+                      : launch_fwd<D, true, false, 1, false, true>(mq, mk, mv, mqr, p, 1, s);
+      }
+      return causal ? launch_fwd<D, false, true, 1, false, true>(mq, mk, mv, mqr, p, 1, s)
+                    : launch_fwd<D, false, false, 1, false, true>(mq, mk, mv, mqr, p, 1, s);
+    }
+  }
 #define FA2_FWD_REP(BF, CA)                                                        \
   switch (rep) {                                                                   \
     case 4: return launch_fwd<D, BF, CA, 4>(mq, mk, mv, mqr, p, n_split, s);       \
@@ -259,7 +272,8 @@ namespace {
 // kernel merges them into O and LSE.
 int fwd_core(const void* Q, const void* K, const void* V, void* O, float* LSE, int BH, int Nq,
              int Nk, int d, float scale, int causal, int window, int dtype, int n_split,
-             int kv_per_split, int rep, float* O_part, float* LSE_part, fa2_stream_t stream) {
+             int kv_per_split, int rep, float* O_part, float* LSE_part, fa2_stream_t stream,
+             bool one = false) {
   int dev = 0;
   int rc = check_device(&dev);
   if (rc != FA2_OK) return rc;
@@ -277,7 +291,8 @@ int fwd_core(const void* Q, const void* K, const void* V, void* O, float* LSE, i
   }
   const int n_part = n_split * rep;
   // One CTA per (query block, batch*head) in x, one per key stretch in y.
-  const long long n_qblk = (Nq + fwd_rows_per_cta(d) - 1) / fwd_rows_per_cta(d);
+  const int rows_per_cta = one ? 128 : fwd_rows_per_cta(d);
+  const long long n_qblk = (Nq + rows_per_cta - 1) / rows_per_cta;
   if (n_qblk * BH > 0x7fffffffll || n_split > 65535) return FA2_ERR_INVALID_ARG;
 
   fa2::FwdParams p{};
@@ -301,10 +316,10 @@ int fwd_core(const void* Q, const void* K, const void* V, void* O, float* LSE, i
   const bool bf = dtype == FA2_BF16;
   const bool ca = causal != 0;
   switch (fwd_tile_dim(d)) {
-    case 64: rc = launch_fwd_any<64>(bf, ca, rep, mq, mk, mv, mqr, p, n_split, s); break;
-    case 128: rc = launch_fwd_any<128>(bf, ca, rep, mq, mk, mv, mqr, p, n_split, s); break;
-    case 192: rc = launch_fwd_any<192>(bf, ca, rep, mq, mk, mv, mqr, p, n_split, s); break;
-    default: rc = launch_fwd_any<256>(bf, ca, rep, mq, mk, mv, mqr, p, n_split, s); break;
+    case 64: rc = launch_fwd_any<64>(bf, ca, rep, one, mq, mk, mv, mqr, p, n_split, s); break;
+    case 128: rc = launch_fwd_any<128>(bf, ca, rep, one, mq, mk, mv, mqr, p, n_split, s); break;
+    case 192: rc = launch_fwd_any<192>(bf, ca, rep, one, mq, mk, mv, mqr, p, n_split, s); break;
+    default: rc = launch_fwd_any<256>(bf, ca, rep, one, mq, mk, mv, mqr, p, n_split, s); break;
   }
   if (rc != FA2_OK || n_part == 1) return rc;
   const long long rows = static_cast<long long>(BH) * Nq;
@@ -336,8 +351,31 @@ int fwd_impl(const void* Q, const void* K, const void* V, void* O, float* LSE, i
       overlaps(LSE, lse_bytes, Q, bytes) || overlaps(LSE, lse_bytes, K, bytes) ||
       overlaps(LSE, lse_bytes, V, bytes))
     return FA2_ERR_INVALID_ARG;
+  // Work-item granularity: two 128-row query tiles per CTA (ping-pong), or one
+  // (twice the CTAs) when that fills the SMs better.  Causal items shrink with
+  // their position, so one-tile items pack well once the two-tile grid is under
+  // one wave; equal items (not causal, or a sliding window) only gain while the
+  // one-tile grid itself fits in one wave.  Measured on B200 (two -> one tile):
+  // causal 1 x 16 x 2048, d = 64: 37.4 -> 29.1 us, d = 128: 43.2 -> 31.2 us;
+  // not causal 1 x 32 x 1024, d = 64: 23.0 -> 29.1 us (so kept at two).
+  bool one = false;
+  if (fwd_tile_dim(d) <= 128) {
+    const int mode = g_fwd_tiles.load();
+    if (mode == 0) {
+      int dev = 0, n_sm = 0;
+      if (cudaGetDevice(&dev) != cudaSuccess ||
+          cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+        cudaGetLastError();
+        return FA2_ERR_CUDA;
+      }
+      const long long two = static_cast<long long>((N + 255) / 256) * BH;
+      one = (causal && window == 0) ? two < n_sm : 2 * two <= n_sm;
+    } else {
+      one = mode == 1;
+    }
+  }
   return fwd_core(Q, K, V, O, LSE, BH, N, N, d, scale, causal, window, dtype, 1, 0, 1, nullptr,
-                  nullptr, stream);
+                  nullptr, stream, one);
 }
 
 // Key tiles per split when the n_kv key tiles are cut into n_split stretches,
@@ -703,6 +741,8 @@ void fa2_debug_set(int fault, unsigned int wait_limit_ms) {
 }
 
 void fa2_debug_set_bwd_grid(int max_ctas) { g_bwd_ctas.store(max_ctas > 0 ? max_ctas : 0); }
+
+void fa2_debug_set_fwd_tiles(int tiles) { g_fwd_tiles.store(tiles == 1 || tiles == 2 ? tiles : 0); }
 
 unsigned long long fa2_launch_count(void) { return g_launches.load(); }
 

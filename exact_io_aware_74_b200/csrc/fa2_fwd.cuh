@@ -82,7 +82,7 @@ struct FwdParams {
   float* LSE_part;
 };
 
-template <int D, bool F8 = false>
+template <int D, bool F8 = false, bool ONE = false>
 struct FwdCfg {
   static_assert(D == 64 || D == 128 || D == 192 || D == 256, "tile head dims");
   static_assert(!F8 || D == 128, "8-bit inputs use 128-byte tiles");
@@ -93,8 +93,10 @@ struct FwdCfg {
   static constexpr int BN = 128;                  // keys per tile
   // Query tiles per CTA: two (ping-pong) up to D = 128; one above, where two
   // D-column output accumulators and two S blocks would exceed TMEM's 512
-  // columns (S double buffer 256 + O D <= 512 still fits).
-  static constexpr int QT = (D <= 128) ? 2 : 1;
+  // columns (S double buffer 256 + O D <= 512 still fits).  ONE asks for one
+  // query tile at D <= 128 too: twice the CTAs, for grids that would otherwise
+  // leave SMs idle.
+  static constexpr int QT = (D <= 128 && !ONE) ? 2 : 1;
   static constexpr int KCH = D * ESZ / 128;       // 128-byte swizzle chunks along d
   static constexpr int CHUNK = 128 * 128;         // bytes of one 128-row x 128-byte chunk
   static constexpr int TILE = 128 * D * ESZ;      // bytes of one 128-row tile
@@ -153,13 +155,13 @@ enum FwdSite : uint32_t {
 // through tmQr (boxes of 128 / REP rows), and copy c scores only key columns
 // [c 128 / REP, (c + 1) 128 / REP) of every key tile, as partial result
 // blockIdx.y * REP + c: a lone query keeps four softmax warps busy, not one.
-template <int D, bool BF16, bool CAUSAL, int REP, bool F8 = false>
+template <int D, bool BF16, bool CAUSAL, int REP, bool F8 = false, bool ONE = false>
 __global__ void __launch_bounds__(384, 1)
 fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmQr,
                const FwdParams p) {
   static_assert(!F8 || (BF16 && REP == 1), "8-bit inputs: bf16 output, no query copies");
-  using C = FwdCfg<D, F8>;
+  using C = FwdCfg<D, F8, ONE>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));

@@ -30,7 +30,7 @@ FA2_BF16 = 1
 EXPORTS = ("fa2_fwd", "fa2_fwd_window", "fa2_fwd_fp8", "fa2_fwd_decode_splits", "fa2_fwd_decode_workspace_size",
            "fa2_fwd_decode", "fa2_bwd_workspace_size", "fa2_bwd", "fa2_bwd_window",
            "fa2_bwd_noalloc", "fa2_get_device_status", "fa2_status_string", "fa2_debug_set",
-           "fa2_debug_set_bwd_grid", "fa2_launch_count")
+           "fa2_debug_set_bwd_grid", "fa2_debug_set_fwd_tiles", "fa2_launch_count")
 
 _lib = None
 
@@ -79,6 +79,8 @@ def load() -> ctypes.CDLL:
     lib.fa2_debug_set.restype = None
     lib.fa2_debug_set_bwd_grid.argtypes = [i]
     lib.fa2_debug_set_bwd_grid.restype = None
+    lib.fa2_debug_set_fwd_tiles.argtypes = [i]
+    lib.fa2_debug_set_fwd_tiles.restype = None
     lib.fa2_launch_count.argtypes = []
     lib.fa2_launch_count.restype = ctypes.c_ulonglong
     _lib = lib
@@ -219,6 +221,11 @@ def fa2_debug_set(fault: int, wait_limit_ms: int = 0) -> None:
 def fa2_debug_set_bwd_grid(max_ctas: int) -> None:
     """Test hook: cap the backward's persistent grid (0 = one CTA per SM)."""
     load().fa2_debug_set_bwd_grid(int(max_ctas))
+
+
+def fa2_debug_set_fwd_tiles(tiles: int) -> None:
+    """Test hook: force 1 or 2 query tiles per forward CTA (0 = the library's choice)."""
+    load().fa2_debug_set_fwd_tiles(int(tiles))
 
 
 def fa2_launch_count() -> int:

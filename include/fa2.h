@@ -261,6 +261,15 @@ void fa2_debug_set(int fault, unsigned int wait_limit_ms);
  */
 void fa2_debug_set_bwd_grid(int max_ctas);
 
+/*
+ * Test hook.  Query tiles (128 rows) per forward CTA for fa2_fwd and
+ * fa2_fwd_window at head dims up to 128: 1 or 2 forces that many; 0, the default,
+ * restores the library's choice (two, unless one fills the SMs better: causal
+ * calls whose two-tile grid is under one wave, other calls whose one-tile grid
+ * fits in one wave).  Results do not depend on it.  Not for production use.
+ */
+void fa2_debug_set_fwd_tiles(int tiles);
+
 /* Number of kernels this library has launched in this process (all devices). */
 unsigned long long fa2_launch_count(void);
 
