@@ -80,6 +80,22 @@ int fwd_tile_dim(int d) { return d <= 64 ? 64 : (d <= 128 ? 128 : (d <= 192 ? 19
 // Query rows per forward CTA: two 128-row tiles up to a tile width of 128, one above.
 int fwd_rows_per_cta(int d) { return fwd_tile_dim(d) <= 128 ? 256 : 128; }
 
+// Query tiles per CTA of a plain (or sliding-window) forward on sm_count SMs:
+// two 128-row tiles (ping-pong), or one (twice the CTAs) when that fills the SMs
+// better.  Causal items shrink with their position, so one-tile items pack well
+// once the two-tile grid is under one wave; equal items (not causal, or a sliding
+// window) only gain while the one-tile grid itself fits in one wave.  Measured on
+// B200 (two -> one tile): causal 1 x 16 x 2048, d = 64: 37.4 -> 29.1 us, d = 128:
+// 43.2 -> 31.2 us; not causal 1 x 32 x 1024, d = 64: 23.0 -> 29.1 us (kept at two).
+int fwd_tiles_per_cta(long long BH, int N, int d, bool causal, int window, int sm_count) {
+  if (fwd_tile_dim(d) > 128) return 1;
+  const int mode = g_fwd_tiles.load();
+  if (mode != 0) return mode;
+  const long long two = static_cast<long long>((N + 255) / 256) * BH;
+  const bool one = (causal && window == 0) ? two < sm_count : 2 * two <= sm_count;
+  return one ? 1 : 2;
+}
+
 // Current device must be compute capability 10.0; returns its ordinal in *dev.
 int check_device(int* dev) {
   if (cudaGetDevice(dev) != cudaSuccess) {
@@ -351,29 +367,13 @@ int fwd_impl(const void* Q, const void* K, const void* V, void* O, float* LSE, i
       overlaps(LSE, lse_bytes, Q, bytes) || overlaps(LSE, lse_bytes, K, bytes) ||
       overlaps(LSE, lse_bytes, V, bytes))
     return FA2_ERR_INVALID_ARG;
-  // Work-item granularity: two 128-row query tiles per CTA (ping-pong), or one
-  // (twice the CTAs) when that fills the SMs better.  Causal items shrink with
-  // their position, so one-tile items pack well once the two-tile grid is under
-  // one wave; equal items (not causal, or a sliding window) only gain while the
-  // one-tile grid itself fits in one wave.  Measured on B200 (two -> one tile):
-  // causal 1 x 16 x 2048, d = 64: 37.4 -> 29.1 us, d = 128: 43.2 -> 31.2 us;
-  // not causal 1 x 32 x 1024, d = 64: 23.0 -> 29.1 us (so kept at two).
-  bool one = false;
-  if (fwd_tile_dim(d) <= 128) {
-    const int mode = g_fwd_tiles.load();
-    if (mode == 0) {
-      int dev = 0, n_sm = 0;
-      if (cudaGetDevice(&dev) != cudaSuccess ||
-          cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
-        cudaGetLastError();
-        return FA2_ERR_CUDA;
-      }
-      const long long two = static_cast<long long>((N + 255) / 256) * BH;
-      one = (causal && window == 0) ? two < n_sm : 2 * two <= n_sm;
-    } else {
-      one = mode == 1;
-    }
+  int dev = 0, n_sm = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+    cudaGetLastError();
+    return FA2_ERR_CUDA;
   }
+  const bool one = fwd_tile_dim(d) <= 128 && fwd_tiles_per_cta(BH, N, d, causal != 0, window, n_sm) == 1;
   return fwd_core(Q, K, V, O, LSE, BH, N, N, d, scale, causal, window, dtype, 1, 0, 1, nullptr,
                   nullptr, stream, one);
 }
@@ -412,6 +412,22 @@ int fa2_fwd_window(const void* Q, const void* K, const void* V, void* O, float* 
   // A window as long as the sequence is plain causal attention.
   return fwd_impl(Q, K, V, O, LSE, B, H, N, d, scale, 1, window >= N ? 0 : window, dtype,
                   stream);
+}
+
+int fa2_fwd_tiles_per_cta(int B, int H, int N, int d, int causal, int window, int sm_count) {
+  if (check_sizes(B, H, N, d, 1.0f, causal, FA2_BF16) != FA2_OK || window < 0) return 0;
+  if (sm_count <= 0) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sm_count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        sm_count <= 0) {
+      cudaGetLastError();
+      return 0;
+    }
+  }
+  // fa2_fwd_window treats a window as long as the sequence as plain causal.
+  const int w = (causal && window > 0 && window < N) ? window : 0;
+  return fwd_tiles_per_cta(static_cast<long long>(B) * H, N, d, causal != 0, w, sm_count);
 }
 
 int fa2_fwd_decode_splits(int B, int H, int Nq, int Nk, int d, int sm_count) {

@@ -667,6 +667,17 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         if (!ok) break;
         tmem_wait_st();
         tc_fence_before();
+        // One tile per CTA: S of the last step was issued before the P V product
+        // of the step before it (phase my_nkv - 2), which may still be pending.
+        // Wait for it here, before this warp hands over the last P: no later
+        // product can complete until then, so the barrier is at most one phase
+        // behind now and at the final wait below.  (Waiting after the hand-over
+        // could find both products complete, two phases on, where a parity wait
+        // no longer tells them apart.)
+        if (single && step == my_nkv - 1 && step >= 1) {
+          ok = __all_sync(0xffffffffu, mbar_wait(&o_done[t], (step - 1) & 1, wc, kSiteSoftOEnd));
+          if (!ok) break;
+        }
       } else if (sep) {
         // Keep the barrier counts: S read; and, like the live warps (which wait
         // for the previous P V product before writing P), arrive for this step's
@@ -682,12 +693,8 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       if (lane == 0) mbar_arrive(&p_ready[buf]);
     }
     // Wait for the last P V product.  A phase-parity wait is only sound while the
-    // barrier is at most one phase behind.  With one tile per CTA, S of the last
-    // step is issued before P V of the step before it, so that product (phase
-    // my_nkv - 2) may still be pending: wait for it first.  (Every earlier one
-    // finished before S of the last step, which this warp has seen.)
-    if (ok && live && single && my_nkv >= 2)
-      ok = __all_sync(0xffffffffu, mbar_wait(&o_done[t], (my_nkv - 2) & 1, wc, kSiteSoftOEnd));
+    // barrier is at most one phase behind: every earlier product has been seen
+    // complete (with one tile per CTA, the one before it inside the last step).
     if (ok && live)
       ok = __all_sync(0xffffffffu, mbar_wait(&o_done[t], (my_nkv - 1) & 1, wc, kSiteSoftOEnd));
     if (ok && live) {

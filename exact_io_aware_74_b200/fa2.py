@@ -27,8 +27,8 @@ FA2_FP16 = 0
 FA2_BF16 = 1
 
 # Every symbol include/fa2.h declares.
-EXPORTS = ("fa2_fwd", "fa2_fwd_window", "fa2_fwd_fp8", "fa2_fwd_decode_splits", "fa2_fwd_decode_workspace_size",
-           "fa2_fwd_decode", "fa2_bwd_workspace_size", "fa2_bwd", "fa2_bwd_window",
+EXPORTS = ("fa2_fwd", "fa2_fwd_window", "fa2_fwd_fp8", "fa2_fwd_tiles_per_cta",
+           "fa2_fwd_decode_splits", "fa2_fwd_decode_workspace_size", "fa2_fwd_decode", "fa2_bwd_workspace_size", "fa2_bwd", "fa2_bwd_window",
            "fa2_bwd_noalloc", "fa2_get_device_status", "fa2_status_string", "fa2_debug_set",
            "fa2_debug_set_bwd_grid", "fa2_debug_set_fwd_tiles", "fa2_launch_count")
 
@@ -57,6 +57,8 @@ def load() -> ctypes.CDLL:
     lib.fa2_fwd_window.restype = i
     lib.fa2_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, f, f, f, vp]
     lib.fa2_fwd_fp8.restype = i
+    lib.fa2_fwd_tiles_per_cta.argtypes = [i, i, i, i, i, i, i]
+    lib.fa2_fwd_tiles_per_cta.restype = i
     lib.fa2_fwd_decode_splits.argtypes = [i, i, i, i, i, i]
     lib.fa2_fwd_decode_splits.restype = i
     lib.fa2_fwd_decode_workspace_size.argtypes = [i, i, i, i, i, i]
@@ -144,6 +146,13 @@ def fa2_fwd_fp8(q, k, v, o, lse, scale: float, causal: bool, q_scale: float, k_s
     return load().fa2_fwd_fp8(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d,
                               float(scale), int(bool(causal)), float(q_scale), float(k_scale),
                               float(v_scale), _stream(stream))
+
+
+def fa2_fwd_tiles_per_cta(B: int, H: int, N: int, d: int, causal: bool, window: int = 0,
+                          sm_count: int = 0) -> int:
+    """Query tiles per CTA the forward uses for these sizes (1 or 2; 0 if rejected)."""
+    return load().fa2_fwd_tiles_per_cta(int(B), int(H), int(N), int(d), int(bool(causal)),
+                                        int(window), int(sm_count))
 
 
 def fa2_fwd_decode_splits(B: int, H: int, Nq: int, Nk: int, d: int, sm_count: int = 0) -> int:

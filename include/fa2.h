@@ -130,6 +130,18 @@ int fa2_fwd_decode(const void* Q, const void* K, const void* V, void* O, float* 
                    void* workspace, size_t workspace_bytes, fa2_stream_t stream);
 
 /*
+ * Query tiles (128 rows) per CTA that fa2_fwd (window = 0) or fa2_fwd_window
+ * uses for these sizes on a GPU with ``sm_count`` SMs (<= 0: the current
+ * device's count): 2 (the softmax of one tile overlaps the other's products), or
+ * 1 (twice the CTAs) for a causal call without a window whose two-tile grid,
+ * ceil(N / 256) x B x H CTAs, is under one wave, or any other call whose one-tile
+ * grid fits in one wave; always 1 for head dims above 128.  The test hook
+ * fa2_debug_set_fwd_tiles overrides it.  Returns 0 for sizes fa2_fwd rejects, or
+ * when sm_count <= 0 and no device can be queried.  Results do not depend on it.
+ */
+int fa2_fwd_tiles_per_cta(int B, int H, int N, int d, int causal, int window, int sm_count);
+
+/*
  * The split count fa2_fwd_decode would best use for these sizes on a GPU with
  * ``sm_count`` SMs (<= 0: the current device's count): as many as keep all CTAs
  * in one wave (one CTA per SM, ceil(Nq / 256) x B x H CTAs per split), but no

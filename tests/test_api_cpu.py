@@ -252,3 +252,35 @@ def test_fp8_validation_without_device(lib):
     if not torch.cuda.is_available():
         for d in (16, 64, 128):
             assert call(d=d) in (fa2.FA2_ERR_CUDA, fa2.FA2_ERR_ARCH)
+
+
+@pytest.mark.parametrize("shape,causal,window,expect", [
+    # causal, two-tile grid under one wave (16 heads x 8 blocks = 128 CTAs): one tile
+    ((1, 16, 2048, 64), True, 0, 1),
+    ((1, 8, 4096, 128), True, 0, 1),
+    # the bench workload (4 x 16 x 4 = 256 two-tile CTAs): two
+    ((4, 16, 1024, 64), True, 0, 2),
+    # not causal: 128 equal two-tile CTAs; one tile would need 256 > 148: two
+    ((1, 32, 1024, 64), False, 0, 2),
+    # not causal, the one-tile grid fits in one wave (2 x 4 x ... = 16 / 64 CTAs): one
+    ((1, 2, 1024, 64), False, 0, 1),
+    ((1, 4, 2048, 128), False, 0, 1),
+    # a sliding window makes the items equal: the one-wave rule for one tile
+    ((1, 16, 2048, 64), True, 512, 2),
+    ((1, 4, 2048, 64), True, 512, 1),
+    # a window as long as the sequence is plain causal
+    ((1, 16, 2048, 64), True, 4096, 1),
+    # head dims above 128 always run one tile per CTA
+    ((8, 16, 4096, 256), True, 0, 1),
+    # the headline shape fills the GPU many times over
+    ((2, 32, 8192, 128), False, 0, 2),
+])
+def test_forward_tiles_per_cta_choice(lib, shape, causal, window, expect):
+    assert fa2.fa2_fwd_tiles_per_cta(*shape, causal, window, 148) == expect
+
+
+def test_forward_tiles_per_cta_rejects_bad_sizes(lib):
+    assert fa2.fa2_fwd_tiles_per_cta(1, 2, 128, 60, True, 0, 148) == 0   # d not a multiple of 8
+    assert fa2.fa2_fwd_tiles_per_cta(0, 2, 128, 64, True, 0, 148) == 0   # B < 1
+    assert fa2.fa2_fwd_tiles_per_cta(1, 2, 128, 64, True, -1, 148) == 0  # negative window
+    assert fa2.fa2_fwd_tiles_per_cta(1, 2, 128, 64, True, 0, 0) == 0     # no device to ask
