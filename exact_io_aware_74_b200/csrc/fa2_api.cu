@@ -647,7 +647,7 @@ int fa2_bwd_window(const void* Q, const void* K, const void* V, const void* O, c
 namespace {
 
 constexpr size_t kNoAllocBytes = static_cast<size_t>(32) << 20;  // 32 MiB
-constexpr size_t kNoAllocStatusBytes = 256;  // status word used when none exists yet
+constexpr size_t kNoAllocStatusBytes = 256;  // the buffer's own status word, then the scratch
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocBytes];
 
@@ -669,9 +669,11 @@ void* noalloc_base(int dev) {
   return g_noalloc_base[dev];
 }
 
-unsigned int* existing_status_word(int dev) {
+// The status word in the buffer (its first 256 bytes), or null before the first
+// fa2_bwd_noalloc call on the device.
+unsigned int* noalloc_status_word(int dev) {
   std::lock_guard<std::mutex> lock(g_mu);
-  return g_status[dev];
+  return static_cast<unsigned int*>(g_noalloc_base[dev]);
 }
 
 }  // namespace
@@ -707,10 +709,9 @@ int fa2_bwd_noalloc(const void* Q, const void* K, const void* V, const void* O, 
   if (rc != FA2_OK) return rc;
   uint8_t* base = static_cast<uint8_t*>(noalloc_base(dev));  // first call on a device: set-up
   if (!base) return FA2_ERR_CUDA;
-  // Timeouts go to the library's status word when it exists (so that
-  // fa2_get_device_status reports them); otherwise to a word in the buffer.
-  unsigned int* st = existing_status_word(dev);
-  if (!st) st = reinterpret_cast<unsigned int*>(base);
+  // Timeouts go to the word at the start of the buffer, which
+  // fa2_get_device_status reads and clears along with the library's own word.
+  unsigned int* st = reinterpret_cast<unsigned int*>(base);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   rc = fa2::launch_bwd(Q, K, V, O, dO, LSE, dQ, dK, dV, base + kNoAllocStatusBytes, BH, N, d,
                        scale, causal != 0, dtype == FA2_BF16, st, wait_ns(), s, 0, g_fault.load(),
@@ -728,13 +729,27 @@ int fa2_get_device_status(fa2_stream_t stream, int* site) {
   }
   if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
     return FA2_ERR_CUDA;
-  unsigned int* st = status_word(dev);
-  if (!st) return FA2_ERR_CUDA;
-  unsigned int w = 0;
-  if (cudaMemcpy(&w, st, sizeof(w), cudaMemcpyDeviceToHost) != cudaSuccess) return FA2_ERR_CUDA;
-  if (w != 0 && cudaMemset(st, 0, sizeof(w)) != cudaSuccess) return FA2_ERR_CUDA;
-  if (site) *site = static_cast<int>((w >> 8) & 0xFFu);
-  const unsigned int code = w & 0xFFu;
+  // Two words may exist: the one the calls with caller-provided memory write (created
+  // by the first of them) and the one in fa2_bwd_noalloc's buffer.  Both are read and
+  // cleared; nothing is allocated here, so a word that does not exist yet has had no
+  // kernel to write it.  The first failure recorded (the library's word first) is
+  // the one returned.
+  unsigned int* words[2] = {nullptr, nullptr};
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    words[0] = g_status[dev];
+  }
+  words[1] = noalloc_status_word(dev);
+  unsigned int first = 0;
+  for (unsigned int* st : words) {
+    if (!st) continue;
+    unsigned int w = 0;
+    if (cudaMemcpy(&w, st, sizeof(w), cudaMemcpyDeviceToHost) != cudaSuccess) return FA2_ERR_CUDA;
+    if (w != 0 && cudaMemset(st, 0, sizeof(w)) != cudaSuccess) return FA2_ERR_CUDA;
+    if (first == 0) first = w;
+  }
+  if (site) *site = static_cast<int>((first >> 8) & 0xFFu);
+  const unsigned int code = first & 0xFFu;
   return code == 0 ? FA2_OK : static_cast<int>(code);
 }
 

@@ -236,9 +236,10 @@ int fa2_bwd_window(const void* Q, const void* K, const void* V, const void* O, c
  *     by the call itself).  Calls that overlap on the GPU -- on different
  *     streams, or from several host threads -- race on the buffer and give
  *     wrong results: serialise them.
- *   - In-kernel wait timeouts are reported by fa2_get_device_status() once any
- *     fa2_fwd / fa2_bwd call has run on the device; before that they are not
- *     observable.
+ *   - In-kernel wait timeouts go to a status word in the first 256 bytes of the
+ *     buffer; fa2_get_device_status() reads and clears it with the library's
+ *     own word and allocates nothing, so a caller that only ever uses this entry
+ *     point sees its timeouts there too.
  */
 int fa2_bwd_noalloc(const void* Q, const void* K, const void* V, const void* O, const void* dO,
                     const float* LSE, void* dQ, void* dK, void* dV, int B, int H, int N, int d,
@@ -246,10 +247,13 @@ int fa2_bwd_noalloc(const void* Q, const void* K, const void* V, const void* O, 
 
 /*
  * Synchronises ``stream``, then returns and clears the current device's status
- * word: FA2_OK, or FA2_ERR_TIMEOUT if a kernel gave up a bounded wait since the
+ * words (the library's, and fa2_bwd_noalloc's if that call has run on the
+ * device): FA2_OK, or FA2_ERR_TIMEOUT if a kernel gave up a bounded wait since the
  * last call (the kernel then skipped its output and exited cleanly; the CUDA
  * context stays usable).  FA2_ERR_CUDA if the synchronisation itself failed.
  * If ``site`` is not NULL it receives the id of the wait that ran out (0 if none).
+ * Allocates nothing.  (``site`` is one argument more than a bare status query
+ * needs; it tells which wait of which kernel ran out.)
  */
 int fa2_get_device_status(fa2_stream_t stream, int* site);
 

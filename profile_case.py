@@ -1,8 +1,8 @@
 """Runs fa2_fwd (and fa2_bwd), or fa2_fwd_decode, a few times on one shape, for profilers.
 
-    python -m exact_io_aware_74_b200.profile_case B H N d causal [reps] [--fwd-only]
-    python -m exact_io_aware_74_b200.profile_case --decode B H Nq Nk d causal [reps] [splits]
-    python -m exact_io_aware_74_b200.profile_case --fp8 B H N d causal [reps]
+    python profile_case.py B H N d causal [reps] [--fwd-only]
+    python profile_case.py --decode B H Nq Nk d causal [reps] [splits]
+    python profile_case.py --fp8 B H N d causal [reps]
 
 Seeded N(0, 1) bf16 inputs; exits non-zero if a call or the device status fails.
 Used to capture Nsight Compute profiles of one kernel on a small case.  With
@@ -12,7 +12,10 @@ Used to capture Nsight Compute profiles of one kernel on a small case.  With
 from __future__ import annotations
 
 import math
+import os
 import sys
+
+sys.path.insert(0, os.path.dirname(os.path.abspath(__file__)))
 
 import torch
 

@@ -284,3 +284,25 @@ def test_forward_tiles_per_cta_rejects_bad_sizes(lib):
     assert fa2.fa2_fwd_tiles_per_cta(0, 2, 128, 64, True, 0, 148) == 0   # B < 1
     assert fa2.fa2_fwd_tiles_per_cta(1, 2, 128, 64, True, -1, 148) == 0  # negative window
     assert fa2.fa2_fwd_tiles_per_cta(1, 2, 128, 64, True, 0, 0) == 0     # no device to ask
+
+
+# ------------------------------------------------------------------ memory linear in N
+#
+# "FlashAttention-2" (systems-analysis.info wiki), "Предпосылки": the tiled method
+# needs memory linear in the sequence length, because no N x N matrix is stored.
+# The forward takes no scratch at all; the backward's scratch is two float rows per
+# query (D and LSE * log2 e, padded to 128 rows) and a float dQ accumulator of one
+# row per query, as wide as the kernel's tile (64 or 128 columns).
+
+@pytest.mark.parametrize("d", [32, 64, 96, 128])
+def test_bwd_workspace_is_linear_in_sequence_length(lib, d):
+    B, H = 2, 3
+    tile = 64 if d <= 64 else 128
+    for N in (128, 1024, 4096, 32768):
+        ws = lib.fa2_bwd_workspace_size(B, H, N, d)
+        rows = B * H * ((N + 127) // 128 * 128)
+        expect = (2 * rows * 4 + 255) // 256 * 256 + (B * H * N * tile * 4 + 255) // 256 * 256
+        assert ws == expect
+        # O(B H N d): at most 8 bytes per head element plus the row statistics
+        assert ws <= B * H * N * (8 * d) + 2 * rows * 4 + 512
+        assert lib.fa2_bwd_workspace_size(B, H, 2 * N, d) == 2 * ws  # doubles with N

@@ -18,8 +18,12 @@ from exact_io_aware_74_b200.workloads import WORKLOADS  # noqa: E402
 
 def test_step_flops_and_default_workload():
     w = WORKLOADS[bench.DEFAULT_WORKLOAD]
-    assert w.backward and w.dtype == "bf16"
-    assert bench.step_flops(w) == pytest.approx(3.5 * 4 * 4 * 16 * 1024 * 1024 * 64 / 2)
+    # the largest forward + backward workload: B=8, H=16, N=4096, d=128, causal
+    assert w.backward and w.dtype == "bf16" and w.causal
+    assert (w.B, w.H, w.N, w.d) == (8, 16, 4096, 128)
+    assert bench.step_flops(w) == pytest.approx(3.5 * 4 * 8 * 16 * 4096 * 4096 * 128 / 2)
+    # its inputs are larger than L2, so no flush buffer is written between steps
+    assert bench.input_bytes(w) * 2 >= 2 * bench.L2_BYTES
     assert bench.HEADLINE_WORKLOAD == "fwd_bf16_b2h32_n8192_d128"
 
 

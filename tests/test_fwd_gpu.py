@@ -64,35 +64,6 @@ def test_fwd_workload_full(name):
     _compare_full(x, w.scale, w.causal, w.dtype)
 
 
-def _sample_rows(N, rng, n=40):
-    fixed = [0, 1, 127, 128, 255, 256, N // 2, N - 129, N - 128, N - 2, N - 1]
-    rows = set(r for r in fixed if 0 <= r < N)
-    rows.update(rng.integers(0, N, size=n).tolist())
-    return sorted(rows)
-
-
-@pytest.mark.slow
-@pytest.mark.parametrize("name", ["fwd_bf16_b2h32_n8192_d128",
-                                  "fwdbwd_bf16_b8h16_n4096_d128_causal",
-                                  "fwd_bf16_b1h32_n32768_d128_causal_outliers"])
-def test_fwd_workload_sampled(name):
-    """Full-size launch as the bench times it; sampled rows checked against the oracle."""
-    w = WORKLOADS[name]
-    x = workload_inputs(w, with_do=False)
-    o, lse = _run(x["q"], x["k"], x["v"], w.scale, w.causal)
-    assert torch.isfinite(o.float()).all() and torch.isfinite(lse).all()
-    rng = np.random.default_rng(w.seed)
-    BH = w.B * w.H
-    for bh in sorted({0, BH - 1, int(rng.integers(0, BH))}):
-        rows = _sample_rows(w.N, rng)
-        ro, rl = oracle.attn_fwd_rows_ref(x["q"], x["k"], x["v"], w.scale, w.causal, bh, rows)
-        b, h = divmod(bh, w.H)
-        go = o[b, h, rows].double().numpy()
-        gl = lse[b, h, rows].double().numpy()
-        assert np.max(np.abs(go - ro)) <= O_TOL[w.dtype]
-        assert np.max(np.abs(gl - rl)) <= LSE_TOL
-
-
 # ------------------------------------------------------------------ invariants on the GPU
 
 def test_fwd_constant_v_and_causal_row0():
