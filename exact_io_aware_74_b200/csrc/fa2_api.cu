@@ -570,11 +570,12 @@ size_t fa2_bwd_workspace_size(int B, int H, int N, int d) {
 
 namespace {
 
-// Shared by fa2_bwd and fa2_bwd_window; window = 0 means no sliding window.
+// Shared by fa2_bwd, fa2_bwd_window and fa2_bwd_ex; window = 0 means no sliding
+// window.
 int bwd_impl(const void* Q, const void* K, const void* V, const void* O, const void* dO,
              const float* LSE, void* dQ, void* dK, void* dV, void* workspace,
              size_t workspace_bytes, int B, int H, int N, int d, float scale, int causal,
-             int window, int dtype, fa2_stream_t stream) {
+             int window, int dtype, fa2_stream_t stream, bool deterministic = false) {
   if (!Q || !K || !V || !O || !dO || !LSE || !dQ || !dK || !dV) return FA2_ERR_INVALID_ARG;
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(dO) ||
       !aligned16(LSE) || !aligned16(dQ) || !aligned16(dK) || !aligned16(dV))
@@ -594,7 +595,7 @@ int bwd_impl(const void* Q, const void* K, const void* V, const void* O, const v
   if (overlaps(dQ, bytes, dK, bytes) || overlaps(dQ, bytes, dV, bytes) ||
       overlaps(dK, bytes, dV, bytes))
     return FA2_ERR_INVALID_ARG;
-  const size_t need = fa2::bwd_workspace_bytes(static_cast<size_t>(BH), N, d);
+  const size_t need = fa2::bwd_workspace_bytes(static_cast<size_t>(BH), N, d, deterministic);
   if (!workspace || workspace_bytes < need ||
       (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
     return FA2_ERR_WORKSPACE;
@@ -606,8 +607,8 @@ int bwd_impl(const void* Q, const void* K, const void* V, const void* O, const v
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   rc = fa2::launch_bwd(Q, K, V, O, dO, LSE, dQ, dK, dV, workspace, BH, N, d, scale, causal != 0,
                        dtype == FA2_BF16, st, wait_ns(), s, window, g_fault.load(),
-                       g_bwd_ctas.load());
-  if (rc == FA2_OK) g_launches.fetch_add(fa2::kBwdKernelsPerCall);
+                       g_bwd_ctas.load(), deterministic);
+  if (rc == FA2_OK) g_launches.fetch_add(fa2::bwd_kernels_per_call(deterministic));
   return rc;
 }
 
@@ -630,6 +631,25 @@ int fa2_bwd_window(const void* Q, const void* K, const void* V, const void* O, c
   if (window < 1) return FA2_ERR_INVALID_ARG;
   return bwd_impl(Q, K, V, O, dO, LSE, dQ, dK, dV, workspace, workspace_bytes, B, H, N, d, scale,
                   1, window >= N ? 0 : window, dtype, stream);
+}
+
+size_t fa2_bwd_ex_workspace_size(int B, int H, int N, int d, int flags) {
+  if ((flags & ~FA2_BWD_DETERMINISTIC) != 0) return 0;
+  if (check_sizes(B, H, N, d, 1.0f, 0, FA2_BF16, kMaxBwdHeadDim) != FA2_OK) return 0;
+  return fa2::bwd_workspace_bytes(static_cast<size_t>(B) * H, N, d,
+                                  (flags & FA2_BWD_DETERMINISTIC) != 0);
+}
+
+int fa2_bwd_ex(const void* Q, const void* K, const void* V, const void* O, const void* dO,
+               const float* LSE, void* dQ, void* dK, void* dV, void* workspace,
+               size_t workspace_bytes, int B, int H, int N, int d, float scale, int causal,
+               int window, int flags, int dtype, fa2_stream_t stream) {
+  if ((flags & ~FA2_BWD_DETERMINISTIC) != 0) return FA2_ERR_INVALID_ARG;
+  if (window < 0 || (window > 0 && causal != 1)) return FA2_ERR_INVALID_ARG;
+  // A window as long as the sequence is plain causal attention.
+  const int w = (window > 0 && window < N) ? window : 0;
+  return bwd_impl(Q, K, V, O, dO, LSE, dQ, dK, dV, workspace, workspace_bytes, B, H, N, d, scale,
+                  causal, w, dtype, stream, (flags & FA2_BWD_DETERMINISTIC) != 0);
 }
 
 }  // extern "C"
@@ -716,7 +736,7 @@ int fa2_bwd_noalloc(const void* Q, const void* K, const void* V, const void* O, 
   rc = fa2::launch_bwd(Q, K, V, O, dO, LSE, dQ, dK, dV, base + kNoAllocStatusBytes, BH, N, d,
                        scale, causal != 0, dtype == FA2_BF16, st, wait_ns(), s, 0, g_fault.load(),
                        g_bwd_ctas.load());
-  if (rc == FA2_OK) g_launches.fetch_add(fa2::kBwdKernelsPerCall);
+  if (rc == FA2_OK) g_launches.fetch_add(fa2::bwd_kernels_per_call(false));
   return rc;
 }
 

@@ -8,45 +8,51 @@
 //   dV = P^T dO,  dP = dO V^T,  D_i = sum_c dO_ic O_ic,
 //   dS = P * (dP - D),  dQ = scale dS K,  dK = scale dS^T Q.
 //
-// Three kernels per call, all on the caller's stream, chained by programmatic
-// dependent launch (each reads nothing before its griddepcontrol.wait):
+// Kernels per call, all on the caller's stream, chained by programmatic dependent
+// launch (each reads nothing before its griddepcontrol.wait):
+//   tile width 64 (d <= 64):
 //   1. fa2_bwd_pre_kernel  : D and LSE * log2(e) per query row (padded to a
 //                            multiple of 128 rows), and a zeroed fp32 dQ
 //                            accumulator;
 //   2. fa2_bwd_kernel      : persistent, at most one CTA per SM.  The key tiles
 //                            (128 keys, batch*head) are listed heaviest first and
 //                            dealt to the CTAs in snake order; each tile loops
-//                            over the query tiles that see its keys;
-//   3. fa2_bwd_dq_kernel   : dQ = scale * accumulator, rounded to 16 bits.
+//                            over the query tiles that see its keys, and adds its
+//                            dQ partials into the accumulator;
+//   3. fa2_bwd_dq_finalise_kernel : dQ = scale * accumulator, rounded to 16 bits.
+//   tile width 128 (64 < d <= 128), where a per-step dQ product no longer fits in
+//   TMEM beside dV and dK:
+//   1. fa2_bwd_dq_kernel (fa2_bwd_dq.cuh): dQ, query-stationary, summed in TMEM;
+//                            it also writes the D and LSE * log2(e) rows;
+//   2. fa2_bwd_kernel      : as above, dK and dV only.
 //
 // Main kernel, CTA layout (320 threads):
 //   warps 0-7 two compute warpgroups g = 0, 1.  Thread r of warpgroup g owns key
 //             row r of the tile for the query columns 64 g .. 64 g + 63 of P^T
-//             and dS^T, and query row r of the current query tile for the head
-//             columns g D/2 .. (g+1) D/2 - 1 when it moves the dQ partial from
-//             TMEM through shared memory into the fp32 accumulator (one TMA
-//             reduce-add per 128 x 32 tile).  Splitting every row between the
-//             two warpgroups halves the per-step chain P^T -> dS^T -> dQ drain
-//             that the products wait on;
+//             and dS^T, and (tile width 64) query row r of the current query tile
+//             for the head columns 32 g .. 32 g + 31 when it moves the dQ partial
+//             from TMEM through shared memory into the fp32 accumulator (one TMA
+//             reduce-add per 128 x 32 tile).  Splitting every row between the two
+//             warpgroups halves the per-step chain P^T -> dS^T -> dQ drain that the
+//             products wait on;
 //   warp  8   TMA producer: K_j and V_j per tile (two buffers at D = 64, the next
 //             tile's loaded during the current one), a 2-stage ring of (Q_i, dO_i)
 //             and the tile's LSE / D rows, across the CTA's tiles;
 //   warp  9   tcgen05 MMA issuer (one thread).
-// TMEM (fp32 columns), D = 128: S^T [0,128), warpgroup g's query columns at
-// [64 g, 64 g + 64); each warpgroup packs its P^T (16-bit pairs) into
-// [64 g, 64 g + 32) and its dS^T into [64 g + 32, 64 g + 64) -- inside its own
-// score columns, which it has fully read by then, never the other warpgroup's;
-// dP^T [128,256), also the dQ partial; dV [256,384); dK [384,512).
-// D = 64: S^T [0,128); dP^T [128,256) with warpgroup g's packed dS^T written over
-// its own dP^T columns [128 + 64 g, + 32); dV [256,320); dK [320,384); dQ
-// [384,448); packed P^T of warpgroup g at [448 + 32 g, + 32).  The score columns
-// are then free once read, and the steps are software-pipelined (BwdCfg::PIPE).
+// TMEM (fp32 columns): S^T [0,128); dP^T [128,256), warpgroup g writing its packed
+// dS^T over its own dP^T columns [128 + 64 g, + 32); dV [256, 256 + D); dK
+// [256 + D, 256 + 2 D).  D = 64: dQ [384,448), packed P^T of warpgroup g at
+// [448 + 32 g, + 32).  D = 128: packed P^T of warpgroup g over its own score
+// columns [64 g, + 32), no dQ.
+// The steps are software-pipelined: the scores of step i + 1 go out right after
+// step i's dV product and its dP^T right after step i's dK product, so that the
+// next step's products overlap this step's dS.
 // Products (M = 128 rows of the first operand, K = 16 per instruction):
 //   S^T  = K_j  Q_i^T   (A = K smem K-major, B = Q smem K-major)
 //   dP^T = V_j  dO_i^T  (A = V smem K-major, B = dO smem K-major)
 //   dV  += P^T  dO_i    (A = P^T TMEM, B = dO smem MN-major)
 //   dK  += dS^T Q_i     (A = dS^T TMEM, B = Q smem MN-major)
-//   dQ_i = dS   K_j     (A = dS^T smem MN-major, B = K smem MN-major)
+//   dQ_i = dS   K_j     (tile width 64: A = dS^T smem MN-major, B = K smem MN-major)
 #pragma once
 
 #include <cuda_fp16.h>
@@ -54,32 +60,28 @@
 #include <algorithm>
 #include <atomic>
 
+#include "fa2_bwd_dq.cuh"
 #include "ptx.cuh"
 
 namespace fa2 {
 
-constexpr int kBwdKernelsPerCall = 3;
-
-// Groups of four probabilities v (of eight per 32 queries) with (v & 3) >=
-// kBwdPolyFrom take the FMA-pipe exp2 polynomial instead of the MUFU unit
-// (4: none).
-#ifndef FA2_BWD_POLY_FROM
-#define FA2_BWD_POLY_FROM 4
-#endif
-constexpr int kBwdPolyFrom = FA2_BWD_POLY_FROM;
-
 // Workspace: D [BH][Npad] f32 | L2 = LSE*log2(e) [BH][Npad] f32 | dQacc [BH][N][Dt] f32,
-// Dt the kernel's tile head dim (64 or 128).
+// Dt the kernel's tile head dim (64 or 128).  The deterministic mode sums dQ in TMEM
+// (fa2_bwd_dq_kernel) and uses the two row statistics alone.
 inline size_t bwd_npad(int N) { return (static_cast<size_t>(N) + 127) / 128 * 128; }
 inline size_t bwd_rowstat_bytes(size_t BH, int N) {
   return (2 * BH * bwd_npad(N) * 4 + 255) / 256 * 256;
 }
 // Kernel head dim for a head dim d <= 128: the tiles are 64 or 128 columns wide.
 inline int bwd_tile_dim(int d) { return d <= 64 ? 64 : 128; }
-inline size_t bwd_workspace_bytes(size_t BH, int N, int d) {
+inline size_t bwd_workspace_bytes(size_t BH, int N, int d, bool deterministic = false) {
+  if (deterministic) return bwd_rowstat_bytes(BH, N);
   return bwd_rowstat_bytes(BH, N) +
          (BH * static_cast<size_t>(N) * bwd_tile_dim(d) * 4 + 255) / 256 * 256;
 }
+// Kernels one backward call launches: preprocess, main and dQ finalisation; in the
+// deterministic mode the dQ kernel and the dK/dV kernel.
+inline int bwd_kernels_per_call(bool deterministic) { return deterministic ? 2 : 3; }
 
 // ------------------------------------------------------------------------------------
 // 1. preprocess
@@ -145,7 +147,7 @@ fa2_bwd_pre_kernel(const uint16_t* __restrict__ O, const uint16_t* __restrict__ 
 
 template <bool BF16>
 __global__ void __launch_bounds__(256)
-fa2_bwd_dq_kernel(const float* __restrict__ dQacc, uint16_t* __restrict__ dQ, float scale,
+fa2_bwd_dq_finalise_kernel(const float* __restrict__ dQacc, uint16_t* __restrict__ dQ, float scale,
                   long long n8, int D, int d) {
   // Thread i converts 8 accumulator columns (group i % (D/8) of row i / (D/8));
   // groups past the head dim d are padding and are dropped.
@@ -184,46 +186,62 @@ struct BwdParams {
   int fault;          // test hook: 1 = skip the K, V load (a consumer's wait runs out)
 };
 
-template <int D>
+template <int D, bool DQ_>
 struct BwdCfg {
   static constexpr int KCH = D / 64;
   static constexpr int CHUNK = 128 * 128;
   static constexpr int TILE = 128 * D * 2;
-  static constexpr int ST = 2;                 // (Q, dO) ring stages
+  static constexpr int ST = 2;                 // (Q, dO) ring stages; dO ring at tile width 128
   // K/V buffers: a CTA runs several key tiles in turn.  At D = 64 the next tile's
   // K and V load into a buffer of their own while the current tile runs; at
   // D = 128 there is room for one, reloaded once the tile's last product has read it.
   static constexpr int KVB = (D == 64) ? 2 : 1;
-  static constexpr int DS_BYTES = 128 * 128 * 2;
+  // DQ: dQ partials from this kernel, added into a float accumulator (the default
+  // mode); otherwise (the deterministic mode, D = 128) fa2_bwd_dq_kernel computes
+  // dQ and this kernel computes dK and dV only.
+  static constexpr bool DQ = DQ_;
+  static_assert(DQ || D == 128, "the dK/dV-only kernel uses 128-wide tiles");
+  // Software-pipelined steps with the dQ product: at D = 64, where TMEM has room.
+  static constexpr bool PIPE = DQ && D == 64;
+  static constexpr int DS_BYTES = DQ ? 128 * 128 * 2 : 0;  // dS^T in shared memory, for dQ
+  // Q tiles: in the (Q, dO) ring at tile width 64; a ring of their own at 128, one
+  // stage deeper than dO's, released by dK (their last reader) -- the next step's
+  // scores are issued as soon as this step's have been read, so the next Q must
+  // already be resident then, while dO is first needed later, by dP^T.
+  static constexpr int QS = DQ ? ST : 3;
   static constexpr int LD_BYTES = ST * 2 * 128 * 4;  // LSE*log2e and D rows of each stage
   static constexpr int CTRL_BYTES = 256;              // barriers, TMEM address, abort flag
   // No alignment slack: the dynamic region must start 1024-byte aligned (checked).
-  static constexpr int SMEM = (2 * KVB + 2 * ST) * TILE + DS_BYTES + LD_BYTES + CTRL_BYTES;
+  static constexpr int SMEM = (2 * KVB + QS + ST) * TILE + DS_BYTES + LD_BYTES + CTRL_BYTES;
+  static_assert(SMEM <= 227 * 1024, "shared memory");
   static constexpr int THREADS = 320;
   static constexpr uint32_t C_S = 0, C_DP = 128;
-  // Software-pipelined steps (D = 64, where TMEM has room): packed P^T of warpgroup
-  // g in columns 448 + 32 g .. + 31 (free at D = 64), packed dS^T in its own dP^T
-  // columns 128 + 64 g .. + 31, so the score columns are free as soon as the scores
-  // have been read and the next step's scores can be computed during this step's
-  // dS.  Otherwise (D = 128, no free columns) P^T and dS^T of warpgroup g sit in
-  // its score columns, 64 g + (0 | 32) .. + 31.
-  static constexpr bool PIPE = (D == 64);
+  // Packed P^T and dS^T of warpgroup g:
+  //   D = 64 (pipelined): P^T in columns 448 + 32 g .. + 31 (free at D = 64), dS^T
+  //     over its own dP^T columns 128 + 64 g .. + 31, so the score columns are free
+  //     as soon as the scores have been read and the next step's scores are
+  //     computed during this step's dS;
+  //   D = 128 with dQ: both inside its own score columns, 64 g + (0 | 32) .. + 31
+  //     (no free columns: dP^T also holds the dQ partial);
+  //   D = 128, dK/dV only: both over its own dP^T columns, dS^T at 128 + 64 g, P^T
+  //     at 128 + 64 g + 32 (P stays in registers until then), so the next step's
+  //     scores are computed during this step's exponentials.
   __host__ __device__ static constexpr uint32_t C_P(int g) {
-    return PIPE ? 448u + 32u * g : 64u * g;
+    return D == 64 ? 448u + 32u * g : (DQ ? 64u * g : C_DP + 64u * g + 32u);
   }
   __host__ __device__ static constexpr uint32_t C_DS(int g) {
-    return PIPE ? C_DP + 64u * g : 64u * g + 32u;
+    return (D == 128 && DQ) ? 64u * g + 32u : C_DP + 64u * g;
   }
   static constexpr uint32_t C_DV = 256, C_DK = 256 + D;
-  static constexpr uint32_t C_DQ = (D == 128) ? 128 : 384;
+  static constexpr uint32_t C_DQ = (D == 128) ? 128 : 384;  // D = 128: shares dP^T's columns
 };
 
 // Control block at the end of the dynamic shared memory (no static shared memory,
 // so that the 1024-byte aligned tiles start at the base of the window).
 template <int ST>
 struct BwdCtrl {
-  uint64_t bar_kv[2], kv_empty[2], acc_free, qdo_full[ST], qdo_empty[ST];
-  uint64_t s_full, dp_full, p_ready, ds_ready, dq_full, dq_drained, drain, fin;
+  uint64_t bar_kv[2], kv_empty[2], acc_free, qdo_full[ST], qdo_empty[ST], q_full[3], q_empty[3];
+  uint64_t s_full, s_read, dp_full, p_ready, ds_ready, dq_full, dq_drained, drain, fin;
   uint32_t tmem_slot;
   int abort_flag;
 };
@@ -243,12 +261,12 @@ enum BwdSite : uint32_t {
   kBSiteProdKV
 };
 
-template <int D, bool BF16, bool CAUSAL>
+template <int D, bool BF16, bool CAUSAL, bool DQ>
 __global__ void __launch_bounds__(320, 1)
 fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
                const __grid_constant__ CUtensorMap tmdQ, const BwdParams p) {
-  using C = BwdCfg<D>;
+  using C = BwdCfg<D, DQ>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   if ((smem_u32(smem_raw) & 1023u) != 0) {
     // The swizzled tiles need a 1024-byte aligned base; report and do nothing.
@@ -261,8 +279,8 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   uint8_t* smem = smem_raw;
   uint8_t* sK = smem;                        // KVB tiles
   uint8_t* sV = sK + C::KVB * C::TILE;       // KVB tiles
-  uint8_t* sQ = sV + C::KVB * C::TILE;       // ST tiles
-  uint8_t* sdO = sQ + C::ST * C::TILE;       // ST tiles
+  uint8_t* sQ = sV + C::KVB * C::TILE;       // QS tiles
+  uint8_t* sdO = sQ + C::QS * C::TILE;       // ST tiles
   uint8_t* sDS = sdO + C::ST * C::TILE;      // dS^T, MN-major for the dQ product
   float* sLD = reinterpret_cast<float*>(sDS + C::DS_BYTES);  // [ST][2][128]: L, D
   BwdCtrl<C::ST>& ctl = *reinterpret_cast<BwdCtrl<C::ST>*>(sDS + C::DS_BYTES + C::LD_BYTES);
@@ -272,9 +290,12 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   uint64_t& acc_free = ctl.acc_free;
   uint64_t* qdo_full = ctl.qdo_full;
   uint64_t* qdo_empty = ctl.qdo_empty;
+  uint64_t* q_full = ctl.q_full;    // tile width 128: the Q ring
+  uint64_t* q_empty = ctl.q_empty;
   uint64_t& s_full = ctl.s_full;
   uint64_t& dp_full = ctl.dp_full;
   uint64_t& p_ready = ctl.p_ready;
+  uint64_t& s_read = ctl.s_read;
   uint64_t& ds_ready = ctl.ds_ready;
   uint64_t& dq_full = ctl.dq_full;
   uint64_t& dq_drained = ctl.dq_drained;
@@ -323,9 +344,11 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     }
     mbar_init(&acc_free, 8);
     for (int s = 0; s < C::ST; ++s) { mbar_init(&qdo_full[s], 1); mbar_init(&qdo_empty[s], 1); }
+    for (int s = 0; s < 3; ++s) { mbar_init(&q_full[s], 1); mbar_init(&q_empty[s], 1); }
     mbar_init(&s_full, 1);
     mbar_init(&dp_full, 1);
     mbar_init(&p_ready, 8);
+    mbar_init(&s_read, 8);
     mbar_init(&ds_ready, 8);
     mbar_init(&dq_full, 1);
     mbar_init(&dq_drained, 8);
@@ -374,6 +397,7 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       load_kv(0);
       if (C::KVB == 2 && tile_of(1) >= 0) load_kv(1);
       int gs = 0;  // query steps issued so far (ring slot and phase)
+      int gq = 0;  // tile width 128: Q loads issued (may run one ahead of gs on an abort)
       bool ok = true;
       for (int k = 0; ok; ++k) {
         const int t = tile_of(k);
@@ -382,19 +406,34 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         const int i0 = q_begin(t / p.BH), n_it = q_end(t / p.BH) - i0;
         for (int it = 0; it < n_it; ++it) {
           const int st = gs % C::ST;
+          const int row = (i0 + it) * 128;
+          if constexpr (!C::DQ) {
+            // Q in a ring of its own (released by dK), loaded before this step's dO.
+            const int qs = gs % C::QS;
+            if (gs >= C::QS &&
+                !mbar_wait(&q_empty[qs], ((gs / C::QS) - 1) & 1, wc, kBSiteProdEmpty)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(&q_full[qs], C::TILE);
+            for (int c = 0; c < C::KCH; ++c)
+              tma_load_3d_hint(sQ + qs * C::TILE + c * C::CHUNK, &tmQ, &q_full[qs], c * 64, row, bh,
+                               keep);
+            ++gq;
+          }
           if (gs >= C::ST &&
               !mbar_wait(&qdo_empty[st], ((gs / C::ST) - 1) & 1, wc, kBSiteProdEmpty)) {
             ok = false;
             break;
           }
-          const int row = (i0 + it) * 128;
-          mbar_arrive_expect_tx(&qdo_full[st], 2 * C::TILE + 2 * 512);
+          mbar_arrive_expect_tx(&qdo_full[st], (C::DQ ? 2 : 1) * C::TILE + 2 * 512);
           const size_t stat = static_cast<size_t>(bh) * p.Npad + row;
           bulk_load_1d(sLD + st * 256, p.Lg + stat, 512, &qdo_full[st]);
           bulk_load_1d(sLD + st * 256 + 128, p.Dg + stat, 512, &qdo_full[st]);
           for (int c = 0; c < C::KCH; ++c) {
-            tma_load_3d_hint(sQ + st * C::TILE + c * C::CHUNK, &tmQ, &qdo_full[st], c * 64, row,
-                             bh, keep);
+            if constexpr (C::DQ)
+              tma_load_3d_hint(sQ + st * C::TILE + c * C::CHUNK, &tmQ, &qdo_full[st], c * 64, row,
+                               bh, keep);
             tma_load_3d_hint(sdO + st * C::TILE + c * C::CHUNK, &tmdO, &qdo_full[st], c * 64,
                              row, bh, keep);
           }
@@ -423,6 +462,10 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       if (!ok) {
         for (int q = max(0, gs - C::ST); q < gs; ++q)
           mbar_wait(&qdo_full[q % C::ST], (q / C::ST) & 1, dw, kBSiteProdDrain);
+        if constexpr (!C::DQ) {
+          for (int q = max(0, gq - C::QS); q < gq; ++q)
+            mbar_wait(&q_full[q % C::QS], (q / C::QS) & 1, dw, kBSiteProdDrain);
+        }
       }
       // Every K, V load lands before exit, even on an aborted run (one at most is
       // in flight per buffer: a reload waits for the previous one to be consumed).
@@ -468,6 +511,8 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         for (int kk = 0; kk < 8; ++kk)
           umma_ts(tbase + C::C_DV, tbase + C::C_P(kk >> 2) + (kk & 3) * 8,
                   sdesc_add(mdO, st * C::TILE + kk * 2048), id_tb, (!first || kk > 0) ? 1u : 0u);
+        // Tile width 128: dV is dO's last reader (its L, D rows were read before ds_ready).
+        if constexpr (!C::DQ) umma_commit(&qdo_empty[st]);
       };
       auto mma_dq = [&](uint32_t kvo) {  // dQ_i = dS K
 #pragma unroll
@@ -476,12 +521,14 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                   id_dq, kk > 0);
         umma_commit(&dq_full);
       };
-      auto mma_dk = [&](int st, bool first) {  // dK += dS^T Q; the step's last read of Q, dO
+      // dK += dS^T Q; the step's last read of Q (and, at tile width 64, of its dO).
+      // qs: the Q slot -- the (Q, dO) ring's at tile width 64, the Q ring's at 128.
+      auto mma_dk = [&](int qs, bool first) {
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
           umma_ts(tbase + C::C_DK, tbase + C::C_DS(kk >> 2) + (kk & 3) * 8,
-                  sdesc_add(mQ, st * C::TILE + kk * 2048), id_tb, (!first || kk > 0) ? 1u : 0u);
-        umma_commit(&qdo_empty[st]);
+                  sdesc_add(mQ, qs * C::TILE + kk * 2048), id_tb, (!first || kk > 0) ? 1u : 0u);
+        umma_commit(C::DQ ? &qdo_empty[qs] : &q_empty[qs]);
       };
       bool ok = true;
       int gs = 0;  // query steps so far
@@ -492,10 +539,41 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         const int b = k % C::KVB;
         const uint32_t kvo = static_cast<uint32_t>(b * C::TILE);  // this tile's K, V buffer
         if (!mbar_wait(&bar_kv[b], kv_par(k), wc, kBSiteMmaKV)) { ok = false; break; }
-        if constexpr (C::PIPE) {
-          // Step g + 1's scores go out once the compute warps have read step g's
-          // (p_ready), so that they overlap step g's dS; step g + 1's dP^T follows
-          // step g's dK, whose dS^T operand sits in the dP^T columns.
+        if constexpr (C::DQ && !C::PIPE) {
+          // Tile width 128 with dQ: TMEM has no free columns, so each step runs in
+          // order -- S^T, dP^T (once the previous dQ partial, in the same columns,
+          // is drained), dV (P^T ready), dQ and dK (dS^T ready).
+          for (int it = 0; it < n_it; ++it, ++gs) {
+            const int st = gs % C::ST;
+            if (!mbar_wait(&qdo_full[st], (gs / C::ST) & 1, wc, kBSiteMmaQ)) { ok = false; break; }
+            tc_fence_after();
+            mma_s(st, kvo);
+            if (gs > 0) {
+              if (!mbar_wait(&dq_drained, (gs - 1) & 1, wc, kBSiteMmaDrained)) { ok = false; break; }
+              tc_fence_after();
+            }
+            mma_dp(st, kvo);
+            if (!mbar_wait(&p_ready, gs & 1, wc, kBSiteMmaP)) { ok = false; break; }
+            tc_fence_after();
+            if (k > 0 && it == 0) {
+              if (!mbar_wait(&acc_free, (k - 1) & 1, wc, kBSiteMmaAcc)) { ok = false; break; }
+              tc_fence_after();
+            }
+            mma_dv(st, it == 0);
+            // dQ_i = dS K first (the drain needs only this one), then dK += dS^T Q (A
+            // from TMEM, so the dQ staging that reuses the dS^T tile of shared memory
+            // cannot race it).
+            if (!mbar_wait(&ds_ready, gs & 1, wc, kBSiteMmaDS)) { ok = false; break; }
+            tc_fence_after();
+            mma_dq(kvo);
+            if (it == n_it - 1) umma_commit(&kv_empty[b]);
+            mma_dk(st, it == 0);
+          }
+        } else if constexpr (C::DQ) {
+          // Tile width 64: step g + 1's scores go out once the compute warps have
+          // read step g's and written P^T (p_ready), right after step g's dV product,
+          // so that they overlap step g's dS; step g + 1's dP^T follows step g's dK,
+          // whose dS^T operand sits in the dP^T columns.
           if (!mbar_wait(&qdo_full[gs % C::ST], (gs / C::ST) & 1, wc, kBSiteMmaQ)) { ok = false; break; }
           tc_fence_after();
           mma_s(gs % C::ST, kvo);
@@ -530,37 +608,48 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             if (it + 1 < n_it) mma_dp((gs + 1) % C::ST, kvo);
           }
         } else {
+          // Tile width 128: S^T(g + 1) as soon as the compute warps have read S^T(g)
+          // (s_read), so that it runs during their exponentials; dV(g) and dK(g) once
+          // P^T and dS^T are packed over the dP^T columns (ds_ready); dP^T(g + 1)
+          // after them, in issue order, since it overwrites those columns.
+          if (!mbar_wait(&q_full[gs % C::QS], (gs / C::QS) & 1, wc, kBSiteMmaQ)) { ok = false; break; }
+          tc_fence_after();
+          mma_s(gs % C::QS, kvo);
+          if (!mbar_wait(&qdo_full[gs % C::ST], (gs / C::ST) & 1, wc, kBSiteMmaQ)) { ok = false; break; }
+          tc_fence_after();
+          mma_dp(gs % C::ST, kvo);
+          // The tile's last reads of K and V are its last S^T and dP^T: the buffer can
+          // take the next tile's K, V during the last dV, dK.
+          if (n_it == 1) umma_commit(&kv_empty[b]);
           for (int it = 0; it < n_it; ++it, ++gs) {
             const int st = gs % C::ST;
-            if (!mbar_wait(&qdo_full[st], (gs / C::ST) & 1, wc, kBSiteMmaQ)) { ok = false; break; }
-            tc_fence_after();
-            mma_s(st, kvo);
-            // dP^T's columns hold the previous dQ partial (D = 128) until drained.
-            if (C::C_DQ == C::C_DP && gs > 0) {
-              if (!mbar_wait(&dq_drained, (gs - 1) & 1, wc, kBSiteMmaDrained)) { ok = false; break; }
+            if (it + 1 < n_it) {
+              const int qs1 = (gs + 1) % C::QS;
+              if (!mbar_wait(&s_read, gs & 1, wc, kBSiteMmaP) ||
+                  !mbar_wait(&q_full[qs1], ((gs + 1) / C::QS) & 1, wc, kBSiteMmaQ)) {
+                ok = false;
+                break;
+              }
               tc_fence_after();
+              mma_s(qs1, kvo);
             }
-            mma_dp(st, kvo);
-            if (!mbar_wait(&p_ready, gs & 1, wc, kBSiteMmaP)) { ok = false; break; }
+            if (!mbar_wait(&ds_ready, gs & 1, wc, kBSiteMmaDS)) { ok = false; break; }
             tc_fence_after();
             if (k > 0 && it == 0) {
+              // A tile's first dV and dK products overwrite the accumulators: the
+              // previous tile's epilogue must have read them out.
               if (!mbar_wait(&acc_free, (k - 1) & 1, wc, kBSiteMmaAcc)) { ok = false; break; }
               tc_fence_after();
             }
             mma_dv(st, it == 0);
-            // dQ_i = dS K first (the drain needs only this one; with its own TMEM
-            // columns, wait for the previous drain), then dK += dS^T Q (A from TMEM,
-            // so the dQ staging that reuses the dS^T tile of shared memory cannot
-            // race it).
-            if (!mbar_wait(&ds_ready, gs & 1, wc, kBSiteMmaDS)) { ok = false; break; }
-            tc_fence_after();
-            if (C::C_DQ != C::C_DP && gs > 0) {
-              if (!mbar_wait(&dq_drained, (gs - 1) & 1, wc, kBSiteMmaDrained)) { ok = false; break; }
+            mma_dk(gs % C::QS, it == 0);
+            if (it + 1 < n_it) {
+              const int st1 = (gs + 1) % C::ST;
+              if (!mbar_wait(&qdo_full[st1], ((gs + 1) / C::ST) & 1, wc, kBSiteMmaQ)) { ok = false; break; }
               tc_fence_after();
+              mma_dp(st1, kvo);
+              if (it + 1 == n_it - 1) umma_commit(&kv_empty[b]);
             }
-            mma_dq(kvo);
-            if (it == n_it - 1) umma_commit(&kv_empty[b]);
-            mma_dk(st, it == 0);
           }
         }
         if (!ok) break;
@@ -610,6 +699,12 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       tmem_wait_ld();
       reg_fence(srr[0]);
       reg_fence(srr[1]);
+      if constexpr (!C::DQ) {
+        // Tile width 128: the score columns may take the next step's scores now.
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s_read);
+      }
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         const uint32_t (&sr)[32] = srr[c];
@@ -644,16 +739,18 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
               (CAUSAL && win > 0 && ip * 128 + qoff + qc - key >= win))
             pr[qc] = 0.f;
       }
-      {
+      if constexpr (C::DQ) {
+        // Tile width 64: P^T goes to its own columns now (dV can start).  At 128 it
+        // stays in registers and is written with dS^T.
         uint32_t pk[32];
 #pragma unroll
         for (int e = 0; e < 32; ++e) pk[e] = pack2<BF16>(pr[2 * e], pr[2 * e + 1]);
         tmem_st32(tmem_addr(tbase, lb, C::C_P(g)), pk);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_ready);
       }
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&p_ready);
       return true;
     };
     // dS^T = P^T * (dP^T - D), 32 queries at a time, written to TMEM (A operand
@@ -664,7 +761,44 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       const float4* D4 = reinterpret_cast<const float4*>(sLD + (gd % C::ST) * 256 + 128 + qoff);
       if (!named_bar_and(wg_bar, 128, mbar_wait(&dp_full, gd & 1, wc, kBSiteCmpDP))) return false;
       tc_fence_after();
-      if (gd > 0) {
+      if constexpr (!C::DQ) {
+        // Tile width 128: all 64 dP^T columns of this warpgroup into registers, then
+        // packed dS^T and P^T over them (the A operands of dK and dV).
+        uint32_t dr[2][32];
+        tmem_ld32(tmem_addr(tbase, lb, C::C_DP + qoff), dr[0]);
+        tmem_ld32(tmem_addr(tbase, lb, C::C_DP + qoff + 32), dr[1]);
+        tmem_wait_ld();
+        reg_fence(dr[0]);
+        reg_fence(dr[1]);
+        uint32_t dsk[32], pk[32];
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+#pragma unroll
+          for (int v = 0; v < 8; ++v) {
+            const float4 d4 = D4[c * 8 + v];
+            const int q0 = c * 32 + v * 4;
+            const uint64_t t01 = f2_sub(f2_pack(__uint_as_float(dr[c][v * 4]), __uint_as_float(dr[c][v * 4 + 1])),
+                                        f2_pack(d4.x, d4.y));
+            const uint64_t t23 = f2_sub(f2_pack(__uint_as_float(dr[c][v * 4 + 2]), __uint_as_float(dr[c][v * 4 + 3])),
+                                        f2_pack(d4.z, d4.w));
+            float a0, a1, a2, a3;
+            f2_unpack(f2_mul(f2_pack(pr[q0], pr[q0 + 1]), t01), a0, a1);
+            f2_unpack(f2_mul(f2_pack(pr[q0 + 2], pr[q0 + 3]), t23), a2, a3);
+            dsk[q0 / 2] = pack2<BF16>(a0, a1);
+            dsk[q0 / 2 + 1] = pack2<BF16>(a2, a3);
+            pk[q0 / 2] = pack2<BF16>(pr[q0], pr[q0 + 1]);
+            pk[q0 / 2 + 1] = pack2<BF16>(pr[q0 + 2], pr[q0 + 3]);
+          }
+        }
+        tmem_st32(tmem_addr(tbase, lb, C::C_DS(g)), dsk);
+        tmem_st32(tmem_addr(tbase, lb, C::C_P(g)), pk);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ds_ready);
+        return true;
+      }
+      if (C::DQ && gd > 0) {
         // This warpgroup's dS^T chunk doubled as the staging tile of the previous
         // dQ reduce: that bulk copy must have finished reading it.
         if (r == 0) tma_store_wait_read();
@@ -692,14 +826,16 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           dsk[2 * v + 1] = pack2<BF16>(a2, a3);
         }
         tmem_st16(tmem_addr(tbase, lb, C::C_DS(g) + 16 * c), dsk);
+        if constexpr (C::DQ) {
 #pragma unroll
-        for (int uu = 0; uu < 4; ++uu) {
-          const int u = c * 4 + uu;
-          const uint4 val = make_uint4(dsk[4 * uu], dsk[4 * uu + 1], dsk[4 * uu + 2], dsk[4 * uu + 3]);
-          *reinterpret_cast<uint4*>(sDS + g * C::CHUNK + r * 128 + ((u ^ (r & 7)) << 4)) = val;
+          for (int uu = 0; uu < 4; ++uu) {
+            const int u = c * 4 + uu;
+            const uint4 val = make_uint4(dsk[4 * uu], dsk[4 * uu + 1], dsk[4 * uu + 2], dsk[4 * uu + 3]);
+            *reinterpret_cast<uint4*>(sDS + g * C::CHUNK + r * 128 + ((u ^ (r & 7)) << 4)) = val;
+          }
         }
       }
-      fence_proxy_async_smem();
+      if constexpr (C::DQ) fence_proxy_async_smem();
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
@@ -721,7 +857,7 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         // One 32-column tile, 16 columns at a time: the next step's P^T is live
         // beside it.  The columns are released once both halves are read.
         static_assert(NCH == 1, "pipelined steps assume D = 64");
-#pragma unroll
+  #pragma unroll
         for (int h = 0; h < 2; ++h) {
           uint32_t q16[16];
           tmem_ld16(tmem_addr(tbase, lb, C::C_DQ + g * HALF + 16 * h), q16);
@@ -732,7 +868,7 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             __syncwarp();
             if (lane == 0) mbar_arrive(&dq_drained);
           }
-#pragma unroll
+  #pragma unroll
           for (int u = 0; u < 4; ++u)
             *reinterpret_cast<uint4*>(stage + r * 128 + (((4 * h + u) ^ (r & 7)) << 4)) =
                 make_uint4(q16[4 * u], q16[4 * u + 1], q16[4 * u + 2], q16[4 * u + 3]);
@@ -823,25 +959,30 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       const int key = j * 128 + r;
       const int i_begin = q_begin(j);
       const int n_it = q_end(j) - i_begin;
-      // Plain order: P, dS, dQ drain of each step.  Pipelined (C::PIPE): P of step
-      // i + 1 between dS and the dQ drain of step i, so that step i's dQ product and
-      // step i + 1's dP product run while the softmax works.
+      // Pipelined order: P of step 0, then per step i: dS(i), P(i + 1), dQ drain(i)
+      // (tile width 64; without dQ no drain), so that step i's dQ product and step
+      // i + 1's dP product run while the softmax works.
       const int g0 = gs;
-      if constexpr (C::PIPE) ok = stage_p(g0, i_begin, j, key);
-      for (int it = 0; it < n_it && ok; ++it) {
-        if constexpr (!C::PIPE) {
+      if constexpr (C::DQ && !C::PIPE) {
+        // Tile width 128 with dQ: P, dS, dQ drain of each step in turn.
+        for (int it = 0; it < n_it && ok; ++it) {
           ok = stage_p(g0 + it, i_begin + it, j, key);
           if (!ok) break;
+          ok = stage_ds(g0 + it);
+          if (!ok) break;
+          ok = stage_dq(g0 + it, i_begin + it, bh);
         }
-        ok = stage_ds(g0 + it);
-        if (!ok) break;
-        if constexpr (C::PIPE) {
+      } else {
+        ok = stage_p(g0, i_begin, j, key);
+        for (int it = 0; it < n_it && ok; ++it) {
+          ok = stage_ds(g0 + it);
+          if (!ok) break;
           if (it + 1 < n_it) {
             ok = stage_p(g0 + it + 1, i_begin + it + 1, j, key);
             if (!ok) break;
           }
+          if constexpr (C::DQ) ok = stage_dq(g0 + it, i_begin + it, bh);
         }
-        ok = stage_dq(g0 + it, i_begin + it, bh);
       }
       gs = g0 + n_it;
       if (!ok) break;
@@ -912,26 +1053,61 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, int smem,
   return e;
 }
 
-template <int D, bool BF16, bool CAUSAL>
+template <int D, bool BF16, bool CAUSAL, bool DQ>
 int launch_bwd_t(const void* Q, const void* K, const void* V, const void* O, const void* dO,
                  const float* LSE, void* dQ, void* dK, void* dV, void* workspace, int BH, int N,
                  int d, float scale, int window, unsigned int* status, unsigned long long wait_ns,
                  int fault, int max_ctas, cudaStream_t stream) {
-  using Cfg = BwdCfg<D>;
+  using Cfg = BwdCfg<D, DQ>;
   const int Npad = static_cast<int>(bwd_npad(N));
   // The tile list (key tiles x heads) is indexed with 32-bit ints in the kernel.
   if (static_cast<long long>(Npad / 128) * BH > (1ll << 30)) return 1;  // FA2_ERR_INVALID_ARG
   float* Dg = static_cast<float*>(workspace);
   float* Lg = Dg + static_cast<size_t>(BH) * Npad;
-  float* dQacc = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
-                                          bwd_rowstat_bytes(static_cast<size_t>(BH), N));
+  // The fp32 dQ accumulator (tile width 64 only) follows the row statistics.
+  float* dQacc = Cfg::DQ ? reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
+                                                    bwd_rowstat_bytes(static_cast<size_t>(BH), N))
+                         : nullptr;
   CUtensorMap mq, mk, mv, mdo, mdq;
   if (!make_tile_map(&mq, Q, BH, N, d, BF16) || !make_tile_map(&mk, K, BH, N, d, BF16) ||
-      !make_tile_map(&mv, V, BH, N, d, BF16) || !make_tile_map(&mdo, dO, BH, N, d, BF16) ||
-      !make_acc_map(&mdq, dQacc, BH, N, D))
+      !make_tile_map(&mv, V, BH, N, d, BF16) || !make_tile_map(&mdo, dO, BH, N, d, BF16))
     return 4;  // FA2_ERR_CUDA
-  // 1. preprocess
-  {
+  if constexpr (Cfg::DQ) {
+    if (!make_acc_map(&mdq, dQacc, BH, N, D)) return 4;
+  } else {
+    mdq = mq;  // not read
+  }
+  if constexpr (!Cfg::DQ) {
+    // 1. dQ (and the D, LSE * log2 e rows), one CTA per (query tile, batch*head)
+    const long long grid = static_cast<long long>(Npad / 128) * BH;
+    if (grid > 0x7fffffffll) return 1;  // FA2_ERR_INVALID_ARG
+    auto kq = fa2_bwd_dq_kernel<BF16, CAUSAL>;
+    static std::atomic<bool> smem_q[kSmemFlagDevices];
+    if (!set_smem_once(kq, BwdDqCfg::SMEM, smem_q)) return 4;
+    BwdDqParams qp{};
+    qp.dQ = dQ;
+    qp.Q = static_cast<const uint16_t*>(Q);
+    qp.O = static_cast<const uint16_t*>(O);
+    qp.dO = static_cast<const uint16_t*>(dO);
+    qp.LSE = LSE;
+    qp.Dg = Dg;
+    qp.Lg = Lg;
+    qp.d = d;
+    qp.N = N;
+    qp.Npad = Npad;
+    qp.BH = BH;
+    qp.n_q = Npad / 128;
+    qp.window = window;
+    qp.scale = scale;
+    qp.scale_log2 = scale * 1.4426950408889634f;
+    qp.status = status;
+    qp.wait_ns = wait_ns;
+    qp.fault = fault;
+    if (launch_pdl(kq, dim3(static_cast<unsigned int>(grid)), dim3(BwdDqCfg::THREADS),
+                   BwdDqCfg::SMEM, stream, mq, mk, mv, mdo, qp) != cudaSuccess)
+      return 4;
+  } else {
+    // 1. preprocess
     const long long rows = static_cast<long long>(BH) * Npad;
     constexpr int RPB = 256 / (D / 8);
     const unsigned int grid = static_cast<unsigned int>((rows + RPB - 1) / RPB);
@@ -940,9 +1116,9 @@ int launch_bwd_t(const void* Q, const void* K, const void* V, const void* O, con
                    dQacc, N, Npad, rows, d) != cudaSuccess)
       return 4;
   }
-  // 2. main
+  // 2. main (dK, dV; and, by default, the dQ partials)
   {
-    auto kern = fa2_bwd_kernel<D, BF16, CAUSAL>;
+    auto kern = fa2_bwd_kernel<D, BF16, CAUSAL, DQ>;
     static std::atomic<bool> smem_set[kSmemFlagDevices];  // this instantiation's flags
     if (!set_smem_once(kern, Cfg::SMEM, smem_set)) return 4;
     BwdParams bp{};
@@ -979,32 +1155,40 @@ int launch_bwd_t(const void* Q, const void* K, const void* V, const void* O, con
       return 4;
   }
   // 3. dQ finalise
-  {
+  if constexpr (Cfg::DQ) {
     const long long n8 = static_cast<long long>(BH) * N * D / 8;
     const unsigned int grid = static_cast<unsigned int>((n8 + 255) / 256);
-    if (launch_pdl(fa2_bwd_dq_kernel<BF16>, dim3(grid), dim3(256), 0, stream, dQacc,
+    if (launch_pdl(fa2_bwd_dq_finalise_kernel<BF16>, dim3(grid), dim3(256), 0, stream, dQacc,
                    static_cast<uint16_t*>(dQ), scale, n8, D, d) != cudaSuccess)
       return 4;
   }
   return 0;
 }
 
+// deterministic: dQ by fa2_bwd_dq_kernel (summed in TMEM in a fixed order) and dK,
+// dV by the dK/dV-only kernel, on 128-wide tiles at every head dim; otherwise the
+// main kernel adds dQ partials into the workspace's accumulator.
 inline int launch_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO,
                       const float* LSE, void* dQ, void* dK, void* dV, void* workspace, int BH,
                       int N, int d, float scale, bool causal, bool bf16, unsigned int* status,
                       unsigned long long wait_ns, cudaStream_t s, int window = 0,
-                      int fault = 0, int max_ctas = 0) {
-#define FA2_BWD_CALL(D_, BF_, CA_)                                                             \
-  return launch_bwd_t<D_, BF_, CA_>(Q, K, V, O, dO, LSE, dQ, dK, dV, workspace, BH, N, d, scale, \
-                                    window, status, wait_ns, fault, max_ctas, s)
-  if (d <= 64) {
-    if (bf16) { if (causal) FA2_BWD_CALL(64, true, true); FA2_BWD_CALL(64, true, false); }
-    if (causal) FA2_BWD_CALL(64, false, true);
-    FA2_BWD_CALL(64, false, false);
+                      int fault = 0, int max_ctas = 0, bool deterministic = false) {
+#define FA2_BWD_CALL(D_, BF_, CA_, DQ_)                                                         \
+  return launch_bwd_t<D_, BF_, CA_, DQ_>(Q, K, V, O, dO, LSE, dQ, dK, dV, workspace, BH, N, d,   \
+                                         scale, window, status, wait_ns, fault, max_ctas, s)
+  if (deterministic) {
+    if (bf16) { if (causal) FA2_BWD_CALL(128, true, true, false); FA2_BWD_CALL(128, true, false, false); }
+    if (causal) FA2_BWD_CALL(128, false, true, false);
+    FA2_BWD_CALL(128, false, false, false);
   }
-  if (bf16) { if (causal) FA2_BWD_CALL(128, true, true); FA2_BWD_CALL(128, true, false); }
-  if (causal) FA2_BWD_CALL(128, false, true);
-  FA2_BWD_CALL(128, false, false);
+  if (d <= 64) {
+    if (bf16) { if (causal) FA2_BWD_CALL(64, true, true, true); FA2_BWD_CALL(64, true, false, true); }
+    if (causal) FA2_BWD_CALL(64, false, true, true);
+    FA2_BWD_CALL(64, false, false, true);
+  }
+  if (bf16) { if (causal) FA2_BWD_CALL(128, true, true, true); FA2_BWD_CALL(128, true, false, true); }
+  if (causal) FA2_BWD_CALL(128, false, true, true);
+  FA2_BWD_CALL(128, false, false, true);
 #undef FA2_BWD_CALL
 }
 

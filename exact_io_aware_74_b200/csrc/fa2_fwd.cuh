@@ -501,7 +501,14 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     const uint32_t lane_base = static_cast<uint32_t>(wq * 32);
     const float sl2 = p.scale_log2;  // > 0 (checked on the host)
     float m = -INFINITY;  // running max, log2 units of scaled scores
-    float l = 0.f;        // running sum of exp2(s * sl2 - m)
+    float l = 0.f;        // running sum of exp2(s * sl2 - m): the log-sum-exp
+    // Running sum of the same values as rounded to 16 bits, the weights the P V
+    // product actually applies: O is divided by this one, so that it is an exact
+    // weighted average of V rows.  (Dividing by the unrounded sum adds the rounding
+    // error of P to O: up to 2^-9 |v| on a row dominated by one key, which the
+    // long-context workload with its x8 key outliers shows.)  8-bit inputs keep the
+    // unrounded sum.
+    float lr = 0.f;
     bool ok = my_nkv > 0;
     const int win = p.window;
     // A warp whose 32 rows are all past Nq only keeps the barrier count: its P
@@ -571,6 +578,7 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           const float f = need ? ex2_approx(m - m_new) : 1.0f;
           if (need) m = m_new;
           l *= f;
+          lr *= f;
           if (!__all_sync(0xffffffffu, mbar_wait(&o_done[t], (step - 1) & 1, wc, kSiteSoftO)))
             return false;
           tc_fence_after();
@@ -593,6 +601,7 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       const float neg_m = (m == -INFINITY) ? 0.f : -m;
       const uint64_t negm2 = f2_pack(neg_m, neg_m);
       uint64_t sum2[4] = {0, 0, 0, 0};
+      [[maybe_unused]] uint64_t sumr2[4] = {0, 0, 0, 0};  // of the 16-bit P values
       // With its own P columns the previous P V product may still be reading them.
       if (sep && step > 0) {
         if (!__all_sync(0xffffffffu, mbar_wait(&o_done[t], (step - 1) & 1, wc, kSiteSoftO)))
@@ -625,8 +634,14 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             e[2 * q] = a;
             e[2 * q + 1] = b;
           }
-          if constexpr (F8) pk[i] = pack4_e4m3(e[0], e[1], e[2], e[3]);
-          else pk[i] = pack2<BF16>(e[0], e[1]);
+          if constexpr (F8) {
+            pk[i] = pack4_e4m3(e[0], e[1], e[2], e[3]);
+          } else {
+            pk[i] = pack2<BF16>(e[0], e[1]);
+            float r0, r1;
+            unpack2<BF16>(pk[i], r0, r1);
+            sumr2[i & 3] = f2_add(sumr2[i & 3], f2_pack(r0, r1));
+          }
         }
         const uint32_t dst = tmem_addr(tbase, lane_base, p_col + col0 / EPC + G * h);
         if constexpr (G == 32) tmem_st32(dst, pk); else tmem_st16(dst, pk);
@@ -648,6 +663,13 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         float lo, hi;
         f2_unpack(s01, lo, hi);
         l += lo + hi;
+        if constexpr (F8) {
+          lr = l;
+        } else {
+          const uint64_t r01 = f2_add(f2_add(sumr2[0], sumr2[1]), f2_add(sumr2[2], sumr2[3]));
+          f2_unpack(r01, lo, hi);
+          lr += lo + hi;
+        }
       }
       return true;
     };
@@ -701,7 +723,7 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       tc_fence_after();
       // A row can see no key of a split (l = 0): it contributes nothing.
       // (8-bit inputs: the scale of V is applied here, once per output element.)
-      const float inv_l = (l > 0.f) ? (F8 ? p.o_scale : 1.0f) / l : 0.f;
+      const float inv_l = (l > 0.f && lr > 0.f) ? (F8 ? p.o_scale : 1.0f) / lr : 0.f;
       const float lse = (l > 0.f) ? (m + __log2f(l)) * 0.69314718055994531f : -INFINITY;
       const size_t orow_idx = static_cast<size_t>(bh) * Nq + row;
       if (!partial) {

@@ -9,6 +9,7 @@
 
 #include <cstdint>
 #include <cuda.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 namespace fa2 {
@@ -509,6 +510,14 @@ __device__ __forceinline__ float exp2_poly3(float x) {
   return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
 }
 
+// Backward passes: groups of four probabilities v with (v & 3) >= kBwdPolyFrom
+// take exp2_poly3 on the FMA pipe instead of the MUFU unit (4: none), so that the
+// exponentials of a step do not all queue on the MUFU unit.
+#ifndef FA2_BWD_POLY_FROM
+#define FA2_BWD_POLY_FROM 4
+#endif
+constexpr int kBwdPolyFrom = FA2_BWD_POLY_FROM;
+
 // Packs two fp32 values into a 32-bit pair of 16-bit values (round to nearest
 // even); ``lo`` goes to the low half.
 template <bool BF16>
@@ -520,6 +529,19 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
     asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   }
   return r;
+}
+
+// The two 16-bit values of a 32-bit pair as floats (exact); the low half first.
+template <bool BF16>
+__device__ __forceinline__ void unpack2(uint32_t v, float& lo, float& hi) {
+  if constexpr (BF16) {
+    lo = __uint_as_float(v << 16);
+    hi = __uint_as_float(v & 0xFFFF0000u);
+  } else {
+    const __half2 h = *reinterpret_cast<const __half2*>(&v);
+    lo = __low2float(h);
+    hi = __high2float(h);
+  }
 }
 
 // Four floats as E4M3 bytes (round to nearest even, saturating to +-448), p0 in

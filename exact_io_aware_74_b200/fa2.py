@@ -25,12 +25,15 @@ FA2_ERR_TIMEOUT = 5
 FA2_ERR_WORKSPACE = 6
 FA2_FP16 = 0
 FA2_BF16 = 1
+FA2_BWD_DETERMINISTIC = 1  # flag of fa2_bwd_ex
 
 # Every symbol include/fa2.h declares.
 EXPORTS = ("fa2_fwd", "fa2_fwd_window", "fa2_fwd_fp8", "fa2_fwd_tiles_per_cta",
-           "fa2_fwd_decode_splits", "fa2_fwd_decode_workspace_size", "fa2_fwd_decode", "fa2_bwd_workspace_size", "fa2_bwd", "fa2_bwd_window",
-           "fa2_bwd_noalloc", "fa2_get_device_status", "fa2_status_string", "fa2_debug_set",
-           "fa2_debug_set_bwd_grid", "fa2_debug_set_fwd_tiles", "fa2_launch_count")
+           "fa2_fwd_decode_splits", "fa2_fwd_decode_workspace_size", "fa2_fwd_decode",
+           "fa2_bwd_workspace_size", "fa2_bwd", "fa2_bwd_window", "fa2_bwd_ex",
+           "fa2_bwd_ex_workspace_size", "fa2_bwd_noalloc", "fa2_get_device_status",
+           "fa2_status_string", "fa2_debug_set", "fa2_debug_set_bwd_grid",
+           "fa2_debug_set_fwd_tiles", "fa2_launch_count")
 
 _lib = None
 
@@ -71,6 +74,10 @@ def load() -> ctypes.CDLL:
     lib.fa2_bwd_workspace_size.restype = sz
     lib.fa2_bwd.argtypes = [vp] * 10 + [sz, i, i, i, i, f, i, i, vp]
     lib.fa2_bwd.restype = i
+    lib.fa2_bwd_ex.argtypes = [vp] * 10 + [sz, i, i, i, i, f, i, i, i, i, vp]
+    lib.fa2_bwd_ex.restype = i
+    lib.fa2_bwd_ex_workspace_size.argtypes = [i, i, i, i, i]
+    lib.fa2_bwd_ex_workspace_size.restype = sz
     lib.fa2_bwd_noalloc.argtypes = [vp] * 9 + [i, i, i, i, f, i, i, vp]
     lib.fa2_bwd_noalloc.restype = i
     lib.fa2_get_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_int)]
@@ -206,6 +213,22 @@ def fa2_bwd(q, k, v, o, do, lse, dq, dk, dv, workspace, scale: float, causal: bo
                           int(bool(causal)), _dtype_code(q), _stream(stream))
 
 
+def fa2_bwd_ex_workspace_size(B: int, H: int, N: int, d: int, flags: int) -> int:
+    return int(load().fa2_bwd_ex_workspace_size(B, H, N, d, int(flags)))
+
+
+def fa2_bwd_ex(q, k, v, o, do, lse, dq, dk, dv, workspace, scale: float, causal: bool,
+               window: int = 0, flags: int = 0, stream=None) -> int:
+    """Raw call of the backward with options (window, FA2_BWD_DETERMINISTIC)."""
+    _check_layout(q, k, v, o, do, lse, dq, dk, dv)
+    B, H, N, d = q.shape
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    return load().fa2_bwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse), _ptr(dq),
+                             _ptr(dk), _ptr(dv), _ptr(workspace), ws_bytes, B, H, N, d,
+                             float(scale), int(bool(causal)), int(window), int(flags),
+                             _dtype_code(q), _stream(stream))
+
+
 def fa2_bwd_noalloc(q, k, v, o, do, lse, dq, dk, dv, scale: float, causal: bool,
                     stream=None) -> int:
     """Raw call of the allocation-free backward (library-owned scratch).  Returns the status."""
@@ -312,14 +335,23 @@ def backward_window(q, k, v, o, do, lse, scale: float, window: int, stream=None)
     return dq, dk, dv
 
 
-def backward(q, k, v, o, do, lse, scale: float, causal: bool, workspace=None, stream=None):
-    """Allocates dQ, dK, dV (and the workspace if not given), calls fa2_bwd."""
+def backward(q, k, v, o, do, lse, scale: float, causal: bool, workspace=None, stream=None,
+             deterministic: bool = False, window: int = 0):
+    """Allocates dQ, dK, dV (and the workspace if not given), calls fa2_bwd, or
+    fa2_bwd_ex when ``deterministic`` or a ``window`` is asked for."""
     B, H, N, d = q.shape
+    flags = FA2_BWD_DETERMINISTIC if deterministic else 0
     if workspace is None:
-        workspace = torch.empty(fa2_bwd_workspace_size(B, H, N, d), dtype=torch.uint8,
+        workspace = torch.empty(fa2_bwd_ex_workspace_size(B, H, N, d, flags), dtype=torch.uint8,
                                 device=q.device)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-    rc = fa2_bwd(q, k, v, o, do, lse, dq, dk, dv, workspace, scale, causal, stream)
+    if flags or window:
+        rc = fa2_bwd_ex(q, k, v, o, do, lse, dq, dk, dv, workspace, scale, causal, window, flags,
+                        stream)
+        where = "fa2_bwd_ex"
+    else:
+        rc = fa2_bwd(q, k, v, o, do, lse, dq, dk, dv, workspace, scale, causal, stream)
+        where = "fa2_bwd"
     if rc != FA2_OK:
-        raise FA2Error(rc, "fa2_bwd")
+        raise FA2Error(rc, where)
     return dq, dk, dv

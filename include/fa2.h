@@ -199,7 +199,8 @@ size_t fa2_bwd_workspace_size(int B, int H, int N, int d);
  *                    256-byte aligned, owned by the caller; its contents on
  *                    entry do not matter and on return are unspecified
  * Other arguments as for fa2_fwd.  dQ is accumulated with float atomics, so it
- * may differ in the last bits from run to run; dK and dV are repeatable.
+ * may differ in the last bits from run to run; dK and dV are repeatable (see
+ * fa2_bwd_ex with FA2_BWD_DETERMINISTIC for a bitwise repeatable dQ).
  */
 int fa2_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO,
             const float* LSE, void* dQ, void* dK, void* dV, void* workspace,
@@ -215,6 +216,38 @@ int fa2_bwd_window(const void* Q, const void* K, const void* V, const void* O, c
                    const float* LSE, void* dQ, void* dK, void* dV, void* workspace,
                    size_t workspace_bytes, int B, int H, int N, int d, float scale, int window,
                    int dtype, fa2_stream_t stream);
+
+/* Flags of fa2_bwd_ex. */
+enum { FA2_BWD_DETERMINISTIC = 1 };
+
+/*
+ * Backward pass with options: the sliding window of fa2_bwd_window (window >= 1,
+ * causal = 1; 0 = no window) and ``flags``:
+ *
+ *   FA2_BWD_DETERMINISTIC  dQ, dK and dV bitwise repeatable run to run.  Source:
+ *     [RU] "Производительность и эффективность" (the method stays exact and
+ *     deterministic).  dQ is then computed by a query-stationary kernel that
+ *     recomputes the scores and dP and sums dQ over the key tiles in tensor memory
+ *     in a fixed order, instead of adding key-tile partials into a float
+ *     accumulator in global memory (whose order of addition varies); dK and dV
+ *     come from a kernel without the dQ product.  Seven matrix products per tile
+ *     pair instead of five, on 128-wide tiles at every head dim: measured on B200
+ *     about 7 % slower than the default at d = 128, about twice the time at d = 64.
+ *     The workspace holds only the two per-row statistics.
+ *
+ * Arguments, layouts, results and errors otherwise as fa2_bwd (and
+ * fa2_bwd_window); flags other than FA2_BWD_DETERMINISTIC, window < 0 or a window
+ * with causal = 0 return FA2_ERR_INVALID_ARG.  The workspace must hold
+ * fa2_bwd_ex_workspace_size(B, H, N, d, flags) bytes.
+ */
+int fa2_bwd_ex(const void* Q, const void* K, const void* V, const void* O, const void* dO,
+               const float* LSE, void* dQ, void* dK, void* dV, void* workspace,
+               size_t workspace_bytes, int B, int H, int N, int d, float scale, int causal,
+               int window, int flags, int dtype, fa2_stream_t stream);
+
+/* Bytes of workspace fa2_bwd_ex needs with ``flags`` (0 for sizes or flags it
+ * rejects); without flags, fa2_bwd_workspace_size. */
+size_t fa2_bwd_ex_workspace_size(int B, int H, int N, int d, int flags);
 
 /*
  * Allocation-free backward.  The paper has no counterpart: this entry point

@@ -84,11 +84,18 @@ def test_fwd_overlap_checks_use_each_buffer_size(lib):
 def test_bwd_validation_without_device(lib):
     ws = fa2.fa2_bwd_workspace_size(2, 3, 1000, 128)
     assert ws > 0 and ws % 256 == 0
-    # D and LSE*log2(e) padded to 128 rows per head, then the fp32 dQ accumulator
-    assert ws >= 2 * 3 * 1000 * 128 * 4
+    # D and LSE*log2(e) padded to 128 rows per head, then the fp32 dQ accumulator, as
+    # wide as the kernel's tile (64 or 128 columns)
+    assert ws == 2 * 2 * 3 * 1024 * 4 + 2 * 3 * 1000 * 128 * 4
+    assert fa2.fa2_bwd_workspace_size(2, 3, 1000, 64) == 2 * 2 * 3 * 1024 * 4 + 2 * 3 * 1000 * 64 * 4
+    # the deterministic mode keeps the two row statistics only
+    assert fa2.fa2_bwd_ex_workspace_size(2, 3, 1000, 128, fa2.FA2_BWD_DETERMINISTIC) == 2 * 2 * 3 * 1024 * 4
+    assert fa2.fa2_bwd_ex_workspace_size(2, 3, 1000, 64, fa2.FA2_BWD_DETERMINISTIC) == 2 * 2 * 3 * 1024 * 4
+    assert fa2.fa2_bwd_ex_workspace_size(2, 3, 1000, 128, 0) == ws
+    assert fa2.fa2_bwd_ex_workspace_size(2, 3, 1000, 128, 2) == 0  # unknown flag
     assert fa2.fa2_bwd_workspace_size(2, 3, 1000, 100) == 0  # d % 8 != 0
     assert fa2.fa2_bwd_workspace_size(2, 3, 1000, 136) == 0  # backward head dims end at 128
-    # d = 96 runs on 128-wide tiles: the fp32 dQ accumulator has 128 columns
+    # d = 96 runs on 128-wide tiles
     assert fa2.fa2_bwd_workspace_size(2, 3, 1000, 96) == fa2.fa2_bwd_workspace_size(2, 3, 1000, 128)
     assert fa2.fa2_bwd_workspace_size(2, 3, 1000, 8) == fa2.fa2_bwd_workspace_size(2, 3, 1000, 64)
     ptrs = [P * (i + 1) for i in range(9)]
@@ -292,7 +299,8 @@ def test_forward_tiles_per_cta_rejects_bad_sizes(lib):
 # needs memory linear in the sequence length, because no N x N matrix is stored.
 # The forward takes no scratch at all; the backward's scratch is two float rows per
 # query (D and LSE * log2 e, padded to 128 rows) and a float dQ accumulator of one
-# row per query, as wide as the kernel's tile (64 or 128 columns).
+# row per query, as wide as the kernel's tile (64 or 128 columns); the deterministic
+# mode, which sums dQ in tensor memory, needs the two rows alone.
 
 @pytest.mark.parametrize("d", [32, 64, 96, 128])
 def test_bwd_workspace_is_linear_in_sequence_length(lib, d):
@@ -303,6 +311,29 @@ def test_bwd_workspace_is_linear_in_sequence_length(lib, d):
         rows = B * H * ((N + 127) // 128 * 128)
         expect = (2 * rows * 4 + 255) // 256 * 256 + (B * H * N * tile * 4 + 255) // 256 * 256
         assert ws == expect
+        assert lib.fa2_bwd_ex_workspace_size(B, H, N, d, 1) == (2 * rows * 4 + 255) // 256 * 256
         # O(B H N d): at most 8 bytes per head element plus the row statistics
         assert ws <= B * H * N * (8 * d) + 2 * rows * 4 + 512
         assert lib.fa2_bwd_workspace_size(B, H, 2 * N, d) == 2 * ws  # doubles with N
+
+
+def test_noalloc_rejects_sizes_beyond_its_buffer_before_any_device_call(lib):
+    # the training shape (8 x 16 heads of 4096 rows, d = 128) needs 258 MiB of scratch
+    B, H, N, d = 8, 16, 4096, 128
+    assert lib.fa2_bwd_workspace_size(B, H, N, d) > (32 << 20) - 256
+    far = 1 << 33  # fake pointers 8 GiB apart: the tensors do not overlap
+    ptrs = [far * (i + 1) for i in range(9)]
+    assert lib.fa2_bwd_noalloc(*ptrs, B, H, N, d, 0.1, 0, 1, None) == fa2.FA2_ERR_WORKSPACE
+
+
+def test_bwd_ex_validation_without_device(lib):
+    ptrs = [P * (i + 1) for i in range(9)]
+    ws = fa2.fa2_bwd_ex_workspace_size(1, 1, 64, 64, fa2.FA2_BWD_DETERMINISTIC)
+    # unknown flag, negative window, a window without causal
+    assert lib.fa2_bwd_ex(*ptrs, 16 * P, ws, 1, 1, 64, 64, 0.1, 1, 0, 2, 1, None) == fa2.FA2_ERR_INVALID_ARG
+    assert lib.fa2_bwd_ex(*ptrs, 16 * P, ws, 1, 1, 64, 64, 0.1, 1, -1, 1, 1, None) == fa2.FA2_ERR_INVALID_ARG
+    assert lib.fa2_bwd_ex(*ptrs, 16 * P, ws, 1, 1, 64, 64, 0.1, 0, 8, 1, 1, None) == fa2.FA2_ERR_INVALID_ARG
+    # the deterministic mode's workspace is the smaller one; too small is still rejected
+    assert lib.fa2_bwd_ex(*ptrs, 16 * P, ws - 256, 1, 1, 64, 64, 0.1, 1, 0, 1, 1, None) == fa2.FA2_ERR_WORKSPACE
+    # head dims end at 128 in both modes
+    assert lib.fa2_bwd_ex(*ptrs, 16 * P, 1 << 20, 1, 1, 64, 136, 0.1, 1, 0, 1, 1, None) == fa2.FA2_ERR_UNSUPPORTED

@@ -78,7 +78,7 @@ def test_bwd_dk_dv_repeatable_and_dq_close():
     runs = [_gpu_fwd_bwd(x, 0.1, True) for _ in range(3)]
     for dq, dk, dv in runs[1:]:
         assert torch.equal(dk, runs[0][1]) and torch.equal(dv, runs[0][2])
-        # dQ sums fp32 partials with atomics: order may change the last bits only
+        # dQ sums fp32 partials with bulk reductions: order may change the last bits only
         assert torch.max(torch.abs(dq.float() - runs[0][0].float())) <= 1e-2 * torch.max(
             torch.abs(runs[0][0].float()))
 

@@ -37,8 +37,8 @@ def _grad_check(got, ref):
 
 
 @pytest.mark.parametrize("d", [64, 128])
-@pytest.mark.parametrize("noalloc", [False, True])
-def test_bwd_timeout_path_reports_and_recovers(d, noalloc):
+@pytest.mark.parametrize("mode", ["default", "noalloc", "deterministic"])
+def test_bwd_timeout_path_reports_and_recovers(d, mode):
     B, H, N = 1, 2, 300
     x = make_inputs(B, H, N, d, "bf16", seed=9500 + d, with_do=True)
     s = 1 / math.sqrt(d)
@@ -48,8 +48,11 @@ def test_bwd_timeout_path_reports_and_recovers(d, noalloc):
     ws = torch.empty(fa2.fa2_bwd_workspace_size(B, H, N, d), dtype=torch.uint8, device="cuda")
 
     def call():
-        if noalloc:
+        if mode == "noalloc":
             return fa2.fa2_bwd_noalloc(q, k, v, o, do, lse, dq, dk, dv, s, True)
+        if mode == "deterministic":
+            return fa2.fa2_bwd_ex(q, k, v, o, do, lse, dq, dk, dv, ws, s, True, 0,
+                                  fa2.FA2_BWD_DETERMINISTIC)
         return fa2.fa2_bwd(q, k, v, o, do, lse, dq, dk, dv, ws, s, True)
 
     rc, status, site = _with_fault(call)

@@ -53,7 +53,7 @@ def _noalloc_matches_backward(name):
     rc = fa2.fa2_bwd_noalloc(q, k, v, o, do, lse, *got, scale, causal)
     assert rc == fa2.FA2_OK, fa2.status_string(rc)
     assert fa2.fa2_get_device_status() == (fa2.FA2_OK, 0)
-    assert fa2.fa2_launch_count() - before == 3
+    assert fa2.fa2_launch_count() - before == 3  # the kernels of one fa2_bwd call
     for g, r in zip(got, ref):
         assert torch.isfinite(g.float()).all()
         assert _close(g, r)
@@ -73,7 +73,7 @@ def test_noalloc_backward_matches_backward_twice(first, second):
 
 
 def test_noalloc_backward_rejects_sizes_beyond_its_buffer():
-    B, H, N, d = 1, 8, 8192, 128  # needs ~32.3 MiB of scratch
+    B, H, N, d = 1, 8, 16384, 64  # needs ~32.5 MiB of scratch (the dQ accumulator)
     assert fa2.fa2_bwd_workspace_size(B, H, N, d) > (32 << 20) - 256
     q = torch.zeros(B, H, N, d, dtype=torch.bfloat16, device="cuda")
     k, v, o, do, dq, dk, dv = (torch.zeros_like(q) for _ in range(7))
