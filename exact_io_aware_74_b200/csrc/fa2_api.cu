@@ -320,6 +320,22 @@ int fwd_core(const void* Q, const void* K, const void* V, void* O, float* LSE, i
   p.off = Nk - Nq;
   p.BH = BH;
   p.n_qblk = static_cast<int>(n_qblk);
+  p.head_group = BH;
+  if (n_split == 1 && window == 0) {
+    // Heads per group of the block order: a group spans about two waves of CTAs
+    // (one CTA per SM), so that the CTAs running together share a few heads.
+    // Measured on B200: headline shape 2.135 -> 2.022 ms, long-context causal 9.15 ->
+    // 8.77 ms, training shape 0.654 -> 0.648 ms; sliding windows (whose blocks read
+    // only their window's keys) 0.397 -> 0.410 ms, so they keep the plain order.
+    int dev_sm = 0;
+    if (cudaDeviceGetAttribute(&dev_sm, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess &&
+        dev_sm > 0) {
+      const long long hg = (2LL * dev_sm + n_qblk - 1) / n_qblk;
+      p.head_group = static_cast<int>(std::min<long long>(BH, std::max<long long>(1, hg)));
+    } else {
+      cudaGetLastError();
+    }
+  }
   p.scale_log2 = scale * 1.4426950408889634f;
   p.status = st;
   p.wait_ns = wait_ns();
@@ -550,6 +566,7 @@ int fa2_fwd_fp8(const void* Q, const void* K, const void* V, void* O, float* LSE
   p.BH = BH;
   if (static_cast<long long>((N + 255) / 256) * BH > 0x7fffffffll) return FA2_ERR_INVALID_ARG;
   p.n_qblk = (N + 255) / 256;
+  p.head_group = BH;
   p.scale_log2 = sl2;
   p.status = st;
   p.wait_ns = wait_ns();

@@ -65,6 +65,7 @@ struct FwdParams {
   int off;                     // causal only: query row i sees keys <= i + off (Nk - Nq)
   int BH;                      // batch * heads
   int n_qblk;                  // ceil(Nq / (128 QT)): query blocks per (batch, head)
+  int head_group;              // heads per group of the block order (1 .. BH)
   float scale_log2;            // scale * log2(e)
   unsigned int* status;        // device status word
   unsigned long long wait_ns;  // budget of one bounded wait
@@ -186,9 +187,18 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   const bool split = p.kv_per_split > 0;    // keys cut into stretches (blockIdx.y)
   const bool partial = p.O_part != nullptr;  // partial results, merged by a second kernel
 
-  // Heaviest query blocks first (they see the most keys when causal).
-  const int qb = p.n_qblk - 1 - static_cast<int>(blockIdx.x) / p.BH;
-  const int bh = static_cast<int>(blockIdx.x) % p.BH;
+  // Block order: head group by head group (head_group heads each, the last group
+  // possibly smaller), and within a group the heaviest query blocks first (they
+  // see the most keys when causal).  A group spans about two waves of CTAs, so the
+  // CTAs running at any one time share a few heads and their K and V tiles come
+  // from L2 (head_group = BH orders every head's blocks together).
+  const int qb_bh_x = static_cast<int>(blockIdx.x);
+  const int grp_blocks = p.head_group * p.n_qblk;
+  const int hgrp = qb_bh_x / grp_blocks;
+  const int hpos = qb_bh_x - hgrp * grp_blocks;
+  const int hcnt = min(p.head_group, p.BH - hgrp * p.head_group);
+  const int qb = p.n_qblk - 1 - hpos / hcnt;
+  const int bh = hgrp * p.head_group + hpos % hcnt;
   const int n_kv_all = (Nk + C::BN - 1) / C::BN;
   // Key tiles of this CTA's split (all of them when the keys are not split).
   const int s_lo = split ? static_cast<int>(blockIdx.y) * p.kv_per_split : 0;
