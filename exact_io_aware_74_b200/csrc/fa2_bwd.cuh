@@ -1164,11 +1164,19 @@ int launch_bwd_t(const void* Q, const void* K, const void* V, const void* O, con
     }
     long long ctas = std::min(static_cast<long long>(bp.n_kv) * BH, static_cast<long long>(n_sm));
     if (max_ctas > 0) ctas = std::min(ctas, static_cast<long long>(max_ctas));
-    // Heads per group: a group of the tile list spans about two rounds of the snake.
-    // Measured on B200 (every head at once -> groups): training-shape backward 2.08 ->
-    // 1.87 ms, its deterministic mode 2.30 -> 2.20 ms, sliding window 1.08 -> 1.05 ms.
-    bp.head_group = static_cast<int>(
-        std::min<long long>(BH, std::max<long long>(1, (2 * ctas + bp.n_kv - 1) / bp.n_kv)));
+    // Heads per group: a group of the tile list spans about two rounds of the snake,
+    // but holds at most ~32 MB of K, V, Q, dO (16-bit) and fp32 dQ rows.  Measured on
+    // B200 (every head at once -> groups of two rounds): training-shape backward 2.08
+    // -> 1.87 ms, its deterministic mode 2.30 -> 2.20 ms, sliding window 1.08 -> 1.05
+    // ms; groups of one round: training shape 1.83 ms but the d = 64 bench-shape
+    // backward 72.7 -> 80.9 us -- the 32 MB cap gives the training shape the smaller
+    // groups (5 heads) and leaves that shape's (37) alone.
+    {
+      long long hg = (2 * ctas + bp.n_kv - 1) / bp.n_kv;
+      const long long per_head = 12LL * N * D;  // bytes of one head's rows (see above)
+      hg = std::min(hg, (32LL << 20) / per_head);
+      bp.head_group = static_cast<int>(std::min<long long>(BH, std::max<long long>(1, hg)));
+    }
     const unsigned int grid = static_cast<unsigned int>(ctas);
     if (launch_pdl(kern, dim3(grid), dim3(Cfg::THREADS), Cfg::SMEM, stream, mq, mk, mv, mdo, mdq,
                    bp) != cudaSuccess)
