@@ -88,7 +88,8 @@ def input_bytes(w) -> int:
 
 
 # Device sources of each C-ABI call's kernels.
-KERNEL_SOURCES = {"fa2_fwd": ("ptx.cuh", "fa2_fwd.cuh"), "fa2_bwd": ("ptx.cuh", "fa2_bwd.cuh"),
+KERNEL_SOURCES = {"fa2_fwd": ("ptx.cuh", "fa2_fwd.cuh"),
+                  "fa2_bwd": ("ptx.cuh", "fa2_bwd.cuh", "fa2_bwd_dq.cuh"),
                   "fa2_fwd_decode": ("ptx.cuh", "fa2_fwd.cuh", "fa2_decode.cuh")}
 
 
