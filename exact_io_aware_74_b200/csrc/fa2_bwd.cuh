@@ -205,12 +205,16 @@ struct BwdCfg {
   // Software-pipelined steps with the dQ product: at D = 64, where TMEM has room.
   static constexpr bool PIPE = DQ && D == 64;
   static constexpr int DS_BYTES = DQ ? 128 * 128 * 2 : 0;  // dS^T in shared memory, for dQ
-  // Q tiles: in the (Q, dO) ring at tile width 64; a ring of their own at 128, one
-  // stage deeper than dO's, released by dK (their last reader) -- the next step's
-  // scores are issued as soon as this step's have been read, so the next Q must
-  // already be resident then, while dO is first needed later, by dP^T.
+  // Q tiles: in the (Q, dO) ring at tile width 64; a ring of their own at 128,
+  // released by dK (their last reader).  Without dQ that ring is one stage deeper
+  // than dO's: the next step's scores are issued as soon as this step's have been
+  // read, so the next Q must already be resident then, while dO is first needed
+  // later, by dP^T.  With dQ (D = 128) the dO tile of a step is released later than
+  // its Q: it doubles as a staging tile of the step's dQ reduce (see the drain).
   static constexpr int QS = DQ ? ST : 3;
-  static constexpr int LD_BYTES = ST * 2 * 128 * 4;  // LSE*log2e and D rows of each stage
+  // LSE*log2e and D rows of each stage: loaded with Q in the fused D = 128 kernel,
+  // with dO otherwise.
+  static constexpr int LD_BYTES = ST * 2 * 128 * 4;
   static constexpr int CTRL_BYTES = 256;              // barriers, TMEM address, abort flag
   // No alignment slack: the dynamic region must start 1024-byte aligned (checked).
   static constexpr int SMEM = (2 * KVB + QS + ST) * TILE + DS_BYTES + LD_BYTES + CTRL_BYTES;
@@ -358,7 +362,10 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       mbar_init(&kv_empty[b], 1);
     }
     mbar_init(&acc_free, 8);
-    for (int s = 0; s < C::ST; ++s) { mbar_init(&qdo_full[s], 1); mbar_init(&qdo_empty[s], 1); }
+    for (int s = 0; s < C::ST; ++s) {
+      mbar_init(&qdo_full[s], 1);
+      mbar_init(&qdo_empty[s], (C::DQ && !C::PIPE) ? 2 : 1);
+    }
     for (int s = 0; s < 3; ++s) { mbar_init(&q_full[s], 1); mbar_init(&q_empty[s], 1); }
     mbar_init(&s_full, 1);
     mbar_init(&dp_full, 1);
@@ -422,7 +429,7 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         for (int it = 0; it < n_it; ++it) {
           const int st = gs % C::ST;
           const int row = (i0 + it) * 128;
-          if constexpr (!C::DQ) {
+          if constexpr (!C::PIPE) {
             // Q in a ring of its own (released by dK), loaded before this step's dO.
             const int qs = gs % C::QS;
             if (gs >= C::QS &&
@@ -430,7 +437,12 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
               ok = false;
               break;
             }
-            mbar_arrive_expect_tx(&q_full[qs], C::TILE);
+            mbar_arrive_expect_tx(&q_full[qs], C::TILE + (C::DQ ? 2 * 512 : 0));
+            if constexpr (C::DQ) {
+              const size_t stq = static_cast<size_t>(bh) * p.Npad + row;
+              bulk_load_1d(sLD + qs * 256, p.Lg + stq, 512, &q_full[qs]);
+              bulk_load_1d(sLD + qs * 256 + 128, p.Dg + stq, 512, &q_full[qs]);
+            }
             for (int c = 0; c < C::KCH; ++c)
               tma_load_3d_hint(sQ + qs * C::TILE + c * C::CHUNK, &tmQ, &q_full[qs], c * 64, row, bh,
                                keep);
@@ -441,12 +453,15 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&qdo_full[st], (C::DQ ? 2 : 1) * C::TILE + 2 * 512);
-          const size_t stat = static_cast<size_t>(bh) * p.Npad + row;
-          bulk_load_1d(sLD + st * 256, p.Lg + stat, 512, &qdo_full[st]);
-          bulk_load_1d(sLD + st * 256 + 128, p.Dg + stat, 512, &qdo_full[st]);
+          constexpr bool LD_WITH_Q = C::DQ && !C::PIPE;
+          mbar_arrive_expect_tx(&qdo_full[st], (C::PIPE ? 2 : 1) * C::TILE + (LD_WITH_Q ? 0 : 2 * 512));
+          if constexpr (!LD_WITH_Q) {
+            const size_t stat = static_cast<size_t>(bh) * p.Npad + row;
+            bulk_load_1d(sLD + st * 256, p.Lg + stat, 512, &qdo_full[st]);
+            bulk_load_1d(sLD + st * 256 + 128, p.Dg + stat, 512, &qdo_full[st]);
+          }
           for (int c = 0; c < C::KCH; ++c) {
-            if constexpr (C::DQ)
+            if constexpr (C::PIPE)
               tma_load_3d_hint(sQ + st * C::TILE + c * C::CHUNK, &tmQ, &qdo_full[st], c * 64, row,
                                bh, keep);
             tma_load_3d_hint(sdO + st * C::TILE + c * C::CHUNK, &tmdO, &qdo_full[st], c * 64,
@@ -477,7 +492,7 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       if (!ok) {
         for (int q = max(0, gs - C::ST); q < gs; ++q)
           mbar_wait(&qdo_full[q % C::ST], (q / C::ST) & 1, dw, kBSiteProdDrain);
-        if constexpr (!C::DQ) {
+        if constexpr (!C::PIPE) {
           for (int q = max(0, gq - C::QS); q < gq; ++q)
             mbar_wait(&q_full[q % C::QS], (q / C::QS) & 1, dw, kBSiteProdDrain);
         }
@@ -526,7 +541,9 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         for (int kk = 0; kk < 8; ++kk)
           umma_ts(tbase + C::C_DV, tbase + C::C_P(kk >> 2) + (kk & 3) * 8,
                   sdesc_add(mdO, st * C::TILE + kk * 2048), id_tb, (!first || kk > 0) ? 1u : 0u);
-        // Tile width 128: dV is dO's last reader (its L, D rows were read before ds_ready).
+        // Without dQ, dV is dO's last reader (its L, D rows were read before
+        // ds_ready).  With dQ at D = 128 the compute warpgroups release dO instead,
+        // once the dQ reduce staged in its tile has been read.
         if constexpr (!C::DQ) umma_commit(&qdo_empty[st]);
       };
       auto mma_dq = [&](uint32_t kvo) {  // dQ_i = dS K
@@ -543,7 +560,7 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         for (int kk = 0; kk < 8; ++kk)
           umma_ts(tbase + C::C_DK, tbase + C::C_DS(kk >> 2) + (kk & 3) * 8,
                   sdesc_add(mQ, qs * C::TILE + kk * 2048), id_tb, (!first || kk > 0) ? 1u : 0u);
-        umma_commit(C::DQ ? &qdo_empty[qs] : &q_empty[qs]);
+        umma_commit(C::PIPE ? &qdo_empty[qs] : &q_empty[qs]);
       };
       bool ok = true;
       int gs = 0;  // query steps so far
@@ -560,13 +577,15 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           // is drained), dV (P^T ready), dQ and dK (dS^T ready).
           for (int it = 0; it < n_it; ++it, ++gs) {
             const int st = gs % C::ST;
-            if (!mbar_wait(&qdo_full[st], (gs / C::ST) & 1, wc, kBSiteMmaQ)) { ok = false; break; }
+            if (!mbar_wait(&q_full[st], (gs / C::QS) & 1, wc, kBSiteMmaQ)) { ok = false; break; }
             tc_fence_after();
             mma_s(st, kvo);
             if (gs > 0) {
               if (!mbar_wait(&dq_drained, (gs - 1) & 1, wc, kBSiteMmaDrained)) { ok = false; break; }
               tc_fence_after();
             }
+            if (!mbar_wait(&qdo_full[st], (gs / C::ST) & 1, wc, kBSiteMmaQ)) { ok = false; break; }
+            tc_fence_after();
             mma_dp(st, kvo);
             if (!mbar_wait(&p_ready, gs & 1, wc, kBSiteMmaP)) { ok = false; break; }
             tc_fence_after();
@@ -695,10 +714,13 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     // must never be left waiting).
     auto stage_p = [&](int gp, int ip, int j, int key) -> bool {
       const int stp = gp % C::ST;
-      // The tile's LSE*log2e and D rows arrive in shared memory with Q_i and dO_i.
+      // The step's LSE*log2e and D rows arrive in shared memory with Q_i (fused
+      // D = 128 kernel) or with dO_i.
       const float4* L4 = reinterpret_cast<const float4*>(sLD + stp * 256 + qoff);
-      if (!named_bar_and(wg_bar, 128, mbar_wait(&qdo_full[stp], (gp / C::ST) & 1, wc, kBSiteCmpQ)))
-        return false;
+      constexpr bool LD_WITH_Q = C::DQ && !C::PIPE;
+      uint64_t* ld_full = LD_WITH_Q ? &q_full[gp % C::QS] : &qdo_full[stp];
+      const uint32_t ld_par = static_cast<uint32_t>((gp / (LD_WITH_Q ? C::QS : C::ST)) & 1);
+      if (!named_bar_and(wg_bar, 128, mbar_wait(ld_full, ld_par, wc, kBSiteCmpQ))) return false;
       if (!named_bar_and(wg_bar, 128, mbar_wait(&s_full, gp & 1, wc, kBSiteCmpS))) return false;
       tc_fence_after();
       // P^T (this warpgroup's 64 query columns): exp2(S^T * scale * log2e - LSE * log2e),
@@ -814,9 +836,14 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         return true;
       }
       if (C::DQ && gd > 0) {
-        // This warpgroup's dS^T chunk doubled as the staging tile of the previous
-        // dQ reduce: that bulk copy must have finished reading it.
-        if (r == 0) tma_store_wait_read();
+        // This warpgroup's dS^T chunk (and, at D = 128, its half of the previous
+        // step's dO tile) held the previous step's dQ reduce: the bulk copies must
+        // have finished reading it.  At D = 128 the dO tile then goes back to the
+        // producer.
+        if (r == 0) {
+          tma_store_wait_read();
+          if constexpr (!C::PIPE) mbar_arrive(&qdo_empty[(gd - 1) % C::ST]);
+        }
         named_bar_sync(wg_bar, 128);
       }
 #pragma unroll
@@ -860,11 +887,11 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     auto stage_dq = [&](int gq, int iq, int bh) -> bool {
       if (!named_bar_and(wg_bar, 128, mbar_wait(&dq_full, gq & 1, wc, kBSiteCmpDQ))) return false;
       tc_fence_after();
-      // dQ partial, head columns g D/2 .. (g+1) D/2 - 1, 32 at a time: TMEM ->
-      // this warpgroup's dS^T chunk of shared memory (free: the dQ product that
-      // read it has completed), laid out as a 128-row x 32-float tile with
-      // 128-byte swizzle -> one TMA reduce-add into the fp32 accumulator (rows
-      // past N are clipped by the tensor map).
+      // dQ partial, head columns g D/2 .. (g+1) D/2 - 1, in 32-column tiles: TMEM ->
+      // shared memory, laid out as a 128-row x 32-float tile with 128-byte swizzle
+      // -> one TMA reduce-add per tile into the fp32 accumulator (rows past N are
+      // clipped by the tensor map).  The first tile goes to this warpgroup's dS^T
+      // chunk (free: the dQ product that read it has completed).
       constexpr int HALF = D / 2;
       constexpr int NCH = HALF / 32;
       uint8_t* stage = sDS + g * C::CHUNK;
@@ -897,7 +924,12 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         __syncwarp();
       } else {
         // All of this warpgroup's TMEM columns first, so that the region is released
-        // (dq_drained) before any staging starts.
+        // (dq_drained) before any staging starts.  The second tile goes to this
+        // warpgroup's half of the step's dO tile (dP^T and dV, its readers, have
+        // completed before dQ; the producer reloads it only after the next step's
+        // release), so that both reduces leave together: with a single staging tile
+        // the second would wait for the first to be read (~1.4k cycles when every SM
+        // is adding into L2).
         uint32_t qr[NCH][32];
 #pragma unroll
         for (int c = 0; c < NCH; ++c)
@@ -908,24 +940,23 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&dq_drained);
+        static_assert(NCH == 2, "two staging tiles");
+        uint8_t* stg[2] = {stage, sdO + (gq % C::ST) * C::TILE + g * C::CHUNK};
 #pragma unroll
         for (int c = 0; c < NCH; ++c) {
-          if (c > 0) {
-            if (r == 0) tma_store_wait_read();
-            named_bar_sync(wg_bar, 128);
-          }
 #pragma unroll
           for (int u = 0; u < 8; ++u)
-            *reinterpret_cast<uint4*>(stage + r * 128 + ((u ^ (r & 7)) << 4)) =
+            *reinterpret_cast<uint4*>(stg[c] + r * 128 + ((u ^ (r & 7)) << 4)) =
                 make_uint4(qr[c][4 * u], qr[c][4 * u + 1], qr[c][4 * u + 2], qr[c][4 * u + 3]);
-          fence_proxy_async_smem();
-          named_bar_sync(wg_bar, 128);
-          if (r == 0) {
-            tma_reduce_add_3d(&tmdQ, stage, g * HALF + 32 * c, iq * 128, bh);
-            tma_store_commit();
-          }
-          __syncwarp();
         }
+        fence_proxy_async_smem();
+        named_bar_sync(wg_bar, 128);
+        if (r == 0) {
+          tma_reduce_add_3d(&tmdQ, stg[0], g * HALF, iq * 128, bh);
+          tma_reduce_add_3d(&tmdQ, stg[1], g * HALF + 32, iq * 128, bh);
+          tma_store_commit();
+        }
+        __syncwarp();
       }
       return true;
     };

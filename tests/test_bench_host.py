@@ -69,7 +69,7 @@ def test_traffic_record_requires_current_kernel_source(tmp_path, monkeypatch):
     (tmp_path / "exact_io_aware_74_b200").mkdir()
     csrc = tmp_path / "exact_io_aware_74_b200" / "csrc"
     csrc.mkdir()
-    for name in ("ptx.cuh", "fa2_fwd.cuh", "fa2_bwd.cuh"):
+    for name in sorted({n for srcs in bench.KERNEL_SOURCES.values() for n in srcs}):
         (csrc / name).write_text(name + " v1")
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     h = bench.csrc_hash("fa2_bwd")
