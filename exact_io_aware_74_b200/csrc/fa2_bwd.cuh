@@ -9,50 +9,55 @@
 //   dS = P * (dP - D),  dQ = scale dS K,  dK = scale dS^T Q.
 //
 // Kernels per call, all on the caller's stream, chained by programmatic dependent
-// launch (each reads nothing before its griddepcontrol.wait):
-//   tile width 64 (d <= 64):
+// launch (each reads nothing before its griddepcontrol.wait).  Tile width 64 for
+// d <= 64, 128 for 64 < d <= 128.
+//   default mode:
 //   1. fa2_bwd_pre_kernel  : D and LSE * log2(e) per query row (padded to a
-//                            multiple of 128 rows), and a zeroed fp32 dQ
-//                            accumulator;
-//   2. fa2_bwd_kernel      : persistent, at most one CTA per SM.  The key tiles
-//                            (128 keys, batch*head) are listed heaviest first and
-//                            dealt to the CTAs in snake order; each tile loops
-//                            over the query tiles that see its keys, and adds its
-//                            dQ partials into the accumulator;
+//                            multiple of 128 rows), a zeroed fp32 dQ accumulator
+//                            and a zeroed tile counter;
+//   2. fa2_bwd_kernel      : persistent, at most one CTA per SM, over the list of
+//                            key tiles (128 keys, batch*head; see the tile
+//                            scheduler); each tile loops over the query tiles that
+//                            see its keys, accumulates dV and dK in TMEM and adds
+//                            its dQ partials into the accumulator (TMA reduce-add);
 //   3. fa2_bwd_dq_finalise_kernel : dQ = scale * accumulator, rounded to 16 bits.
-//   tile width 128 (64 < d <= 128), where a per-step dQ product no longer fits in
-//   TMEM beside dV and dK:
-//   1. fa2_bwd_dq_kernel (fa2_bwd_dq.cuh): dQ, query-stationary, summed in TMEM;
-//                            it also writes the D and LSE * log2(e) rows;
+//   deterministic mode (tile width 128 at every d):
+//   1. fa2_bwd_dq_kernel (fa2_bwd_dq.cuh): dQ, query-stationary, summed in TMEM in a
+//                            fixed order; it also writes the D and LSE * log2(e)
+//                            rows and zeroes the tile counter;
 //   2. fa2_bwd_kernel      : as above, dK and dV only.
 //
 // Main kernel, CTA layout (320 threads):
 //   warps 0-7 two compute warpgroups g = 0, 1.  Thread r of warpgroup g owns key
 //             row r of the tile for the query columns 64 g .. 64 g + 63 of P^T
-//             and dS^T, and (tile width 64) query row r of the current query tile
-//             for the head columns 32 g .. 32 g + 31 when it moves the dQ partial
-//             from TMEM through shared memory into the fp32 accumulator (one TMA
-//             reduce-add per 128 x 32 tile).  Splitting every row between the two
-//             warpgroups halves the per-step chain P^T -> dS^T -> dQ drain that the
-//             products wait on;
+//             and dS^T, and query row r of the current query tile for the head
+//             columns g D/2 .. (g+1) D/2 - 1 when it moves the dQ partial from TMEM
+//             through shared memory into the fp32 accumulator (one TMA reduce-add
+//             per 128 x 32 tile).  Splitting every row between the two warpgroups
+//             halves the per-step chain P^T -> dS^T -> dQ drain that the products
+//             wait on;
 //   warp  8   TMA producer: K_j and V_j per tile (two buffers at D = 64, the next
-//             tile's loaded during the current one), a 2-stage ring of (Q_i, dO_i)
-//             and the tile's LSE / D rows, across the CTA's tiles;
+//             tile's loaded during the current one), the (Q_i, dO_i) tiles and LSE /
+//             D rows of each step in 2-stage rings, across the CTA's tiles;
 //   warp  9   tcgen05 MMA issuer (one thread).
-// TMEM (fp32 columns): S^T [0,128); dP^T [128,256), warpgroup g writing its packed
-// dS^T over its own dP^T columns [128 + 64 g, + 32); dV [256, 256 + D); dK
-// [256 + D, 256 + 2 D).  D = 64: dQ [384,448), packed P^T of warpgroup g at
-// [448 + 32 g, + 32).  D = 128: packed P^T of warpgroup g over its own score
-// columns [64 g, + 32), no dQ.
-// The steps are software-pipelined: the scores of step i + 1 go out right after
-// step i's dV product and its dP^T right after step i's dK product, so that the
-// next step's products overlap this step's dS.
+// TMEM (fp32 columns): S^T [0,128); dP^T [128,256); dV [256, 256 + D); dK
+// [256 + D, 256 + 2 D).
+//   D = 64: dQ [384,448); packed P^T of warpgroup g at [448 + 32 g, + 32), its dS^T
+//     over its own dP^T columns [128 + 64 g, + 32).  The steps are software-
+//     pipelined: the scores of step i + 1 go out right after step i's dV product and
+//     its dP^T right after step i's dK product, so that the next step's products
+//     overlap this step's dS.
+//   D = 128 with dQ: no free columns; packed P^T and dS^T of warpgroup g over its
+//     own score columns [64 g, + 32), [64 g + 32, + 32); the dQ partial over dP^T.
+//     Each step runs its products in order (S^T, dP^T, dV, dQ, dK).
+//   D = 128, dK/dV only: packed dS^T and P^T over warpgroup g's dP^T columns, so
+//     that step i + 1's scores run during step i's exponentials.
 // Products (M = 128 rows of the first operand, K = 16 per instruction):
 //   S^T  = K_j  Q_i^T   (A = K smem K-major, B = Q smem K-major)
 //   dP^T = V_j  dO_i^T  (A = V smem K-major, B = dO smem K-major)
 //   dV  += P^T  dO_i    (A = P^T TMEM, B = dO smem MN-major)
 //   dK  += dS^T Q_i     (A = dS^T TMEM, B = Q smem MN-major)
-//   dQ_i = dS   K_j     (tile width 64: A = dS^T smem MN-major, B = K smem MN-major)
+//   dQ_i = dS   K_j     (A = dS^T smem MN-major, B = K smem MN-major)
 #pragma once
 
 #include <cuda_fp16.h>
@@ -65,9 +70,11 @@
 
 namespace fa2 {
 
-// Workspace: D [BH][Npad] f32 | L2 = LSE*log2(e) [BH][Npad] f32 | dQacc [BH][N][Dt] f32,
-// Dt the kernel's tile head dim (64 or 128).  The deterministic mode sums dQ in TMEM
-// (fa2_bwd_dq_kernel) and uses the two row statistics alone.
+// Workspace: D [BH][Npad] f32 | L2 = LSE*log2(e) [BH][Npad] f32 | dQacc [BH][N][Dt] f32
+// | tile counter (256 bytes), Dt the kernel's tile head dim (64 or 128).  The
+// deterministic mode sums dQ in TMEM (fa2_bwd_dq_kernel) and uses the row statistics
+// and the counter alone.  The counter hands out the key tiles of the persistent grid
+// (see the tile scheduler); the first kernel of a call zeroes it.
 inline size_t bwd_npad(int N) { return (static_cast<size_t>(N) + 127) / 128 * 128; }
 inline size_t bwd_rowstat_bytes(size_t BH, int N) {
   return (2 * BH * bwd_npad(N) * 4 + 255) / 256 * 256;
@@ -75,9 +82,9 @@ inline size_t bwd_rowstat_bytes(size_t BH, int N) {
 // Kernel head dim for a head dim d <= 128: the tiles are 64 or 128 columns wide.
 inline int bwd_tile_dim(int d) { return d <= 64 ? 64 : 128; }
 inline size_t bwd_workspace_bytes(size_t BH, int N, int d, bool deterministic = false) {
-  if (deterministic) return bwd_rowstat_bytes(BH, N);
-  return bwd_rowstat_bytes(BH, N) +
-         (BH * static_cast<size_t>(N) * bwd_tile_dim(d) * 4 + 255) / 256 * 256;
+  const size_t acc =
+      deterministic ? 0 : (BH * static_cast<size_t>(N) * bwd_tile_dim(d) * 4 + 255) / 256 * 256;
+  return bwd_rowstat_bytes(BH, N) + acc + 256;
 }
 // Kernels one backward call launches: preprocess, main and dQ finalisation; in the
 // deterministic mode the dQ kernel and the dK/dV kernel.
@@ -91,8 +98,8 @@ template <int D, bool BF16>
 __global__ void __launch_bounds__(256)
 fa2_bwd_pre_kernel(const uint16_t* __restrict__ O, const uint16_t* __restrict__ dO,
                    const float* __restrict__ LSE, float* __restrict__ Dg,
-                   float* __restrict__ Lg, float* __restrict__ dQacc, int N, int Npad,
-                   long long total_rows, int d) {
+                   float* __restrict__ Lg, float* __restrict__ dQacc, unsigned int* __restrict__ tile_ctr,
+                   int N, int Npad, long long total_rows, int d) {
   constexpr int TPR = D / 8;  // threads per row, 8 elements (16 bytes) each
   constexpr int RPB = 256 / TPR;
   // Launched behind the caller's previous kernel (the forward, typically) with
@@ -100,6 +107,7 @@ fa2_bwd_pre_kernel(const uint16_t* __restrict__ O, const uint16_t* __restrict__ 
   // for O and LSE.
   griddep_launch_dependents();
   griddep_wait();
+  if (blockIdx.x == 0 && threadIdx.x == 0) *tile_ctr = 0u;
   const int sub = threadIdx.x % TPR;
   const long long r = static_cast<long long>(blockIdx.x) * RPB + threadIdx.x / TPR;
   const bool in_range = r < total_rows;  // no early exit: the shuffle below is warp-wide
@@ -185,6 +193,8 @@ struct BwdParams {
   unsigned int* status;
   unsigned long long wait_ns;
   int fault;          // test hook: 1 = skip the K, V load (a consumer's wait runs out)
+  unsigned int* tile_ctr;  // tiles handed out past the first two rounds (zeroed by the first kernel)
+  int dynamic;        // 1: tiles past the first two rounds from tile_ctr; 0: snake order
 };
 
 template <int D, bool DQ_>
@@ -215,7 +225,7 @@ struct BwdCfg {
   // LSE*log2e and D rows of each stage: loaded with Q in the fused D = 128 kernel,
   // with dO otherwise.
   static constexpr int LD_BYTES = ST * 2 * 128 * 4;
-  static constexpr int CTRL_BYTES = 256;              // barriers, TMEM address, abort flag
+  static constexpr int CTRL_BYTES = 512;  // barriers, tile ring, TMEM address, abort flag
   // No alignment slack: the dynamic region must start 1024-byte aligned (checked).
   static constexpr int SMEM = (2 * KVB + QS + ST) * TILE + DS_BYTES + LD_BYTES + CTRL_BYTES;
   static_assert(SMEM <= 227 * 1024, "shared memory");
@@ -243,10 +253,16 @@ struct BwdCfg {
 
 // Control block at the end of the dynamic shared memory (no static shared memory,
 // so that the 1024-byte aligned tiles start at the base of the window).
+// Depth of the ring through which the producer hands the CTA's tile sequence to the
+// MMA and compute roles.
+constexpr int kTileRing = 4;
+
 template <int ST>
 struct BwdCtrl {
   uint64_t bar_kv[2], kv_empty[2], acc_free, qdo_full[ST], qdo_empty[ST], q_full[3], q_empty[3];
   uint64_t s_full, s_read, dp_full, p_ready, ds_ready, dq_full, dq_drained, drain, fin;
+  uint64_t tile_full[kTileRing], tile_empty[kTileRing];
+  int tile_ring[kTileRing];
   uint32_t tmem_slot;
   int abort_flag;
 };
@@ -263,7 +279,7 @@ __device__ __forceinline__ void bulk_load_1d(void* smem_dst, const void* gmem_sr
 enum BwdSite : uint32_t {
   kBSiteAlign = 31, kBSiteProdEmpty = 32, kBSiteMmaKV, kBSiteMmaQ, kBSiteMmaDrained, kBSiteMmaP, kBSiteMmaDS,
   kBSiteMmaDrain, kBSiteCmpQ, kBSiteCmpS, kBSiteCmpDP, kBSiteCmpDQ, kBSiteProdDrain, kBSiteMmaAcc,
-  kBSiteProdKV
+  kBSiteProdKV, kBSiteProdTile, kBSiteMmaTile, kBSiteCmpTile
 };
 
 template <int D, bool BF16, bool CAUSAL, bool DQ>
@@ -318,11 +334,18 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   // (causal: key tile j is seen by query tiles j .. n - 1, so the work falls with
   // j): list position t of group g0 = t / (HG n) is tile j = p / hg of head
   // g0 HG + p % hg, p = t mod HG n, hg the group's head count.  The grid has at most
-  // one CTA per SM, and CTA c runs tiles c, 2G - 1 - c, 2G + c, 4G - 1 - c, ... of
-  // the list (G CTAs: a snake over it), so that every CTA gets about the same number
-  // of query steps and pays its set-up once.  A group spans about two rounds of the
-  // snake, so the CTAs running at any one time share a few heads, whose K, V, Q, dO
-  // and dQ accumulator rows then stay in L2 (HG = BH lists every head at once).
+  // one CTA per SM; CTA c starts with positions c and 2G - 1 - c (G CTAs: a heavy
+  // and a light tile of the first two rounds).  Its later tiles (p.dynamic) are the
+  // next free positions of the list, taken from a counter in global memory by the
+  // producer as the CTA starts the tile two before (the atomic's latency stays off
+  // the critical path, and the next tile's K and V can be loaded ahead): the CTAs
+  // work down the list together, each taking new work as it finishes, so that they
+  // end within about a tile of each other whatever the mix of tile sizes.  Otherwise
+  // they continue the snake, 2G + c, 4G - 1 - c, ..., which balances lists of equal
+  // tiles and short lists.  The CTAs running at any one time share a few heads,
+  // whose K, V, Q, dO and dQ accumulator rows then stay in L2 (HG = BH lists every
+  // head at once).  The producer passes the sequence to the other roles through a
+  // ring in shared memory; -1 ends it.
   // (The helpers below copy what they need from p: capturing the kernel parameter
   // itself would take its address and copy it to local memory.)
   const int G = static_cast<int>(gridDim.x);
@@ -330,9 +353,10 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   const int BH = p.BH;
   const int win = p.window;
   const int T = n_q * BH;
-  auto tile_of = [=](int k) {
-    const int t = k * G + ((k & 1) ? G - 1 - cta : cta);
-    return t < T ? t : -1;
+  const bool dyn = p.dynamic != 0;
+  auto snake_tile = [=](int k) {  // the CTA's tile k in snake order (-1: none)
+    const long long t = static_cast<long long>(k) * G + ((k & 1) ? G - 1 - cta : cta);
+    return t < T ? static_cast<int>(t) : -1;
   };
   const int HG = p.head_group;
   auto tile_j = [=](int t) {  // key tile of list position t
@@ -367,6 +391,8 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       mbar_init(&qdo_empty[s], (C::DQ && !C::PIPE) ? 2 : 1);
     }
     for (int s = 0; s < 3; ++s) { mbar_init(&q_full[s], 1); mbar_init(&q_empty[s], 1); }
+    // a tile id is read by the MMA thread and by the 8 compute warps
+    for (int s = 0; s < kTileRing; ++s) { mbar_init(&ctl.tile_full[s], 1); mbar_init(&ctl.tile_empty[s], 9); }
     mbar_init(&s_full, 1);
     mbar_init(&dp_full, 1);
     mbar_init(&p_ready, 8);
@@ -398,9 +424,8 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       // K and V of the CTA's tile k into its buffer (the test hook skips them: a
       // consumer's wait then runs out).
       const bool skip_kv = p.fault == 1;
-      auto load_kv = [&](int k) {
+      auto load_kv = [&](int k, int t) {
         if (skip_kv) return;
-        const int t = tile_of(k);
         const int b = k % C::KVB;
         const int row = tile_j(t) * 128, bh = tile_bh(t);
         mbar_arrive_expect_tx(&bar_kv[b], 2 * C::TILE);
@@ -415,15 +440,37 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       // with an early trigger) may still be writing K or V.  The L, D rows and the
       // zeroed dQ accumulator come from the preprocess itself.
       const uint64_t keep = policy_evict_last();
-      griddep_wait();
-      load_kv(0);
-      if (C::KVB == 2 && tile_of(1) >= 0) load_kv(1);
+      // The CTA's tile kk >= 2 (-1 past the end of the list): the next free list
+      // position past the first two rounds, or the snake's; and tile k's id into the
+      // ring.
+      auto grab = [&](int kk) -> int {
+        if (!dyn) return snake_tile(kk);
+        const long long t = 2LL * G + atomicAdd(p.tile_ctr, 1u);
+        return t < T ? static_cast<int>(t) : -1;
+      };
+      // Tiles 0 and 1 are the snake's in both modes: the ring carries tiles 2, 3, ...
+      auto publish = [&](int k, int t) -> bool {
+        if (!dyn) return true;  // the other roles follow the snake themselves
+        const int q = k - 2, s = q % kTileRing;
+        if (q >= kTileRing &&
+            !mbar_wait(&ctl.tile_empty[s], ((q / kTileRing) - 1) & 1, wc, kBSiteProdTile))
+          return false;
+        ctl.tile_ring[s] = t;
+        mbar_arrive(&ctl.tile_full[s]);
+        return true;
+      };
+      griddep_wait();  // also orders the counter's zeroing before the first grab
+      // Tiles k, k + 1 and k + 2 of the CTA (-1: none).
+      int t_cur = snake_tile(0);
+      int t_nx = t_cur >= 0 ? snake_tile(1) : -1;
+      int t_nx2 = -1;
+      bool ok = true;
+      if (t_cur >= 0) load_kv(0, t_cur);
+      if (C::KVB == 2 && t_nx >= 0) load_kv(1, t_nx);
       int gs = 0;  // query steps issued so far (ring slot and phase)
       int gq = 0;  // tile width 128: Q loads issued (may run one ahead of gs on an abort)
-      bool ok = true;
-      for (int k = 0; ok; ++k) {
-        const int t = tile_of(k);
-        if (t < 0) break;
+      for (int k = 0; ok && t_cur >= 0; ++k) {
+        const int t = t_cur;
         const int bh = tile_bh(t);
         const int i0 = q_begin(tile_j(t)), n_it = q_end(tile_j(t)) - i0;
         for (int it = 0; it < n_it; ++it) {
@@ -468,24 +515,35 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                              row, bh, keep);
           }
           ++gs;
+          // Tile k + 2 is taken once tile k's first loads are out, and handed on at
+          // the end of tile k (the atomic's result is not waited for before then).
+          if (it == 0 && t_nx >= 0) t_nx2 = grab(k + 2);
           // The next K, V load.  Two buffers: tile k + 1's, a step or two into tile
           // k, once tile k - 1 has released the buffer.  One buffer: tile k's own,
           // right after its first (Q, dO) load, once tile k - 1's last product has
           // read the buffer.
-          int nk = -1;
+          int nk = -1, nt = -1;
           if (C::KVB == 2) {
-            if (k >= 1 && it == min(C::ST, n_it - 1) && tile_of(k + 1) >= 0) nk = k + 1;
+            if (k >= 1 && it == min(C::ST, n_it - 1) && t_nx >= 0) nk = k + 1, nt = t_nx;
           } else if (k >= 1 && it == 0) {
-            nk = k;
+            nk = k, nt = t;
           }
           if (nk >= 0) {
             if (!mbar_wait(&kv_empty[nk % C::KVB], kv_par(nk - C::KVB), wc, kBSiteProdKV)) {
               ok = false;
               break;
             }
-            load_kv(nk);
+            load_kv(nk, nt);
           }
         }
+        if (!ok) break;
+        if (t_nx >= 0 && !publish(k + 2, t_nx2)) {
+          ok = false;
+          break;
+        }
+        t_cur = t_nx;
+        t_nx = t_nx2;
+        t_nx2 = -1;
       }
       volatile int no_abort = 0;
       WaitCtl dw{p.status, &no_abort, 100000000ull};
@@ -565,7 +623,13 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       bool ok = true;
       int gs = 0;  // query steps so far
       for (int k = 0; ok; ++k) {
-        const int t = tile_of(k);
+        int t = snake_tile(k);
+        if (dyn && k >= 2) {
+          const int ts = (k - 2) % kTileRing;
+          if (!mbar_wait(&ctl.tile_full[ts], ((k - 2) / kTileRing) & 1, wc, kBSiteMmaTile)) { ok = false; break; }
+          t = ctl.tile_ring[ts];
+          mbar_arrive(&ctl.tile_empty[ts]);
+        }
         if (t < 0) break;
         const int n_it = q_end(tile_j(t)) - q_begin(tile_j(t));
         const int b = k % C::KVB;
@@ -999,7 +1063,18 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       return true;
     };
     for (int k = 0; ok; ++k) {
-      const int t = tile_of(k);
+      int t = snake_tile(k);
+      if (dyn && k >= 2) {
+        const int ts = (k - 2) % kTileRing;
+        if (!named_bar_and(wg_bar, 128,
+                           mbar_wait(&ctl.tile_full[ts], ((k - 2) / kTileRing) & 1, wc, kBSiteCmpTile))) {
+          ok = false;
+          break;
+        }
+        t = ctl.tile_ring[ts];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ctl.tile_empty[ts]);
+      }
       if (t < 0) break;
       const int j = tile_j(t), bh = tile_bh(t);
       const int key = j * 128 + r;
@@ -1110,6 +1185,9 @@ int launch_bwd_t(const void* Q, const void* K, const void* V, const void* O, con
   if (static_cast<long long>(Npad / 128) * BH > (1ll << 30)) return 1;  // FA2_ERR_INVALID_ARG
   float* Dg = static_cast<float*>(workspace);
   float* Lg = Dg + static_cast<size_t>(BH) * Npad;
+  unsigned int* tile_ctr = reinterpret_cast<unsigned int*>(
+      static_cast<uint8_t*>(workspace) +
+      bwd_workspace_bytes(static_cast<size_t>(BH), N, d, !Cfg::DQ) - 256);
   // The fp32 dQ accumulator (tile width 64 only) follows the row statistics.
   float* dQacc = Cfg::DQ ? reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
                                                     bwd_rowstat_bytes(static_cast<size_t>(BH), N))
@@ -1149,6 +1227,7 @@ int launch_bwd_t(const void* Q, const void* K, const void* V, const void* O, con
     qp.status = status;
     qp.wait_ns = wait_ns;
     qp.fault = fault;
+    qp.tile_ctr = tile_ctr;
     if (launch_pdl(kq, dim3(static_cast<unsigned int>(grid)), dim3(BwdDqCfg::THREADS),
                    BwdDqCfg::SMEM, stream, mq, mk, mv, mdo, qp) != cudaSuccess)
       return 4;
@@ -1159,7 +1238,7 @@ int launch_bwd_t(const void* Q, const void* K, const void* V, const void* O, con
     const unsigned int grid = static_cast<unsigned int>((rows + RPB - 1) / RPB);
     if (launch_pdl(fa2_bwd_pre_kernel<D, BF16>, dim3(grid), dim3(256), 0, stream,
                    static_cast<const uint16_t*>(O), static_cast<const uint16_t*>(dO), LSE, Dg, Lg,
-                   dQacc, N, Npad, rows, d) != cudaSuccess)
+                   dQacc, tile_ctr, N, Npad, rows, d) != cudaSuccess)
       return 4;
   }
   // 2. main (dK, dV; and, by default, the dQ partials)
@@ -1184,6 +1263,7 @@ int launch_bwd_t(const void* Q, const void* K, const void* V, const void* O, con
     bp.status = status;
     bp.wait_ns = wait_ns;
     bp.fault = fault;
+    bp.tile_ctr = tile_ctr;
     // Persistent grid: one CTA per SM at most (the kernel's shared memory and TMEM
     // admit one per SM), each running its share of the tile list.
     int dev = 0, n_sm = 0;
@@ -1195,17 +1275,26 @@ int launch_bwd_t(const void* Q, const void* K, const void* V, const void* O, con
     }
     long long ctas = std::min(static_cast<long long>(bp.n_kv) * BH, static_cast<long long>(n_sm));
     if (max_ctas > 0) ctas = std::min(ctas, static_cast<long long>(max_ctas));
-    // Heads per group: a group of the tile list spans about two rounds of the snake,
-    // but holds at most ~32 MB of K, V, Q, dO (16-bit) and fp32 dQ rows.  Measured on
-    // B200 (every head at once -> groups of two rounds): training-shape backward 2.08
-    // -> 1.87 ms, its deterministic mode 2.30 -> 2.20 ms, sliding window 1.08 -> 1.05
-    // ms; groups of one round: training shape 1.83 ms but the d = 64 bench-shape
-    // backward 72.7 -> 80.9 us -- the 32 MB cap gives the training shape the smaller
-    // groups (5 heads) and leaves that shape's (37) alone.
+    // Tiles past the first two rounds from the counter (dynamic) on causal lists of
+    // at least 8 tiles per CTA, whose tile sizes vary; the snake otherwise (equal
+    // tiles, or too few for the counter to pay).  Heads per group: dynamic, about
+    // 192 MB of K, V, Q, dO (16-bit) and fp32 dQ rows, and at least two rounds of
+    // tiles; snake, about two rounds, capped at ~32 MB of rows.  Measured on B200
+    // (backward, ms; snake with the capped groups -> dynamic): training shape B8 H16
+    // N4096 d128 causal 1.772 (5 heads) -> 1.729 (32), its deterministic mode 2.236
+    // -> 2.160 (32), B1 H16 N16384 causal 3.69 (1) -> 2.99 (8); dynamic with the
+    // snake's groups was slower on the training shape (1.82) and the counter on the
+    // d = 64 bench shape B4 H16 N1024 (512 tiles) 70.6 -> 80.9 us.  The snake's
+    // groups: every head at once -> two rounds took the training shape from 2.08 to
+    // 1.87 ms; one round gave 1.83 ms but slowed the d = 64 shape 72.7 -> 80.9 us,
+    // hence the 32 MB cap (5 heads there, that shape's 37 untouched).
     {
-      long long hg = (2 * ctas + bp.n_kv - 1) / bp.n_kv;
+      const long long T = static_cast<long long>(bp.n_kv) * BH;
+      bp.dynamic = (CAUSAL && T >= 8 * ctas) ? 1 : 0;
       const long long per_head = 12LL * N * D;  // bytes of one head's rows (see above)
-      hg = std::min(hg, (32LL << 20) / per_head);
+      const long long two_rounds = (2 * ctas + bp.n_kv - 1) / bp.n_kv;
+      const long long hg = bp.dynamic ? std::max(two_rounds, (192LL << 20) / per_head)
+                                      : std::min(two_rounds, (32LL << 20) / per_head);
       bp.head_group = static_cast<int>(std::min<long long>(BH, std::max<long long>(1, hg)));
     }
     const unsigned int grid = static_cast<unsigned int>(ctas);

@@ -59,6 +59,7 @@ struct BwdDqParams {
   unsigned int* status;
   unsigned long long wait_ns;
   int fault;             // test hook: 1 = skip the first K load (a wait runs out)
+  unsigned int* tile_ctr;  // the dK/dV kernel's tile counter, zeroed here (it runs next)
 };
 
 struct BwdDqCfg {
@@ -163,8 +164,10 @@ fa2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
       tma_prefetch_desc(&tmV);
       tma_prefetch_desc(&tmdO);
       // Nothing is read before the previous grid on the stream (the forward that
-      // wrote O and LSE, typically) has completed.
+      // wrote O and LSE, typically) has completed; the counter is zeroed after it
+      // too (that grid may be the previous call's dK/dV kernel, still using it).
       griddep_wait();
+      if (blockIdx.x == 0) *p.tile_ctr = 0u;
       mbar_arrive_expect_tx(&ctl.bar_qdo, C::TILE);
       for (int c = 0; c < C::KCH; ++c)
         tma_load_3d(sdO + c * C::CHUNK, &tmdO, &ctl.bar_qdo, c * 64, row0, bh);

@@ -181,7 +181,8 @@ int fa2_fwd_fp8(const void* Q, const void* K, const void* V, void* O, float* LSE
 
 /*
  * Bytes of device workspace fa2_bwd needs for these sizes (the per-row
- * D = rowsum(dO * O) and a float32 dQ accumulator), a multiple of 256.
+ * D = rowsum(dO * O) and LSE * log2 e, a 256-byte counter that hands out the
+ * key tiles, and a float32 dQ accumulator), a multiple of 256.
  * Returns 0 for sizes fa2_bwd would reject.
  */
 size_t fa2_bwd_workspace_size(int B, int H, int N, int d);
@@ -233,7 +234,7 @@ enum { FA2_BWD_DETERMINISTIC = 1 };
  *     come from a kernel without the dQ product.  Seven matrix products per tile
  *     pair instead of five, on 128-wide tiles at every head dim: measured on B200
  *     about 7 % slower than the default at d = 128, about twice the time at d = 64.
- *     The workspace holds only the two per-row statistics.
+ *     The workspace holds only the two per-row statistics and the tile counter.
  *
  * Arguments, layouts, results and errors otherwise as fa2_bwd (and
  * fa2_bwd_window); flags other than FA2_BWD_DETERMINISTIC, window < 0 or a window

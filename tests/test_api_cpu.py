@@ -84,13 +84,13 @@ def test_fwd_overlap_checks_use_each_buffer_size(lib):
 def test_bwd_validation_without_device(lib):
     ws = fa2.fa2_bwd_workspace_size(2, 3, 1000, 128)
     assert ws > 0 and ws % 256 == 0
-    # D and LSE*log2(e) padded to 128 rows per head, then the fp32 dQ accumulator, as
-    # wide as the kernel's tile (64 or 128 columns)
-    assert ws == 2 * 2 * 3 * 1024 * 4 + 2 * 3 * 1000 * 128 * 4
-    assert fa2.fa2_bwd_workspace_size(2, 3, 1000, 64) == 2 * 2 * 3 * 1024 * 4 + 2 * 3 * 1000 * 64 * 4
-    # the deterministic mode keeps the two row statistics only
-    assert fa2.fa2_bwd_ex_workspace_size(2, 3, 1000, 128, fa2.FA2_BWD_DETERMINISTIC) == 2 * 2 * 3 * 1024 * 4
-    assert fa2.fa2_bwd_ex_workspace_size(2, 3, 1000, 64, fa2.FA2_BWD_DETERMINISTIC) == 2 * 2 * 3 * 1024 * 4
+    # D and LSE*log2(e) padded to 128 rows per head, the 256-byte tile counter, then
+    # the fp32 dQ accumulator, as wide as the kernel's tile (64 or 128 columns)
+    assert ws == 2 * 2 * 3 * 1024 * 4 + 256 + 2 * 3 * 1000 * 128 * 4
+    assert fa2.fa2_bwd_workspace_size(2, 3, 1000, 64) == 2 * 2 * 3 * 1024 * 4 + 256 + 2 * 3 * 1000 * 64 * 4
+    # the deterministic mode keeps the two row statistics and the counter only
+    assert fa2.fa2_bwd_ex_workspace_size(2, 3, 1000, 128, fa2.FA2_BWD_DETERMINISTIC) == 2 * 2 * 3 * 1024 * 4 + 256
+    assert fa2.fa2_bwd_ex_workspace_size(2, 3, 1000, 64, fa2.FA2_BWD_DETERMINISTIC) == 2 * 2 * 3 * 1024 * 4 + 256
     assert fa2.fa2_bwd_ex_workspace_size(2, 3, 1000, 128, 0) == ws
     assert fa2.fa2_bwd_ex_workspace_size(2, 3, 1000, 128, 2) == 0  # unknown flag
     assert fa2.fa2_bwd_workspace_size(2, 3, 1000, 100) == 0  # d % 8 != 0
@@ -298,9 +298,10 @@ def test_forward_tiles_per_cta_rejects_bad_sizes(lib):
 # "FlashAttention-2" (systems-analysis.info wiki), "Предпосылки": the tiled method
 # needs memory linear in the sequence length, because no N x N matrix is stored.
 # The forward takes no scratch at all; the backward's scratch is two float rows per
-# query (D and LSE * log2 e, padded to 128 rows) and a float dQ accumulator of one
-# row per query, as wide as the kernel's tile (64 or 128 columns); the deterministic
-# mode, which sums dQ in tensor memory, needs the two rows alone.
+# query (D and LSE * log2 e, padded to 128 rows), a 256-byte tile counter and a float
+# dQ accumulator of one row per query, as wide as the kernel's tile (64 or 128
+# columns); the deterministic mode, which sums dQ in tensor memory, needs the rows and
+# the counter alone.
 
 @pytest.mark.parametrize("d", [32, 64, 96, 128])
 def test_bwd_workspace_is_linear_in_sequence_length(lib, d):
@@ -309,12 +310,13 @@ def test_bwd_workspace_is_linear_in_sequence_length(lib, d):
     for N in (128, 1024, 4096, 32768):
         ws = lib.fa2_bwd_workspace_size(B, H, N, d)
         rows = B * H * ((N + 127) // 128 * 128)
-        expect = (2 * rows * 4 + 255) // 256 * 256 + (B * H * N * tile * 4 + 255) // 256 * 256
+        expect = (2 * rows * 4 + 255) // 256 * 256 + 256 + (B * H * N * tile * 4 + 255) // 256 * 256
         assert ws == expect
-        assert lib.fa2_bwd_ex_workspace_size(B, H, N, d, 1) == (2 * rows * 4 + 255) // 256 * 256
+        assert lib.fa2_bwd_ex_workspace_size(B, H, N, d, 1) == (2 * rows * 4 + 255) // 256 * 256 + 256
         # O(B H N d): at most 8 bytes per head element plus the row statistics
-        assert ws <= B * H * N * (8 * d) + 2 * rows * 4 + 512
-        assert lib.fa2_bwd_workspace_size(B, H, 2 * N, d) == 2 * ws  # doubles with N
+        assert ws <= B * H * N * (8 * d) + 2 * rows * 4 + 768
+        # all but the counter doubles with N
+        assert lib.fa2_bwd_workspace_size(B, H, 2 * N, d) - 256 == 2 * (ws - 256)
 
 
 def test_noalloc_rejects_sizes_beyond_its_buffer_before_any_device_call(lib):

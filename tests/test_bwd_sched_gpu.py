@@ -1,11 +1,11 @@
 """GPU parity of the backward's persistent tile scheduler.
 
-The backward runs at most one CTA per SM; each CTA walks its share of the key
-tiles (heaviest first, in snake order over the CTAs), carrying its barrier phases,
-its (Q, dO) ring and its K/V buffers from one tile to the next.  Small problems
-have fewer tiles than SMs, so the test hook ``fa2_debug_set_bwd_grid`` caps the
-grid to make every CTA run many tiles: one CTA running all of them, and counts
-that do not divide the tile count.  dK and dV of a key tile do not depend on which
+The backward runs at most one CTA per SM; each CTA starts with one key tile and
+then takes the next free one from a counter in the workspace, carrying its barrier
+phases, its (Q, dO) ring, its K/V buffers and its tile ring from one tile to the
+next.  Small problems have fewer tiles than SMs, so the test hook
+``fa2_debug_set_bwd_grid`` caps the grid to make every CTA run many tiles: one CTA
+running all of them, and counts that do not divide the tile count.  dK and dV of a key tile do not depend on which
 CTA computed them (bitwise equal to the uncapped run); dQ is summed by float
 reductions whose order may change (checked against the oracle).  Tolerances as
 elsewhere: gradients 1e-2 x max|reference|.
