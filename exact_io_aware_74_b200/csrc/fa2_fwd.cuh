@@ -236,7 +236,13 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 
   WaitCtl wc{p.status, &abort_flag, p.wait_ns};
 
-  if (threadIdx.x == 0) {
+  // The producer thread sets up the barriers and sends Q and the first K tile out
+  // at once, so that their latency overlaps the TMEM allocation and the block-wide
+  // barrier (a CTA's set-up up to its first scores took 2.8 us on the training
+  // shape, 0.9 us of it before the first load).
+  const bool prod0 = warp == 8 && lane == 0;
+  bool k0_early = false;  // K tile 0 issued in the set-up
+  if (prod0) {
     abort_flag = 0;
     mbar_init(&bar_q, 1);
     for (int s = 0; s < C::KS; ++s) { mbar_init(&k_full[s], 1); mbar_init(&k_empty[s], 1); }
@@ -249,6 +255,36 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     }
     mbar_init(&drain, 1);
     fence_mbar_init();
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+    uint32_t q_bytes = 0;
+    for (int t = 0; t < 2; ++t) q_bytes += (j_hi[t] > 0) ? C::TILE : 0;
+    // (A CTA whose split holds no key any of its rows sees loads nothing.)
+    mbar_arrive_expect_tx(&bar_q, q_bytes);
+    if constexpr (REP > 1) {
+      // REP copies of rows 0 .. 128/REP - 1 (tile 0 only), one box each.
+      if (j_hi[0] > 0) {
+        tma_prefetch_desc(&tmQr);
+        constexpr int qr = C::BM / REP;
+        for (int r = 0; r < REP; ++r)
+          for (int c = 0; c < C::KCH; ++c)
+            tma_load_3d(sQ + c * C::CHUNK + r * qr * 128, &tmQr, &bar_q, c * C::CHUNK_COLS, 0, bh);
+      }
+    } else {
+      for (int t = 0; t < 2; ++t) {
+        if (j_hi[t] == 0) continue;
+        for (int c = 0; c < C::KCH; ++c)
+          tma_load_3d(sQ + t * C::TILE + c * C::CHUNK, &tmQ, &bar_q, c * C::CHUNK_COLS, row0[t], bh);
+      }
+    }
+    if (n_steps > 0 && p.fault != 1) {  // the test hook skips K tile 0 (see load_k)
+      const uint64_t keep = policy_evict_last();
+      mbar_arrive_expect_tx(&k_full[0], C::TILE);
+      for (int c = 0; c < C::KCH; ++c)
+        tma_load_3d_hint(sK + c * C::CHUNK, &tmK, &k_full[0], c * 64, j0 * C::BN, bh, keep);
+      k0_early = true;
+    }
   }
   if (warp == 0) {
     tmem_alloc(&tmem_slot, 512);
@@ -267,34 +303,16 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   } else if (warp == 8) {
     // ------------------------------------------------------------------ producer
     if (lane == 0) {
-      tma_prefetch_desc(&tmQ);
-      tma_prefetch_desc(&tmK);
-      tma_prefetch_desc(&tmV);
+      // Q and K tile 0 went out in the set-up.
       const uint64_t keep = policy_evict_last();
-      uint32_t q_bytes = 0;
-      for (int t = 0; t < 2; ++t) q_bytes += (j_hi[t] > 0) ? C::TILE : 0;
-      // (A CTA whose split holds no key any of its rows sees loads nothing.)
-      mbar_arrive_expect_tx(&bar_q, q_bytes);
-      if constexpr (REP > 1) {
-        // REP copies of rows 0 .. 128/REP - 1 (tile 0 only), one box each.
-        if (j_hi[0] > 0) {
-          tma_prefetch_desc(&tmQr);
-          constexpr int qr = C::BM / REP;
-          for (int r = 0; r < REP; ++r)
-            for (int c = 0; c < C::KCH; ++c)
-              tma_load_3d(sQ + c * C::CHUNK + r * qr * 128, &tmQr, &bar_q, c * C::CHUNK_COLS, 0, bh);
-        }
-      } else {
-        for (int t = 0; t < 2; ++t) {
-          if (j_hi[t] == 0) continue;
-          for (int c = 0; c < C::KCH; ++c)
-            tma_load_3d(sQ + t * C::TILE + c * C::CHUNK, &tmQ, &bar_q, c * C::CHUNK_COLS, row0[t], bh);
-        }
-      }
       // With one query tile the second Q slot (if any) is one more V stage.
       const int vring = single ? C::VS + C::VX : C::VS;
       int k_issued = 0, v_issued = 0;  // loads issued so far
       auto load_k = [&](int jj) -> bool {
+        if (jj == 0 && k0_early) {
+          k_issued = 1;
+          return true;
+        }
         const int ks = jj % C::KS;
         if (jj >= C::KS && !mbar_wait(&k_empty[ks], ((jj / C::KS) - 1) & 1, wc, kSiteProdKEmpty))
           return false;
