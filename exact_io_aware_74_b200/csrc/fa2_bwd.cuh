@@ -344,8 +344,9 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   // they continue the snake, 2G + c, 4G - 1 - c, ..., which balances lists of equal
   // tiles and short lists.  The CTAs running at any one time share a few heads,
   // whose K, V, Q, dO and dQ accumulator rows then stay in L2 (HG = BH lists every
-  // head at once).  The producer passes the sequence to the other roles through a
-  // ring in shared memory; -1 ends it.
+  // head at once).  With the counter, the producer passes tiles 2, 3, ... to the
+  // other roles through a ring in shared memory (-1 ends the sequence); snake
+  // positions every role computes itself.
   // (The helpers below copy what they need from p: capturing the kernel parameter
   // itself would take its address and copy it to local memory.)
   const int G = static_cast<int>(gridDim.x);
